@@ -1,0 +1,86 @@
+// af_internal.h -- declarations shared by the library's translation units.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace af {
+
+// Epilogues fused into the tensor-core GEMM.
+enum GemmMode : int {
+  EPI_STORE = 0,     // C = acc (bf16), optional output row remap
+  EPI_GATE_RES = 1,  // x += gate[b] * acc   (adaLN-Zero gated residual)
+  EPI_SWIGLU = 2,    // h = silu(acc[W1 half]) * acc[W2 half]
+  EPI_QKV = 3,       // per-head LayerNorm of Q and K, scatter to [B, H, N, hd]
+};
+
+struct GemmParams {
+  int M, N, K;        // acc[M, N] = A[M, K] * W[N, K]^T  (EPI_SWIGLU: N = output width F)
+  int mode;
+  int rows_per_batch;      // sample index of GEMM row r is r / rows_per_batch
+  int out_rows_per_batch;  // output rows per sample
+  int out_row_off;         // first output row of each sample
+  uint16_t* out;           // STORE / SWIGLU output, GATE_RES residual (in/out)
+  int ldo;                 // row stride of `out` in elements
+  const float* gate;       // GATE_RES: gate of sample b at gate[b * gate_stride + col]
+  int gate_stride;
+  uint16_t* q;             // QKV: destinations [B, heads, n_total, hd]
+  uint16_t* k;
+  uint16_t* v;
+  int heads, hd, n_total, qkv_row_off, D;
+  float eps;
+  int swiglu_w2_row;       // SWIGLU: first row of W2 inside the packed weight
+  int num_m_tiles, num_n_tiles, num_tiles;
+  int* err;                // device error word
+};
+
+constexpr int GEMM_BM = 128;
+constexpr int GEMM_BN = 256;
+constexpr int GEMM_BK = 64;
+constexpr int GEMM_STAGES = 4;
+constexpr int GEMM_THREADS = 192;
+constexpr int GEMM_SMEM_BYTES = GEMM_STAGES * (GEMM_BM + GEMM_BN) * GEMM_BK * 2 + 1024 /*barriers*/ + 1024 /*align*/;
+
+// Host helpers (gemm.cu)
+bool encode_tmap_2d(CUtensorMap* map, const void* ptr, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                    uint32_t box_inner, uint32_t box_outer);
+bool encode_tmap_3d(CUtensorMap* map, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1_bytes,
+                    uint64_t s2_bytes, uint32_t b0, uint32_t b1, uint32_t b2);
+cudaError_t launch_gemm(const GemmParams& p_in, const void* A, const void* W, int W_rows, cudaStream_t stream,
+                        int num_sms);
+int device_sm_count();
+
+// Attention (attention.cu)
+struct AttnParams {
+  int B, H, N, hd;
+  // output row r (< N) of sample b goes to
+  //   r <  split: out_a + (b * split + r) * ldo + h * hd
+  //   r >= split: out_b + (b * (N - split) + r - split) * ldo + h * hd
+  uint16_t* out_a;
+  uint16_t* out_b;
+  int split;
+  int ldo;
+  float scale_log2;  // softmax scale * log2(e)
+  int* err;
+};
+cudaError_t launch_attention(const AttnParams& p, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                             cudaStream_t stream);
+
+// Small kernels (kernels.cu)
+cudaError_t launch_ln_modulate(const uint16_t* x, const float* shift, const float* scale, int mod_stride,
+                               uint16_t* y, int rows, int rows_per_batch, int D, float eps, cudaStream_t s);
+cudaError_t launch_timestep_mlp(const float* t, int B, const uint16_t* w1, const uint16_t* b1, const uint16_t* w2,
+                                const uint16_t* b2, int C, int D, float* feat, float* h1, float* temb, cudaStream_t s);
+cudaError_t launch_modulation(const float* temb, int B, int D, const uint16_t* w, int rows, float* out,
+                              cudaStream_t s);
+cudaError_t launch_patch_embed(const float* lat, int B, int C, int H, int W, int p, const uint16_t* w_pe,
+                               const uint16_t* pos, int G, int D, uint16_t* out, int out_rows_per_batch,
+                               int out_row_off, cudaStream_t s);
+cudaError_t launch_output_stage(const uint16_t* x, int rows_per_batch, int row_off, int B, int hp, int wp, int D,
+                                const float* scale, const float* shift, int mod_stride, const uint16_t* w_out,
+                                int p, int C, float* vel, cudaStream_t s);
+cudaError_t launch_fill(float* dst, int n, float value, cudaStream_t s);
+cudaError_t launch_euler_cfg(float* lat, const float* v, int Bi, int64_t per_sample, float g, float sigma,
+                             float sigma_next, cudaStream_t s);
+
+}  // namespace af

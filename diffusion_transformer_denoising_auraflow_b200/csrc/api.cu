@@ -1,0 +1,901 @@
+// api.cu -- the C ABI (include/af.h): weight pack, scratch, block and forward
+// orchestration.  Every compute step runs in this library's kernels
+// (gemm.cu, attention.cu, kernels.cu); this file only checks arguments,
+// lays out memory and sequences launches on the caller's stream.
+//
+// Sequencing follows "Diffusers 中的 AuraFlowTransformer2DModel架构解析与源码级
+// 使用指南", §前向传播流程 (embed -> joint blocks -> cat(text, image) ->
+// single blocks -> image slice -> pre-final -> proj_out -> unpatchify), with
+// the block internals of §联合注意力块 / §单 DiT 块.
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <unordered_map>
+#include <vector>
+
+#include "af.h"
+#include "af_internal.h"
+
+using namespace af;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+af_status cuda_fail(cudaError_t e) {
+  g_last_error = cudaGetErrorString(e);
+  return AF_ERR_CUDA;
+}
+
+#define AF_CUDA(x)                              \
+  do {                                          \
+    cudaError_t e_ = (x);                       \
+    if (e_ != cudaSuccess) return cuda_fail(e_); \
+  } while (0)
+
+int isqrt_exact(int n) {
+  int g = 0;
+  while ((g + 1) * (g + 1) <= n) ++g;
+  return g * g == n ? g : -1;
+}
+
+int find_multiple(int n, int k) { return n % k == 0 ? n : n + k - n % k; }
+
+struct Derived {
+  int D, F, G, H, hd;
+};
+
+af_status derive(const af_config* c, Derived* d) {
+  if (!c) return AF_ERR_INVALID_ARG;
+  if (c->patch_size <= 0 || c->in_channels <= 0 || c->out_channels <= 0 || c->num_mmdit_layers < 0 ||
+      c->num_single_dit_layers < 0 || c->attention_head_dim <= 0 || c->num_attention_heads <= 0 ||
+      c->joint_attention_dim <= 0 || c->pos_embed_max_size <= 0 || c->num_register_tokens < 0 ||
+      c->timestep_channels <= 0 || c->timestep_channels % 2 != 0 || c->ffn_inner < 0 || !(c->ln_eps >= 0.f))
+    return AF_ERR_INVALID_ARG;
+  d->H = c->num_attention_heads;
+  d->hd = c->attention_head_dim;
+  d->D = d->H * d->hd;
+  d->F = c->ffn_inner > 0 ? c->ffn_inner : find_multiple(static_cast<int>(2.0 * (4.0 * d->D) / 3.0), 256);
+  d->G = isqrt_exact(c->pos_embed_max_size);
+  if (d->G <= 0) return AF_ERR_INVALID_ARG;
+  return AF_OK;
+}
+
+struct TensorInfo {
+  std::string name;
+  int ndim;
+  int64_t shape[2];
+  size_t offset;  // bytes into the pack
+  size_t numel() const { return ndim == 1 ? shape[0] : static_cast<size_t>(shape[0]) * shape[1]; }
+};
+
+}  // namespace
+
+struct af_weights {
+  af_config cfg;
+  Derived d;
+  int device;
+  uint8_t* base = nullptr;
+  size_t bytes = 0;
+  std::vector<TensorInfo> tensors;
+  std::unordered_map<std::string, int> index;
+  // adaLN region: rows of every modulation linear, contiguous, in unit order
+  size_t ada_rows = 0;
+  std::vector<size_t> unit_row;  // first row of unit u (joint i: 2i img, 2i+1 txt; single j: 2J + j)
+  size_t pf_row = 0;             // first row of norm_out
+
+  const uint16_t* ptr(const std::string& n) const {
+    auto it = index.find(n);
+    return it == index.end() ? nullptr : reinterpret_cast<const uint16_t*>(base + tensors[it->second].offset);
+  }
+};
+
+struct af_scratch {
+  const af_weights* w;
+  int max_b, max_ni, max_l, max_nt, max_n;
+  int device;
+  uint8_t* base = nullptr;
+  size_t bytes = 0;
+  int* err;
+  float *temb, *h1, *mods, *tfeat;
+  uint16_t *y, *q, *k, *v, *o, *h;
+  uint16_t *img, *txt, *x;
+  float *lat2, *vel, *tvec;  // denoise step: CFG-duplicated latents, velocity, model times
+  int sms;
+  // launch accounting / profiling (kernel classes: GEMM, attention, LN, other)
+  int64_t launches[AF_NUM_KERNEL_CLASSES] = {0, 0, 0, 0};
+  bool profiling = false;
+  std::vector<cudaEvent_t> pool;
+  size_t pool_used = 0;
+  struct Rec {
+    int cls;
+    size_t e0;
+    int n;
+    double work;
+  };
+  std::vector<Rec> recs;
+};
+
+namespace {
+
+void add_tensor(af_weights* w, size_t& off, const std::string& name, int64_t r, int64_t c, bool align = true) {
+  if (align) off = (off + 255) & ~size_t(255);
+  TensorInfo t;
+  t.name = name;
+  t.ndim = c > 0 ? 2 : 1;
+  t.shape[0] = r;
+  t.shape[1] = c > 0 ? c : 0;
+  t.offset = off;
+  w->index[name] = static_cast<int>(w->tensors.size());
+  w->tensors.push_back(t);
+  off += t.numel() * 2;
+}
+
+void build_layout(af_weights* w) {
+  const af_config& c = w->cfg;
+  const int D = w->d.D, F = w->d.F, p = c.patch_size;
+  size_t off = 0;
+  // adaLN-Zero / pre-final linears, one contiguous [rows, D] matrix
+  size_t row = 0;
+  w->unit_row.clear();
+  for (int i = 0; i < c.num_mmdit_layers; ++i) {
+    const std::string b = "joint_transformer_blocks." + std::to_string(i) + ".";
+    w->unit_row.push_back(row);
+    add_tensor(w, off, b + "norm1.linear.weight", 6 * D, D, row == 0);
+    row += 6 * D;
+    w->unit_row.push_back(row);
+    add_tensor(w, off, b + "norm1_context.linear.weight", 6 * D, D, false);
+    row += 6 * D;
+  }
+  for (int i = 0; i < c.num_single_dit_layers; ++i) {
+    w->unit_row.push_back(row);
+    add_tensor(w, off, "single_transformer_blocks." + std::to_string(i) + ".norm1.linear.weight", 6 * D, D,
+               row == 0);
+    row += 6 * D;
+  }
+  w->pf_row = row;
+  add_tensor(w, off, "norm_out.linear.weight", 2 * D, D, row == 0);
+  row += 2 * D;
+  w->ada_rows = row;
+  // blocks: q,k,v contiguous (fused QKV), linear_1, linear_2 contiguous (SwiGLU up)
+  for (int i = 0; i < c.num_mmdit_layers; ++i) {
+    const std::string b = "joint_transformer_blocks." + std::to_string(i) + ".";
+    add_tensor(w, off, b + "attn.to_q.weight", D, D);
+    add_tensor(w, off, b + "attn.to_k.weight", D, D, false);
+    add_tensor(w, off, b + "attn.to_v.weight", D, D, false);
+    add_tensor(w, off, b + "attn.add_q_proj.weight", D, D);
+    add_tensor(w, off, b + "attn.add_k_proj.weight", D, D, false);
+    add_tensor(w, off, b + "attn.add_v_proj.weight", D, D, false);
+    add_tensor(w, off, b + "attn.to_out.0.weight", D, D);
+    add_tensor(w, off, b + "attn.to_add_out.weight", D, D);
+    add_tensor(w, off, b + "ff.linear_1.weight", F, D);
+    add_tensor(w, off, b + "ff.linear_2.weight", F, D, false);
+    add_tensor(w, off, b + "ff.out_projection.weight", D, F);
+    add_tensor(w, off, b + "ff_context.linear_1.weight", F, D);
+    add_tensor(w, off, b + "ff_context.linear_2.weight", F, D, false);
+    add_tensor(w, off, b + "ff_context.out_projection.weight", D, F);
+  }
+  for (int i = 0; i < c.num_single_dit_layers; ++i) {
+    const std::string b = "single_transformer_blocks." + std::to_string(i) + ".";
+    add_tensor(w, off, b + "attn.to_q.weight", D, D);
+    add_tensor(w, off, b + "attn.to_k.weight", D, D, false);
+    add_tensor(w, off, b + "attn.to_v.weight", D, D, false);
+    add_tensor(w, off, b + "attn.to_out.0.weight", D, D);
+    add_tensor(w, off, b + "ff.linear_1.weight", F, D);
+    add_tensor(w, off, b + "ff.linear_2.weight", F, D, false);
+    add_tensor(w, off, b + "ff.out_projection.weight", D, F);
+  }
+  add_tensor(w, off, "pos_embed.proj.weight", D, p * p * c.in_channels);
+  add_tensor(w, off, "pos_embed.pos_embed", c.pos_embed_max_size, D);
+  add_tensor(w, off, "time_step_proj.linear_1.weight", D, c.timestep_channels);
+  add_tensor(w, off, "time_step_proj.linear_1.bias", D, 0);
+  add_tensor(w, off, "time_step_proj.linear_2.weight", D, D);
+  add_tensor(w, off, "time_step_proj.linear_2.bias", D, 0);
+  add_tensor(w, off, "context_embedder.weight", D, c.joint_attention_dim);
+  add_tensor(w, off, "register_tokens", c.num_register_tokens, D);
+  add_tensor(w, off, "proj_out.weight", p * p * c.out_channels, D);
+  w->bytes = (off + 255) & ~size_t(255);
+}
+
+const uint16_t* ada_base(const af_weights* w) {
+  return reinterpret_cast<const uint16_t*>(w->base + w->tensors[0].offset);
+}
+
+af_status check_scratch(const af_weights* w, af_scratch* s) {
+  if (!w || !s || s->w != w) return AF_ERR_INVALID_ARG;
+  return AF_OK;
+}
+
+enum { KC_GEMM = 0, KC_ATTN = 1, KC_LN = 2, KC_OTHER = 3 };
+
+// Counts the launches made inside its scope and, while profiling, brackets
+// them with a CUDA event pair on `st`.
+struct LaunchScope {
+  af_scratch* s;
+  cudaStream_t st;
+  size_t e0 = SIZE_MAX;
+  LaunchScope(af_scratch* s_, int cls, double work, cudaStream_t st_, int n = 1) : s(s_), st(st_) {
+    s->launches[cls] += n;
+    if (!s->profiling) return;
+    while (s->pool.size() < s->pool_used + 2) {
+      cudaEvent_t e;
+      if (cudaEventCreate(&e) != cudaSuccess) return;
+      s->pool.push_back(e);
+    }
+    e0 = s->pool_used;
+    s->pool_used += 2;
+    cudaEventRecord(s->pool[e0], st);
+    s->recs.push_back({cls, e0, n, work});
+  }
+  ~LaunchScope() {
+    if (e0 != SIZE_MAX) cudaEventRecord(s->pool[e0 + 1], st);
+  }
+};
+
+// ---------------------------------------------------------------- GEMM helpers
+GemmParams gemm_base(const af_scratch* s, int M, int N, int K, int mode, int rows_per_batch) {
+  GemmParams p;
+  memset(&p, 0, sizeof(p));
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.mode = mode;
+  p.rows_per_batch = rows_per_batch > 0 ? rows_per_batch : (M > 0 ? M : 1);
+  p.out_rows_per_batch = p.rows_per_batch;
+  p.out_row_off = 0;
+  p.err = s->err;
+  return p;
+}
+
+af_status run_gemm(af_scratch* s, const GemmParams& p, const void* A, const void* W, int W_rows,
+                   cudaStream_t st) {
+  const double ncols = p.mode == EPI_SWIGLU ? 2.0 * p.N : static_cast<double>(p.N);
+  LaunchScope ls(s, KC_GEMM, 2.0 * p.M * ncols * p.K, st);
+  cudaError_t e = launch_gemm(p, A, W, W_rows, st, s->sms);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return AF_OK;
+}
+
+// QKV projection of one stream with per-head LayerNorm of Q and K.
+af_status qkv(const af_weights* w, af_scratch* s, const uint16_t* y, int B, int rows, const uint16_t* wqkv,
+              int row_off, int n_total, cudaStream_t st) {
+  const Derived& d = w->d;
+  GemmParams p = gemm_base(s, B * rows, 3 * d.D, d.D, EPI_QKV, rows);
+  p.q = s->q;
+  p.k = s->k;
+  p.v = s->v;
+  p.heads = d.H;
+  p.hd = d.hd;
+  p.n_total = n_total;
+  p.qkv_row_off = row_off;
+  p.D = d.D;
+  p.eps = w->cfg.ln_eps;
+  return run_gemm(s, p, y, wqkv, 3 * d.D, st);
+}
+
+// x += gate[b] * (A W^T)
+af_status gated_residual(af_scratch* s, const uint16_t* A, int B, int rows, int K, const uint16_t* W, int N,
+                         uint16_t* x, const float* gate, int gate_stride, cudaStream_t st) {
+  GemmParams p = gemm_base(s, B * rows, N, K, EPI_GATE_RES, rows);
+  p.out = x;
+  p.ldo = N;
+  p.gate = gate;
+  p.gate_stride = gate_stride;
+  return run_gemm(s, p, A, W, N, st);
+}
+
+// h = silu(y W1^T) * (y W2^T), W1 and W2 stacked in one [2F, D] matrix
+af_status swiglu(const af_weights* w, af_scratch* s, const uint16_t* y, int M, const uint16_t* w12,
+                 uint16_t* h, cudaStream_t st) {
+  const Derived& d = w->d;
+  GemmParams p = gemm_base(s, M, d.F, d.D, EPI_SWIGLU, M);
+  p.out = h;
+  p.ldo = d.F;
+  p.swiglu_w2_row = d.F;
+  return run_gemm(s, p, y, w12, 2 * d.F, st);
+}
+
+af_status attention(const af_weights* w, af_scratch* s, int B, int N, uint16_t* out_a, uint16_t* out_b, int split,
+                    cudaStream_t st) {
+  const Derived& d = w->d;
+  AttnParams p;
+  p.B = B;
+  p.H = d.H;
+  p.N = N;
+  p.hd = d.hd;
+  p.out_a = out_a;
+  p.out_b = out_b;
+  p.split = split;
+  p.ldo = d.D;
+  p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(d.hd));
+  p.err = s->err;
+  LaunchScope ls(s, KC_ATTN, 4.0 * B * d.H * static_cast<double>(N) * N * d.hd, st);
+  cudaError_t e = launch_attention(p, s->q, s->k, s->v, st);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return AF_OK;
+}
+
+af_status ln_mod(af_scratch* s, const uint16_t* x, const float* shift, const float* scale, int mod_stride, uint16_t* y,
+                 int rows, int rows_per_batch, int D, float eps, cudaStream_t st) {
+  LaunchScope ls(s, KC_LN, 4.0 * rows * D, st);
+  cudaError_t e = launch_ln_modulate(x, shift, scale, mod_stride, y, rows, rows_per_batch, D, eps, st);
+  return e == cudaSuccess ? AF_OK : cuda_fail(e);
+}
+
+#define AF_TRY(x)                  \
+  do {                             \
+    af_status st_ = (x);           \
+    if (st_ != AF_OK) return st_;  \
+  } while (0)
+
+// One joint block given the modulation vectors of both streams (mods rows
+// [unit_row, +6D) per sample, sample stride mod_stride).
+af_status joint_block_impl(const af_weights* w, af_scratch* s, int layer, uint16_t* img, uint16_t* txt,
+                           const float* mi, const float* mt, int mod_stride, int B, int Ni, int Nt,
+                           cudaStream_t st) {
+  const Derived& d = w->d;
+  const int D = d.D;
+  const float eps = w->cfg.ln_eps;
+  const std::string pre = "joint_transformer_blocks." + std::to_string(layer) + ".";
+  const int N = Nt + Ni;
+  uint16_t* y_img = s->y;
+  uint16_t* y_txt = s->y + static_cast<size_t>(B) * Ni * D;
+  uint16_t* o_img = s->o;
+  uint16_t* o_txt = s->o + static_cast<size_t>(B) * Ni * D;
+  uint16_t* h_img = s->h;
+  uint16_t* h_txt = s->h + static_cast<size_t>(B) * Ni * d.F;
+
+  AF_TRY(ln_mod(s, img, mi + 0 * D, mi + 1 * D, mod_stride, y_img, B * Ni, Ni, D, eps, st));
+  AF_TRY(ln_mod(s, txt, mt + 0 * D, mt + 1 * D, mod_stride, y_txt, B * Nt, Nt, D, eps, st));
+  AF_TRY(qkv(w, s, y_txt, B, Nt, w->ptr(pre + "attn.add_q_proj.weight"), 0, N, st));
+  AF_TRY(qkv(w, s, y_img, B, Ni, w->ptr(pre + "attn.to_q.weight"), Nt, N, st));
+  AF_TRY(attention(w, s, B, N, o_txt, o_img, Nt, st));
+  AF_TRY(gated_residual(s, o_img, B, Ni, D, w->ptr(pre + "attn.to_out.0.weight"), D, img, mi + 2 * D, mod_stride, st));
+  AF_TRY(gated_residual(s, o_txt, B, Nt, D, w->ptr(pre + "attn.to_add_out.weight"), D, txt, mt + 2 * D, mod_stride,
+                        st));
+  AF_TRY(ln_mod(s, img, mi + 3 * D, mi + 4 * D, mod_stride, y_img, B * Ni, Ni, D, eps, st));
+  AF_TRY(ln_mod(s, txt, mt + 3 * D, mt + 4 * D, mod_stride, y_txt, B * Nt, Nt, D, eps, st));
+  AF_TRY(swiglu(w, s, y_img, B * Ni, w->ptr(pre + "ff.linear_1.weight"), h_img, st));
+  AF_TRY(swiglu(w, s, y_txt, B * Nt, w->ptr(pre + "ff_context.linear_1.weight"), h_txt, st));
+  AF_TRY(gated_residual(s, h_img, B, Ni, d.F, w->ptr(pre + "ff.out_projection.weight"), D, img, mi + 5 * D,
+                        mod_stride, st));
+  AF_TRY(gated_residual(s, h_txt, B, Nt, d.F, w->ptr(pre + "ff_context.out_projection.weight"), D, txt, mt + 5 * D,
+                        mod_stride, st));
+  return AF_OK;
+}
+
+af_status single_block_impl(const af_weights* w, af_scratch* s, int layer, uint16_t* x, const float* m,
+                            int mod_stride, int B, int N, cudaStream_t st) {
+  const Derived& d = w->d;
+  const int D = d.D;
+  const float eps = w->cfg.ln_eps;
+  const std::string pre = "single_transformer_blocks." + std::to_string(layer) + ".";
+  AF_TRY(ln_mod(s, x, m + 0 * D, m + 1 * D, mod_stride, s->y, B * N, N, D, eps, st));
+  AF_TRY(qkv(w, s, s->y, B, N, w->ptr(pre + "attn.to_q.weight"), 0, N, st));
+  AF_TRY(attention(w, s, B, N, s->o, s->o, 0, st));
+  AF_TRY(gated_residual(s, s->o, B, N, D, w->ptr(pre + "attn.to_out.0.weight"), D, x, m + 2 * D, mod_stride, st));
+  AF_TRY(ln_mod(s, x, m + 3 * D, m + 4 * D, mod_stride, s->y, B * N, N, D, eps, st));
+  AF_TRY(swiglu(w, s, s->y, B * N, w->ptr(pre + "ff.linear_1.weight"), s->h, st));
+  AF_TRY(gated_residual(s, s->h, B, N, d.F, w->ptr(pre + "ff.out_projection.weight"), D, x, m + 5 * D, mod_stride,
+                        st));
+  return AF_OK;
+}
+
+af_status check_dev_ptr(const void* p) {
+  if (!p) return AF_ERR_INVALID_ARG;
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();
+    return AF_ERR_INVALID_ARG;
+  }
+  if (a.type != cudaMemoryTypeDevice && a.type != cudaMemoryTypeManaged) return AF_ERR_INVALID_ARG;
+  return AF_OK;
+}
+
+}  // namespace
+
+// =========================================================================== C ABI
+
+extern "C" {
+
+const char* af_status_string(af_status st) {
+  switch (st) {
+    case AF_OK: return "ok";
+    case AF_ERR_INVALID_ARG: return "invalid argument";
+    case AF_ERR_SHAPE: return "shape error";
+    case AF_ERR_UNSUPPORTED: return "unsupported configuration";
+    case AF_ERR_OOM: return "out of device memory";
+    case AF_ERR_CUDA: return "CUDA error";
+    case AF_ERR_TIMEOUT: return "device wait timed out";
+    case AF_ERR_NOT_FOUND: return "tensor not found";
+  }
+  return "unknown status";
+}
+
+const char* af_last_error(void) { return g_last_error.c_str(); }
+
+af_status af_config_default(af_config* c) {
+  if (!c) return AF_ERR_INVALID_ARG;
+  c->patch_size = 2;
+  c->in_channels = 4;
+  c->out_channels = 4;
+  c->num_mmdit_layers = 4;
+  c->num_single_dit_layers = 32;
+  c->attention_head_dim = 256;
+  c->num_attention_heads = 12;
+  c->joint_attention_dim = 2048;
+  c->pos_embed_max_size = 1024;
+  c->num_register_tokens = 8;
+  c->timestep_channels = 256;
+  c->ffn_inner = 0;
+  c->ln_eps = 1e-6f;
+  return AF_OK;
+}
+
+af_status af_config_derive(const af_config* c, int* inner_dim, int* ffn_inner, int* grid_side) {
+  Derived d;
+  AF_TRY(derive(c, &d));
+  if (inner_dim) *inner_dim = d.D;
+  if (ffn_inner) *ffn_inner = d.F;
+  if (grid_side) *grid_side = d.G;
+  return AF_OK;
+}
+
+af_status af_weights_create(const af_config* cfg, int device, af_weights** out) {
+  if (!out) return AF_ERR_INVALID_ARG;
+  *out = nullptr;
+  Derived d;
+  AF_TRY(derive(cfg, &d));
+  // kernel coverage of this build
+  if (d.D % 32 != 0 || d.F % 128 != 0 || cfg->joint_attention_dim % 8 != 0) return AF_ERR_UNSUPPORTED;
+  if (!(d.hd == 256 || d.hd == 8 || d.hd == 16 || d.hd == 32 || d.hd == 64)) return AF_ERR_UNSUPPORTED;
+  if (cfg->patch_size * cfg->patch_size * cfg->in_channels > 64) return AF_ERR_UNSUPPORTED;
+  af_weights* w = new af_weights();
+  w->cfg = *cfg;
+  w->d = d;
+  w->device = device;
+  build_layout(w);
+  int prev = 0;
+  cudaGetDevice(&prev);
+  if (cudaSetDevice(device) != cudaSuccess) {
+    delete w;
+    return AF_ERR_INVALID_ARG;
+  }
+  cudaError_t e = cudaMalloc(&w->base, w->bytes);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    cudaSetDevice(prev);
+    delete w;
+    return AF_ERR_OOM;
+  }
+  e = cudaMemset(w->base, 0, w->bytes);
+  cudaSetDevice(prev);
+  if (e != cudaSuccess) {
+    cudaFree(w->base);
+    delete w;
+    return cuda_fail(e);
+  }
+  *out = w;
+  return AF_OK;
+}
+
+void af_weights_destroy(af_weights* w) {
+  if (!w) return;
+  if (w->base) cudaFree(w->base);
+  delete w;
+}
+
+af_status af_weights_num_tensors(const af_weights* w, int* n) {
+  if (!w || !n) return AF_ERR_INVALID_ARG;
+  *n = static_cast<int>(w->tensors.size());
+  return AF_OK;
+}
+
+af_status af_weights_tensor_info(const af_weights* w, int id, char* name, size_t name_cap, int* ndim,
+                                 int64_t shape[2]) {
+  if (!w || id < 0 || id >= static_cast<int>(w->tensors.size())) return AF_ERR_INVALID_ARG;
+  const TensorInfo& t = w->tensors[id];
+  if (name && name_cap > 0) {
+    strncpy(name, t.name.c_str(), name_cap - 1);
+    name[name_cap - 1] = '\0';
+  }
+  if (ndim) *ndim = t.ndim;
+  if (shape) {
+    shape[0] = t.shape[0];
+    shape[1] = t.shape[1];
+  }
+  return AF_OK;
+}
+
+af_status af_weights_find(const af_weights* w, const char* name, int* id) {
+  if (!w || !name || !id) return AF_ERR_INVALID_ARG;
+  auto it = w->index.find(name);
+  if (it == w->index.end()) return AF_ERR_NOT_FOUND;
+  *id = it->second;
+  return AF_OK;
+}
+
+af_status af_weights_set(af_weights* w, int id, const uint16_t* src, int src_is_device, void* stream) {
+  if (!w || !src || id < 0 || id >= static_cast<int>(w->tensors.size())) return AF_ERR_INVALID_ARG;
+  const TensorInfo& t = w->tensors[id];
+  const size_t bytes = t.numel() * 2;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (src_is_device) {
+    AF_TRY(check_dev_ptr(src));
+    AF_CUDA(cudaMemcpyAsync(w->base + t.offset, src, bytes, cudaMemcpyDeviceToDevice, st));
+  } else {
+    AF_CUDA(cudaMemcpy(w->base + t.offset, src, bytes, cudaMemcpyHostToDevice));
+  }
+  return AF_OK;
+}
+
+af_status af_weights_bytes(const af_weights* w, size_t* bytes) {
+  if (!w || !bytes) return AF_ERR_INVALID_ARG;
+  *bytes = w->bytes;
+  return AF_OK;
+}
+
+af_status af_scratch_create(const af_weights* w, int max_batch, int max_img_tokens, int max_text_len,
+                            af_scratch** out) {
+  if (!w || !out || max_batch <= 0 || max_img_tokens <= 0 || max_text_len < 0) return AF_ERR_INVALID_ARG;
+  *out = nullptr;
+  const Derived& d = w->d;
+  af_scratch* s = new af_scratch();
+  s->w = w;
+  s->max_b = max_batch;
+  s->max_ni = max_img_tokens;
+  s->max_l = max_text_len;
+  s->max_nt = max_text_len + w->cfg.num_register_tokens;
+  s->max_n = s->max_nt + max_img_tokens;
+  s->device = w->device;
+  const size_t B = max_batch, N = s->max_n, D = d.D, F = d.F;
+  const size_t rowsN = B * N;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = (off + bytes + 255) & ~size_t(255);
+    return o;
+  };
+  const size_t o_err = take(256);
+  const size_t o_temb = take(B * D * 4);
+  const size_t o_h1 = take(B * D * 4);
+  const size_t o_tfeat = take(B * w->cfg.timestep_channels * 4);
+  const size_t o_mods = take(B * w->ada_rows * 4);
+  const size_t o_y = take(rowsN * D * 2);
+  const size_t o_q = take(rowsN * D * 2);
+  const size_t o_k = take(rowsN * D * 2);
+  const size_t o_v = take(rowsN * D * 2);
+  const size_t o_o = take(rowsN * D * 2);
+  const size_t o_h = take(rowsN * F * 2);
+  const size_t o_img = take(B * s->max_ni * D * 2);
+  const size_t o_txt = take(B * s->max_nt * D * 2);
+  const size_t o_x = take(rowsN * D * 2);
+  const int cmax = w->cfg.in_channels > w->cfg.out_channels ? w->cfg.in_channels : w->cfg.out_channels;
+  const size_t lat_elems = B * static_cast<size_t>(cmax) * s->max_ni * w->cfg.patch_size * w->cfg.patch_size;
+  const size_t o_lat2 = take(lat_elems * 4);
+  const size_t o_vel = take(lat_elems * 4);
+  const size_t o_tvec = take(B * 4);
+  s->bytes = off;
+  int prev = 0;
+  cudaGetDevice(&prev);
+  cudaSetDevice(w->device);
+  cudaError_t e = cudaMalloc(&s->base, s->bytes);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    cudaSetDevice(prev);
+    delete s;
+    return AF_ERR_OOM;
+  }
+  e = cudaMemset(s->base, 0, s->bytes);
+  s->sms = device_sm_count();
+  cudaSetDevice(prev);
+  if (e != cudaSuccess) {
+    cudaFree(s->base);
+    delete s;
+    return cuda_fail(e);
+  }
+  s->err = reinterpret_cast<int*>(s->base + o_err);
+  s->temb = reinterpret_cast<float*>(s->base + o_temb);
+  s->h1 = reinterpret_cast<float*>(s->base + o_h1);
+  s->tfeat = reinterpret_cast<float*>(s->base + o_tfeat);
+  s->mods = reinterpret_cast<float*>(s->base + o_mods);
+  s->y = reinterpret_cast<uint16_t*>(s->base + o_y);
+  s->q = reinterpret_cast<uint16_t*>(s->base + o_q);
+  s->k = reinterpret_cast<uint16_t*>(s->base + o_k);
+  s->v = reinterpret_cast<uint16_t*>(s->base + o_v);
+  s->o = reinterpret_cast<uint16_t*>(s->base + o_o);
+  s->h = reinterpret_cast<uint16_t*>(s->base + o_h);
+  s->img = reinterpret_cast<uint16_t*>(s->base + o_img);
+  s->txt = reinterpret_cast<uint16_t*>(s->base + o_txt);
+  s->x = reinterpret_cast<uint16_t*>(s->base + o_x);
+  s->lat2 = reinterpret_cast<float*>(s->base + o_lat2);
+  s->vel = reinterpret_cast<float*>(s->base + o_vel);
+  s->tvec = reinterpret_cast<float*>(s->base + o_tvec);
+  *out = s;
+  return AF_OK;
+}
+
+void af_scratch_destroy(af_scratch* s) {
+  if (!s) return;
+  for (cudaEvent_t e : s->pool) cudaEventDestroy(e);
+  if (s->base) cudaFree(s->base);
+  delete s;
+}
+
+af_status af_sync(af_scratch* s, void* stream) {
+  if (!s) return AF_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  AF_CUDA(cudaStreamSynchronize(st));
+  int h = 0;
+  AF_CUDA(cudaMemcpy(&h, s->err, sizeof(int), cudaMemcpyDeviceToHost));
+  if (h != 0) {
+    AF_CUDA(cudaMemset(s->err, 0, sizeof(int)));
+    return AF_ERR_TIMEOUT;
+  }
+  return AF_OK;
+}
+
+af_status af_timestep_embed(const af_weights* w, af_scratch* s, const float* t, int B, float* temb, void* stream) {
+  AF_TRY(check_scratch(w, s));
+  if (!t || !temb || B <= 0) return AF_ERR_INVALID_ARG;
+  if (B > s->max_b) return AF_ERR_SHAPE;
+  const Derived& d = w->d;
+  LaunchScope ls(s, KC_OTHER, 2.0 * d.D * (w->cfg.timestep_channels + d.D), static_cast<cudaStream_t>(stream), 3);
+  AF_CUDA(launch_timestep_mlp(t, B, w->ptr("time_step_proj.linear_1.weight"), w->ptr("time_step_proj.linear_1.bias"),
+                              w->ptr("time_step_proj.linear_2.weight"), w->ptr("time_step_proj.linear_2.bias"),
+                              w->cfg.timestep_channels, d.D, s->tfeat, s->h1, temb, static_cast<cudaStream_t>(stream)));
+  return AF_OK;
+}
+
+af_status af_patch_embed(const af_weights* w, af_scratch* s, const float* latents, int B, int H, int W,
+                         uint16_t* img_tokens, void* stream) {
+  AF_TRY(check_scratch(w, s));
+  if (!latents || !img_tokens || B <= 0 || H <= 0 || W <= 0) return AF_ERR_INVALID_ARG;
+  const int p = w->cfg.patch_size;
+  if (H % p || W % p || H / p > w->d.G || W / p > w->d.G) return AF_ERR_SHAPE;
+  const int Ni = (H / p) * (W / p);
+  LaunchScope ls(s, KC_OTHER, 4.0 * B * Ni * w->d.D + 4.0 * B * w->cfg.in_channels * H * W,
+                 static_cast<cudaStream_t>(stream));
+  AF_CUDA(launch_patch_embed(latents, B, w->cfg.in_channels, H, W, p, w->ptr("pos_embed.proj.weight"),
+                             w->ptr("pos_embed.pos_embed"), w->d.G, w->d.D, img_tokens, Ni, 0,
+                             static_cast<cudaStream_t>(stream)));
+  return AF_OK;
+}
+
+af_status af_joint_block(const af_weights* w, af_scratch* s, int layer, uint16_t* img, uint16_t* txt,
+                         const float* temb, int B, int Ni, int Nt, void* stream) {
+  AF_TRY(check_scratch(w, s));
+  if (!img || !txt || !temb || B <= 0 || Ni <= 0 || Nt <= 0) return AF_ERR_INVALID_ARG;
+  if (layer < 0 || layer >= w->cfg.num_mmdit_layers) return AF_ERR_INVALID_ARG;
+  if (B > s->max_b || Ni + Nt > s->max_n || Ni > s->max_n) return AF_ERR_SHAPE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int D = w->d.D;
+  // modulation of this block's two streams only
+  const size_t r_img = w->unit_row[2 * layer];
+  const uint16_t* ada = ada_base(w);
+  {
+    LaunchScope ls(s, KC_OTHER, 2.0 * 12 * D * D, st, (B + 7) / 8);
+    AF_CUDA(launch_modulation(temb, B, D, ada + r_img * D, 12 * D, s->mods, st));
+  }
+  const float* mi = s->mods;
+  const float* mt = s->mods + 6 * D;
+  return joint_block_impl(w, s, layer, img, txt, mi, mt, 12 * D, B, Ni, Nt, st);
+}
+
+af_status af_single_block(const af_weights* w, af_scratch* s, int layer, uint16_t* x, const float* temb, int B,
+                          int N, void* stream) {
+  AF_TRY(check_scratch(w, s));
+  if (!x || !temb || B <= 0 || N <= 0) return AF_ERR_INVALID_ARG;
+  if (layer < 0 || layer >= w->cfg.num_single_dit_layers) return AF_ERR_INVALID_ARG;
+  if (B > s->max_b || N > s->max_n) return AF_ERR_SHAPE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int D = w->d.D;
+  const size_t r = w->unit_row[2 * w->cfg.num_mmdit_layers + layer];
+  {
+    LaunchScope ls(s, KC_OTHER, 2.0 * 6 * D * D, st, (B + 7) / 8);
+    AF_CUDA(launch_modulation(temb, B, D, ada_base(w) + r * D, 6 * D, s->mods, st));
+  }
+  return single_block_impl(w, s, layer, x, s->mods, 6 * D, B, N, st);
+}
+
+static af_status forward_impl(const af_weights* w, af_scratch* s, const float* latents, const uint16_t* text_emb,
+                              const float* t, int B, int H, int W, int L, float* velocity, cudaStream_t st) {
+  AF_TRY(check_scratch(w, s));
+  if (!latents || !text_emb || !t || !velocity || B <= 0 || H <= 0 || W <= 0 || L < 0) return AF_ERR_INVALID_ARG;
+  const af_config& c = w->cfg;
+  const Derived& d = w->d;
+  const int p = c.patch_size;
+  if (H % p || W % p || H / p > d.G || W / p > d.G) return AF_ERR_SHAPE;
+  const int hp = H / p, wp = W / p, Ni = hp * wp;
+  const int R = c.num_register_tokens, Nt = R + L, N = Nt + Ni;
+  if (B > s->max_b || Ni > s->max_ni || L > s->max_l) return AF_ERR_SHAPE;
+  if (Nt <= 0) return AF_ERR_SHAPE;
+  const int D = d.D;
+  const size_t R_ada = w->ada_rows;
+
+  // embedding stage
+  {
+    LaunchScope ls(s, KC_OTHER, 2.0 * D * (c.timestep_channels + D), st, 3);
+    AF_CUDA(launch_timestep_mlp(t, B, w->ptr("time_step_proj.linear_1.weight"),
+                                w->ptr("time_step_proj.linear_1.bias"), w->ptr("time_step_proj.linear_2.weight"),
+                                w->ptr("time_step_proj.linear_2.bias"), c.timestep_channels, D, s->tfeat, s->h1,
+                                s->temb, st));
+  }
+  {
+    LaunchScope ls(s, KC_OTHER, 2.0 * R_ada * D, st, (B + 7) / 8);
+    AF_CUDA(launch_modulation(s->temb, B, D, ada_base(w), static_cast<int>(R_ada), s->mods, st));
+  }
+  {
+    LaunchScope ls(s, KC_OTHER, 4.0 * B * Ni * D + 4.0 * B * c.in_channels * H * W, st);
+    AF_CUDA(launch_patch_embed(latents, B, c.in_channels, H, W, p, w->ptr("pos_embed.proj.weight"),
+                               w->ptr("pos_embed.pos_embed"), d.G, D, s->img, Ni, 0, st));
+  }
+  for (int b = 0; b < B && R > 0; ++b)  // register tokens at the head of every sample's text stream
+    AF_CUDA(cudaMemcpyAsync(s->txt + static_cast<size_t>(b) * Nt * D, w->ptr("register_tokens"),
+                            static_cast<size_t>(R) * D * 2, cudaMemcpyDeviceToDevice, st));
+  if (L > 0) {
+    GemmParams gp = gemm_base(s, B * L, D, c.joint_attention_dim, EPI_STORE, L);
+    gp.out = s->txt;
+    gp.ldo = D;
+    gp.out_rows_per_batch = Nt;
+    gp.out_row_off = R;
+    AF_TRY(run_gemm(s, gp, text_emb, w->ptr("context_embedder.weight"), D, st));
+  }
+  // joint blocks
+  for (int i = 0; i < c.num_mmdit_layers; ++i) {
+    const float* mi = s->mods + w->unit_row[2 * i];
+    const float* mt = s->mods + w->unit_row[2 * i + 1];
+    AF_TRY(joint_block_impl(w, s, i, s->img, s->txt, mi, mt, static_cast<int>(R_ada), B, Ni, Nt, st));
+  }
+  // x = cat(text, image) per sample
+  AF_CUDA(cudaMemcpy2DAsync(s->x, static_cast<size_t>(N) * D * 2, s->txt, static_cast<size_t>(Nt) * D * 2,
+                            static_cast<size_t>(Nt) * D * 2, B, cudaMemcpyDeviceToDevice, st));
+  AF_CUDA(cudaMemcpy2DAsync(s->x + static_cast<size_t>(Nt) * D, static_cast<size_t>(N) * D * 2, s->img,
+                            static_cast<size_t>(Ni) * D * 2, static_cast<size_t>(Ni) * D * 2, B,
+                            cudaMemcpyDeviceToDevice, st));
+  for (int i = 0; i < c.num_single_dit_layers; ++i) {
+    const float* m = s->mods + w->unit_row[2 * c.num_mmdit_layers + i];
+    AF_TRY(single_block_impl(w, s, i, s->x, m, static_cast<int>(R_ada), B, N, st));
+  }
+  // pre-final (scale first, then shift), proj_out, unpatchify on the image rows
+  const float* pf = s->mods + w->pf_row;
+  LaunchScope ls(s, KC_OTHER, 2.0 * B * Ni * D + 4.0 * B * c.out_channels * H * W, st);
+  AF_CUDA(launch_output_stage(s->x, N, Nt, B, hp, wp, D, pf, pf + D, static_cast<int>(R_ada),
+                              w->ptr("proj_out.weight"), p, c.out_channels, velocity, st));
+  return AF_OK;
+}
+
+af_status af_transformer_forward(const af_weights* w, af_scratch* s, const float* latents, const uint16_t* text_emb,
+                                 const float* t, int B, int H, int W, int L, float* velocity, void* stream) {
+  return forward_impl(w, s, latents, text_emb, t, B, H, W, L, velocity, static_cast<cudaStream_t>(stream));
+}
+
+af_status af_denoise_step(const af_weights* w, af_scratch* s, float* latents, const uint16_t* text_emb, int Bi, int H,
+                          int W, int L, float guidance, float sigma, float sigma_next, void* stream) {
+  AF_TRY(check_scratch(w, s));
+  if (!latents || !text_emb || Bi <= 0 || H <= 0 || W <= 0 || L < 0) return AF_ERR_INVALID_ARG;
+  const int B = 2 * Bi;
+  const int p = w->cfg.patch_size;
+  if (H % p || W % p) return AF_ERR_SHAPE;
+  if (B > s->max_b || (H / p) * (W / p) > s->max_ni) return AF_ERR_SHAPE;
+  if (w->cfg.in_channels != w->cfg.out_channels) return AF_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t per = static_cast<size_t>(w->cfg.in_channels) * H * W;
+  // CFG batch [uncond; text] shares the latents
+  AF_CUDA(cudaMemcpyAsync(s->lat2, latents, per * Bi * 4, cudaMemcpyDeviceToDevice, st));
+  AF_CUDA(cudaMemcpyAsync(s->lat2 + per * Bi, latents, per * Bi * 4, cudaMemcpyDeviceToDevice, st));
+  {
+    LaunchScope ls(s, KC_OTHER, 4.0 * B, st);
+    AF_CUDA(launch_fill(s->tvec, B, sigma, st));
+  }
+  AF_TRY(forward_impl(w, s, s->lat2, text_emb, s->tvec, B, H, W, L, s->vel, st));
+  LaunchScope ls(s, KC_OTHER, 16.0 * per * Bi, st);
+  AF_CUDA(launch_euler_cfg(latents, s->vel, Bi, static_cast<int64_t>(per), guidance, sigma, sigma_next, st));
+  return AF_OK;
+}
+
+af_status af_sigma_schedule(int n_steps, float shift, int num_train_timesteps, float* out) {
+  if (!out || n_steps <= 0 || num_train_timesteps <= 0 || !(shift > 0.f)) return AF_ERR_INVALID_ARG;
+  const double lo = 1.0 / num_train_timesteps;
+  for (int i = 0; i < n_steps; ++i) {
+    const double s = n_steps == 1 ? 1.0 : 1.0 + (lo - 1.0) * i / (n_steps - 1);
+    out[i] = static_cast<float>(shift * s / (1.0 + (shift - 1.0) * s));
+  }
+  out[n_steps] = 0.f;
+  return AF_OK;
+}
+
+af_status af_launch_counts(const af_scratch* s, int64_t counts[AF_NUM_KERNEL_CLASSES]) {
+  if (!s || !counts) return AF_ERR_INVALID_ARG;
+  for (int i = 0; i < AF_NUM_KERNEL_CLASSES; ++i) counts[i] = s->launches[i];
+  return AF_OK;
+}
+
+af_status af_profile_begin(af_scratch* s) {
+  if (!s) return AF_ERR_INVALID_ARG;
+  s->profiling = true;
+  s->pool_used = 0;
+  s->recs.clear();
+  return AF_OK;
+}
+
+af_status af_profile_end(af_scratch* s, void* stream, double ms[AF_NUM_KERNEL_CLASSES],
+                         int64_t launches[AF_NUM_KERNEL_CLASSES], double work[AF_NUM_KERNEL_CLASSES]) {
+  if (!s) return AF_ERR_INVALID_ARG;
+  s->profiling = false;
+  AF_CUDA(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+  double t[AF_NUM_KERNEL_CLASSES] = {0, 0, 0, 0}, wk[AF_NUM_KERNEL_CLASSES] = {0, 0, 0, 0};
+  int64_t n[AF_NUM_KERNEL_CLASSES] = {0, 0, 0, 0};
+  for (const auto& r : s->recs) {
+    float e = 0.f;
+    AF_CUDA(cudaEventElapsedTime(&e, s->pool[r.e0], s->pool[r.e0 + 1]));
+    t[r.cls] += e;
+    n[r.cls] += r.n;
+    wk[r.cls] += r.work;
+  }
+  s->recs.clear();
+  s->pool_used = 0;
+  for (int i = 0; i < AF_NUM_KERNEL_CLASSES; ++i) {
+    if (ms) ms[i] = t[i];
+    if (launches) launches[i] = n[i];
+    if (work) work[i] = wk[i];
+  }
+  return AF_OK;
+}
+
+af_status af_euler_cfg_step(float* latents, const float* velocity, int Bi, int C, int H, int W, float guidance,
+                            float sigma, float sigma_next, void* stream) {
+  if (!latents || !velocity || Bi <= 0 || C <= 0 || H <= 0 || W <= 0) return AF_ERR_INVALID_ARG;
+  AF_CUDA(launch_euler_cfg(latents, velocity, Bi, static_cast<int64_t>(C) * H * W, guidance, sigma, sigma_next,
+                           static_cast<cudaStream_t>(stream)));
+  return AF_OK;
+}
+
+af_status af_ln_modulate(const uint16_t* x, const float* shift, const float* scale, int mod_stride, uint16_t* y,
+                         int B, int N, int D, float eps, void* stream) {
+  if (!x || !shift || !scale || !y || B <= 0 || N <= 0 || D <= 0 || mod_stride < 0) return AF_ERR_INVALID_ARG;
+  if (D % 8 != 0 || D > 4096) return AF_ERR_UNSUPPORTED;
+  AF_CUDA(launch_ln_modulate(x, shift, scale, mod_stride, y, B * N, N, D, eps, static_cast<cudaStream_t>(stream)));
+  return AF_OK;
+}
+
+af_status af_linear(const uint16_t* A, const uint16_t* W, uint16_t* C, int M, int N, int K, void* stream) {
+  if (!A || !W || !C || M <= 0 || N <= 0 || K <= 0) return AF_ERR_INVALID_ARG;
+  if (K % 8 != 0 || N % 8 != 0) return AF_ERR_UNSUPPORTED;
+  GemmParams p;
+  memset(&p, 0, sizeof(p));
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.mode = EPI_STORE;
+  p.rows_per_batch = M;
+  p.out_rows_per_batch = M;
+  p.out = C;
+  p.ldo = N;
+  p.err = nullptr;
+  static int sms = 0;
+  if (!sms) sms = device_sm_count();
+  AF_CUDA(launch_gemm(p, A, W, N, static_cast<cudaStream_t>(stream), sms));
+  return AF_OK;
+}
+
+af_status af_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* o, int B, int H, int N,
+                       int hd, void* stream) {
+  if (!q || !k || !v || !o || B <= 0 || H <= 0 || N <= 0) return AF_ERR_INVALID_ARG;
+  if (!(hd == 256 || hd == 8 || hd == 16 || hd == 32 || hd == 64)) return AF_ERR_UNSUPPORTED;
+  AttnParams p;
+  p.B = B;
+  p.H = H;
+  p.N = N;
+  p.hd = hd;
+  p.out_a = o;
+  p.out_b = o;
+  p.split = 0;
+  p.ldo = H * hd;
+  p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(hd));
+  p.err = nullptr;
+  AF_CUDA(launch_attention(p, q, k, v, static_cast<cudaStream_t>(stream)));
+  return AF_OK;
+}
+
+}  // extern "C"

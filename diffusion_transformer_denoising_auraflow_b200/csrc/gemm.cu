@@ -1,0 +1,448 @@
+// gemm.cu -- persistent tcgen05 GEMM for sm_100a with fused epilogues.
+//
+//   acc[M, N] = A[M, K] * W[N, K]^T      (bf16 operands, fp32 accumulation in TMEM)
+//
+// These are the bias-free projections of the AuraFlow blocks: fused QKV and
+// added-KV ("Diffusers 中的 AuraFlowTransformer2DModel架构解析与源码级使用指南",
+// §模型概述 and §注意力处理器与 QKV 融合), the output projections and the
+// SiLU-gated FFN (§FeedForward), gated by adaLN-Zero (§联合注意力块).
+//
+// Structure (one CTA per SM, persistent over 128 x 256 output tiles):
+//   warp 0      TMA producer: A tile 128x64 and W tile 256x64 per k-block,
+//               128-byte swizzled, into a 4-stage shared-memory ring.
+//   warp 1      allocates 512 TMEM columns; one thread issues
+//               tcgen05.mma (M=128, N=256, K=16) into one of two 256-column
+//               fp32 accumulators, committing each stage back to the producer.
+//   warps 2..5  epilogue: tcgen05.ld of their 32-lane quarter (one thread =
+//               one output row), fused epilogue, global stores; the other
+//               accumulator is being filled meanwhile.
+// Every wait is bounded (ptx.cuh); a timeout sets the error word and the CTA
+// drains its outstanding copies and MMAs before releasing TMEM.
+#include <cstdio>
+#include <mutex>
+
+#include <cudaTypedefs.h>
+
+#include "af_internal.h"
+#include "ptx.cuh"
+
+namespace af {
+
+// ----------------------------------------------------------------- host: TMA descriptors
+
+static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+bool encode_tmap_2d(CUtensorMap* map, const void* ptr, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                    uint32_t box_inner, uint32_t box_outer) {
+  auto enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool encode_tmap_3d(CUtensorMap* map, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1_bytes,
+                    uint64_t s2_bytes, uint32_t b0, uint32_t b1, uint32_t b2) {
+  auto enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {s1_bytes, s2_bytes};
+  cuuint32_t box[3] = {b0, b1, b2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int device_sm_count() {
+  int dev = 0, n = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+// ----------------------------------------------------------------- device: tiles
+
+constexpr uint32_t A_STAGE_BYTES = GEMM_BM * GEMM_BK * 2;  // 16 KB
+constexpr uint32_t B_STAGE_BYTES = GEMM_BN * GEMM_BK * 2;  // 32 KB
+constexpr int GROUP_N = 8;                                  // n-tiles per raster group
+
+__device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int& mb, int& nb) {
+  const int per_group = GROUP_N * num_m;
+  const int g = t / per_group;
+  const int r = t - g * per_group;
+  const int n_first = g * GROUP_N;
+  const int gw = min(GROUP_N, num_n - n_first);
+  mb = r / gw;
+  nb = n_first + (r - mb * gw);
+}
+
+__device__ __forceinline__ float silu_f(float a) { return a / (1.0f + __expf(-a)); }
+
+__device__ __forceinline__ void store_bf16x32(uint16_t* dst, const float* v) {
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint4 u;
+    u.x = pack_bf16(v[8 * i + 0], v[8 * i + 1]);
+    u.y = pack_bf16(v[8 * i + 2], v[8 * i + 3]);
+    u.z = pack_bf16(v[8 * i + 4], v[8 * i + 5]);
+    u.w = pack_bf16(v[8 * i + 6], v[8 * i + 7]);
+    d[i] = u;
+  }
+}
+
+// Store `n` (< 32 allowed at a ragged right edge) bf16 values.
+__device__ __forceinline__ void store_bf16_n(uint16_t* dst, const float* v, int n) {
+  if (n >= 32 && (reinterpret_cast<uintptr_t>(dst) & 15u) == 0) {
+    store_bf16x32(dst, v);
+    return;
+  }
+  for (int i = 0; i < n && i < 32; ++i) {
+    uint32_t p = pack_bf16(v[i], 0.f);
+    dst[i] = static_cast<uint16_t>(p & 0xFFFFu);
+  }
+}
+
+// QK-norm epilogue for one output row: columns [c0, c0 + width) of the tile
+// hold (256 / hd) heads of Q, K or V.  Q and K are LayerNorm-ed over each
+// head's hd values (two passes over TMEM: mean, then variance), V is stored as is.
+__device__ __forceinline__ void epilogue_qkv(const GemmParams& p, uint32_t tbase, int n0, bool row_ok, int b,
+                                             int n_in) {
+  const int hd = p.hd;
+  const int tok = p.qkv_row_off + n_in;
+  if (hd >= 32) {
+    const int chunks = hd >> 5;
+    for (int h0 = 0; h0 < GEMM_BN; h0 += hd) {
+      const int col = n0 + h0;
+      if (col >= p.N) break;                       // uniform across the warp
+      const int which = col / p.D;
+      const int head = (col - which * p.D) / hd;
+      uint16_t* base = which == 0 ? p.q : (which == 1 ? p.k : p.v);
+      uint16_t* dst = base + ((static_cast<size_t>(b) * p.heads + head) * p.n_total + tok) * hd;
+      float mean = 0.f, rstd = 1.f;
+      uint32_t r[32];
+      if (which < 2) {
+        float s = 0.f;
+        for (int c = 0; c < chunks; ++c) {
+          tmem_ld32(tbase + h0 + c * 32, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) s += __uint_as_float(r[j]);
+        }
+        mean = s / hd;
+        float ss = 0.f;
+        for (int c = 0; c < chunks; ++c) {
+          tmem_ld32(tbase + h0 + c * 32, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float d = __uint_as_float(r[j]) - mean;
+            ss += d * d;
+          }
+        }
+        rstd = rsqrtf(ss / hd + p.eps);
+      }
+      for (int c = 0; c < chunks; ++c) {
+        tmem_ld32(tbase + h0 + c * 32, r);
+        tmem_wait_ld();
+        float v[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = (__uint_as_float(r[j]) - mean) * rstd;
+        if (row_ok) store_bf16x32(dst + c * 32, v);
+      }
+    }
+  } else {
+    // small heads (hd in {8, 16}): each 32-column chunk holds 32 / hd heads
+    for (int c = 0; c < GEMM_BN / 32; ++c) {
+      if (n0 + c * 32 >= p.N) break;
+      uint32_t r[32];
+      tmem_ld32(tbase + c * 32, r);
+      tmem_wait_ld();
+      for (int s0 = 0; s0 < 32; s0 += hd) {
+        const int col = n0 + c * 32 + s0;
+        if (col >= p.N) break;
+        const int which = col / p.D;
+        const int head = (col - which * p.D) / hd;
+        uint16_t* base = which == 0 ? p.q : (which == 1 ? p.k : p.v);
+        uint16_t* dst = base + ((static_cast<size_t>(b) * p.heads + head) * p.n_total + tok) * hd;
+        float v[32];
+        float mean = 0.f, rstd = 1.f;
+        if (which < 2) {
+          float s = 0.f;
+          for (int j = 0; j < hd; ++j) s += __uint_as_float(r[s0 + j]);
+          mean = s / hd;
+          float ss = 0.f;
+          for (int j = 0; j < hd; ++j) {
+            const float d = __uint_as_float(r[s0 + j]) - mean;
+            ss += d * d;
+          }
+          rstd = rsqrtf(ss / hd + p.eps);
+        }
+        for (int j = 0; j < hd; ++j) v[j] = (__uint_as_float(r[s0 + j]) - mean) * rstd;
+        if (row_ok)
+          for (int j = 0; j < hd; ++j) dst[j] = static_cast<uint16_t>(pack_bf16(v[j], 0.f) & 0xFFFFu);
+      }
+    }
+  }
+}
+
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+    gemm_bf16_tcgen05(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                      const GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + GEMM_STAGES * A_STAGE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + GEMM_STAGES * B_STAGE_BYTES);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + GEMM_STAGES;
+  uint64_t* acc_full = bars + 2 * GEMM_STAGES;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* mma_done = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < GEMM_STAGES; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&empty[s]), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(smem_u32(&acc_full[a]), 1);
+      mbar_init(smem_u32(&acc_empty[a]), 128);
+    }
+    mbar_init(smem_u32(mma_done), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int num_k = (p.K + GEMM_BK - 1) / GEMM_BK;
+  volatile int never = 0;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, armed = 0, armed_par = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+        int mb, nb;
+        tile_coords(t, p.num_m_tiles, p.num_n_tiles, mb, nb);
+        int wrow0, wrow1;
+        if (p.mode == EPI_SWIGLU) {
+          wrow0 = nb * 128;
+          wrow1 = p.swiglu_w2_row + nb * 128;
+        } else {
+          wrow0 = nb * GEMM_BN;
+          wrow1 = wrow0 + 128;
+        }
+        for (int kb = 0; kb < num_k; ++kb) {
+          if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, p.err, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = smem_u32(&full[stage]);
+          mbar_arrive_expect_tx(fb, A_STAGE_BYTES + B_STAGE_BYTES);
+          armed |= 1u << stage;
+          armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+          const uint32_t a_dst = smem_u32(sA + stage * A_STAGE_BYTES);
+          const uint32_t b_dst = smem_u32(sB + stage * B_STAGE_BYTES);
+          tma_load_2d(a_dst, &tmA, fb, kb * GEMM_BK, mb * GEMM_BM);
+          tma_load_2d(b_dst, &tmB, fb, kb * GEMM_BK, wrow0);
+          tma_load_2d(b_dst + B_STAGE_BYTES / 2, &tmB, fb, kb * GEMM_BK, wrow1);
+          if (++stage == GEMM_STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {  // drain copies still in flight before the CTA exits
+        for (int s = 0; s < GEMM_STAGES; ++s)
+          if (armed & (1u << s))
+            mbar_wait(smem_u32(&full[s]), (armed_par >> s) & 1u, nullptr, &never, 100000000ull);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = make_idesc_bf16(GEMM_BM, GEMM_BN, false, false);
+      int stage = 0;
+      uint32_t phase = 0, acc = 0, acc_phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+        if (!mbar_wait(smem_u32(&acc_empty[acc]), acc_phase ^ 1u, p.err, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d = tmem + acc * GEMM_BN;
+        for (int kb = 0; kb < num_k; ++kb) {
+          if (!mbar_wait(smem_u32(&full[stage]), phase, p.err, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t adesc = make_sdesc(smem_u32(sA + stage * A_STAGE_BYTES), 16, 1024, SWZ_128B);
+          const uint64_t bdesc = make_sdesc(smem_u32(sB + stage * B_STAGE_BYTES), 16, 1024, SWZ_128B);
+#pragma unroll
+          for (int k = 0; k < GEMM_BK / 16; ++k)
+            mma_bf16_ss(d, adesc + 2 * k, bdesc + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+          mma_commit(smem_u32(&empty[stage]));
+          if (++stage == GEMM_STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        mma_commit(smem_u32(&acc_full[acc]));
+        acc ^= 1u;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      // all MMAs issued by this thread must finish before TMEM is released
+      mma_commit(smem_u32(mma_done));
+      mbar_wait(smem_u32(mma_done), 0, nullptr, &never, 100000000ull);
+    }
+  } else {
+    // ---------------------------------------------------------- epilogue warps
+    const int quarter = warp & 3;
+    const int row_in_tile = quarter * 32 + lane;
+    uint32_t acc = 0, acc_phase = 0;
+    for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
+      int mb, nb;
+      tile_coords(t, p.num_m_tiles, p.num_n_tiles, mb, nb);
+      const bool got = mbar_wait(smem_u32(&acc_full[acc]), acc_phase, p.err, abort_flag);
+      __syncwarp();
+      if (!__all_sync(0xffffffffu, got)) break;
+      tc_fence_after();
+      const uint32_t tbase = tmem + acc * GEMM_BN + (static_cast<uint32_t>(quarter * 32) << 16);
+      const int r = mb * GEMM_BM + row_in_tile;
+      const bool row_ok = r < p.M;
+      const int b = r / p.rows_per_batch;
+      const int n_in = r - b * p.rows_per_batch;
+      const size_t orow = static_cast<size_t>(b) * p.out_rows_per_batch + p.out_row_off + n_in;
+
+      if (p.mode == EPI_QKV) {
+        epilogue_qkv(p, tbase, nb * GEMM_BN, row_ok, b, n_in);
+      } else if (p.mode == EPI_SWIGLU) {
+        const int col0 = nb * 128;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t ra[32], rb[32];
+          tmem_ld32(tbase + c * 32, ra);
+          tmem_ld32(tbase + 128 + c * 32, rb);
+          tmem_wait_ld();
+          float v[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = silu_f(__uint_as_float(ra[j])) * __uint_as_float(rb[j]);
+          const int col = col0 + c * 32;
+          if (row_ok && col < p.N) store_bf16_n(p.out + orow * p.ldo + col, v, p.N - col);
+        }
+      } else {
+        const int col0 = nb * GEMM_BN;
+#pragma unroll 1
+        for (int c = 0; c < GEMM_BN / 32; ++c) {
+          const int col = col0 + c * 32;
+          if (col >= p.N) break;  // uniform
+          uint32_t ra[32];
+          tmem_ld32(tbase + c * 32, ra);
+          tmem_wait_ld();
+          float v[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(ra[j]);
+          if (!row_ok) continue;
+          uint16_t* dst = p.out + orow * p.ldo + col;
+          const int n = min(32, p.N - col);
+          if (p.mode == EPI_GATE_RES) {
+            const float* g = p.gate + static_cast<size_t>(b) * p.gate_stride + col;
+            if (n == 32) {
+              const uint4* xs = reinterpret_cast<const uint4*>(dst);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const uint4 xv = xs[i];
+                const float4 g0 = *reinterpret_cast<const float4*>(g + 8 * i);
+                const float4 g1 = *reinterpret_cast<const float4*>(g + 8 * i + 4);
+                v[8 * i + 0] = bf16_lo(xv.x) + g0.x * v[8 * i + 0];
+                v[8 * i + 1] = bf16_hi(xv.x) + g0.y * v[8 * i + 1];
+                v[8 * i + 2] = bf16_lo(xv.y) + g0.z * v[8 * i + 2];
+                v[8 * i + 3] = bf16_hi(xv.y) + g0.w * v[8 * i + 3];
+                v[8 * i + 4] = bf16_lo(xv.z) + g1.x * v[8 * i + 4];
+                v[8 * i + 5] = bf16_hi(xv.z) + g1.y * v[8 * i + 5];
+                v[8 * i + 6] = bf16_lo(xv.w) + g1.z * v[8 * i + 6];
+                v[8 * i + 7] = bf16_hi(xv.w) + g1.w * v[8 * i + 7];
+              }
+            } else {
+              for (int j = 0; j < n; ++j) v[j] = __uint_as_float(static_cast<uint32_t>(dst[j]) << 16) + g[j] * v[j];
+            }
+          }
+          store_bf16_n(dst, v, n);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(smem_u32(&acc_empty[acc]));
+      acc ^= 1u;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ----------------------------------------------------------------- host launch
+
+cudaError_t launch_gemm(const GemmParams& p_in, const void* A, const void* W, int W_rows, cudaStream_t stream,
+                        int num_sms) {
+  GemmParams p = p_in;
+  if (p.M <= 0 || p.N <= 0) return cudaSuccess;
+  if (p.K <= 0 || (p.K % 8) != 0) return cudaErrorInvalidValue;
+  CUtensorMap ta, tb;
+  if (!encode_tmap_2d(&ta, A, p.K, p.M, static_cast<uint64_t>(p.K) * 2, GEMM_BK, GEMM_BM)) return cudaErrorInvalidValue;
+  if (!encode_tmap_2d(&tb, W, p.K, W_rows, static_cast<uint64_t>(p.K) * 2, GEMM_BK, 128)) return cudaErrorInvalidValue;
+  p.num_m_tiles = (p.M + GEMM_BM - 1) / GEMM_BM;
+  p.num_n_tiles = p.mode == EPI_SWIGLU ? (p.N + 127) / 128 : (p.N + GEMM_BN - 1) / GEMM_BN;
+  p.num_tiles = p.num_m_tiles * p.num_n_tiles;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_bf16_tcgen05, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         GEMM_SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  const int grid = p.num_tiles < num_sms ? p.num_tiles : num_sms;
+  gemm_bf16_tcgen05<<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, stream>>>(ta, tb, p);
+  return cudaGetLastError();
+}
+
+}  // namespace af

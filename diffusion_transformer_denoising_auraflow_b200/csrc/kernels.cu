@@ -1,0 +1,388 @@
+// kernels.cu -- the HBM-bound kernels of the AuraFlow forward on sm_100a.
+//
+// Page cited: "Diffusers 中的 AuraFlowTransformer2DModel架构解析与源码级使用指南"
+// (sections named per kernel) and "Diffusers 中 AuraFlow 管线实战" (CFG).
+//
+//   ln_modulate      FP32 LayerNorm (no affine) + adaLN (1 + scale), + shift
+//                    (§调制与归一化).  One warp per row, 16-byte loads, the
+//                    row kept in registers, two-pass mean / variance with
+//                    warp shuffles.
+//   gemv_rows        out[b, j] = act(W[j] . in(x[b]) + bias[j]) for the
+//                    timestep MLP and every adaLN-Zero / pre-final linear
+//                    (§前向传播流程, §联合注意力块): one warp per weight row,
+//                    weights streamed once for the whole batch.
+//   patch_embed      patch gather + Linear(p*p*C -> D) + centre-cropped
+//                    learned position row (§Patch Embedding).
+//   output_stage     pre-final x * (1 + scale) + shift, proj_out and the
+//                    unpatchify scatter (§调制与归一化, §前向传播流程).
+//   euler_cfg        v = v_u + g (v_c - v_u); x += (sigma' - sigma) v.
+#include "af_internal.h"
+#include "ptx.cuh"
+
+namespace af {
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// ------------------------------------------------------------------ LN + modulate
+template <int VPL>  // 8-element vectors per lane
+__global__ void __launch_bounds__(256) ln_modulate_kernel(const uint16_t* __restrict__ x,
+                                                          const float* __restrict__ shift,
+                                                          const float* __restrict__ scale, int mod_stride,
+                                                          uint16_t* __restrict__ y, int rows, int rows_per_batch,
+                                                          int D, float eps) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= rows) return;
+  const int nvec = D >> 3;
+  const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<size_t>(warp) * D);
+  float v[VPL][8];
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    const int vi = i * 32 + lane;
+    if (vi < nvec) {
+      const uint4 u = xr[vi];
+      v[i][0] = bf16_lo(u.x); v[i][1] = bf16_hi(u.x); v[i][2] = bf16_lo(u.y); v[i][3] = bf16_hi(u.y);
+      v[i][4] = bf16_lo(u.z); v[i][5] = bf16_hi(u.z); v[i][6] = bf16_lo(u.w); v[i][7] = bf16_hi(u.w);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) s += v[i][e];
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v[i][e] = 0.f;
+    }
+  }
+  const float mean = warp_sum(s) / D;
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    if (i * 32 + lane < nvec) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float d = v[i][e] - mean;
+        ss += d * d;
+      }
+    }
+  }
+  const float rstd = rsqrtf(warp_sum(ss) / D + eps);
+  const int b = warp / rows_per_batch;
+  const float* sh = shift + static_cast<size_t>(b) * mod_stride;
+  const float* sc = scale + static_cast<size_t>(b) * mod_stride;
+  uint4* yr = reinterpret_cast<uint4*>(y + static_cast<size_t>(warp) * D);
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    const int vi = i * 32 + lane;
+    if (vi < nvec) {
+      const float4 s0 = *reinterpret_cast<const float4*>(sc + vi * 8);
+      const float4 s1 = *reinterpret_cast<const float4*>(sc + vi * 8 + 4);
+      const float4 h0 = *reinterpret_cast<const float4*>(sh + vi * 8);
+      const float4 h1 = *reinterpret_cast<const float4*>(sh + vi * 8 + 4);
+      const float scv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+      const float shv[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+      float o[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) o[e] = (v[i][e] - mean) * rstd * (1.0f + scv[e]) + shv[e];
+      uint4 u;
+      u.x = pack_bf16(o[0], o[1]);
+      u.y = pack_bf16(o[2], o[3]);
+      u.z = pack_bf16(o[4], o[5]);
+      u.w = pack_bf16(o[6], o[7]);
+      yr[vi] = u;
+    }
+  }
+}
+
+cudaError_t launch_ln_modulate(const uint16_t* x, const float* shift, const float* scale, int mod_stride,
+                               uint16_t* y, int rows, int rows_per_batch, int D, float eps, cudaStream_t s) {
+  if (rows <= 0) return cudaSuccess;
+  if (D % 8 != 0) return cudaErrorInvalidValue;
+  const int nvec = D / 8;
+  const int vpl = (nvec + 31) / 32;
+  const int blocks = (rows + 7) / 8;
+#define AF_LN_CASE(N)                                                                                    \
+  if (vpl <= N) {                                                                                        \
+    ln_modulate_kernel<N><<<blocks, 256, 0, s>>>(x, shift, scale, mod_stride, y, rows, rows_per_batch, D, \
+                                                 eps);                                                   \
+    return cudaGetLastError();                                                                           \
+  }
+  AF_LN_CASE(1)
+  AF_LN_CASE(2)
+  AF_LN_CASE(4)
+  AF_LN_CASE(8)
+  AF_LN_CASE(12)
+  AF_LN_CASE(16)
+#undef AF_LN_CASE
+  return cudaErrorInvalidValue;
+}
+
+// ------------------------------------------------------------------ batched GEMV
+// out[b * out_stride + j] = post(sum_k W[j, k] * pre(x[b, k]) + bias[j]),  j < rows
+// pre/post: 0 = identity, 1 = SiLU.  x is staged once per CTA in shared memory.
+constexpr int GEMV_MAX_B = 8;
+
+__global__ void __launch_bounds__(256) gemv_rows_kernel(const float* __restrict__ x, int B, int K,
+                                                        const uint16_t* __restrict__ W,
+                                                        const uint16_t* __restrict__ bias, int rows, int pre,
+                                                        int post, float* __restrict__ out, int out_stride) {
+  extern __shared__ float xs[];  // [B, K]
+  for (int i = threadIdx.x; i < B * K; i += blockDim.x) {
+    float a = x[i];
+    if (pre == 1) a = a / (1.0f + __expf(-a));
+    xs[i] = a;
+  }
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int wpb = blockDim.x >> 5;
+  const int nvec = K >> 3;
+  for (int j = blockIdx.x * wpb + (threadIdx.x >> 5); j < rows; j += gridDim.x * wpb) {
+    const uint4* wr = reinterpret_cast<const uint4*>(W + static_cast<size_t>(j) * K);
+    float acc[GEMV_MAX_B];
+#pragma unroll
+    for (int bb = 0; bb < GEMV_MAX_B; ++bb) acc[bb] = 0.f;
+    for (int vi = lane; vi < nvec; vi += 32) {
+      const uint4 u = __ldg(wr + vi);
+      const float w[8] = {bf16_lo(u.x), bf16_hi(u.x), bf16_lo(u.y), bf16_hi(u.y),
+                          bf16_lo(u.z), bf16_hi(u.z), bf16_lo(u.w), bf16_hi(u.w)};
+#pragma unroll
+      for (int bb = 0; bb < GEMV_MAX_B; ++bb) {
+        if (bb < B) {
+          const float* xb = xs + bb * K + vi * 8;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[bb] += w[e] * xb[e];
+        }
+      }
+    }
+#pragma unroll
+    for (int bb = 0; bb < GEMV_MAX_B; ++bb) {
+      if (bb < B) {
+        float r = warp_sum(acc[bb]);
+        if (lane == 0) {
+          if (bias) r += __uint_as_float(static_cast<uint32_t>(bias[j]) << 16);
+          if (post == 1) r = r / (1.0f + __expf(-r));
+          out[static_cast<size_t>(bb) * out_stride + j] = r;
+        }
+      }
+    }
+  }
+}
+
+static cudaError_t gemv(const float* x, int B, int K, const uint16_t* W, const uint16_t* bias, int rows, int pre,
+                        int post, float* out, int out_stride, cudaStream_t s) {
+  if (K % 8 != 0) return cudaErrorInvalidValue;
+  static int sms = 0;
+  if (!sms) sms = device_sm_count();
+  for (int b0 = 0; b0 < B; b0 += GEMV_MAX_B) {
+    const int nb = B - b0 < GEMV_MAX_B ? B - b0 : GEMV_MAX_B;
+    const size_t smem = static_cast<size_t>(nb) * K * sizeof(float);
+    if (smem > 48 * 1024) {
+      cudaError_t e = cudaFuncSetAttribute(gemv_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(smem));
+      if (e != cudaSuccess) return e;
+    }
+    int blocks = (rows + 7) / 8;
+    const int cap = sms * 8;
+    if (blocks > cap) blocks = cap;
+    gemv_rows_kernel<<<blocks, 256, smem, s>>>(x + static_cast<size_t>(b0) * K, nb, K, W, bias, rows, pre, post,
+                                               out + static_cast<size_t>(b0) * out_stride, out_stride);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+// ------------------------------------------------------------------ timestep embedding
+// e = [cos(1000 t w_j), sin(1000 t w_j)], w_j = exp(-ln(10000) j / half)   (§前向传播流程)
+__global__ void timestep_features_kernel(const float* __restrict__ t, int B, int C, float* __restrict__ e) {
+  const int half = C / 2;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < B * half; i += gridDim.x * blockDim.x) {
+    const int b = i / half, j = i - b * half;
+    const float w = expf(-9.210340371976184f * static_cast<float>(j) / static_cast<float>(half));
+    const float a = 1000.0f * t[b] * w;
+    e[b * C + j] = cosf(a);
+    e[b * C + half + j] = sinf(a);
+  }
+}
+
+cudaError_t launch_timestep_mlp(const float* t, int B, const uint16_t* w1, const uint16_t* b1, const uint16_t* w2,
+                                const uint16_t* b2, int C, int D, float* feat, float* h1, float* temb, cudaStream_t s) {
+  timestep_features_kernel<<<(B * C / 2 + 255) / 256, 256, 0, s>>>(t, B, C, feat);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  e = gemv(feat, B, C, w1, b1, D, 0, 1, h1, D, s);  // h1 = silu(W1 e + b1)
+  if (e != cudaSuccess) return e;
+  return gemv(h1, B, D, w2, b2, D, 0, 0, temb, D, s);  // temb = W2 h1 + b2
+}
+
+cudaError_t launch_modulation(const float* temb, int B, int D, const uint16_t* w, int rows, float* out,
+                              cudaStream_t s) {
+  return gemv(temb, B, D, w, nullptr, rows, 1, 0, out, rows, s);  // out[b, r] = W[r] . silu(temb[b])
+}
+
+// ------------------------------------------------------------------ patch embedding
+// img[b, n, d] = sum_k W[d, k] patch(b, n)[k] + PE[(r0 + n / wp) * G + c0 + n % wp, d]
+// patch vector index k = (py * p + px) * C + c  <->  latent[b, c, hp * p + py, wp * p + px]
+__global__ void __launch_bounds__(128) patch_embed_kernel(const float* __restrict__ lat, int C, int H, int W, int p,
+                                                          const uint16_t* __restrict__ wpe,
+                                                          const uint16_t* __restrict__ pos, int G, int D,
+                                                          uint16_t* __restrict__ out, int out_rows_per_batch,
+                                                          int out_row_off) {
+  __shared__ float patch[64];
+  const int n = blockIdx.x, b = blockIdx.y;
+  const int hpn = H / p, wpn = W / p;
+  const int hp = n / wpn, wp = n - hp * wpn;
+  const int KP = p * p * C;
+  for (int k = threadIdx.x; k < KP; k += blockDim.x) {
+    const int c = k % C, pq = k / C;
+    const int py = pq / p, px = pq - py * p;
+    patch[k] = lat[((static_cast<size_t>(b) * C + c) * H + hp * p + py) * W + wp * p + px];
+  }
+  __syncthreads();
+  const int r0 = (G - hpn) / 2, c0 = (G - wpn) / 2;
+  const size_t prow = static_cast<size_t>(r0 + hp) * G + c0 + wp;
+  uint16_t* orow = out + (static_cast<size_t>(b) * out_rows_per_batch + out_row_off + n) * D;
+  const int nvec = D / 8;
+  for (int vi = threadIdx.x; vi < nvec; vi += blockDim.x) {
+    const uint4 pu = *reinterpret_cast<const uint4*>(pos + prow * D + vi * 8);
+    float acc[8] = {bf16_lo(pu.x), bf16_hi(pu.x), bf16_lo(pu.y), bf16_hi(pu.y),
+                    bf16_lo(pu.z), bf16_hi(pu.z), bf16_lo(pu.w), bf16_hi(pu.w)};
+    float mm[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    for (int e = 0; e < 8; ++e) {
+      const uint16_t* wr = wpe + static_cast<size_t>(vi * 8 + e) * KP;
+      float a = 0.f;
+      for (int k = 0; k < KP; ++k) a += __uint_as_float(static_cast<uint32_t>(wr[k]) << 16) * patch[k];
+      mm[e] = a;
+    }
+    uint4 u;
+    u.x = pack_bf16(mm[0] + acc[0], mm[1] + acc[1]);
+    u.y = pack_bf16(mm[2] + acc[2], mm[3] + acc[3]);
+    u.z = pack_bf16(mm[4] + acc[4], mm[5] + acc[5]);
+    u.w = pack_bf16(mm[6] + acc[6], mm[7] + acc[7]);
+    *reinterpret_cast<uint4*>(orow + vi * 8) = u;
+  }
+}
+
+cudaError_t launch_patch_embed(const float* lat, int B, int C, int H, int W, int p, const uint16_t* w_pe,
+                               const uint16_t* pos, int G, int D, uint16_t* out, int out_rows_per_batch,
+                               int out_row_off, cudaStream_t s) {
+  if (p * p * C > 64 || D % 8 != 0) return cudaErrorInvalidValue;
+  dim3 grid((H / p) * (W / p), B);
+  patch_embed_kernel<<<grid, 128, 0, s>>>(lat, C, H, W, p, w_pe, pos, G, D, out, out_rows_per_batch, out_row_off);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ output stage
+// z = x * (1 + scale[b]) + shift[b];  o[k] = W_out[k] . z  (k < p*p*C);
+// velocity[b, c, hp * p + py, wp * p + px] = o[(py * p + px) * C + c]
+template <int VPL>
+__global__ void __launch_bounds__(256) output_stage_kernel(const uint16_t* __restrict__ x, int rows_per_batch,
+                                                           int row_off, int B, int hpn, int wpn, int D,
+                                                           const float* __restrict__ scale,
+                                                           const float* __restrict__ shift, int mod_stride,
+                                                           const uint16_t* __restrict__ wout, int p, int C,
+                                                           float* __restrict__ vel) {
+  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const int ntok = hpn * wpn;
+  if (gw >= B * ntok) return;
+  const int b = gw / ntok, n = gw - b * ntok;
+  const uint4* xr = reinterpret_cast<const uint4*>(x + (static_cast<size_t>(b) * rows_per_batch + row_off + n) * D);
+  const float* sc = scale + static_cast<size_t>(b) * mod_stride;
+  const float* sh = shift + static_cast<size_t>(b) * mod_stride;
+  const int nvec = D >> 3;
+  float z[VPL][8];
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    const int vi = i * 32 + lane;
+    if (vi < nvec) {
+      const uint4 u = xr[vi];
+      const float xv[8] = {bf16_lo(u.x), bf16_hi(u.x), bf16_lo(u.y), bf16_hi(u.y),
+                           bf16_lo(u.z), bf16_hi(u.z), bf16_lo(u.w), bf16_hi(u.w)};
+#pragma unroll
+      for (int e = 0; e < 8; ++e) z[i][e] = xv[e] * (1.0f + sc[vi * 8 + e]) + sh[vi * 8 + e];
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) z[i][e] = 0.f;
+    }
+  }
+  const int KP = p * p * C;
+  const int hp = n / wpn, wp = n - hp * wpn;
+  const int H = hpn * p, W = wpn * p;
+  for (int k = 0; k < KP; ++k) {
+    const uint4* wr = reinterpret_cast<const uint4*>(wout + static_cast<size_t>(k) * D);
+    float a = 0.f;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const int vi = i * 32 + lane;
+      if (vi < nvec) {
+        const uint4 u = __ldg(wr + vi);
+        a += bf16_lo(u.x) * z[i][0] + bf16_hi(u.x) * z[i][1] + bf16_lo(u.y) * z[i][2] + bf16_hi(u.y) * z[i][3] +
+             bf16_lo(u.z) * z[i][4] + bf16_hi(u.z) * z[i][5] + bf16_lo(u.w) * z[i][6] + bf16_hi(u.w) * z[i][7];
+      }
+    }
+    a = warp_sum(a);
+    if (lane == 0) {
+      const int c = k % C, pq = k / C;
+      const int py = pq / p, px = pq - py * p;
+      vel[((static_cast<size_t>(b) * C + c) * H + hp * p + py) * W + wp * p + px] = a;
+    }
+  }
+}
+
+cudaError_t launch_output_stage(const uint16_t* x, int rows_per_batch, int row_off, int B, int hp, int wp, int D,
+                                const float* scale, const float* shift, int mod_stride, const uint16_t* w_out, int p,
+                                int C, float* vel, cudaStream_t s) {
+  if (D % 8 != 0) return cudaErrorInvalidValue;
+  const int warps = B * hp * wp;
+  const int blocks = (warps + 7) / 8;
+  const int vpl = (D / 8 + 31) / 32;
+#define AF_OUT_CASE(N)                                                                                        \
+  if (vpl <= N) {                                                                                             \
+    output_stage_kernel<N><<<blocks, 256, 0, s>>>(x, rows_per_batch, row_off, B, hp, wp, D, scale, shift,     \
+                                                  mod_stride, w_out, p, C, vel);                              \
+    return cudaGetLastError();                                                                                \
+  }
+  AF_OUT_CASE(1)
+  AF_OUT_CASE(4)
+  AF_OUT_CASE(12)
+  AF_OUT_CASE(16)
+#undef AF_OUT_CASE
+  return cudaErrorInvalidValue;
+}
+
+// ------------------------------------------------------------------ fill (model time of a CFG batch)
+__global__ void fill_kernel(float* __restrict__ dst, int n, float value) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) dst[i] = value;
+}
+
+cudaError_t launch_fill(float* dst, int n, float value, cudaStream_t s) {
+  fill_kernel<<<(n + 255) / 256, 256, 0, s>>>(dst, n, value);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ Euler + CFG
+__global__ void euler_cfg_kernel(float* __restrict__ x, const float* __restrict__ v, int64_t n_total,
+                                 int64_t per_sample, float g, float dt) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n_total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float vu = v[i];
+    const float vc = v[i + n_total];
+    (void)per_sample;
+    x[i] = x[i] + dt * (vu + g * (vc - vu));
+  }
+}
+
+cudaError_t launch_euler_cfg(float* lat, const float* v, int Bi, int64_t per_sample, float g, float sigma,
+                             float sigma_next, cudaStream_t s) {
+  const int64_t n = static_cast<int64_t>(Bi) * per_sample;
+  if (n <= 0) return cudaSuccess;
+  int blocks = static_cast<int>((n + 255) / 256);
+  if (blocks > 4096) blocks = 4096;
+  euler_cfg_kernel<<<blocks, 256, 0, s>>>(lat, v, n, per_sample, g, sigma_next - sigma);
+  return cudaGetLastError();
+}
+
+}  // namespace af

@@ -1,0 +1,250 @@
+/*
+ * af.h -- C ABI of the B200 (sm_100a) AuraFlow denoising forward.
+ *
+ * The library computes the AuraFlowTransformer2DModel forward and the
+ * flow-match Euler + classifier-free-guidance step on one GPU with
+ * hand-written CUDA kernels.  Citations name the page title and section of
+ * the description the operation follows:
+ *
+ *   [ARCH] "Diffusers 中的 AuraFlowTransformer2DModel架构解析与源码级使用指南"
+ *   [PIPE] "Diffusers 中 AuraFlow 管线实战：从 bitsandbytes 量化到 torch.compile 加速"
+ *   [DEEP] "【深度拆解】AuraFlow从基座到技术实现：开源文生图新范式"
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Tensors are caller-owned, contiguous, row-major.  "device" pointers
+ *    must be CUDA device memory of the device the weight pack lives on.
+ *    bf16 tensors are passed as uint16_t bit patterns.
+ *  - Compute calls are asynchronous on `stream` (a cudaStream_t passed as
+ *    void*; NULL = legacy default stream).  They return once all work is
+ *    enqueued.
+ *  - Argument and shape errors are detected on the host, before anything is
+ *    launched, and reported as AF_ERR_INVALID_ARG / AF_ERR_SHAPE /
+ *    AF_ERR_UNSUPPORTED; nothing is modified in that case.
+ *  - A CUDA launch or runtime failure returns AF_ERR_CUDA; af_last_error()
+ *    then holds the CUDA error text.
+ *  - Every device-side wait in the kernels is bounded.  A wait that runs out
+ *    records an error word in the scratch handle; af_sync() reports it as
+ *    AF_ERR_TIMEOUT.
+ *  - Only *_create calls allocate device memory.  A scratch handle must not
+ *    be used by two streams at once (calls on it would race).
+ */
+#ifndef AF_H_
+#define AF_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  AF_OK = 0,
+  AF_ERR_INVALID_ARG = 1,  /* null handle/pointer, bad enum, negative size */
+  AF_ERR_SHAPE = 2,        /* sizes inconsistent with the model or over capacity */
+  AF_ERR_UNSUPPORTED = 3,  /* configuration this build does not implement */
+  AF_ERR_OOM = 4,          /* device allocation failed in a *_create call */
+  AF_ERR_CUDA = 5,         /* CUDA runtime error (see af_last_error) */
+  AF_ERR_TIMEOUT = 6,      /* a bounded device-side wait expired (from af_sync) */
+  AF_ERR_NOT_FOUND = 7     /* unknown tensor name */
+} af_status;
+
+/* Model configuration: the constructor parameters of
+ * AuraFlowTransformer2DModel ([ARCH] §构造参数详解).
+ *   inner_dim D = num_attention_heads * attention_head_dim.
+ *   ffn_inner  = 0 selects find_multiple(int(2 * 4D / 3), 256) ([ARCH]
+ *                §FeedForward); any other value is used as given.
+ *   pos_embed_max_size = G*G, the size of the learned position grid
+ *                ([ARCH] §Patch Embedding); must be a perfect square.
+ *   num_register_tokens: learned tokens at the head of the text sequence
+ *                ([ARCH] §Register Tokens), 8 in the model.
+ *   timestep_channels: sinusoidal timestep channels, 256 ([ARCH] §前向传播流程).
+ *   ln_eps: epsilon of every LayerNorm (adaLN and QK-norm). */
+typedef struct {
+  int patch_size;
+  int in_channels;
+  int out_channels;
+  int num_mmdit_layers;
+  int num_single_dit_layers;
+  int attention_head_dim;
+  int num_attention_heads;
+  int joint_attention_dim;
+  int pos_embed_max_size;
+  int num_register_tokens;
+  int timestep_channels;
+  int ffn_inner;
+  float ln_eps;
+} af_config;
+
+typedef struct af_weights af_weights; /* device-resident weight pack (bf16) */
+typedef struct af_scratch af_scratch; /* device work buffers + error word */
+
+/* Fill *cfg with the page's defaults (patch 2, 4 -> 4 channels, 4 joint +
+ * 32 single blocks, 12 heads x 256, joint_attention_dim 2048,
+ * pos_embed_max_size 1024, 8 registers, 256 timestep channels, eps 1e-6). */
+af_status af_config_default(af_config* cfg);
+
+/* Derived sizes: inner_dim D, FFN width F, position grid side G.
+ * AF_ERR_INVALID_ARG if the configuration is malformed. */
+af_status af_config_derive(const af_config* cfg, int* inner_dim, int* ffn_inner, int* grid_side);
+
+/* ---- weight pack --------------------------------------------------------
+ * One device allocation holding every parameter in bf16.  Tensors are
+ * addressed by the diffusers-style names listed by af_weights_tensor_info
+ * (e.g. "single_transformer_blocks.3.attn.to_q.weight"), each with the
+ * nn.Linear layout [out, in].  Freshly created packs are zero-filled. */
+af_status af_weights_create(const af_config* cfg, int device, af_weights** out);
+void af_weights_destroy(af_weights* w);
+af_status af_weights_num_tensors(const af_weights* w, int* n);
+/* name: written NUL-terminated into name[0..name_cap); shape: up to 2 dims
+ * (ndim = 1 or 2). */
+af_status af_weights_tensor_info(const af_weights* w, int id, char* name, size_t name_cap,
+                                 int* ndim, int64_t shape[2]);
+af_status af_weights_find(const af_weights* w, const char* name, int* id);
+/* Copy one tensor (bf16 bit patterns, numel elements as listed) into the
+ * pack.  src_is_device != 0: src is device memory on the pack's device,
+ * else host memory.  Asynchronous on `stream` for device sources; host
+ * sources are copied synchronously. */
+af_status af_weights_set(af_weights* w, int id, const uint16_t* src, int src_is_device, void* stream);
+/* Total bytes of the pack (for reporting). */
+af_status af_weights_bytes(const af_weights* w, size_t* bytes);
+
+/* ---- scratch ------------------------------------------------------------
+ * Work buffers for batches up to max_batch with at most max_img_tokens
+ * image tokens ((H/p)*(W/p)) and at most max_text_len text tokens (before
+ * the registers are prepended). */
+af_status af_scratch_create(const af_weights* w, int max_batch, int max_img_tokens, int max_text_len,
+                            af_scratch** out);
+void af_scratch_destroy(af_scratch* s);
+/* Synchronise `stream`, then read and clear the device error word.
+ * Returns AF_ERR_TIMEOUT if a bounded device wait expired since the last
+ * af_sync, AF_ERR_CUDA on a CUDA error, else AF_OK. */
+af_status af_sync(af_scratch* s, void* stream);
+
+/* ---- the forward path ---------------------------------------------------*/
+
+/* Timestep embedding: temb[b] = W2 silu(W1 e(t_b) + b1) + b2 with e the
+ * 256-channel sinusoid of 1000*t_b (cosines first).  [ARCH] §前向传播流程
+ * (Timesteps -> TimestepEmbedding), §在 AuraFlowPipeline 中的实际调用 (the
+ * model receives timestep/1000).
+ *   t:    device float[B], model time in [0, 1] (1 = pure noise).
+ *   temb: device float[B, D] (output). */
+af_status af_timestep_embed(const af_weights* w, af_scratch* s, const float* t, int B, float* temb,
+                            void* stream);
+
+/* Patch embedding with centre-cropped learned positions ([ARCH] §Patch
+ * Embedding): img[b, n] = W_pe patch(b, n) + PE[(r0 + n / wp) * G + c0 + n % wp]
+ * with r0 = (G - H/p) / 2, c0 = (G - W/p) / 2 (floor); patch vector order
+ * (row-in-patch, col-in-patch, channel); tokens row-major over the patch grid.
+ *   latents:    device float[B, C_in, H, W].
+ *   img_tokens: device bf16[B, (H/p)(W/p), D] (output).
+ * AF_ERR_SHAPE if H or W is not a multiple of p or the patch grid exceeds
+ * the G x G position grid ([PIPE] §AuraFlowPipeline 核心参数详解, the
+ * resolution check). */
+af_status af_patch_embed(const af_weights* w, af_scratch* s, const float* latents, int B, int H, int W,
+                         uint16_t* img_tokens, void* stream);
+
+/* One AuraFlowJointTransformerBlock ([ARCH] §联合注意力块, §注意力处理器与
+ * QKV 融合), in place on both residual streams:
+ *   per stream: adaLN-Zero (6 vectors from W silu(temb)), FP32 LayerNorm,
+ *   bias-free Q/K/V with per-head LayerNorm on Q and K, joint attention over
+ *   [text; image] (text first), gated output projection, gated SiLU FFN.
+ *   img:  device bf16[B, Ni, D] in/out (image stream).
+ *   txt:  device bf16[B, Nt, D] in/out (text stream incl. registers).
+ *   temb: device float[B, D].
+ *   layer in [0, num_mmdit_layers). */
+af_status af_joint_block(const af_weights* w, af_scratch* s, int layer, uint16_t* img, uint16_t* txt,
+                         const float* temb, int B, int Ni, int Nt, void* stream);
+
+/* One AuraFlowSingleTransformerBlock ([ARCH] §单 DiT 块) in place on the
+ * concatenated sequence x = [text; image]:
+ *   x: device bf16[B, N, D] in/out; temb: device float[B, D];
+ *   layer in [0, num_single_dit_layers). */
+af_status af_single_block(const af_weights* w, af_scratch* s, int layer, uint16_t* x, const float* temb,
+                          int B, int N, void* stream);
+
+/* The whole AuraFlowTransformer2DModel forward ([ARCH] §前向传播流程):
+ * patch embed, timestep embed, context_embedder (bias-free 2048 -> D) with
+ * the register tokens prepended, the joint blocks, concatenation
+ * [text; image], the single blocks, the image slice, the pre-final
+ * modulation x * (1 + scale) + shift, proj_out (bias-free) and unpatchify.
+ *   latents:  device float[B, C_in, H, W]
+ *   text_emb: device bf16[B, L, joint_attention_dim]
+ *   t:        device float[B] (timestep / 1000)
+ *   velocity: device float[B, C_out, H, W] (output) */
+af_status af_transformer_forward(const af_weights* w, af_scratch* s, const float* latents,
+                                 const uint16_t* text_emb, const float* t, int B, int H, int W, int L,
+                                 float* velocity, void* stream);
+
+/* Classifier-free guidance combine and flow-match Euler step ([PIPE]
+ * §AuraFlowPipeline 核心参数详解 (CFG formula), [ARCH] §在 AuraFlowPipeline
+ * 中的实际调用 (uncond half first), [DEEP] §2.3 (FlowMatchEulerDiscreteScheduler)):
+ *   v = v[uncond] + guidance (v[text] - v[uncond]);  x += (sigma_next - sigma) v
+ *   latents:  device float[Bi, C, H, W] in/out
+ *   velocity: device float[2 Bi, C, H, W], the uncond half first.
+ * With guidance disabled pass the B = Bi velocity twice-concatenated or
+ * guidance = 1 and any uncond half. */
+af_status af_euler_cfg_step(float* latents, const float* velocity, int Bi, int C, int H, int W,
+                            float guidance, float sigma, float sigma_next, void* stream);
+
+/* One step of the sampling loop ([ARCH] §在 AuraFlowPipeline 中的实际调用):
+ * the latents are duplicated into a CFG batch [uncond; text], the forward
+ * runs at model time t = sigma on the 2 Bi batch, and af_euler_cfg_step
+ * updates the latents in place with sigma_next.
+ *   latents:  device float[Bi, C_in, H, W] in/out
+ *   text_emb: device bf16[2 Bi, L, joint_attention_dim], uncond rows first.
+ * Needs a scratch created with max_batch >= 2 Bi. */
+af_status af_denoise_step(const af_weights* w, af_scratch* s, float* latents, const uint16_t* text_emb, int Bi,
+                          int H, int W, int L, float guidance, float sigma, float sigma_next, void* stream);
+
+/* Host-side sigma schedule of the flow-match Euler sampler ([DEEP] §2.3:
+ * num_train_timesteps 1000, shift 1.73, 25 steps): n_steps + 1 values
+ * sigma_i = k s_i / (1 + (k - 1) s_i) with s = linspace(1, 1/num_train,
+ * n_steps), then a final 0.  The model time of step i is t_i = sigma_i.
+ * out: host float[n_steps + 1].  No device work. */
+af_status af_sigma_schedule(int n_steps, float shift, int num_train_timesteps, float* out);
+
+/* ---- launch accounting and per-kernel-class timing ----------------------
+ * Kernel classes: 0 tensor-core GEMM, 1 attention, 2 LayerNorm+modulate,
+ * 3 other kernels (timestep/modulation GEMV, patch embed, output stage,
+ * Euler/CFG).  af_launch_counts returns the number of this library's kernel
+ * launches made through `s` since it was created (always counted).
+ * Between af_profile_begin and af_profile_end, a CUDA event pair is
+ * recorded around every launch; af_profile_end synchronises `stream` and
+ * returns, per class, the summed device time (ms), the number of launches
+ * and the algorithmic work (FLOPs for classes 0/1, bytes moved for 2/3). */
+#define AF_NUM_KERNEL_CLASSES 4
+af_status af_launch_counts(const af_scratch* s, int64_t counts[AF_NUM_KERNEL_CLASSES]);
+af_status af_profile_begin(af_scratch* s);
+af_status af_profile_end(af_scratch* s, void* stream, double ms[AF_NUM_KERNEL_CLASSES],
+                         int64_t launches[AF_NUM_KERNEL_CLASSES], double work[AF_NUM_KERNEL_CLASSES]);
+
+/* ---- building blocks (the kernels the forward is made of) --------------*/
+
+/* y = LN(x) * (1 + scale[b]) + shift[b]: FP32 LayerNorm without affine
+ * weights ([ARCH] §调制与归一化), then the adaLN modulation.
+ *   x, y: device bf16[B*N, D];  shift, scale: device float, element (b, d)
+ *   at shift[b * mod_stride + d]. */
+af_status af_ln_modulate(const uint16_t* x, const float* shift, const float* scale, int mod_stride,
+                         uint16_t* y, int B, int N, int D, float eps, void* stream);
+
+/* C = A W^T on the tcgen05 tensor cores, bf16 in, fp32 accumulate, bf16 out.
+ *   A: device bf16[M, K]; W: device bf16[N, K]; C: device bf16[M, N].
+ *   K must be a multiple of 8 (16-byte rows for the TMA engine). */
+af_status af_linear(const uint16_t* A, const uint16_t* W, uint16_t* C, int M, int N, int K, void* stream);
+
+/* Non-causal softmax(q k^T / sqrt(hd)) v per (batch, head) ([ARCH]
+ * §注意力处理器与 QKV 融合).
+ *   q, k, v: device bf16[B, H, N, hd];  o: device bf16[B, N, H*hd]. */
+af_status af_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* o, int B,
+                       int H, int N, int hd, void* stream);
+
+const char* af_status_string(af_status st);
+/* Text of the last CUDA error seen by this thread's calls ("" if none). */
+const char* af_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* AF_H_ */

@@ -329,11 +329,11 @@ def attention(q, k, v, scale=None):
     q, k, v = _f(q), _f(k), _f(v)
     if scale is None:
         scale = 1.0 / math.sqrt(q.shape[-1])
-    s = np.einsum("bhqd,bhkd->bhqk", q, k) * scale
+    s = (q @ np.swapaxes(k, -1, -2)) * scale
     s = s - s.max(axis=-1, keepdims=True)
     p = np.exp(s)
     p = p / p.sum(axis=-1, keepdims=True)
-    return np.einsum("bhqk,bhkd->bhqd", p, v)
+    return p @ v
 
 
 def qkv_normed(y, wq, wk, wv, heads: int, eps: float):

@@ -1,0 +1,150 @@
+"""GPU parity of whole blocks against the fp64 oracle.
+
+The tolerance per block is relative L2 <= 2e-2 (bf16 path).  Small token
+counts with a ragged tail exercise several tiles; the full single-block and
+joint-block workloads (B = 2, 4096 image + 256 text tokens, D = 3072,
+F = 8192) are checked on sampled rows, which the oracle computes from all
+keys and values.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import synth
+from helpers import af_config, block_names, draw_weights, full_config, to_bf16, to_f32, to_np, upload
+
+pytestmark = pytest.mark.gpu
+
+BLOCK_TOL = 2e-2
+
+
+@pytest.fixture(scope="module")
+def af():
+    import diffusion_transformer_denoising_auraflow_b200 as m
+    return m
+
+
+@pytest.fixture(scope="module")
+def single_setup(af):
+    cfg = full_config(num_mmdit_layers=0, num_single_dit_layers=1)
+    w = af.Weights(af_config(cfg))
+    drawn = draw_weights(cfg, 2, block_names(cfg, "single", 0))
+    upload(w, drawn)
+    s = af.Scratch(w, 2, 4096, 256)
+    return cfg, w, s, drawn
+
+
+@pytest.fixture(scope="module")
+def joint_setup(af):
+    cfg = full_config(num_mmdit_layers=1, num_single_dit_layers=0)
+    w = af.Weights(af_config(cfg))
+    drawn = draw_weights(cfg, 3, block_names(cfg, "joint", 0))
+    upload(w, drawn)
+    s = af.Scratch(w, 2, 4096, 256)
+    return cfg, w, s, drawn
+
+
+def _run_single(af, setup, x, temb):
+    cfg, w, s, drawn = setup
+    xt = to_bf16(x)
+    af.single_block(w, s, 0, xt, to_f32(temb))
+    s.sync()
+    return to_np(xt)
+
+
+@pytest.mark.parametrize("N", [300, 129])
+def test_single_block_small(af, single_setup, N):
+    cfg, w, s, drawn = single_setup
+    x = synth.activations(2, f"x{N}", (2, N, 3072))
+    temb = synth.conditioning(2, (2, 3072))
+    got = _run_single(af, single_setup, x, temb)
+    ref = O.single_block(x, temb, drawn, "single_transformer_blocks.0.", cfg)
+    err = O.rel_l2(got - x, ref - x)   # the block's update, the harder comparison
+    assert O.rel_l2(got, ref) < BLOCK_TOL and err < 5e-2, err
+
+
+def test_single_block_zero_gates_identity(af, single_setup):
+    cfg, w, s, drawn = single_setup
+    name = "single_transformer_blocks.0.norm1.linear.weight"
+    W = drawn[name].copy()
+    W[2 * 3072:3 * 3072] = 0.0
+    W[5 * 3072:6 * 3072] = 0.0
+    w.set(name, to_bf16(W))
+    try:
+        x = synth.activations(3, "xz", (2, 77, 3072))
+        got = _run_single(af, single_setup, x, synth.conditioning(3, (2, 3072)))
+        assert np.array_equal(got, x.astype(np.float64))
+    finally:
+        w.set(name, to_bf16(drawn[name]))
+
+
+def test_single_block_batch_independence(af, single_setup):
+    x = synth.activations(4, "xb", (2, 140, 3072))
+    temb = synth.conditioning(4, (2, 3072))
+    both = _run_single(af, single_setup, x, temb)
+    for b in range(2):
+        one = _run_single(af, single_setup, x[b:b + 1], temb[b:b + 1])
+        assert np.array_equal(both[b:b + 1], one)
+
+
+def test_single_block_full_size_sampled_rows(af, single_setup):
+    """The single-block workload: B = 2, 256 text + 4096 image tokens."""
+    cfg, w, s, drawn = single_setup
+    N = 4352
+    x = synth.activations(5, "xfull", (2, N, 3072))
+    temb = synth.conditioning(5, (2, 3072))
+    got = _run_single(af, single_setup, x, temb)
+    rows = [0, 1, 127, 128, 255, 256, 1000, 2047, 2048, 3333, 4223, 4224, 4351]
+    ref = O.single_block_rows(x, temb, drawn, "single_transformer_blocks.0.", cfg, rows)
+    assert O.rel_l2(got[:, rows], ref) < BLOCK_TOL
+
+
+def _run_joint(af, setup, img, txt, temb):
+    cfg, w, s, drawn = setup
+    it, tt = to_bf16(img), to_bf16(txt)
+    af.joint_block(w, s, 0, it, tt, to_f32(temb))
+    s.sync()
+    return to_np(tt), to_np(it)
+
+
+def test_joint_block_small(af, joint_setup):
+    cfg, w, s, drawn = joint_setup
+    img = synth.activations(6, "img", (2, 200, 3072))
+    txt = synth.activations(6, "txt", (2, 37, 3072))
+    temb = synth.conditioning(6, (2, 3072))
+    gt, gi = _run_joint(af, joint_setup, img, txt, temb)
+    rt, ri = O.joint_block(img, txt, temb, drawn, "joint_transformer_blocks.0.", cfg)
+    assert O.rel_l2(gi, ri) < BLOCK_TOL and O.rel_l2(gt, rt) < BLOCK_TOL
+    assert O.rel_l2(gi - img, ri - img) < 5e-2 and O.rel_l2(gt - txt, rt - txt) < 5e-2
+
+
+def test_joint_block_zero_gates_identity(af, joint_setup):
+    cfg, w, s, drawn = joint_setup
+    names = ["joint_transformer_blocks.0.norm1.linear.weight", "joint_transformer_blocks.0.norm1_context.linear.weight"]
+    for n in names:
+        W = drawn[n].copy()
+        W[2 * 3072:3 * 3072] = 0.0
+        W[5 * 3072:6 * 3072] = 0.0
+        w.set(n, to_bf16(W))
+    try:
+        img = synth.activations(7, "img", (2, 64, 3072))
+        txt = synth.activations(7, "txt", (2, 20, 3072))
+        gt, gi = _run_joint(af, joint_setup, img, txt, synth.conditioning(7, (2, 3072)))
+        assert np.array_equal(gi, img.astype(np.float64)) and np.array_equal(gt, txt.astype(np.float64))
+    finally:
+        for n in names:
+            w.set(n, to_bf16(drawn[n]))
+
+
+def test_joint_block_full_size_sampled_rows(af, joint_setup):
+    """The joint-block workload: B = 2, image stream 4096 tokens, text stream 256."""
+    cfg, w, s, drawn = joint_setup
+    img = synth.activations(8, "imgfull", (2, 4096, 3072))
+    txt = synth.activations(8, "txtfull", (2, 256, 3072))
+    temb = synth.conditioning(8, (2, 3072))
+    gt, gi = _run_joint(af, joint_setup, img, txt, temb)
+    ir = [0, 127, 128, 1500, 4095]
+    tr = [0, 7, 8, 128, 255]
+    rt, ri = O.joint_block_rows(img, txt, temb, drawn, "joint_transformer_blocks.0.", cfg, ir, tr)
+    assert O.rel_l2(gi[:, ir], ri) < BLOCK_TOL and O.rel_l2(gt[:, tr], rt) < BLOCK_TOL

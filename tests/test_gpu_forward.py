@@ -1,0 +1,126 @@
+"""GPU parity of the whole forward (+ CFG / Euler step) against the oracle.
+
+Tolerance for the full stack on the bf16 path: relative L2 <= 5e-2.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import synth
+from helpers import af_config, draw_weights, tiny_config, to_bf16, to_f32, to_np, upload
+
+pytestmark = pytest.mark.gpu
+
+STACK_TOL = 5e-2
+
+
+@pytest.fixture(scope="module")
+def af():
+    import diffusion_transformer_denoising_auraflow_b200 as m
+    return m
+
+
+def _forward(af, cfg, seed, B, H, W, L, t, with_step=None):
+    w = af.Weights(af_config(cfg))
+    drawn = draw_weights(cfg, seed)
+    upload(w, drawn)
+    s = af.Scratch(w, B, (H // 2) * (W // 2), L)
+    lat = synth.latents(seed, (B, 4, H, W))
+    text = synth.text_embeddings(seed, (B, L, cfg.joint_attention_dim))
+    tt = np.full((B,), t, dtype=np.float32)
+    vel = torch.empty(B, 4, H, W, dtype=torch.float32, device="cuda")
+    af.transformer_forward(w, s, to_f32(lat), to_bf16(text), to_f32(tt), vel)
+    s.sync()
+    ref = O.transformer_forward(lat, text, tt, drawn, cfg)
+    return w, s, drawn, lat, text, to_np(vel), ref
+
+
+def test_tiny_forward_matches_oracle(af):
+    """Tiny model: 1 joint + 1 single block, D = 32 (4 x 8), F = 256, 8 x 8 grid,
+    latent 4 x 16 x 16 (64 image tokens), 8 text tokens, timestep 500."""
+    cfg = tiny_config()
+    *_, got, ref = _forward(af, cfg, 1, 1, 16, 16, 8, 0.5)
+    assert O.rel_l2(got, ref) < STACK_TOL
+
+
+def test_tiny_forward_cfg_euler_step(af):
+    cfg = tiny_config()
+    w, s, drawn, lat, text, got, ref = _forward(af, cfg, 9, 2, 16, 16, 8, 1.0)
+    x = synth.latents(10, (1, 4, 16, 16))
+    xt = to_f32(x)
+    sig = O.sigma_schedule(25, 1.73)
+    af.euler_cfg_step(xt, to_f32(got.astype(np.float32)), 3.5, sig[0], sig[1])
+    torch.cuda.synchronize()
+    ref_x = O.euler_cfg_step(x, ref, 3.5, sig[0], sig[1])
+    assert O.rel_l2(to_np(xt) - x, ref_x - x) < STACK_TOL
+
+
+def test_tiny_forward_batch_independence(af):
+    cfg = tiny_config()
+    w = af.Weights(af_config(cfg))
+    upload(w, draw_weights(cfg, 11))
+    s = af.Scratch(w, 2, 64, 8)
+    lat = to_f32(synth.latents(11, (2, 4, 16, 16)))
+    text = to_bf16(synth.text_embeddings(11, (2, 8, 32)))
+    t = to_f32(np.array([0.3, 0.9], np.float32))
+    both = torch.empty(2, 4, 16, 16, device="cuda")
+    af.transformer_forward(w, s, lat, text, t, both)
+    for b in range(2):
+        one = torch.empty(1, 4, 16, 16, device="cuda")
+        af.transformer_forward(w, s, lat[b:b + 1].contiguous(), text[b:b + 1].contiguous(), t[b:b + 1].contiguous(),
+                               one)
+        s.sync()
+        assert torch.equal(both[b:b + 1], one)
+
+
+def test_forward_rejects_bad_shapes(af):
+    cfg = tiny_config()
+    w = af.Weights(af_config(cfg))
+    s = af.Scratch(w, 1, 64, 8)
+    vel = torch.empty(1, 4, 18, 18, device="cuda")
+    with pytest.raises(af.AFError):
+        af.transformer_forward(w, s, torch.zeros(1, 4, 18, 18, device="cuda"),
+                               torch.zeros(1, 8, 32, dtype=torch.bfloat16, device="cuda"),
+                               torch.zeros(1, device="cuda"), vel)
+    with pytest.raises(af.AFError):   # text longer than the scratch was sized for
+        af.transformer_forward(w, s, torch.zeros(1, 4, 16, 16, device="cuda"),
+                               torch.zeros(1, 9, 32, dtype=torch.bfloat16, device="cuda"),
+                               torch.zeros(1, device="cuda"), torch.empty(1, 4, 16, 16, device="cuda"))
+
+
+def test_real_width_forward_small_latent(af):
+    """Full model width and depth (4 joint + 32 single blocks, D = 3072) on a
+    16 x 16 latent (64 image tokens) with 24 text tokens, CFG batch 2.  The
+    oracle runs block by block so only one block's weights are held at a time."""
+    from helpers import block_names
+    cfg = O.Config(pos_embed_max_size=64 * 64)
+    B, H, W, L, seed = 2, 16, 16, 24, 4
+    w = af.Weights(af_config(cfg))
+    blocks = set()
+    for i in range(cfg.num_mmdit_layers):
+        blocks |= set(block_names(cfg, "joint", i))
+    for i in range(cfg.num_single_dit_layers):
+        blocks |= set(block_names(cfg, "single", i))
+    misc = draw_weights(cfg, seed, [n for n, _ in O.weight_specs(cfg) if n not in blocks])
+    upload(w, misc)
+    lat = synth.latents(seed, (B, 4, H, W))
+    text = synth.text_embeddings(seed, (B, L, cfg.joint_attention_dim))
+    tt = np.array([1.0, 1.0], dtype=np.float32)
+    img, txt, temb = O.embed(lat, text, tt, misc, cfg)
+    for i in range(cfg.num_mmdit_layers):
+        blk = draw_weights(cfg, seed, block_names(cfg, "joint", i))
+        upload(w, blk)
+        txt, img = O.joint_block(img, txt, temb, blk, f"joint_transformer_blocks.{i}.", cfg)
+    nt = txt.shape[1]
+    x = np.concatenate([txt, img], axis=1)
+    for i in range(cfg.num_single_dit_layers):
+        blk = draw_weights(cfg, seed, block_names(cfg, "single", i))
+        upload(w, blk)
+        x = O.single_block(x, temb, blk, f"single_transformer_blocks.{i}.", cfg)
+    ref = O.output_stage(x[:, nt:], temb, misc, cfg, H, W)
+    s = af.Scratch(w, B, (H // 2) * (W // 2), L)
+    vel = torch.empty(B, 4, H, W, dtype=torch.float32, device="cuda")
+    af.transformer_forward(w, s, to_f32(lat), to_bf16(text), to_f32(tt), vel)
+    s.sync()
+    assert O.rel_l2(to_np(vel), ref) < STACK_TOL
