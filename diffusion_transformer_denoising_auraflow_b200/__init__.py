@@ -67,6 +67,7 @@ _SIGS = {
     "af_scratch_destroy": [_P],
     "af_sync": [_P, _P],
     "af_timestep_embed": [_P, _P, _P, _I, _P, _P],
+    "af_timestep_embed_noalloc": [_P, _P, _I, _P, _P],
     "af_patch_embed": [_P, _P, _P, _I, _I, _I, _P, _P],
     "af_joint_block": [_P, _P, _I, _P, _P, _P, _I, _I, _I, _P],
     "af_single_block": [_P, _P, _I, _P, _P, _I, _I, _P],
@@ -229,6 +230,14 @@ class Scratch:
 def timestep_embed(w: Weights, s: Scratch, t, temb, stream=None):
     _check(lib.af_timestep_embed(w.handle, s.handle, _dev(t, torch.float32, "t"), t.numel(),
                                  _dev(temb, torch.float32, "temb"), _stream(stream)), "af_timestep_embed")
+
+
+def timestep_embed_noalloc(w: Weights, t, temb, stream=None):
+    """af_timestep_embed without a scratch handle: nothing is allocated (fixed device array)."""
+    st = lib.af_timestep_embed_noalloc(w.handle, _dev(t, torch.float32, "t"), t.numel(),
+                                       _dev(temb, torch.float32, "temb"), _stream(stream))
+    if st != AF_OK:
+        raise AFError(st, "af_timestep_embed_noalloc", lib.af_last_error().decode())
 
 
 def patch_embed(w: Weights, s: Scratch, latents, img, stream=None):

@@ -3,6 +3,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cstdint>
+#include <string>
 
 namespace af {
 
@@ -83,4 +84,15 @@ cudaError_t launch_fill(float* dst, int n, float value, cudaStream_t s);
 cudaError_t launch_euler_cfg(float* lat, const float* v, int Bi, int64_t per_sample, float g, float sigma,
                              float sigma_next, cudaStream_t s);
 
+}  // namespace af
+
+// Read-only accessors of the weight pack and the thread's last-error text,
+// for entry points defined outside api.cu.
+struct af_weights;
+namespace af {
+const uint16_t* weights_tensor(const af_weights* w, const char* name);
+int weights_device(const af_weights* w);
+int weights_inner_dim(const af_weights* w);
+int weights_timestep_channels(const af_weights* w);
+void set_last_error(const std::string& msg);
 }  // namespace af

@@ -394,6 +394,14 @@ af_status check_dev_ptr(const void* p) {
 
 }  // namespace
 
+namespace af {
+const uint16_t* weights_tensor(const af_weights* w, const char* name) { return w->ptr(name); }
+int weights_device(const af_weights* w) { return w->device; }
+int weights_inner_dim(const af_weights* w) { return w->d.D; }
+int weights_timestep_channels(const af_weights* w) { return w->cfg.timestep_channels; }
+void set_last_error(const std::string& msg) { g_last_error = msg; }
+}  // namespace af
+
 // =========================================================================== C ABI
 
 extern "C" {

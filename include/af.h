@@ -133,6 +133,23 @@ af_status af_sync(af_scratch* s, void* stream);
 af_status af_timestep_embed(const af_weights* w, af_scratch* s, const float* t, int B, float* temb,
                             void* stream);
 
+/* Same result as af_timestep_embed, for callers that cannot allocate device
+ * memory (their device memory is owned and budgeted by another allocator,
+ * they run a latency-critical loop where cudaMalloc/cudaFree may stall the
+ * device, or they may only allocate at initialisation): no af_scratch is
+ * needed and nothing is allocated.  The architecture description has no
+ * counterpart of this call.  Its intermediates live in one fixed 256 KB
+ * device array (65536 floats) that every GPU loading the library holds until
+ * exit; a call needs B * (timestep_channels + inner_dim) floats of it and
+ * larger requests return AF_ERR_SHAPE (text in af_last_error) before any
+ * launch.  All calls on a device share that array and it keeps the last
+ * call's contents (nothing in it needs to start at zero), so calls that
+ * overlap on the GPU race and must be serialised by the caller.  The first
+ * call on each device looks up the array's device address; make it before
+ * any stream capture.
+ *   t: device float[B]; temb: device float[B, D] (output). */
+af_status af_timestep_embed_noalloc(const af_weights* w, const float* t, int B, float* temb, void* stream);
+
 /* Patch embedding with centre-cropped learned positions ([ARCH] §Patch
  * Embedding): img[b, n] = W_pe patch(b, n) + PE[(r0 + n / wp) * G + c0 + n % wp]
  * with r0 = (G - H/p) / 2, c0 = (G - W/p) / 2 (floor); patch vector order
