@@ -80,7 +80,7 @@ _SIGS = {
     "af_profile_end": [_P, _P, _P, _P, _P],
     "af_ln_modulate": [_P, _P, _P, _I, _P, _I, _I, _I, _F, _P],
     "af_linear": [_P, _P, _P, _I, _I, _I, _P],
-    "af_attention": [_P, _P, _P, _P, _I, _I, _I, _I, _P],
+    "af_attention": [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P],
     "af_status_string": [_I],
     "af_last_error": [],
 }
@@ -311,7 +311,8 @@ def linear(A, W, C, stream=None):
                          M, N, K, _stream(stream)), "af_linear")
 
 
-def attention(q, k, v, o, stream=None):
+def attention(q, k, v, o, qk_normalized: bool = False, stream=None):
     B, H, N, hd = q.shape
     _check(lib.af_attention(_dev(q, torch.bfloat16, "q"), _dev(k, torch.bfloat16, "k"), _dev(v, torch.bfloat16, "v"),
-                            _dev(o, torch.bfloat16, "o"), B, H, N, hd, _stream(stream)), "af_attention")
+                            _dev(o, torch.bfloat16, "o"), B, H, N, hd, 1 if qk_normalized else 0, _stream(stream)),
+           "af_attention")

@@ -30,8 +30,7 @@ struct GemmParams {
   uint16_t* v;
   int heads, hd, n_total, qkv_row_off, D;
   float eps;
-  int swiglu_w2_row;       // SWIGLU: first row of W2 inside the packed weight
-  int num_m_tiles, num_n_tiles, num_tiles;
+  int num_m_tiles, num_n_tiles, num_tiles, group_n;
   int* err;                // device error word
 };
 
@@ -62,6 +61,8 @@ struct AttnParams {
   int split;
   int ldo;
   float scale_log2;  // softmax scale * log2(e)
+  int qk_normalized; // nonzero: every q, k row has L2 norm <= sqrt(hd) (per-head LayerNorm output)
+  const uint16_t* q; // [B, H, N, hd] (read directly by the QK-normalised kernel)
   int* err;
 };
 cudaError_t launch_attention(const AttnParams& p, const uint16_t* q, const uint16_t* k, const uint16_t* v,

@@ -66,6 +66,11 @@ struct TensorInfo {
   int ndim;
   int64_t shape[2];
   size_t offset;  // bytes into the pack
+  // FFN up-projection pairs (linear_1, linear_2) are stored interleaved in
+  // 128-row groups, [W1 g | W2 g] for g = 0, 1, ..., so one 256-row tile of
+  // the pair feeds both halves of the SwiGLU epilogue: 1 = W1, 2 = W2.
+  int interleave = 0;
+  size_t pair_base = 0;
   size_t numel() const { return ndim == 1 ? shape[0] : static_cast<size_t>(shape[0]) * shape[1]; }
 };
 
@@ -131,6 +136,14 @@ void add_tensor(af_weights* w, size_t& off, const std::string& name, int64_t r, 
   off += t.numel() * 2;
 }
 
+void mark_pair(af_weights* w, const std::string& w1, const std::string& w2) {
+  TensorInfo& a = w->tensors[w->index[w1]];
+  TensorInfo& b = w->tensors[w->index[w2]];
+  a.interleave = 1;
+  b.interleave = 2;
+  a.pair_base = b.pair_base = a.offset;
+}
+
 void build_layout(af_weights* w) {
   const af_config& c = w->cfg;
   const int D = w->d.D, F = w->d.F, p = c.patch_size;
@@ -174,6 +187,8 @@ void build_layout(af_weights* w) {
     add_tensor(w, off, b + "ff_context.linear_1.weight", F, D);
     add_tensor(w, off, b + "ff_context.linear_2.weight", F, D, false);
     add_tensor(w, off, b + "ff_context.out_projection.weight", D, F);
+    mark_pair(w, b + "ff.linear_1.weight", b + "ff.linear_2.weight");
+    mark_pair(w, b + "ff_context.linear_1.weight", b + "ff_context.linear_2.weight");
   }
   for (int i = 0; i < c.num_single_dit_layers; ++i) {
     const std::string b = "single_transformer_blocks." + std::to_string(i) + ".";
@@ -184,6 +199,7 @@ void build_layout(af_weights* w) {
     add_tensor(w, off, b + "ff.linear_1.weight", F, D);
     add_tensor(w, off, b + "ff.linear_2.weight", F, D, false);
     add_tensor(w, off, b + "ff.out_projection.weight", D, F);
+    mark_pair(w, b + "ff.linear_1.weight", b + "ff.linear_2.weight");
   }
   add_tensor(w, off, "pos_embed.proj.weight", D, p * p * c.in_channels);
   add_tensor(w, off, "pos_embed.pos_embed", c.pos_embed_max_size, D);
@@ -284,14 +300,13 @@ af_status gated_residual(af_scratch* s, const uint16_t* A, int B, int rows, int 
   return run_gemm(s, p, A, W, N, st);
 }
 
-// h = silu(y W1^T) * (y W2^T), W1 and W2 stacked in one [2F, D] matrix
+// h = silu(y W1^T) * (y W2^T), W1 and W2 interleaved in 128-row groups ([2F, D])
 af_status swiglu(const af_weights* w, af_scratch* s, const uint16_t* y, int M, const uint16_t* w12,
                  uint16_t* h, cudaStream_t st) {
   const Derived& d = w->d;
   GemmParams p = gemm_base(s, M, d.F, d.D, EPI_SWIGLU, M);
   p.out = h;
   p.ldo = d.F;
-  p.swiglu_w2_row = d.F;
   return run_gemm(s, p, y, w12, 2 * d.F, st);
 }
 
@@ -308,8 +323,10 @@ af_status attention(const af_weights* w, af_scratch* s, int B, int N, uint16_t* 
   p.split = split;
   p.ldo = d.D;
   p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(d.hd));
+  p.qk_normalized = 1;  // q and k come from the QK-norm epilogue of the QKV GEMM
   p.err = s->err;
   LaunchScope ls(s, KC_ATTN, 4.0 * B * d.H * static_cast<double>(N) * N * d.hd, st);
+  p.q = s->q;
   cudaError_t e = launch_attention(p, s->q, s->k, s->v, st);
   if (e != cudaSuccess) return cuda_fail(e);
   return AF_OK;
@@ -528,8 +545,19 @@ af_status af_weights_set(af_weights* w, int id, const uint16_t* src, int src_is_
   const TensorInfo& t = w->tensors[id];
   const size_t bytes = t.numel() * 2;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (src_is_device) AF_TRY(check_dev_ptr(src));
+  if (t.interleave) {
+    // 128-row groups of this half go to every other 128-row slot of the pair
+    const size_t group = static_cast<size_t>(128) * t.shape[1] * 2;
+    uint8_t* dst = w->base + t.pair_base + (t.interleave == 2 ? group : 0);
+    const size_t groups = static_cast<size_t>(t.shape[0]) / 128;
+    if (src_is_device)
+      AF_CUDA(cudaMemcpy2DAsync(dst, 2 * group, src, group, group, groups, cudaMemcpyDeviceToDevice, st));
+    else
+      AF_CUDA(cudaMemcpy2D(dst, 2 * group, src, group, group, groups, cudaMemcpyHostToDevice));
+    return AF_OK;
+  }
   if (src_is_device) {
-    AF_TRY(check_dev_ptr(src));
     AF_CUDA(cudaMemcpyAsync(w->base + t.offset, src, bytes, cudaMemcpyDeviceToDevice, st));
   } else {
     AF_CUDA(cudaMemcpy(w->base + t.offset, src, bytes, cudaMemcpyHostToDevice));
@@ -888,7 +916,7 @@ af_status af_linear(const uint16_t* A, const uint16_t* W, uint16_t* C, int M, in
 }
 
 af_status af_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* o, int B, int H, int N,
-                       int hd, void* stream) {
+                       int hd, int qk_normalized, void* stream) {
   if (!q || !k || !v || !o || B <= 0 || H <= 0 || N <= 0) return AF_ERR_INVALID_ARG;
   if (!(hd == 256 || hd == 8 || hd == 16 || hd == 32 || hd == 64)) return AF_ERR_UNSUPPORTED;
   AttnParams p;
@@ -901,6 +929,8 @@ af_status af_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, 
   p.split = 0;
   p.ldo = H * hd;
   p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(hd));
+  p.qk_normalized = qk_normalized ? 1 : 0;
+  p.q = q;
   p.err = nullptr;
   AF_CUDA(launch_attention(p, q, k, v, static_cast<cudaStream_t>(stream)));
   return AF_OK;

@@ -6,21 +6,27 @@
 // §注意力处理器与 QKV 融合: text and image tokens are concatenated and
 // attended jointly with SDPA, dropout 0, is_causal False.)
 //
-// attn_hd256_tcgen05: one CTA = 128 query rows of one (sample, head).
+// attn_hd256_online (any q, k) and attn_hd256_qknorm (per-head LayerNorm-ed
+// q, k; see below): one CTA = 128 query rows of one (sample, head).
 //   smem: Q 128x256 (64 KB, loaded once), K and V tiles of 64 keys x 256
 //   double-buffered (2 x 32 KB each), P 128x64 bf16 (16 KB); all 128-byte
 //   swizzled.  TMEM (512 columns): O 128x256 fp32 in columns [0,256), two
 //   S buffers 128x64 fp32 in [256,384).
-//   warp 0      TMA producer (Q once, then K_j, V_j).
+//   warp 0      TMA producer of Q (once) and the K tiles; warp 10 of the V
+//               tiles (independent rings, so a K load never waits for a V
+//               buffer release).
 //   warp 1      one thread issues S_{j+1} = Q K_{j+1}^T (M=128, N=64, K=256)
 //               before O += P_j V_j (M=128, N=256, K=64, V read MN-major),
 //               so the tensor core works on the next scores while the
 //               softmax warps handle the current ones.
-//   warps 2..5  softmax: thread = query row; loads its S row from TMEM,
-//               masks keys >= N, fp32 online softmax in the exp2 domain with
-//               a lazy running max (O is rescaled only when the max grows by
-//               more than 2^8), writes P (bf16) into shared memory, and at the
-//               end normalises O and stores it.
+//   warps 2..9  softmax, two warpgroups: warpgroup g owns key columns
+//               [32g, 32g+32) of every S tile and O columns [128g, 128g+128);
+//               thread = query row.  Partial row maxima (and at the end the
+//               partial row sums) are exchanged through shared memory.  fp32
+//               online softmax in the exp2 domain with a lazy running max
+//               (O is rescaled only when the max grows by more than 2^8), P
+//               written as bf16 into swizzled shared memory, O normalised at
+//               the end.
 // attn_small_simt: one thread per query row, for head_dim <= 64 (used by
 //   small test models only).
 #include "af_internal.h"
@@ -34,12 +40,21 @@ constexpr int AT_HD = 256;
 constexpr uint32_t AT_Q_BYTES = AT_BM * AT_HD * 2;   // 64 KB
 constexpr uint32_t AT_KV_BYTES = AT_BN * AT_HD * 2;  // 32 KB
 constexpr uint32_t AT_P_BYTES = AT_BM * AT_BN * 2;   // 16 KB
-constexpr int AT_THREADS = 192;
-constexpr int AT_SMEM = AT_Q_BYTES + 4 * AT_KV_BYTES + AT_P_BYTES + 512 + 1024;
+constexpr int AT_SOFTMAX_WARPS = 8;
+constexpr int AT_V_WARP = 2 + AT_SOFTMAX_WARPS;            // V producer (after the softmax warps)
+constexpr int AT_THREADS = 32 * (AT_V_WARP + 1);
+constexpr uint32_t AT_XCH_BYTES = 3 * 2 * AT_BM * 4;  // row-max slots [2][2][128] + row-sum [2][128]
+constexpr int AT_SMEM = AT_Q_BYTES + 4 * AT_KV_BYTES + AT_P_BYTES + AT_XCH_BYTES + 512 + 1024;
 constexpr float LAZY_RESCALE_LOG2 = 8.0f;
 
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __global__ void __launch_bounds__(AT_THREADS, 1)
-    attn_hd256_tcgen05(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+    attn_hd256_online(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -47,7 +62,9 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
   uint8_t* sK = sQ + AT_Q_BYTES;            // 2 buffers
   uint8_t* sV = sK + 2 * AT_KV_BYTES;       // 2 buffers
   uint8_t* sP = sV + 2 * AT_KV_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + AT_P_BYTES);
+  float* xmax = reinterpret_cast<float*>(sP + AT_P_BYTES);  // [slot 2][wg 2][row 128]
+  float* xsum = xmax + 4 * AT_BM;                           // [wg 2][row 128]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + AT_P_BYTES + AT_XCH_BYTES);
   uint64_t* q_full = bars + 0;
   uint64_t* k_full = bars + 1;    // [2]
   uint64_t* v_full = bars + 3;    // [2]
@@ -58,7 +75,9 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
   uint64_t* p_full = bars + 13;
   uint64_t* o_done = bars + 14;
   uint64_t* mma_done = bars + 15;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  uint64_t* xbar = bars + 16;     // [2] row-max exchange
+  uint64_t* lbar = bars + 18;     // row-sum exchange
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 19);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -76,11 +95,13 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       mbar_init(smem_u32(&k_empty[i]), 1);
       mbar_init(smem_u32(&v_empty[i]), 1);
       mbar_init(smem_u32(&s_full[i]), 1);
-      mbar_init(smem_u32(&s_empty[i]), 128);
+      mbar_init(smem_u32(&s_empty[i]), AT_SOFTMAX_WARPS);
+      mbar_init(smem_u32(&xbar[i]), AT_SOFTMAX_WARPS);
     }
-    mbar_init(smem_u32(p_full), 128);
+    mbar_init(smem_u32(p_full), AT_SOFTMAX_WARPS);
     mbar_init(smem_u32(o_done), 1);
     mbar_init(smem_u32(mma_done), 1);
+    mbar_init(smem_u32(lbar), AT_SOFTMAX_WARPS);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -101,35 +122,36 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
   const uint32_t tS = tmem + 256;
   volatile int never = 0;
 
-  if (warp == 0) {
+  if (warp == 0 || warp == AT_V_WARP) {
+    // warp 0 streams Q then the K tiles, the last warp streams the V tiles, so
+    // neither ring waits behind the other's buffer release
     if (lane == 0) {
-      uint32_t armedK = 0, armedV = 0, parK = 0, parV = 0;
+      const bool is_k = warp == 0;
+      uint64_t* full = is_k ? k_full : v_full;
+      uint64_t* empty = is_k ? k_empty : v_empty;
+      const void* tm = is_k ? static_cast<const void*>(&tmK) : static_cast<const void*>(&tmV);
+      uint8_t* buf = is_k ? sK : sV;
+      uint32_t armed = 0, par = 0;
       bool ok = true;
-      mbar_arrive_expect_tx(smem_u32(q_full), AT_Q_BYTES);
-      for (int c = 0; c < 4; ++c)
-        tma_load_3d(smem_u32(sQ + c * (AT_BM * 128)), &tmQ, smem_u32(q_full), c * 64, q0, bh);
-      for (int j = 0; j < nkv && ok; ++j) {
+      if (is_k) {
+        mbar_arrive_expect_tx(smem_u32(q_full), AT_Q_BYTES);
+        for (int c = 0; c < 4; ++c)
+          tma_load_3d(smem_u32(sQ + c * (AT_BM * 128)), &tmQ, smem_u32(q_full), c * 64, q0, bh);
+      }
+      for (int j = 0; j < nkv; ++j) {
         const int s = j & 1;
         const uint32_t ph = (j >> 1) & 1;
-        if (!mbar_wait(smem_u32(&k_empty[s]), ph ^ 1u, p.err, abort_flag)) { ok = false; break; }
-        mbar_arrive_expect_tx(smem_u32(&k_full[s]), AT_KV_BYTES);
-        armedK |= 1u << s; parK = (parK & ~(1u << s)) | (ph << s);
+        if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1u, p.err, abort_flag)) { ok = false; break; }
+        mbar_arrive_expect_tx(smem_u32(&full[s]), AT_KV_BYTES);
+        armed |= 1u << s; par = (par & ~(1u << s)) | (ph << s);
         for (int c = 0; c < 4; ++c)
-          tma_load_3d(smem_u32(sK + s * AT_KV_BYTES + c * (AT_BN * 128)), &tmK, smem_u32(&k_full[s]), c * 64,
-                      j * AT_BN, bh);
-        if (!mbar_wait(smem_u32(&v_empty[s]), ph ^ 1u, p.err, abort_flag)) { ok = false; break; }
-        mbar_arrive_expect_tx(smem_u32(&v_full[s]), AT_KV_BYTES);
-        armedV |= 1u << s; parV = (parV & ~(1u << s)) | (ph << s);
-        for (int c = 0; c < 4; ++c)
-          tma_load_3d(smem_u32(sV + s * AT_KV_BYTES + c * (AT_BN * 128)), &tmV, smem_u32(&v_full[s]), c * 64,
+          tma_load_3d(smem_u32(buf + s * AT_KV_BYTES + c * (AT_BN * 128)), tm, smem_u32(&full[s]), c * 64,
                       j * AT_BN, bh);
       }
       if (!ok) {
-        mbar_wait(smem_u32(q_full), 0, nullptr, &never, 100000000ull);
-        for (int s = 0; s < 2; ++s) {
-          if (armedK & (1u << s)) mbar_wait(smem_u32(&k_full[s]), (parK >> s) & 1u, nullptr, &never, 100000000ull);
-          if (armedV & (1u << s)) mbar_wait(smem_u32(&v_full[s]), (parV >> s) & 1u, nullptr, &never, 100000000ull);
-        }
+        if (is_k) mbar_wait(smem_u32(q_full), 0, nullptr, &never, 100000000ull);
+        for (int s = 0; s < 2; ++s)
+          if (armed & (1u << s)) mbar_wait(smem_u32(&full[s]), (par >> s) & 1u, nullptr, &never, 100000000ull);
       }
     }
   } else if (warp == 1) {
@@ -178,10 +200,12 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       mbar_wait(smem_u32(mma_done), 0, nullptr, &never, 100000000ull);
     }
   } else {
-    // ---------------------------------------------------------------- softmax warps
+    // ---------------------------------------------------------------- softmax warpgroups
+    const int wg = (warp - 2) >> 2;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const float c = p.scale_log2;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     uint8_t* prow = sP + row * 128;
@@ -191,27 +215,28 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       __syncwarp();
       if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
       tc_fence_after();
-      uint32_t r0[32], r1[32];
-      tmem_ld32(tS + s * AT_BN + lane_off, r0);
-      tmem_ld32(tS + s * AT_BN + 32 + lane_off, r1);
+      uint32_t r[32];
+      tmem_ld32(tS + s * AT_BN + 32 * wg + lane_off, r);
       tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(smem_u32(&s_empty[s]));
-      float x[64];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&s_empty[s]));
+      float x[32];
+      const int kvalid = p.N - j * AT_BN - 32 * wg;   // valid key columns in this half
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        x[i] = __uint_as_float(r0[i]) * p.scale_log2;
-        x[32 + i] = __uint_as_float(r1[i]) * p.scale_log2;
-      }
-      const int kvalid = p.N - j * AT_BN;
-      if (kvalid < AT_BN) {
+      for (int i = 0; i < 32; ++i) x[i] = (i < kvalid) ? __uint_as_float(r[i]) : -INFINITY;
+      float mr = x[0];
 #pragma unroll
-        for (int i = 0; i < 64; ++i)
-          if (i >= kvalid) x[i] = -INFINITY;
-      }
-      float mt = x[0];
-#pragma unroll
-      for (int i = 1; i < 64; ++i) mt = fmaxf(mt, x[i]);
+      for (int i = 1; i < 32; ++i) mr = fmaxf(mr, x[i]);
+      // exchange the partial row max with the other warpgroup
+      float* slot = xmax + (j & 1) * 2 * AT_BM;
+      slot[wg * AT_BM + row] = mr * c;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&xbar[j & 1]));
+      const bool gx = mbar_wait(smem_u32(&xbar[j & 1]), (j >> 1) & 1, p.err, abort_flag);
+      __syncwarp();
+      if (!__all_sync(0xffffffffu, gx)) { ok = false; break; }
+      const float mt = fmaxf(mr * c, slot[(wg ^ 1) * AT_BM + row]);
       float m_new = m;
       bool rescale = false;
       if (j == 0) {
@@ -221,11 +246,11 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
         rescale = true;
       }
       float rs = 0.f;
-      uint32_t pk[32];
+      uint32_t pk[16];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const float e0 = exp2f(x[2 * i] - m_new);
-        const float e1 = exp2f(x[2 * i + 1] - m_new);
+      for (int i = 0; i < 16; ++i) {
+        const float e0 = ex2_approx(fmaf(x[2 * i], c, -m_new));
+        const float e1 = ex2_approx(fmaf(x[2 * i + 1], c, -m_new));
         rs += e0 + e1;
         pk[i] = pack_bf16(e0, e1);
       }
@@ -237,14 +262,15 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
         tc_fence_after();
       }
       if (__any_sync(0xffffffffu, rescale)) {
-        const float alpha = rescale ? exp2f(m - m_new) : 1.0f;
-        for (int c = 0; c < AT_HD / 32; ++c) {
+        const float alpha = rescale ? ex2_approx(m - m_new) : 1.0f;
+        for (int cc = 0; cc < 4; ++cc) {
+          const uint32_t ta = tO + 128 * wg + cc * 32 + lane_off;
           uint32_t o[32];
-          tmem_ld32(tO + c * 32 + lane_off, o);
+          tmem_ld32(ta, o);
           tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(tO + c * 32 + lane_off, o);
+          tmem_st32(ta, o);
         }
         tmem_wait_st();
         l *= alpha;
@@ -252,19 +278,27 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       m = m_new;
       l += rs;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint4 v = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-        *reinterpret_cast<uint4*>(prow + ((c ^ (row & 7)) << 4)) = v;
+      for (int q = 0; q < 4; ++q) {
+        const int chunk = 4 * wg + q;
+        uint4 v = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+        *reinterpret_cast<uint4*>(prow + ((chunk ^ (row & 7)) << 4)) = v;
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(smem_u32(p_full));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(p_full));
     }
     if (ok) {
-      const bool g3 = mbar_wait(smem_u32(o_done), (nkv - 1) & 1, p.err, abort_flag);
+      // total row sum from both warpgroups
+      xsum[wg * AT_BM + row] = l;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(lbar));
+      const bool g3 = mbar_wait(smem_u32(lbar), 0, p.err, abort_flag) &&
+                      mbar_wait(smem_u32(o_done), (nkv - 1) & 1, p.err, abort_flag);
       __syncwarp();
       if (__all_sync(0xffffffffu, g3)) {
         tc_fence_after();
+        const float inv = 1.0f / (l + xsum[(wg ^ 1) * AT_BM + row]);
         const int qrow = q0 + row;
         const bool row_ok = qrow < p.N;
         uint16_t* dst = nullptr;
@@ -273,14 +307,312 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
             dst = p.out_a + (static_cast<size_t>(b) * p.split + qrow) * p.ldo + h * AT_HD;
           else
             dst = p.out_b + (static_cast<size_t>(b) * (p.N - p.split) + (qrow - p.split)) * p.ldo + h * AT_HD;
+          dst += 128 * wg;
         }
-        const float inv = 1.0f / l;
-        for (int c = 0; c < AT_HD / 32; ++c) {
+        for (int cc = 0; cc < 4; ++cc) {
           uint32_t o[32];
-          tmem_ld32(tO + c * 32 + lane_off, o);
+          tmem_ld32(tO + 128 * wg + cc * 32 + lane_off, o);
           tmem_wait_ld();
           if (row_ok) {
-            uint4* d = reinterpret_cast<uint4*>(dst + c * 32);
+            uint4* d = reinterpret_cast<uint4*>(dst + cc * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              uint4 u;
+              u.x = pack_bf16(__uint_as_float(o[8 * i + 0]) * inv, __uint_as_float(o[8 * i + 1]) * inv);
+              u.y = pack_bf16(__uint_as_float(o[8 * i + 2]) * inv, __uint_as_float(o[8 * i + 3]) * inv);
+              u.z = pack_bf16(__uint_as_float(o[8 * i + 4]) * inv, __uint_as_float(o[8 * i + 5]) * inv);
+              u.w = pack_bf16(__uint_as_float(o[8 * i + 6]) * inv, __uint_as_float(o[8 * i + 7]) * inv);
+              d[i] = u;
+            }
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------- QK-normalised inputs
+// When every q and k row is a per-head LayerNorm output (||q||, ||k|| <=
+// sqrt(hd), up to bf16 rounding), every logit satisfies
+// |q.k| / sqrt(hd) <= sqrt(hd) * (1 + 2^-9)^2, i.e. <= 23.2 in log2 units
+// for hd = 256.  Softmax is invariant to a common shift, so the fixed shift
+// QKN_OFFSET_LOG2 = 24 replaces the running maximum exactly: probabilities
+// lie in [2^-48, 1) (normal fp32/bf16 numbers) and no rescaling of O is ever
+// needed.  The two softmax warpgroups then work on alternate KV tiles (group
+// g takes tiles j = g mod 2, full 64-key rows) with one P buffer each, and
+// their partial row sums are added at the end.
+//
+// Q is kept in TMEM (columns [384, 512), two bf16 per column) and S = Q K^T
+// is issued with A read from TMEM, so the 16 K-steps of a tile only stream
+// the K tile from shared memory (re-reading a 128 x 16 Q slice from shared
+// memory for every step made the N = 64 product bandwidth-bound).  TMEM:
+// O [0, 256), S0 [256, 320), S1 [320, 384), Q [384, 512).  The freed shared
+// memory holds a third K and V stage.
+//
+// The CTAs of one (sample, head) all stream the same K and V; each starts its
+// KV loop at a different tile (kv_tile(j) below) so that concurrently running
+// CTAs request different lines instead of hammering the same L2 slices.
+constexpr float QKN_OFFSET_LOG2 = 24.0f;
+constexpr int QKN_THREADS = AT_THREADS;
+constexpr int QKN_STAGES = 3;
+constexpr uint32_t QKN_XCH_BYTES = 2 * AT_BM * 4;
+constexpr int QKN_SMEM = 2 * QKN_STAGES * AT_KV_BYTES + 2 * AT_P_BYTES + QKN_XCH_BYTES + 256 + 1024;
+
+__global__ void __launch_bounds__(QKN_THREADS, 1)
+    attn_hd256_qknorm(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                      const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sK = smem;                               // QKN_STAGES buffers
+  uint8_t* sV = sK + QKN_STAGES * AT_KV_BYTES;      // QKN_STAGES buffers
+  uint8_t* sP = sV + QKN_STAGES * AT_KV_BYTES;      // 2 buffers
+  float* xsum = reinterpret_cast<float*>(sP + 2 * AT_P_BYTES);  // [wg 2][row 128]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + 2 * AT_P_BYTES + QKN_XCH_BYTES);
+  uint64_t* q_full = bars + 0;
+  uint64_t* k_full = bars + 1;    // [QKN_STAGES]
+  uint64_t* v_full = bars + 4;    // [QKN_STAGES]
+  uint64_t* k_empty = bars + 7;   // [QKN_STAGES]
+  uint64_t* v_empty = bars + 10;  // [QKN_STAGES]
+  uint64_t* s_full = bars + 13;   // [2]
+  uint64_t* s_empty = bars + 15;  // [2]
+  uint64_t* p_full = bars + 17;   // [2]
+  uint64_t* pv_done = bars + 19;  // [2]
+  uint64_t* mma_done = bars + 21;
+  uint64_t* lbar = bars + 22;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 23);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int bh = b * p.H + h;
+  const int q0 = qt * AT_BM;
+  const int nkv = (p.N + AT_BN - 1) / AT_BN;
+  const int kv0 = static_cast<int>((static_cast<long long>(qt) * nkv) / gridDim.x);
+  auto kv_tile = [&](int j) { const int t = j + kv0; return t < nkv ? t : t - nkv; };
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(q_full), 4);
+    for (int i = 0; i < QKN_STAGES; ++i) {
+      mbar_init(smem_u32(&k_full[i]), 1);
+      mbar_init(smem_u32(&v_full[i]), 1);
+      mbar_init(smem_u32(&k_empty[i]), 1);
+      mbar_init(smem_u32(&v_empty[i]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&s_full[i]), 1);
+      mbar_init(smem_u32(&s_empty[i]), 4);
+      mbar_init(smem_u32(&p_full[i]), 4);
+      mbar_init(smem_u32(&pv_done[i]), 1);
+    }
+    mbar_init(smem_u32(mma_done), 1);
+    mbar_init(smem_u32(lbar), AT_SOFTMAX_WARPS);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tO = tmem;
+  const uint32_t tS = tmem + 256;
+  const uint32_t tQ = tmem + 384;
+  volatile int never = 0;
+
+  if (warp == 0 || warp == AT_V_WARP) {
+    if (lane == 0) {
+      const bool is_k = warp == 0;
+      uint64_t* full = is_k ? k_full : v_full;
+      uint64_t* empty = is_k ? k_empty : v_empty;
+      const void* tm = is_k ? static_cast<const void*>(&tmK) : static_cast<const void*>(&tmV);
+      uint8_t* buf = is_k ? sK : sV;
+      uint32_t armed = 0, par = 0;
+      bool ok = true;
+      for (int j = 0; j < nkv; ++j) {
+        const int s = j % QKN_STAGES;
+        const uint32_t ph = (j / QKN_STAGES) & 1;
+        if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1u, p.err, abort_flag)) { ok = false; break; }
+        mbar_arrive_expect_tx(smem_u32(&full[s]), AT_KV_BYTES);
+        armed |= 1u << s; par = (par & ~(1u << s)) | (ph << s);
+        for (int c = 0; c < 4; ++c)
+          tma_load_3d(smem_u32(buf + s * AT_KV_BYTES + c * (AT_BN * 128)), tm, smem_u32(&full[s]), c * 64,
+                      kv_tile(j) * AT_BN, bh);
+      }
+      if (!ok) {
+        for (int s = 0; s < QKN_STAGES; ++s)
+          if (armed & (1u << s)) mbar_wait(smem_u32(&full[s]), (par >> s) & 1u, nullptr, &never, 100000000ull);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc_qk = make_idesc_bf16(AT_BM, AT_BN, false, false);
+      const uint32_t idesc_pv = make_idesc_bf16(AT_BM, AT_HD, false, true);
+      bool ok = mbar_wait(smem_u32(q_full), 0, p.err, abort_flag);
+      tc_fence_after();
+      auto issue_s = [&](int j) -> bool {
+        const int kb = j % QKN_STAGES;
+        const int s = j & 1;
+        if (!mbar_wait(smem_u32(&k_full[kb]), (j / QKN_STAGES) & 1, p.err, abort_flag)) return false;
+        if (!mbar_wait(smem_u32(&s_empty[s]), ((j >> 1) & 1) ^ 1u, p.err, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t kaddr = smem_u32(sK + kb * AT_KV_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < AT_HD / 16; ++kk) {
+          const uint32_t c = kk >> 2, off = (kk & 3) * 32;
+          const uint64_t bd = make_sdesc(kaddr + c * (AT_BN * 128) + off, 16, 1024, SWZ_128B);
+          mma_bf16_ts(tS + s * AT_BN, tQ + kk * 8, bd, idesc_qk, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(smem_u32(&s_full[s]));
+        mma_commit(smem_u32(&k_empty[kb]));
+        return true;
+      };
+      if (ok) ok = issue_s(0);
+      for (int j = 0; j < nkv && ok; ++j) {
+        if (j + 1 < nkv && !issue_s(j + 1)) { ok = false; break; }
+        const int s = j & 1;
+        const int vb = j % QKN_STAGES;
+        if (!mbar_wait(smem_u32(&p_full[s]), (j >> 1) & 1, p.err, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(smem_u32(&v_full[vb]), (j / QKN_STAGES) & 1, p.err, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t paddr = smem_u32(sP + s * AT_P_BYTES);
+        const uint32_t vaddr = smem_u32(sV + vb * AT_KV_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < AT_BN / 16; ++kk) {
+          const uint64_t ad = make_sdesc(paddr + kk * 32, 16, 1024, SWZ_128B);
+          const uint64_t bd = make_sdesc(vaddr + kk * (16 * 128), AT_BN * 128, 1024, SWZ_128B);
+          mma_bf16_ss(tO, ad, bd, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(smem_u32(&pv_done[s]));
+        mma_commit(smem_u32(&v_empty[vb]));
+      }
+      mma_commit(smem_u32(mma_done));
+      mbar_wait(smem_u32(mma_done), 0, nullptr, &never, 100000000ull);
+    }
+  } else {
+    // ---------------------------------------------------------------- softmax: group g takes tiles j = g (mod 2)
+    const int wg = (warp - 2) >> 2;
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const float c = p.scale_log2;
+    const float off = -QKN_OFFSET_LOG2;
+    float l = 0.f;
+    bool ok = true;
+    uint8_t* prow = sP + wg * AT_P_BYTES + row * 128;
+    if (wg == 0) {
+      // this row of Q into TMEM (zeros beyond N), then release the MMA warp
+      const int qrow = q0 + row;
+      const uint4* src = reinterpret_cast<const uint4*>(p.q + (static_cast<size_t>(bh) * p.N + qrow) * AT_HD);
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t qv[32];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const uint4 u = qrow < p.N ? src[cc * 8 + i] : make_uint4(0, 0, 0, 0);
+          qv[4 * i] = u.x;
+          qv[4 * i + 1] = u.y;
+          qv[4 * i + 2] = u.z;
+          qv[4 * i + 3] = u.w;
+        }
+        tmem_st32(tQ + cc * 32 + lane_off, qv);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(q_full));
+    }
+    for (int j = wg; j < nkv; j += 2) {
+      const uint32_t ph = (j >> 1) & 1;
+      const bool got = mbar_wait(smem_u32(&s_full[wg]), ph, p.err, abort_flag);
+      __syncwarp();
+      if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t r0[32], r1[32];
+      tmem_ld32(tS + wg * AT_BN + lane_off, r0);
+      tmem_ld32(tS + wg * AT_BN + 32 + lane_off, r1);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&s_empty[wg]));
+      const int kvalid = p.N - kv_tile(j) * AT_BN;
+      uint32_t pk[32];
+      float rs = 0.f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        float e0 = ex2_approx(fmaf(__uint_as_float(r0[2 * i]), c, off));
+        float e1 = ex2_approx(fmaf(__uint_as_float(r0[2 * i + 1]), c, off));
+        float e2 = ex2_approx(fmaf(__uint_as_float(r1[2 * i]), c, off));
+        float e3 = ex2_approx(fmaf(__uint_as_float(r1[2 * i + 1]), c, off));
+        if (kvalid < AT_BN) {
+          if (2 * i >= kvalid) e0 = 0.f;
+          if (2 * i + 1 >= kvalid) e1 = 0.f;
+          if (32 + 2 * i >= kvalid) e2 = 0.f;
+          if (32 + 2 * i + 1 >= kvalid) e3 = 0.f;
+        }
+        rs += (e0 + e1) + (e2 + e3);
+        pk[i] = pack_bf16(e0, e1);
+        pk[16 + i] = pack_bf16(e2, e3);
+      }
+      l += rs;
+      // P buffer wg is free once PV_{j-2} has completed
+      if (j >= 2) {
+        const bool g2 = mbar_wait(smem_u32(&pv_done[wg]), ph ^ 1u, p.err, abort_flag);
+        __syncwarp();
+        if (!__all_sync(0xffffffffu, g2)) { ok = false; break; }
+      }
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        uint4 v = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+        *reinterpret_cast<uint4*>(prow + ((q ^ (row & 7)) << 4)) = v;
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&p_full[wg]));
+    }
+    if (ok) {
+      xsum[wg * AT_BM + row] = l;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(lbar));
+      const int jl = nkv - 1;
+      const bool g3 = mbar_wait(smem_u32(lbar), 0, p.err, abort_flag) &&
+                      mbar_wait(smem_u32(&pv_done[jl & 1]), (jl >> 1) & 1, p.err, abort_flag);
+      __syncwarp();
+      if (__all_sync(0xffffffffu, g3)) {
+        tc_fence_after();
+        const float inv = 1.0f / (l + xsum[(wg ^ 1) * AT_BM + row]);
+        const int qrow = q0 + row;
+        const bool row_ok = qrow < p.N;
+        uint16_t* dst = nullptr;
+        if (row_ok) {
+          if (qrow < p.split)
+            dst = p.out_a + (static_cast<size_t>(b) * p.split + qrow) * p.ldo + h * AT_HD;
+          else
+            dst = p.out_b + (static_cast<size_t>(b) * (p.N - p.split) + (qrow - p.split)) * p.ldo + h * AT_HD;
+          dst += 128 * wg;
+        }
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t o[32];
+          tmem_ld32(tO + 128 * wg + cc * 32 + lane_off, o);
+          tmem_wait_ld();
+          if (row_ok) {
+            uint4* d = reinterpret_cast<uint4*>(dst + cc * 32);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               uint4 u;
@@ -347,12 +679,17 @@ cudaError_t launch_attention(const AttnParams& p, const uint16_t* q, const uint1
     if (!encode_tmap_3d(&tv, v, AT_HD, p.N, bh, rb, sb, 64, AT_BN, 1)) return cudaErrorInvalidValue;
     static bool attr = false;
     if (!attr) {
-      cudaError_t e = cudaFuncSetAttribute(attn_hd256_tcgen05, cudaFuncAttributeMaxDynamicSharedMemorySize, AT_SMEM);
+      cudaError_t e = cudaFuncSetAttribute(attn_hd256_online, cudaFuncAttributeMaxDynamicSharedMemorySize, AT_SMEM);
+      if (e != cudaSuccess) return e;
+      e = cudaFuncSetAttribute(attn_hd256_qknorm, cudaFuncAttributeMaxDynamicSharedMemorySize, QKN_SMEM);
       if (e != cudaSuccess) return e;
       attr = true;
     }
     dim3 grid((p.N + AT_BM - 1) / AT_BM, p.H, p.B);
-    attn_hd256_tcgen05<<<grid, AT_THREADS, AT_SMEM, stream>>>(tq, tk, tv, p);
+    if (p.qk_normalized)
+      attn_hd256_qknorm<<<grid, QKN_THREADS, QKN_SMEM, stream>>>(tq, tk, tv, p);
+    else
+      attn_hd256_online<<<grid, AT_THREADS, AT_SMEM, stream>>>(tq, tk, tv, p);
     return cudaGetLastError();
   }
   dim3 grid((p.N + 127) / 128, p.H, p.B);

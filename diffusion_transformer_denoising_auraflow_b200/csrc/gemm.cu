@@ -8,8 +8,10 @@
 // SiLU-gated FFN (§FeedForward), gated by adaLN-Zero (§联合注意力块).
 //
 // Structure (one CTA per SM, persistent over 128 x 256 output tiles):
-//   warp 0      TMA producer: A tile 128x64 and W tile 256x64 per k-block,
-//               128-byte swizzled, into a 4-stage shared-memory ring.
+//   warp 0      TMA producer: A tile 128x64 and W tile 256x64 per k-block
+//               (one box each: the TMA engine's cost is per box, so the W
+//               tile is never split), 128-byte swizzled, into a 4-stage
+//               shared-memory ring.
 //   warp 1      allocates 512 TMEM columns; one thread issues
 //               tcgen05.mma (M=128, N=256, K=16) into one of two 256-column
 //               fp32 accumulators, committing each stage back to the producer.
@@ -82,14 +84,15 @@ int device_sm_count() {
 
 constexpr uint32_t A_STAGE_BYTES = GEMM_BM * GEMM_BK * 2;  // 16 KB
 constexpr uint32_t B_STAGE_BYTES = GEMM_BN * GEMM_BK * 2;  // 32 KB
-constexpr int GROUP_N = 8;                                  // n-tiles per raster group
-
-__device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int& mb, int& nb) {
-  const int per_group = GROUP_N * num_m;
+// Tile order: n-tiles are taken in groups of `group_n`; inside a group the
+// tiles run m-major, so the CTAs in flight share a few A panels and the
+// group's weight panels stay resident in L2.
+__device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int group_n, int& mb, int& nb) {
+  const int per_group = group_n * num_m;
   const int g = t / per_group;
   const int r = t - g * per_group;
-  const int n_first = g * GROUP_N;
-  const int gw = min(GROUP_N, num_n - n_first);
+  const int n_first = g * group_n;
+  const int gw = min(group_n, num_n - n_first);
   mb = r / gw;
   nb = n_first + (r - mb * gw);
 }
@@ -204,6 +207,75 @@ __device__ __forceinline__ void epilogue_qkv(const GemmParams& p, uint32_t tbase
   }
 }
 
+// Epilogue of one accumulator tile for one output row (thread = TMEM lane):
+// tbase addresses this warp's 32-lane quarter of the accumulator, m0 is the
+// first GEMM row of the tile half held in this CTA's TMEM, nb the n-tile.
+__device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tbase, int m0, int nb, int row_in_tile) {
+  const int r = m0 + row_in_tile;
+  const bool row_ok = r < p.M;
+  const int b = r / p.rows_per_batch;
+  const int n_in = r - b * p.rows_per_batch;
+  const size_t orow = static_cast<size_t>(b) * p.out_rows_per_batch + p.out_row_off + n_in;
+
+  if (p.mode == EPI_QKV) {
+    epilogue_qkv(p, tbase, nb * GEMM_BN, row_ok, b, n_in);
+  } else if (p.mode == EPI_SWIGLU) {
+    const int col0 = nb * 128;
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+      uint32_t ra[32], rb[32];
+      tmem_ld32(tbase + c * 32, ra);
+      tmem_ld32(tbase + 128 + c * 32, rb);
+      tmem_wait_ld();
+      float v[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = silu_f(__uint_as_float(ra[j])) * __uint_as_float(rb[j]);
+      const int col = col0 + c * 32;
+      if (row_ok && col < p.N) store_bf16_n(p.out + orow * p.ldo + col, v, p.N - col);
+    }
+  } else {
+    const int col0 = nb * GEMM_BN;
+#pragma unroll 1
+    for (int c = 0; c < GEMM_BN / 32; ++c) {
+      const int col = col0 + c * 32;
+      if (col >= p.N) break;  // uniform across the warp
+      uint32_t ra[32];
+      tmem_ld32(tbase + c * 32, ra);
+      tmem_wait_ld();
+      float v[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(ra[j]);
+      if (!row_ok) continue;
+      uint16_t* dst = p.out + orow * p.ldo + col;
+      const int n = min(32, p.N - col);
+      if (p.mode == EPI_GATE_RES) {
+        const float* g = p.gate + static_cast<size_t>(b) * p.gate_stride + col;
+        if (n == 32) {
+          const uint4* xs = reinterpret_cast<const uint4*>(dst);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const uint4 xv = xs[i];
+            const float4 g0 = *reinterpret_cast<const float4*>(g + 8 * i);
+            const float4 g1 = *reinterpret_cast<const float4*>(g + 8 * i + 4);
+            v[8 * i + 0] = bf16_lo(xv.x) + g0.x * v[8 * i + 0];
+            v[8 * i + 1] = bf16_hi(xv.x) + g0.y * v[8 * i + 1];
+            v[8 * i + 2] = bf16_lo(xv.y) + g0.z * v[8 * i + 2];
+            v[8 * i + 3] = bf16_hi(xv.y) + g0.w * v[8 * i + 3];
+            v[8 * i + 4] = bf16_lo(xv.z) + g1.x * v[8 * i + 4];
+            v[8 * i + 5] = bf16_hi(xv.z) + g1.y * v[8 * i + 5];
+            v[8 * i + 6] = bf16_lo(xv.w) + g1.z * v[8 * i + 6];
+            v[8 * i + 7] = bf16_hi(xv.w) + g1.w * v[8 * i + 7];
+          }
+        } else {
+          for (int j = 0; j < n; ++j) v[j] = __uint_as_float(static_cast<uint32_t>(dst[j]) << 16) + g[j] * v[j];
+        }
+      }
+      store_bf16_n(dst, v, n);
+    }
+  }
+}
+
+
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_bf16_tcgen05(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                       const GemmParams p) {
@@ -258,15 +330,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       bool ok = true;
       for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
         int mb, nb;
-        tile_coords(t, p.num_m_tiles, p.num_n_tiles, mb, nb);
-        int wrow0, wrow1;
-        if (p.mode == EPI_SWIGLU) {
-          wrow0 = nb * 128;
-          wrow1 = p.swiglu_w2_row + nb * 128;
-        } else {
-          wrow0 = nb * GEMM_BN;
-          wrow1 = wrow0 + 128;
-        }
+        tile_coords(t, p.num_m_tiles, p.num_n_tiles, p.group_n, mb, nb);
+        const int wrow = nb * GEMM_BN;  // SwiGLU: W1/W2 are interleaved per 128 rows in the pack
         for (int kb = 0; kb < num_k; ++kb) {
           if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, p.err, abort_flag)) {
             ok = false;
@@ -279,8 +344,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           const uint32_t a_dst = smem_u32(sA + stage * A_STAGE_BYTES);
           const uint32_t b_dst = smem_u32(sB + stage * B_STAGE_BYTES);
           tma_load_2d(a_dst, &tmA, fb, kb * GEMM_BK, mb * GEMM_BM);
-          tma_load_2d(b_dst, &tmB, fb, kb * GEMM_BK, wrow0);
-          tma_load_2d(b_dst + B_STAGE_BYTES / 2, &tmB, fb, kb * GEMM_BK, wrow1);
+          tma_load_2d(b_dst, &tmB, fb, kb * GEMM_BK, wrow);
           if (++stage == GEMM_STAGES) {
             stage = 0;
             phase ^= 1u;
@@ -336,74 +400,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     uint32_t acc = 0, acc_phase = 0;
     for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
       int mb, nb;
-      tile_coords(t, p.num_m_tiles, p.num_n_tiles, mb, nb);
+      tile_coords(t, p.num_m_tiles, p.num_n_tiles, p.group_n, mb, nb);
       const bool got = mbar_wait(smem_u32(&acc_full[acc]), acc_phase, p.err, abort_flag);
       __syncwarp();
       if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
       const uint32_t tbase = tmem + acc * GEMM_BN + (static_cast<uint32_t>(quarter * 32) << 16);
-      const int r = mb * GEMM_BM + row_in_tile;
-      const bool row_ok = r < p.M;
-      const int b = r / p.rows_per_batch;
-      const int n_in = r - b * p.rows_per_batch;
-      const size_t orow = static_cast<size_t>(b) * p.out_rows_per_batch + p.out_row_off + n_in;
-
-      if (p.mode == EPI_QKV) {
-        epilogue_qkv(p, tbase, nb * GEMM_BN, row_ok, b, n_in);
-      } else if (p.mode == EPI_SWIGLU) {
-        const int col0 = nb * 128;
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t ra[32], rb[32];
-          tmem_ld32(tbase + c * 32, ra);
-          tmem_ld32(tbase + 128 + c * 32, rb);
-          tmem_wait_ld();
-          float v[32];
-#pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = silu_f(__uint_as_float(ra[j])) * __uint_as_float(rb[j]);
-          const int col = col0 + c * 32;
-          if (row_ok && col < p.N) store_bf16_n(p.out + orow * p.ldo + col, v, p.N - col);
-        }
-      } else {
-        const int col0 = nb * GEMM_BN;
-#pragma unroll 1
-        for (int c = 0; c < GEMM_BN / 32; ++c) {
-          const int col = col0 + c * 32;
-          if (col >= p.N) break;  // uniform
-          uint32_t ra[32];
-          tmem_ld32(tbase + c * 32, ra);
-          tmem_wait_ld();
-          float v[32];
-#pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(ra[j]);
-          if (!row_ok) continue;
-          uint16_t* dst = p.out + orow * p.ldo + col;
-          const int n = min(32, p.N - col);
-          if (p.mode == EPI_GATE_RES) {
-            const float* g = p.gate + static_cast<size_t>(b) * p.gate_stride + col;
-            if (n == 32) {
-              const uint4* xs = reinterpret_cast<const uint4*>(dst);
-#pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                const uint4 xv = xs[i];
-                const float4 g0 = *reinterpret_cast<const float4*>(g + 8 * i);
-                const float4 g1 = *reinterpret_cast<const float4*>(g + 8 * i + 4);
-                v[8 * i + 0] = bf16_lo(xv.x) + g0.x * v[8 * i + 0];
-                v[8 * i + 1] = bf16_hi(xv.x) + g0.y * v[8 * i + 1];
-                v[8 * i + 2] = bf16_lo(xv.y) + g0.z * v[8 * i + 2];
-                v[8 * i + 3] = bf16_hi(xv.y) + g0.w * v[8 * i + 3];
-                v[8 * i + 4] = bf16_lo(xv.z) + g1.x * v[8 * i + 4];
-                v[8 * i + 5] = bf16_hi(xv.z) + g1.y * v[8 * i + 5];
-                v[8 * i + 6] = bf16_lo(xv.w) + g1.z * v[8 * i + 6];
-                v[8 * i + 7] = bf16_hi(xv.w) + g1.w * v[8 * i + 7];
-              }
-            } else {
-              for (int j = 0; j < n; ++j) v[j] = __uint_as_float(static_cast<uint32_t>(dst[j]) << 16) + g[j] * v[j];
-            }
-          }
-          store_bf16_n(dst, v, n);
-        }
-      }
+      epilogue_tile(p, tbase, mb * GEMM_BM, nb, row_in_tile);
       tc_fence_before();
       mbar_arrive(smem_u32(&acc_empty[acc]));
       acc ^= 1u;
@@ -420,6 +423,176 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   }
 }
 
+// ----------------------------------------------------------------- CTA-pair variant
+// Two CTAs of a cluster compute one 256 x 256 tile with tcgen05.mma.cta_group::2:
+// each CTA loads its 128 rows of A and its 128-row half of the W tile (32 KB
+// per stage instead of 48 KB for the same FLOPs per SM, so the TMA engine
+// keeps up with the tensor core), the leader CTA issues the M = 256 MMAs
+// and its commits arrive on both CTAs' barriers; each CTA's epilogue warps
+// read the 128 x 256 accumulator half in their own TMEM.  The TMA loads of
+// both CTAs complete on the leader's stage barrier; the follower's epilogue
+// warps release the accumulator on the leader's barrier.
+constexpr int G2_STAGES = 6;
+constexpr uint32_t G2_A_BYTES = 128 * GEMM_BK * 2;  // 16 KB
+constexpr uint32_t G2_B_BYTES = 128 * GEMM_BK * 2;  // 16 KB
+constexpr int GEMM2_SMEM = G2_STAGES * (G2_A_BYTES + G2_B_BYTES) + 1024 + 1024;
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
+    gemm_bf16_tcgen05_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                           const GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + G2_STAGES * G2_A_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + G2_STAGES * G2_B_BYTES);
+  uint64_t* full = bars;                         // [G2_STAGES], used in the leader
+  uint64_t* empty = bars + G2_STAGES;            // [G2_STAGES], both CTAs
+  uint64_t* acc_full = bars + 2 * G2_STAGES;     // [2], both CTAs
+  uint64_t* acc_empty = acc_full + 2;            // [2], used in the leader
+  uint64_t* mma_done = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int cl = blockIdx.x >> 1;
+  const int ncl = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < G2_STAGES; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&empty[s]), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(smem_u32(&acc_full[a]), 1);
+      mbar_init(smem_u32(&acc_empty[a]), 8);  // 4 epilogue warps in each CTA
+    }
+    mbar_init(smem_u32(mma_done), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(tmem_slot), 512);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // the partner's barriers exist before anything signals them
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int num_k = (p.K + GEMM_BK - 1) / GEMM_BK;
+  volatile int never = 0;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true, issued = false;
+      for (int t = cl; t < p.num_tiles && ok; t += ncl) {
+        int mb, nb;
+        tile_coords(t, p.num_m_tiles, p.num_n_tiles, p.group_n, mb, nb);
+        const int arow = mb * 256 + static_cast<int>(rank) * 128;
+        const int wrow = nb * GEMM_BN + static_cast<int>(rank) * 128;
+        for (int kb = 0; kb < num_k; ++kb) {
+          if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, p.err, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb_local = smem_u32(&full[stage]);
+          if (leader) mbar_arrive_expect_tx(fb_local, 2 * (G2_A_BYTES + G2_B_BYTES));
+          const uint32_t fb = mapa_shared(fb_local, 0);
+          tma_load_2d_pair(smem_u32(sA + stage * G2_A_BYTES), &tmA, fb, kb * GEMM_BK, arow);
+          tma_load_2d_pair(smem_u32(sB + stage * G2_B_BYTES), &tmB, fb, kb * GEMM_BK, wrow);
+          issued = true;
+          if (++stage == G2_STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok && issued) {  // let copies still in flight land before the CTA leaves
+        const uint64_t t0 = globaltimer();
+        while (globaltimer() - t0 < 200000ull) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      const uint32_t idesc = make_idesc_bf16(256, GEMM_BN, false, false);
+      int stage = 0;
+      uint32_t phase = 0, acc = 0, acc_phase = 0;
+      bool ok = true;
+      for (int t = cl; t < p.num_tiles && ok; t += ncl) {
+        if (!mbar_wait(smem_u32(&acc_empty[acc]), acc_phase ^ 1u, p.err, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d = tmem + acc * GEMM_BN;
+        for (int kb = 0; kb < num_k; ++kb) {
+          if (!mbar_wait(smem_u32(&full[stage]), phase, p.err, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t adesc = make_sdesc(smem_u32(sA + stage * G2_A_BYTES), 16, 1024, SWZ_128B);
+          const uint64_t bdesc = make_sdesc(smem_u32(sB + stage * G2_B_BYTES), 16, 1024, SWZ_128B);
+#pragma unroll
+          for (int k = 0; k < GEMM_BK / 16; ++k)
+            mma_bf16_ss_pair(d, adesc + 2 * k, bdesc + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+          mma_commit_pair(smem_u32(&empty[stage]), 0x3);
+          if (++stage == G2_STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        mma_commit_pair(smem_u32(&acc_full[acc]), 0x3);
+        acc ^= 1u;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      mma_commit_pair(smem_u32(mma_done), 0x1);
+      mbar_wait(smem_u32(mma_done), 0, nullptr, &never, 100000000ull);
+    }
+  } else {
+    const int quarter = warp & 3;
+    const int row_in_tile = quarter * 32 + lane;
+    uint32_t acc = 0, acc_phase = 0;
+    for (int t = cl; t < p.num_tiles; t += ncl) {
+      int mb, nb;
+      tile_coords(t, p.num_m_tiles, p.num_n_tiles, p.group_n, mb, nb);
+      const bool got = mbar_wait(smem_u32(&acc_full[acc]), acc_phase, p.err, abort_flag);
+      __syncwarp();
+      if (!__all_sync(0xffffffffu, got)) break;
+      tc_fence_after();
+      const uint32_t tbase = tmem + acc * GEMM_BN + (static_cast<uint32_t>(quarter * 32) << 16);
+      epilogue_tile(p, tbase, mb * 256 + static_cast<int>(rank) * 128, nb, row_in_tile);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (leader)
+          mbar_arrive(smem_u32(&acc_empty[acc]));
+        else
+          mbar_arrive_cluster(mapa_shared(smem_u32(&acc_empty[acc]), 0));
+      }
+      acc ^= 1u;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // neither CTA leaves while its partner may still signal it
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, 512);
+  }
+}
+
 // ----------------------------------------------------------------- host launch
 
 cudaError_t launch_gemm(const GemmParams& p_in, const void* A, const void* W, int W_rows, cudaStream_t stream,
@@ -429,17 +602,31 @@ cudaError_t launch_gemm(const GemmParams& p_in, const void* A, const void* W, in
   if (p.K <= 0 || (p.K % 8) != 0) return cudaErrorInvalidValue;
   CUtensorMap ta, tb;
   if (!encode_tmap_2d(&ta, A, p.K, p.M, static_cast<uint64_t>(p.K) * 2, GEMM_BK, GEMM_BM)) return cudaErrorInvalidValue;
-  if (!encode_tmap_2d(&tb, W, p.K, W_rows, static_cast<uint64_t>(p.K) * 2, GEMM_BK, 128)) return cudaErrorInvalidValue;
-  p.num_m_tiles = (p.M + GEMM_BM - 1) / GEMM_BM;
-  p.num_n_tiles = p.mode == EPI_SWIGLU ? (p.N + 127) / 128 : (p.N + GEMM_BN - 1) / GEMM_BN;
-  p.num_tiles = p.num_m_tiles * p.num_n_tiles;
+  const bool pair = p.M >= 1024 && num_sms >= 2;
+  if (!encode_tmap_2d(&tb, W, p.K, W_rows, static_cast<uint64_t>(p.K) * 2, GEMM_BK, pair ? 128 : GEMM_BN))
+    return cudaErrorInvalidValue;
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(gemm_bf16_tcgen05, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          GEMM_SMEM_BYTES);
     if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(gemm_bf16_tcgen05_pair, cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM2_SMEM);
+    if (e != cudaSuccess) return e;
     attr_set = true;
   }
+  p.num_n_tiles = p.mode == EPI_SWIGLU ? (p.N + 127) / 128 : (p.N + GEMM_BN - 1) / GEMM_BN;
+  p.group_n = p.num_n_tiles < 16 ? p.num_n_tiles : 16;
+  if (p.M >= 1024 && num_sms >= 2) {
+    // CTA pairs on 256-row tiles
+    p.num_m_tiles = (p.M + 255) / 256;
+    p.num_tiles = p.num_m_tiles * p.num_n_tiles;
+    const int pairs = num_sms / 2;
+    const int grid = 2 * (p.num_tiles < pairs ? p.num_tiles : pairs);
+    gemm_bf16_tcgen05_pair<<<grid, GEMM_THREADS, GEMM2_SMEM, stream>>>(ta, tb, p);
+    return cudaGetLastError();
+  }
+  p.num_m_tiles = (p.M + GEMM_BM - 1) / GEMM_BM;
+  p.num_tiles = p.num_m_tiles * p.num_n_tiles;
   const int grid = p.num_tiles < num_sms ? p.num_tiles : num_sms;
   gemm_bf16_tcgen05<<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, stream>>>(ta, tb, p);
   return cudaGetLastError();

@@ -123,6 +123,7 @@ cudaError_t launch_ln_modulate(const uint16_t* x, const float* shift, const floa
 // pre/post: 0 = identity, 1 = SiLU.  x is staged once per CTA in shared memory.
 constexpr int GEMV_MAX_B = 8;
 
+template <int VPL>  // 16-byte weight vectors per lane (K = VPL * 256), all issued before use
 __global__ void __launch_bounds__(256) gemv_rows_kernel(const float* __restrict__ x, int B, int K,
                                                         const uint16_t* __restrict__ W,
                                                         const uint16_t* __restrict__ bias, int rows, int pre,
@@ -136,22 +137,26 @@ __global__ void __launch_bounds__(256) gemv_rows_kernel(const float* __restrict_
   __syncthreads();
   const int lane = threadIdx.x & 31;
   const int wpb = blockDim.x >> 5;
-  const int nvec = K >> 3;
   for (int j = blockIdx.x * wpb + (threadIdx.x >> 5); j < rows; j += gridDim.x * wpb) {
     const uint4* wr = reinterpret_cast<const uint4*>(W + static_cast<size_t>(j) * K);
+    const int nvec = K >> 3;
+    uint4 u[VPL];
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) u[i] = (i * 32 + lane < nvec) ? __ldg(wr + i * 32 + lane) : make_uint4(0, 0, 0, 0);
     float acc[GEMV_MAX_B];
 #pragma unroll
     for (int bb = 0; bb < GEMV_MAX_B; ++bb) acc[bb] = 0.f;
-    for (int vi = lane; vi < nvec; vi += 32) {
-      const uint4 u = __ldg(wr + vi);
-      const float w[8] = {bf16_lo(u.x), bf16_hi(u.x), bf16_lo(u.y), bf16_hi(u.y),
-                          bf16_lo(u.z), bf16_hi(u.z), bf16_lo(u.w), bf16_hi(u.w)};
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const float w[8] = {bf16_lo(u[i].x), bf16_hi(u[i].x), bf16_lo(u[i].y), bf16_hi(u[i].y),
+                          bf16_lo(u[i].z), bf16_hi(u[i].z), bf16_lo(u[i].w), bf16_hi(u[i].w)};
 #pragma unroll
       for (int bb = 0; bb < GEMV_MAX_B; ++bb) {
-        if (bb < B) {
-          const float* xb = xs + bb * K + vi * 8;
-#pragma unroll
-          for (int e = 0; e < 8; ++e) acc[bb] += w[e] * xb[e];
+        if (bb < B && i * 32 + lane < nvec) {
+          const float4* xb = reinterpret_cast<const float4*>(xs + bb * K + (i * 32 + lane) * 8);
+          const float4 x0 = xb[0], x1 = xb[1];
+          acc[bb] += w[0] * x0.x + w[1] * x0.y + w[2] * x0.z + w[3] * x0.w + w[4] * x1.x + w[5] * x1.y +
+                     w[6] * x1.z + w[7] * x1.w;
         }
       }
     }
@@ -169,6 +174,19 @@ __global__ void __launch_bounds__(256) gemv_rows_kernel(const float* __restrict_
   }
 }
 
+template <int VPL>
+static cudaError_t gemv_launch(const float* x, int nb, int K, const uint16_t* W, const uint16_t* bias, int rows,
+                               int pre, int post, float* out, int out_stride, cudaStream_t s, int blocks) {
+  const size_t smem = static_cast<size_t>(nb) * K * sizeof(float);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(gemv_rows_kernel<VPL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  gemv_rows_kernel<VPL><<<blocks, 256, smem, s>>>(x, nb, K, W, bias, rows, pre, post, out, out_stride);
+  return cudaGetLastError();
+}
+
 static cudaError_t gemv(const float* x, int B, int K, const uint16_t* W, const uint16_t* bias, int rows, int pre,
                         int post, float* out, int out_stride, cudaStream_t s) {
   if (K % 8 != 0) return cudaErrorInvalidValue;
@@ -176,18 +194,22 @@ static cudaError_t gemv(const float* x, int B, int K, const uint16_t* W, const u
   if (!sms) sms = device_sm_count();
   for (int b0 = 0; b0 < B; b0 += GEMV_MAX_B) {
     const int nb = B - b0 < GEMV_MAX_B ? B - b0 : GEMV_MAX_B;
-    const size_t smem = static_cast<size_t>(nb) * K * sizeof(float);
-    if (smem > 48 * 1024) {
-      cudaError_t e = cudaFuncSetAttribute(gemv_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           static_cast<int>(smem));
-      if (e != cudaSuccess) return e;
-    }
     int blocks = (rows + 7) / 8;
     const int cap = sms * 8;
     if (blocks > cap) blocks = cap;
-    gemv_rows_kernel<<<blocks, 256, smem, s>>>(x + static_cast<size_t>(b0) * K, nb, K, W, bias, rows, pre, post,
-                                               out + static_cast<size_t>(b0) * out_stride, out_stride);
-    cudaError_t e = cudaGetLastError();
+    const float* xb = x + static_cast<size_t>(b0) * K;
+    float* ob = out + static_cast<size_t>(b0) * out_stride;
+    cudaError_t e;
+    const int vpl = (K / 8 + 31) / 32;
+    switch (vpl <= 2 ? vpl : (vpl <= 4 ? 4 : (vpl <= 8 ? 8 : (vpl <= 12 ? 12 : (vpl <= 16 ? 16 : -1))))) {
+      case 1: e = gemv_launch<1>(xb, nb, K, W, bias, rows, pre, post, ob, out_stride, s, blocks); break;
+      case 2: e = gemv_launch<2>(xb, nb, K, W, bias, rows, pre, post, ob, out_stride, s, blocks); break;
+      case 4: e = gemv_launch<4>(xb, nb, K, W, bias, rows, pre, post, ob, out_stride, s, blocks); break;
+      case 8: e = gemv_launch<8>(xb, nb, K, W, bias, rows, pre, post, ob, out_stride, s, blocks); break;
+      case 12: e = gemv_launch<12>(xb, nb, K, W, bias, rows, pre, post, ob, out_stride, s, blocks); break;
+      case 16: e = gemv_launch<16>(xb, nb, K, W, bias, rows, pre, post, ob, out_stride, s, blocks); break;
+      default: return cudaErrorInvalidValue;
+    }
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
@@ -264,10 +286,85 @@ __global__ void __launch_bounds__(128) patch_embed_kernel(const float* __restric
   }
 }
 
+// Fast path for p*p*C = 16 (patch 2, 4 channels): a thread owns 8 output
+// columns and keeps their 8 x 16 projection weights in registers; the block
+// walks PE_TOK tokens whose patch vectors are staged in shared memory.
+constexpr int PE_TOK = 32;
+constexpr int PE_KP = 16;
+
+__global__ void __launch_bounds__(128) patch_embed16_kernel(const float* __restrict__ lat, int C, int H, int W,
+                                                            int p, const uint16_t* __restrict__ wpe,
+                                                            const uint16_t* __restrict__ pos, int G, int D,
+                                                            uint16_t* __restrict__ out, int out_rows_per_batch,
+                                                            int out_row_off) {
+  __shared__ float patch[PE_TOK][PE_KP];
+  const int b = blockIdx.z;
+  const int hpn = H / p, wpn = W / p, ntok = hpn * wpn;
+  const int t0 = blockIdx.x * PE_TOK;
+  for (int i = threadIdx.x; i < PE_TOK * PE_KP; i += blockDim.x) {
+    const int tt = i / PE_KP, k = i - tt * PE_KP;
+    const int n = t0 + tt;
+    float v = 0.f;
+    if (n < ntok) {
+      const int hp = n / wpn, wp = n - hp * wpn;
+      const int c = k % C, pq = k / C;
+      const int py = pq / p, px = pq - py * p;
+      v = lat[((static_cast<size_t>(b) * C + c) * H + hp * p + py) * W + wp * p + px];
+    }
+    patch[tt][k] = v;
+  }
+  __syncthreads();
+  const int vi = blockIdx.y * blockDim.x + threadIdx.x;
+  if (vi >= D / 8) return;
+  float wv[8][PE_KP];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const uint4* wr = reinterpret_cast<const uint4*>(wpe + static_cast<size_t>(vi * 8 + e) * PE_KP);
+    const uint4 a = wr[0], c = wr[1];
+    const uint32_t q[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      wv[e][2 * k] = bf16_lo(q[k]);
+      wv[e][2 * k + 1] = bf16_hi(q[k]);
+    }
+  }
+  const int r0 = (G - hpn) / 2, c0 = (G - wpn) / 2;
+  for (int tt = 0; tt < PE_TOK; ++tt) {
+    const int n = t0 + tt;
+    if (n >= ntok) break;
+    const int hp = n / wpn, wp = n - hp * wpn;
+    const size_t prow = static_cast<size_t>(r0 + hp) * G + c0 + wp;
+    const uint4 pu = *reinterpret_cast<const uint4*>(pos + prow * D + vi * 8);
+    const float pe[8] = {bf16_lo(pu.x), bf16_hi(pu.x), bf16_lo(pu.y), bf16_hi(pu.y),
+                         bf16_lo(pu.z), bf16_hi(pu.z), bf16_lo(pu.w), bf16_hi(pu.w)};
+    float o[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      float a = 0.f;
+#pragma unroll
+      for (int k = 0; k < PE_KP; ++k) a += wv[e][k] * patch[tt][k];
+      o[e] = a + pe[e];
+    }
+    uint4 u;
+    u.x = pack_bf16(o[0], o[1]);
+    u.y = pack_bf16(o[2], o[3]);
+    u.z = pack_bf16(o[4], o[5]);
+    u.w = pack_bf16(o[6], o[7]);
+    *reinterpret_cast<uint4*>(out + (static_cast<size_t>(b) * out_rows_per_batch + out_row_off + n) * D + vi * 8) = u;
+  }
+}
+
 cudaError_t launch_patch_embed(const float* lat, int B, int C, int H, int W, int p, const uint16_t* w_pe,
                                const uint16_t* pos, int G, int D, uint16_t* out, int out_rows_per_batch,
                                int out_row_off, cudaStream_t s) {
   if (p * p * C > 64 || D % 8 != 0) return cudaErrorInvalidValue;
+  if (p * p * C == PE_KP) {
+    const int ntok = (H / p) * (W / p);
+    dim3 grid((ntok + PE_TOK - 1) / PE_TOK, (D / 8 + 127) / 128, B);
+    patch_embed16_kernel<<<grid, 128, 0, s>>>(lat, C, H, W, p, w_pe, pos, G, D, out, out_rows_per_batch,
+                                              out_row_off);
+    return cudaGetLastError();
+  }
   dim3 grid((H / p) * (W / p), B);
   patch_embed_kernel<<<grid, 128, 0, s>>>(lat, C, H, W, p, w_pe, pos, G, D, out, out_rows_per_batch, out_row_off);
   return cudaGetLastError();

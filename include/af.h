@@ -253,9 +253,13 @@ af_status af_linear(const uint16_t* A, const uint16_t* W, uint16_t* C, int M, in
 
 /* Non-causal softmax(q k^T / sqrt(hd)) v per (batch, head) ([ARCH]
  * §注意力处理器与 QKV 融合).
- *   q, k, v: device bf16[B, H, N, hd];  o: device bf16[B, N, H*hd]. */
+ *   q, k, v: device bf16[B, H, N, hd];  o: device bf16[B, N, H*hd].
+ *   qk_normalized: nonzero promises that every q and k row has L2 norm at
+ *   most sqrt(hd) (up to bf16 rounding), as the per-head LayerNorm (QK-norm)
+ *   guarantees; the kernel then uses a fixed softmax shift instead of a
+ *   running maximum.  Pass 0 for arbitrary inputs. */
 af_status af_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* o, int B,
-                       int H, int N, int hd, void* stream);
+                       int H, int N, int hd, int qk_normalized, void* stream);
 
 const char* af_status_string(af_status st);
 /* Text of the last CUDA error seen by this thread's calls ("" if none). */

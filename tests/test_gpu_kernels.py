@@ -28,7 +28,9 @@ def af():
 # ---------------------------------------------------------------- GEMM (tcgen05)
 
 @pytest.mark.parametrize("M,N,K", [(300, 520, 200), (1000, 3072, 3072), (64, 96, 32), (129, 256, 64),
-                                   (528, 9216, 3072), (8, 16, 2048)])
+                                   (528, 9216, 3072), (8, 16, 2048),
+                                   # M >= 1024 runs on CTA pairs (256-row tiles, cta_group::2)
+                                   (1100, 776, 520), (4096, 3072, 3072), (2304, 16, 64), (8720, 1024, 8192)])
 def test_linear_matches_fp64(af, M, N, K):
     A = synth.normal(11, f"A{M}_{N}_{K}", (M, K), 1.0)
     W = synth.normal(12, f"W{M}_{N}_{K}", (N, K), 0.02)
@@ -52,10 +54,15 @@ def test_linear_rejects_unaligned_k(af):
 
 # ---------------------------------------------------------------- attention
 
-@pytest.mark.parametrize("B,H,N,hd,qscale", [(2, 2, 1, 256, 1.0), (1, 2, 7, 256, 1.0), (2, 1, 64, 256, 1.0),
-                                             (1, 2, 129, 256, 1.0), (2, 2, 264, 256, 3.0), (1, 3, 600, 256, 1.0),
-                                             (1, 4, 80, 8, 1.0), (2, 2, 33, 16, 1.0)])
-def test_attention_matches_oracle(af, B, H, N, hd, qscale):
+ATTN_CASES = [(2, 2, 1, 256, 1.0), (1, 2, 7, 256, 1.0), (2, 1, 64, 256, 1.0), (1, 2, 129, 256, 1.0),
+              (2, 2, 264, 256, 3.0), (1, 3, 600, 256, 1.0), (1, 4, 80, 8, 1.0), (2, 2, 33, 16, 1.0)]
+
+
+@pytest.mark.parametrize("qkn", [False, True])
+@pytest.mark.parametrize("B,H,N,hd,qscale", ATTN_CASES)
+def test_attention_matches_oracle(af, B, H, N, hd, qscale, qkn):
+    if qkn and qscale != 1.0:
+        pytest.skip("the fixed-shift kernel requires per-head LayerNorm-ed q and k")
     q = synth.normal(21, f"q{N}", (B, H, N, hd), 1.0)
     k = synth.normal(22, f"k{N}", (B, H, N, hd), 1.0)
     v = synth.normal(23, f"v{N}", (B, H, N, hd), 1.0)
@@ -63,9 +70,23 @@ def test_attention_matches_oracle(af, B, H, N, hd, qscale):
     qn = synth.bf16_round((O.layer_norm(q, 1e-6) * qscale).astype(np.float32))
     kn = synth.bf16_round(O.layer_norm(k, 1e-6).astype(np.float32))
     o = torch.empty(B, N, H * hd, dtype=torch.bfloat16, device="cuda")
-    af.attention(to_bf16(qn), to_bf16(kn), to_bf16(v), o)
+    af.attention(to_bf16(qn), to_bf16(kn), to_bf16(v), o, qk_normalized=qkn)
     torch.cuda.synchronize()
     ref = O.merge_heads(O.attention(qn, kn, v))
+    assert O.rel_l2(to_np(o), ref) < 1e-2
+
+
+@pytest.mark.parametrize("qkn", [False, True])
+def test_attention_extreme_logits(af, qkn):
+    """q = k (LayerNorm-ed): every diagonal logit is at the bound |q.k|/16 = 16."""
+    B, H, N, hd = 1, 2, 300, 256
+    q = synth.normal(26, "qe", (B, H, N, hd), 1.0)
+    qn = synth.bf16_round(O.layer_norm(q, 1e-6).astype(np.float32))
+    v = synth.normal(27, "ve", (B, H, N, hd), 1.0)
+    o = torch.empty(B, N, H * hd, dtype=torch.bfloat16, device="cuda")
+    af.attention(to_bf16(qn), to_bf16(qn), to_bf16(v), o, qk_normalized=qkn)
+    torch.cuda.synchronize()
+    ref = O.merge_heads(O.attention(qn, qn, v))
     assert O.rel_l2(to_np(o), ref) < 1e-2
 
 
