@@ -637,6 +637,308 @@ __global__ void __launch_bounds__(QKN_THREADS, 1)
   }
 }
 
+// ---------------------------------------------------------------- QK-normalised inputs on CTA pairs
+// attn_hd256_qknorm_pair: a cluster of two CTAs takes 256 query rows of one
+// (sample, head), 128 per CTA, and walks the keys in tiles of 128 with
+// tcgen05.mma.cta_group::2 issued by the leader CTA:
+//   S = Q K^T   M = 256, N = 128, K = 256: each CTA supplies its 128 Q rows
+//               and half of the K tile (64 keys); each CTA's TMEM receives
+//               its 128 x 128 block of S.
+//   O += P V    M = 256, N = 256, K = 128: each CTA supplies its 128 rows of
+//               P and half of the V tile (128 head-dim columns); each CTA's
+//               TMEM accumulates its 128 x 256 block of O.
+// Per SM that is 64 KB of K/V per 128 keys instead of 128 KB, and every MMA
+// has N >= 128 (full tensor-core rate).  TMEM per CTA: O [0, 256), S0
+// [256, 384), S1 [384, 512).  Shared memory per CTA: Q 64 KB, K and V halves
+// double-buffered (4 x 32 KB), one P buffer (128 x 128 bf16, 32 KB).
+// Softmax (fixed shift, as for attn_hd256_qknorm): warpgroup g of each CTA
+// owns keys [64 g, 64 g + 64) of every S tile; their partial row sums are
+// added at the end.  The leader issues S_0, S_1, then per tile PV_j followed
+// by S_{j+2}, so the tensor core computes the next scores while the softmax
+// warps publish P_{j+1}.  Barriers that gather both CTAs live in the leader
+// (TMA completions, S/P handshakes); commits are multicast to both CTAs.
+// The follower's softmax warps arrive directly on the leader's S/P barriers
+// (CTA-scope release; a cluster-scope release there costs ~1.2k cycles).
+constexpr int AP_BN = 128;
+constexpr uint32_t AP_Q_BYTES = 128 * AT_HD * 2;      // 64 KB
+constexpr uint32_t AP_KH_BYTES = 64 * AT_HD * 2;      // 32 KB: 64 keys x 256
+constexpr uint32_t AP_VH_BYTES = AP_BN * 128 * 2;     // 32 KB: 128 keys x 128 columns
+constexpr uint32_t AP_P_BYTES = 128 * AP_BN * 2;      // 32 KB
+constexpr int AP_SMEM = AP_Q_BYTES + 2 * AP_KH_BYTES + 2 * AP_VH_BYTES + AP_P_BYTES + 2 * 128 * 4 + 256 + 1024;
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
+    attn_hd256_qknorm_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                           const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sK = sQ + AP_Q_BYTES;          // 2 buffers
+  uint8_t* sV = sK + 2 * AP_KH_BYTES;     // 2 buffers
+  uint8_t* sP = sV + 2 * AP_VH_BYTES;
+  float* xsum = reinterpret_cast<float*>(sP + AP_P_BYTES);  // [wg 2][row 128]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + AP_P_BYTES + 2 * 128 * 4);
+  uint64_t* q_full = bars + 0;     // leader: both CTAs' Q loads
+  uint64_t* k_full = bars + 1;     // [2] leader: both K halves
+  uint64_t* v_full = bars + 3;     // [2] leader: both V halves
+  uint64_t* k_empty = bars + 5;    // [2] both CTAs (multicast commit)
+  uint64_t* v_empty = bars + 7;    // [2] both CTAs
+  uint64_t* s_full = bars + 9;     // [2] both CTAs
+  uint64_t* s_empty = bars + 11;   // [2] leader: 16 softmax warps of both CTAs
+  uint64_t* p_full = bars + 13;    // leader: 16 softmax warps of both CTAs
+  uint64_t* pv_done = bars + 14;   // both CTAs
+  uint64_t* mma_done = bars + 15;  // leader
+  uint64_t* lbar = bars + 16;      // per CTA: 8 softmax warps
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int bh = b * p.H + h;
+  const int q0 = pair * 256 + static_cast<int>(rank) * 128;
+  const int nkv = (p.N + AP_BN - 1) / AP_BN;
+  const int kv0 = static_cast<int>((static_cast<long long>(pair) * nkv) / npairs);
+  auto kv_tile = [&](int j) { const int t = j + kv0; return t < nkv ? t : t - nkv; };
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(q_full), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&k_full[i]), 1);
+      mbar_init(smem_u32(&v_full[i]), 1);
+      mbar_init(smem_u32(&k_empty[i]), 1);
+      mbar_init(smem_u32(&v_empty[i]), 1);
+      mbar_init(smem_u32(&s_full[i]), 1);
+      mbar_init(smem_u32(&s_empty[i]), 2 * AT_SOFTMAX_WARPS);
+    }
+    mbar_init(smem_u32(p_full), 2 * AT_SOFTMAX_WARPS);
+    mbar_init(smem_u32(pv_done), 1);
+    mbar_init(smem_u32(mma_done), 1);
+    mbar_init(smem_u32(lbar), AT_SOFTMAX_WARPS);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(tmem_slot), 512);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tO = tmem;
+  const uint32_t tS = tmem + 256;
+  volatile int never = 0;
+
+  if (warp == 0 || warp == AT_V_WARP) {
+    // warp 0: Q then the K halves (keys [64 rank, +64) of each tile);
+    // last warp: the V halves (head-dim columns [128 rank, +128)).
+    if (lane == 0) {
+      const bool is_k = warp == 0;
+      uint64_t* full = is_k ? k_full : v_full;
+      uint64_t* empty = is_k ? k_empty : v_empty;
+      const uint32_t half = is_k ? AP_KH_BYTES : AP_VH_BYTES;
+      uint8_t* buf = is_k ? sK : sV;
+      bool ok = true, issued = false;
+      if (is_k) {
+        const uint32_t qb = mapa_shared(smem_u32(q_full), 0);
+        if (leader) mbar_arrive_expect_tx(smem_u32(q_full), 2 * AP_Q_BYTES);
+        for (int c = 0; c < 4; ++c)
+          tma_load_3d_pair(smem_u32(sQ + c * (128 * 128)), &tmQ, qb, c * 64, q0, bh);
+        issued = true;
+      }
+      for (int j = 0; j < nkv; ++j) {
+        const int s = j & 1;
+        const uint32_t ph = (j >> 1) & 1;
+        if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1u, p.err, abort_flag)) { ok = false; break; }
+        if (leader) mbar_arrive_expect_tx(smem_u32(&full[s]), 2 * half);
+        const uint32_t fb = mapa_shared(smem_u32(&full[s]), 0);
+        const int key0 = kv_tile(j) * AP_BN;
+        if (is_k) {
+          for (int c = 0; c < 4; ++c)
+            tma_load_3d_pair(smem_u32(buf + s * half + c * (64 * 128)), &tmK, fb, c * 64,
+                             key0 + static_cast<int>(rank) * 64, bh);
+        } else {
+          for (int c = 0; c < 2; ++c)
+            tma_load_3d_pair(smem_u32(buf + s * half + c * (AP_BN * 128)), &tmV, fb,
+                             static_cast<int>(rank) * 128 + c * 64, key0, bh);
+        }
+        issued = true;
+      }
+      if (!ok && issued) {
+        const uint64_t t0 = globaltimer();
+        while (globaltimer() - t0 < 200000ull) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      const uint32_t idesc_qk = make_idesc_bf16(256, AP_BN, false, false);
+      const uint32_t idesc_pv = make_idesc_bf16(256, AT_HD, false, true);
+      const uint32_t qaddr = smem_u32(sQ);
+      const uint32_t paddr = smem_u32(sP);
+      bool ok = mbar_wait(smem_u32(q_full), 0, p.err, abort_flag);
+      auto issue_s = [&](int j) -> bool {
+        const int s = j & 1;
+        const uint32_t ph = (j >> 1) & 1;
+        if (!mbar_wait(smem_u32(&k_full[s]), ph, p.err, abort_flag)) return false;
+        if (!mbar_wait(smem_u32(&s_empty[s]), ph ^ 1u, p.err, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t kaddr = smem_u32(sK + s * AP_KH_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < AT_HD / 16; ++kk) {
+          const uint32_t c = kk >> 2, off = (kk & 3) * 32;
+          const uint64_t ad = make_sdesc(qaddr + c * (128 * 128) + off, 16, 1024, SWZ_128B);
+          const uint64_t bd = make_sdesc(kaddr + c * (64 * 128) + off, 16, 1024, SWZ_128B);
+          mma_bf16_ss_pair(tS + s * AP_BN, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
+        }
+        mma_commit_pair(smem_u32(&s_full[s]), 0x3);
+        mma_commit_pair(smem_u32(&k_empty[s]), 0x3);
+        return true;
+      };
+      if (ok) ok = issue_s(0);
+      if (ok && nkv > 1) ok = issue_s(1);
+      for (int j = 0; j < nkv && ok; ++j) {
+        const int s = j & 1;
+        if (!mbar_wait(smem_u32(p_full), j & 1, p.err, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(smem_u32(&v_full[s]), (j >> 1) & 1, p.err, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t vaddr = smem_u32(sV + s * AP_VH_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < AP_BN / 16; ++kk) {
+          const uint32_t c = kk >> 2, off = (kk & 3) * 32;
+          const uint64_t ad = make_sdesc(paddr + c * (128 * 128) + off, 16, 1024, SWZ_128B);
+          const uint64_t bd = make_sdesc(vaddr + kk * (16 * 128), AP_BN * 128, 1024, SWZ_128B);
+          mma_bf16_ss_pair(tO, ad, bd, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit_pair(smem_u32(pv_done), 0x3);
+        mma_commit_pair(smem_u32(&v_empty[s]), 0x3);
+        if (j + 2 < nkv && !issue_s(j + 2)) { ok = false; break; }
+      }
+      mma_commit_pair(smem_u32(mma_done), 0x1);
+      mbar_wait(smem_u32(mma_done), 0, nullptr, &never, 100000000ull);
+    }
+  } else {
+    // ---------------------------------------------------------------- softmax: group g owns keys [64 g, 64 g + 64)
+    const int wg = (warp - 2) >> 2;
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const float c = p.scale_log2;
+    const float off = -QKN_OFFSET_LOG2;
+    const uint32_t s_empty_l = mapa_shared(smem_u32(s_empty), 0);
+    const uint32_t p_full_l = mapa_shared(smem_u32(p_full), 0);
+    float l = 0.f;
+    bool ok = true;
+    uint8_t* prow = sP + wg * (128 * 128) + row * 128;
+    for (int j = 0; j < nkv; ++j) {
+      const int s = j & 1;
+      const bool got = mbar_wait(smem_u32(&s_full[s]), (j >> 1) & 1, p.err, abort_flag);
+      __syncwarp();
+      if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t r0[32], r1[32];
+      tmem_ld32(tS + s * AP_BN + 64 * wg + lane_off, r0);
+      tmem_ld32(tS + s * AP_BN + 64 * wg + 32 + lane_off, r1);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(s_empty_l + s * 8);
+      const int kvalid = p.N - kv_tile(j) * AP_BN - 64 * wg;
+      uint32_t pk[32];
+      float rs = 0.f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        float e0 = ex2_approx(fmaf(__uint_as_float(r0[2 * i]), c, off));
+        float e1 = ex2_approx(fmaf(__uint_as_float(r0[2 * i + 1]), c, off));
+        float e2 = ex2_approx(fmaf(__uint_as_float(r1[2 * i]), c, off));
+        float e3 = ex2_approx(fmaf(__uint_as_float(r1[2 * i + 1]), c, off));
+        if (kvalid < 64) {
+          if (2 * i >= kvalid) e0 = 0.f;
+          if (2 * i + 1 >= kvalid) e1 = 0.f;
+          if (32 + 2 * i >= kvalid) e2 = 0.f;
+          if (32 + 2 * i + 1 >= kvalid) e3 = 0.f;
+        }
+        rs += (e0 + e1) + (e2 + e3);
+        pk[i] = pack_bf16(e0, e1);
+        pk[16 + i] = pack_bf16(e2, e3);
+      }
+      l += rs;
+      // the P buffer is free once PV_{j-1} has completed
+      if (j >= 1) {
+        const bool g2 = mbar_wait(smem_u32(pv_done), (j - 1) & 1, p.err, abort_flag);
+        __syncwarp();
+        if (!__all_sync(0xffffffffu, g2)) { ok = false; break; }
+      }
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        uint4 v = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+        *reinterpret_cast<uint4*>(prow + ((q ^ (row & 7)) << 4)) = v;
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(p_full_l);
+    }
+    if (ok) {
+      xsum[wg * 128 + row] = l;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(lbar));
+      const bool g3 = mbar_wait(smem_u32(lbar), 0, p.err, abort_flag) &&
+                      mbar_wait(smem_u32(pv_done), (nkv - 1) & 1, p.err, abort_flag);
+      __syncwarp();
+      if (__all_sync(0xffffffffu, g3)) {
+        tc_fence_after();
+        const float inv = 1.0f / (l + xsum[(wg ^ 1) * 128 + row]);
+        const int qrow = q0 + row;
+        const bool row_ok = qrow < p.N;
+        uint16_t* dst = nullptr;
+        if (row_ok) {
+          if (qrow < p.split)
+            dst = p.out_a + (static_cast<size_t>(b) * p.split + qrow) * p.ldo + h * AT_HD;
+          else
+            dst = p.out_b + (static_cast<size_t>(b) * (p.N - p.split) + (qrow - p.split)) * p.ldo + h * AT_HD;
+          dst += 128 * wg;
+        }
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t o[32];
+          tmem_ld32(tO + 128 * wg + cc * 32 + lane_off, o);
+          tmem_wait_ld();
+          if (row_ok) {
+            uint4* d = reinterpret_cast<uint4*>(dst + cc * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              uint4 u;
+              u.x = pack_bf16(__uint_as_float(o[8 * i + 0]) * inv, __uint_as_float(o[8 * i + 1]) * inv);
+              u.y = pack_bf16(__uint_as_float(o[8 * i + 2]) * inv, __uint_as_float(o[8 * i + 3]) * inv);
+              u.z = pack_bf16(__uint_as_float(o[8 * i + 4]) * inv, __uint_as_float(o[8 * i + 5]) * inv);
+              u.w = pack_bf16(__uint_as_float(o[8 * i + 6]) * inv, __uint_as_float(o[8 * i + 7]) * inv);
+              d[i] = u;
+            }
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, 512);
+  }
+}
+
 // ---------------------------------------------------------------- small heads (SIMT)
 template <int HD>
 __global__ void attn_small_simt(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
@@ -683,7 +985,16 @@ cudaError_t launch_attention(const AttnParams& p, const uint16_t* q, const uint1
       if (e != cudaSuccess) return e;
       e = cudaFuncSetAttribute(attn_hd256_qknorm, cudaFuncAttributeMaxDynamicSharedMemorySize, QKN_SMEM);
       if (e != cudaSuccess) return e;
+      e = cudaFuncSetAttribute(attn_hd256_qknorm_pair, cudaFuncAttributeMaxDynamicSharedMemorySize, AP_SMEM);
+      if (e != cudaSuccess) return e;
       attr = true;
+    }
+    if (p.qk_normalized && p.N >= 256) {
+      CUtensorMap tv2;  // V halves: 128 keys x 64 columns per box
+      if (!encode_tmap_3d(&tv2, v, AT_HD, p.N, bh, rb, sb, 64, AP_BN, 1)) return cudaErrorInvalidValue;
+      dim3 grid2(2 * ((p.N + 255) / 256), p.H, p.B);
+      attn_hd256_qknorm_pair<<<grid2, AT_THREADS, AP_SMEM, stream>>>(tq, tk, tv2, p);
+      return cudaGetLastError();
     }
     dim3 grid((p.N + AT_BM - 1) / AT_BM, p.H, p.B);
     if (p.qk_normalized)

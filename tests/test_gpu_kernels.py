@@ -55,7 +55,9 @@ def test_linear_rejects_unaligned_k(af):
 # ---------------------------------------------------------------- attention
 
 ATTN_CASES = [(2, 2, 1, 256, 1.0), (1, 2, 7, 256, 1.0), (2, 1, 64, 256, 1.0), (1, 2, 129, 256, 1.0),
-              (2, 2, 264, 256, 3.0), (1, 3, 600, 256, 1.0), (1, 4, 80, 8, 1.0), (2, 2, 33, 16, 1.0)]
+              (2, 2, 264, 256, 3.0), (1, 3, 600, 256, 1.0), (1, 4, 80, 8, 1.0), (2, 2, 33, 16, 1.0),
+              # N >= 256 with QK-normalised inputs runs on CTA pairs (256 query rows, 128-key tiles)
+              (1, 2, 256, 256, 1.0), (2, 1, 257, 256, 1.0), (1, 2, 1000, 256, 1.0), (1, 1, 4360, 256, 1.0)]
 
 
 @pytest.mark.parametrize("qkn", [False, True])
