@@ -314,19 +314,22 @@ def run_af(args, rank, world, local_rank):
     attn_tflops = work[1] / (ms[1] * 1e-3) / 1e12 if ms[1] > 0 else None
     ln_gbs = work[2] / (ms[2] * 1e-3) / 1e9 if ms[2] > 0 else None
     traffic = None
-    tpath = os.path.join(ROOT, "profiles", "gemm_traffic.json")
+    tpath = os.path.join(ROOT, "profiles", "gemm_traffic.txt")
     if os.path.exists(tpath):
         try:
             import hashlib
             with open(tpath) as f:
-                tr = json.load(f)
-            src = open(os.path.join(ROOT, "diffusion_transformer_denoising_auraflow_b200", "csrc", "gemm.cu"),
-                       "rb").read()
-            if tr.get("gemm_cu_sha1") == hashlib.sha1(src).hexdigest():
-                traffic = tr.get("bytes_per_launch")
-        except Exception:
+                tr = dict(ln.split(":", 1) for ln in f.read().splitlines() if ln and not ln.startswith("#"))
+            h = hashlib.sha1()
+            for name in ("gemm.cu", "ptx.cuh", "af_internal.h"):
+                with open(os.path.join(ROOT, "diffusion_transformer_denoising_auraflow_b200", "csrc", name), "rb") as f:
+                    h.update(f.read())
+            if tr.get("sources_sha1", "").strip() == h.hexdigest():   # stale once the kernel changes
+                traffic = float(tr["bytes_per_launch"])
+        except (OSError, ValueError, KeyError):
             traffic = None
-    roofline = {"bound": "tensor", "kernel": "gemm_bf16_tcgen05", "achieved": gemm_tflops,
+    roofline = {"bound": "tensor", "kernel": "gemm_bf16_tcgen05_pair (M >= 1024) / gemm_bf16_tcgen05",
+                "achieved": gemm_tflops,
                 "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s", "frac": gemm_tflops / pk["bf16_tflops_sustained"],
                 "traffic": traffic, "peak_source": f"{pk['source']} (sustained cuBLAS bf16)",
                 "flops_per_launch": gemm_flops_launch, "ms_per_launch": gemm_ms_launch}
