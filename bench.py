@@ -56,6 +56,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--seed", type=int, default=4)
+    ap.add_argument("--direct", action="store_true",
+                    help="time the per-step entry point (af_denoise_step) instead of the sampler plan")
     ap.add_argument("--case", default="step", choices=["step", "single_block"],
                     help="single_block: time one full-shape AuraFlowSingleTransformerBlock only "
                          "(a small command for profiler captures)")
@@ -252,7 +254,8 @@ def run_af(args, rank, world, local_rank):
     w = af.Weights(cfg, local_rank)
     make_weights(af, torch, w, args.seed, device)
     s = af.Scratch(w, 2, Ni, L)
-    stream = torch.cuda.current_stream()
+    stream = torch.cuda.Stream(device)
+    torch.cuda.set_stream(stream)   # graphs cannot be captured on the legacy default stream
 
     gen = torch.Generator(device=device)
     gen.manual_seed(args.seed * 7919 + rank)
@@ -260,10 +263,24 @@ def run_af(args, rank, world, local_rank):
     text = torch.randn(2, L, 2048, generator=gen, device=device).to(torch.bfloat16)
     lat = lat0.clone()
     sig = af.sigma_schedule(N_SCHED, SHIFT)
+    lat_d = torch.empty_like(lat0)
+    text_d = torch.empty_like(text)
+    # the product path: the sampler plan (all modulations in one GEMM per
+    # 25-step run, every step a CUDA graph), one plan per bound latent buffer
+    plans = {} if args.direct else {id(lat): af.Sampler(w, s, lat, text, sig, GUIDANCE, use_graphs=True),
+                                    id(lat_d): af.Sampler(w, s, lat_d, text_d, sig, GUIDANCE, use_graphs=True)}
+
+    def direct_step(i, latents, text_emb):
+        j = i % N_SCHED
+        af.denoise_step(w, s, latents, text_emb, GUIDANCE, sig[j], sig[j + 1], stream)
 
     def step(i, latents, text_emb):
-        j = i % N_SCHED
-        af.denoise_step(w, s, latents, text_emb, GUIDANCE, sig[j], sig[j + 1])
+        if args.direct:
+            return direct_step(i, latents, text_emb)
+        plan, j = plans[id(latents)], i % N_SCHED
+        if j == 0:
+            plan.prepare(stream)    # modulation table of the whole run, timed with its first step
+        plan.step(j, stream)
 
     def barrier():
         if world > 1:
@@ -277,6 +294,15 @@ def run_af(args, rank, world, local_rank):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         return float(t.item())
 
+    # build the plans: capture and instantiate all N_SCHED step graphs (untimed)
+    for plan_lat, plan_txt in ((lat, text), (lat_d, text_d)):
+        if args.direct:
+            break
+        plan_lat.copy_(lat0)
+        plan_txt.copy_(text)
+        for i in range(N_SCHED):
+            step(i, plan_lat, plan_txt)
+    lat.copy_(lat0)
     # warm-up
     for i in range(args.warmup):
         step(i, lat, text)
@@ -300,12 +326,27 @@ def run_af(args, rank, world, local_rank):
     value = world * args.steps / t_max
     clocks = clk.summary()
 
-    # ---- per-kernel-class device time over a few more steps (live roofline)
+    # ---- the per-step path (no plan, no graphs): same kernels, modulations by GEMV each step
+    direct = None
+    if not args.direct:
+        for i in range(2):
+            direct_step(i, lat, text)
+        barrier()
+        e4, e5 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e4.record(stream)
+        for i in range(args.steps):
+            direct_step(i, lat, text)
+        e5.record(stream)
+        barrier()
+        direct = world * args.steps / max_over_ranks(e4.elapsed_time(e5) / 1000.0)
+
+    # ---- per-kernel-class device time over a few more steps (live roofline);
+    # the event profiler brackets every launch, so it runs on the per-step path
     n_prof = max(3, min(args.steps, 5))
     barrier()
     s.profile_begin()
     for i in range(n_prof):
-        step(i, lat, text)
+        direct_step(i, lat, text)
     ms, nl, work = s.profile_end()
     pk = peaks()
     gemm_ms_launch = ms[0] / max(nl[0], 1)
@@ -341,8 +382,6 @@ def run_af(args, rank, world, local_rank):
         lat_h = lat0.cpu().pin_memory()
         text_h = text.cpu().pin_memory()
         out_h = torch.empty_like(lat_h).pin_memory()
-        lat_d = torch.empty_like(lat0)
-        text_d = torch.empty_like(text)
         for i in range(2):
             lat_d.copy_(lat_h, non_blocking=True)
             text_d.copy_(text_h, non_blocking=True)
@@ -383,7 +422,12 @@ def run_af(args, rank, world, local_rank):
                                    "ln_modulate": step_ms_classes[2], "other": step_ms_classes[3]},
             "kernel_rates": {"attention_tflops": attn_tflops, "ln_modulate_gbs": ln_gbs},
             "e2e": e2e,
+            "path": ("per-step calls (af_denoise_step)" if args.direct else
+                     "af_sampler: modulations of all 25 steps in one GEMM per run (timed), steps as CUDA graphs"),
+            "per_step_path_steps_per_s": direct,
         }
+    for plan in plans.values():
+        plan.close()
     s.close()
     w.close()
     return line

@@ -75,6 +75,10 @@ _SIGS = {
     "af_euler_cfg_step": [_P, _P, _I, _I, _I, _I, _F, _F, _F, _P],
     "af_denoise_step": [_P, _P, _P, _P, _I, _I, _I, _I, _F, _F, _F, _P],
     "af_sigma_schedule": [_I, _F, _I, _P],
+    "af_sampler_create": [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _F, _I, _P],
+    "af_sampler_prepare": [_P, _P],
+    "af_sampler_step": [_P, _I, _P],
+    "af_sampler_destroy": [_P],
     "af_launch_counts": [_P, _P],
     "af_profile_begin": [_P],
     "af_profile_end": [_P, _P, _P, _P, _P],
@@ -99,6 +103,7 @@ def _load():
         fn.restype = _I
     L.af_weights_destroy.restype = None
     L.af_scratch_destroy.restype = None
+    L.af_sampler_destroy.restype = None
     L.af_status_string.restype = ctypes.c_char_p
     L.af_last_error.restype = ctypes.c_char_p
     return L
@@ -288,6 +293,42 @@ def denoise_step(w: Weights, s: Scratch, latents, text_emb, guidance: float, sig
     _check(lib.af_denoise_step(w.handle, s.handle, _dev(latents, torch.float32, "latents"),
                                _dev(text_emb, torch.bfloat16, "text_emb"), Bi, H, W, L, float(guidance), float(sigma),
                                float(sigma_next), _stream(stream)), "af_denoise_step")
+
+
+class Sampler:
+    """The denoising loop as a plan (af_sampler): modulations of every step
+    precomputed by prepare(), steps optionally replayed as CUDA graphs."""
+
+    def __init__(self, w: Weights, s: Scratch, latents, text_emb, sigmas, guidance: float, use_graphs: bool = True):
+        Bi, C, H, W = latents.shape
+        L = text_emb.shape[1]
+        if text_emb.shape[0] != 2 * Bi:
+            raise ValueError("text_emb must hold 2*Bi rows (uncond first)")
+        self.n_steps = len(sigmas) - 1
+        sig = (ctypes.c_float * len(sigmas))(*[float(x) for x in sigmas])
+        h = ctypes.c_void_p()
+        _check(lib.af_sampler_create(w.handle, s.handle, _dev(latents, torch.float32, "latents"),
+                                     _dev(text_emb, torch.bfloat16, "text_emb"), Bi, H, W, L, self.n_steps, sig,
+                                     float(guidance), 1 if use_graphs else 0, ctypes.byref(h)), "af_sampler_create")
+        self.handle = h
+        self._keep = (w, s, latents, text_emb)
+
+    def prepare(self, stream=None):
+        _check(lib.af_sampler_prepare(self.handle, _stream(stream)), "af_sampler_prepare")
+
+    def step(self, i: int, stream=None):
+        _check(lib.af_sampler_step(self.handle, int(i), _stream(stream)), "af_sampler_step")
+
+    def close(self):
+        if self.handle:
+            lib.af_sampler_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 def sigma_schedule(n_steps: int, shift: float = 1.73, num_train_timesteps: int = 1000):

@@ -13,6 +13,7 @@ enum GemmMode : int {
   EPI_GATE_RES = 1,  // x += gate[b] * acc   (adaLN-Zero gated residual)
   EPI_SWIGLU = 2,    // h = silu(acc[W1 half]) * acc[W2 half]
   EPI_QKV = 3,       // per-head LayerNorm of Q and K, scatter to [B, H, N, hd]
+  EPI_STORE_F32 = 4, // C = acc (fp32) into out_f32
 };
 
 struct GemmParams {
@@ -22,6 +23,7 @@ struct GemmParams {
   int out_rows_per_batch;  // output rows per sample
   int out_row_off;         // first output row of each sample
   uint16_t* out;           // STORE / SWIGLU output, GATE_RES residual (in/out)
+  float* out_f32;          // STORE_F32 output
   int ldo;                 // row stride of `out` in elements
   const float* gate;       // GATE_RES: gate of sample b at gate[b * gate_stride + col]
   int gate_stride;
@@ -82,6 +84,10 @@ cudaError_t launch_output_stage(const uint16_t* x, int rows_per_batch, int row_o
                                 const float* scale, const float* shift, int mod_stride, const uint16_t* w_out,
                                 int p, int C, float* vel, cudaStream_t s);
 cudaError_t launch_fill(float* dst, int n, float value, cudaStream_t s);
+cudaError_t launch_silu_bf16(const float* x, int n, uint16_t* y, cudaStream_t s);
+cudaError_t gemm_set_attributes();
+cudaError_t attention_set_attributes();
+cudaError_t small_kernels_set_attributes();
 cudaError_t launch_euler_cfg(float* lat, const float* v, int Bi, int64_t per_sample, float g, float sigma,
                              float sigma_next, cudaStream_t s);
 

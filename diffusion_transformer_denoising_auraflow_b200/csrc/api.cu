@@ -7,6 +7,7 @@
 // 使用指南", §前向传播流程 (embed -> joint blocks -> cat(text, image) ->
 // single blocks -> image slice -> pre-final -> proj_out -> unpatchify), with
 // the block internals of §联合注意力块 / §单 DiT 块.
+#include <array>
 #include <cstdio>
 #include <cstring>
 #include <string>
@@ -734,8 +735,13 @@ af_status af_single_block(const af_weights* w, af_scratch* s, int layer, uint16_
   return single_block_impl(w, s, layer, x, s->mods, 6 * D, B, N, st);
 }
 
+// premods != nullptr: every adaLN / pre-final modulation of this step was
+// precomputed (rows in the adaLN unit order, element (b, r) at
+// premods[b * pre_stride + r]); the timestep MLP and the modulation GEMV are
+// skipped and `t` is not read.
 static af_status forward_impl(const af_weights* w, af_scratch* s, const float* latents, const uint16_t* text_emb,
-                              const float* t, int B, int H, int W, int L, float* velocity, cudaStream_t st) {
+                              const float* t, int B, int H, int W, int L, float* velocity, cudaStream_t st,
+                              const float* premods = nullptr, int pre_stride = 0) {
   AF_TRY(check_scratch(w, s));
   if (!latents || !text_emb || !t || !velocity || B <= 0 || H <= 0 || W <= 0 || L < 0) return AF_ERR_INVALID_ARG;
   const af_config& c = w->cfg;
@@ -748,16 +754,18 @@ static af_status forward_impl(const af_weights* w, af_scratch* s, const float* l
   if (Nt <= 0) return AF_ERR_SHAPE;
   const int D = d.D;
   const size_t R_ada = w->ada_rows;
+  const float* mods = premods ? premods : s->mods;
+  const int mstride = premods ? pre_stride : static_cast<int>(R_ada);
 
   // embedding stage
-  {
+  if (!premods) {
     LaunchScope ls(s, KC_OTHER, 2.0 * D * (c.timestep_channels + D), st, 3);
     AF_CUDA(launch_timestep_mlp(t, B, w->ptr("time_step_proj.linear_1.weight"),
                                 w->ptr("time_step_proj.linear_1.bias"), w->ptr("time_step_proj.linear_2.weight"),
                                 w->ptr("time_step_proj.linear_2.bias"), c.timestep_channels, D, s->tfeat, s->h1,
                                 s->temb, st));
   }
-  {
+  if (!premods) {
     LaunchScope ls(s, KC_OTHER, 2.0 * R_ada * D, st, (B + 7) / 8);
     AF_CUDA(launch_modulation(s->temb, B, D, ada_base(w), static_cast<int>(R_ada), s->mods, st));
   }
@@ -779,9 +787,9 @@ static af_status forward_impl(const af_weights* w, af_scratch* s, const float* l
   }
   // joint blocks
   for (int i = 0; i < c.num_mmdit_layers; ++i) {
-    const float* mi = s->mods + w->unit_row[2 * i];
-    const float* mt = s->mods + w->unit_row[2 * i + 1];
-    AF_TRY(joint_block_impl(w, s, i, s->img, s->txt, mi, mt, static_cast<int>(R_ada), B, Ni, Nt, st));
+    const float* mi = mods + w->unit_row[2 * i];
+    const float* mt = mods + w->unit_row[2 * i + 1];
+    AF_TRY(joint_block_impl(w, s, i, s->img, s->txt, mi, mt, mstride, B, Ni, Nt, st));
   }
   // x = cat(text, image) per sample
   AF_CUDA(cudaMemcpy2DAsync(s->x, static_cast<size_t>(N) * D * 2, s->txt, static_cast<size_t>(Nt) * D * 2,
@@ -790,13 +798,13 @@ static af_status forward_impl(const af_weights* w, af_scratch* s, const float* l
                             static_cast<size_t>(Ni) * D * 2, static_cast<size_t>(Ni) * D * 2, B,
                             cudaMemcpyDeviceToDevice, st));
   for (int i = 0; i < c.num_single_dit_layers; ++i) {
-    const float* m = s->mods + w->unit_row[2 * c.num_mmdit_layers + i];
-    AF_TRY(single_block_impl(w, s, i, s->x, m, static_cast<int>(R_ada), B, N, st));
+    const float* m = mods + w->unit_row[2 * c.num_mmdit_layers + i];
+    AF_TRY(single_block_impl(w, s, i, s->x, m, mstride, B, N, st));
   }
   // pre-final (scale first, then shift), proj_out, unpatchify on the image rows
-  const float* pf = s->mods + w->pf_row;
+  const float* pf = mods + w->pf_row;
   LaunchScope ls(s, KC_OTHER, 2.0 * B * Ni * D + 4.0 * B * c.out_channels * H * W, st);
-  AF_CUDA(launch_output_stage(s->x, N, Nt, B, hp, wp, D, pf, pf + D, static_cast<int>(R_ada),
+  AF_CUDA(launch_output_stage(s->x, N, Nt, B, hp, wp, D, pf, pf + D, mstride,
                               w->ptr("proj_out.weight"), p, c.out_channels, velocity, st));
   return AF_OK;
 }
@@ -806,27 +814,187 @@ af_status af_transformer_forward(const af_weights* w, af_scratch* s, const float
   return forward_impl(w, s, latents, text_emb, t, B, H, W, L, velocity, static_cast<cudaStream_t>(stream));
 }
 
-af_status af_denoise_step(const af_weights* w, af_scratch* s, float* latents, const uint16_t* text_emb, int Bi, int H,
-                          int W, int L, float guidance, float sigma, float sigma_next, void* stream) {
-  AF_TRY(check_scratch(w, s));
-  if (!latents || !text_emb || Bi <= 0 || H <= 0 || W <= 0 || L < 0) return AF_ERR_INVALID_ARG;
+static af_status denoise_step_impl(const af_weights* w, af_scratch* s, float* latents, const uint16_t* text_emb,
+                                   int Bi, int H, int W, int L, float guidance, float sigma, float sigma_next,
+                                   cudaStream_t st, const float* premods = nullptr) {
   const int B = 2 * Bi;
-  const int p = w->cfg.patch_size;
-  if (H % p || W % p) return AF_ERR_SHAPE;
-  if (B > s->max_b || (H / p) * (W / p) > s->max_ni) return AF_ERR_SHAPE;
-  if (w->cfg.in_channels != w->cfg.out_channels) return AF_ERR_UNSUPPORTED;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
   const size_t per = static_cast<size_t>(w->cfg.in_channels) * H * W;
   // CFG batch [uncond; text] shares the latents
   AF_CUDA(cudaMemcpyAsync(s->lat2, latents, per * Bi * 4, cudaMemcpyDeviceToDevice, st));
   AF_CUDA(cudaMemcpyAsync(s->lat2 + per * Bi, latents, per * Bi * 4, cudaMemcpyDeviceToDevice, st));
-  {
+  if (!premods) {
     LaunchScope ls(s, KC_OTHER, 4.0 * B, st);
     AF_CUDA(launch_fill(s->tvec, B, sigma, st));
   }
-  AF_TRY(forward_impl(w, s, s->lat2, text_emb, s->tvec, B, H, W, L, s->vel, st));
+  AF_TRY(forward_impl(w, s, s->lat2, text_emb, s->tvec, B, H, W, L, s->vel, st, premods, 0));
   LaunchScope ls(s, KC_OTHER, 16.0 * per * Bi, st);
   AF_CUDA(launch_euler_cfg(latents, s->vel, Bi, static_cast<int64_t>(per), guidance, sigma, sigma_next, st));
+  return AF_OK;
+}
+
+static af_status check_step_args(const af_weights* w, af_scratch* s, const float* latents, const uint16_t* text_emb,
+                                 int Bi, int H, int W, int L) {
+  AF_TRY(check_scratch(w, s));
+  if (!latents || !text_emb || Bi <= 0 || H <= 0 || W <= 0 || L < 0) return AF_ERR_INVALID_ARG;
+  const int p = w->cfg.patch_size;
+  if (H % p || W % p || H / p > w->d.G || W / p > w->d.G) return AF_ERR_SHAPE;
+  if (2 * Bi > s->max_b || (H / p) * (W / p) > s->max_ni || L > s->max_l) return AF_ERR_SHAPE;
+  if (w->cfg.in_channels != w->cfg.out_channels) return AF_ERR_UNSUPPORTED;
+  return AF_OK;
+}
+
+af_status af_denoise_step(const af_weights* w, af_scratch* s, float* latents, const uint16_t* text_emb, int Bi, int H,
+                          int W, int L, float guidance, float sigma, float sigma_next, void* stream) {
+  AF_TRY(check_step_args(w, s, latents, text_emb, Bi, H, W, L));
+  return denoise_step_impl(w, s, latents, text_emb, Bi, H, W, L, guidance, sigma, sigma_next,
+                           static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------- sampler
+struct af_sampler {
+  const af_weights* w = nullptr;
+  af_scratch* s = nullptr;
+  float* latents = nullptr;
+  const uint16_t* text = nullptr;
+  int Bi = 0, H = 0, W = 0, L = 0, n_steps = 0;
+  float guidance = 1.f;
+  bool use_graphs = false;
+  std::vector<float> sigmas;  // n_steps + 1
+  uint8_t* base = nullptr;
+  float *t_dev = nullptr, *feat = nullptr, *h1 = nullptr, *temb = nullptr, *mods = nullptr;
+  uint16_t* silu = nullptr;
+  std::vector<cudaGraphExec_t> graphs;
+  std::vector<std::array<int64_t, AF_NUM_KERNEL_CLASSES>> graph_launches;
+};
+
+extern "C" {
+
+af_status af_sampler_create(const af_weights* w, af_scratch* s, float* latents, const uint16_t* text_emb, int Bi,
+                            int H, int W, int L, int n_steps, const float* sigmas, float guidance, int use_graphs,
+                            af_sampler** out) {
+  if (!out) return AF_ERR_INVALID_ARG;
+  *out = nullptr;
+  AF_TRY(check_step_args(w, s, latents, text_emb, Bi, H, W, L));
+  if (n_steps <= 0 || !sigmas) return AF_ERR_INVALID_ARG;
+  af_sampler* m = new af_sampler();
+  m->w = w;
+  m->s = s;
+  m->latents = latents;
+  m->text = text_emb;
+  m->Bi = Bi;
+  m->H = H;
+  m->W = W;
+  m->L = L;
+  m->n_steps = n_steps;
+  m->guidance = guidance;
+  m->use_graphs = use_graphs != 0;
+  m->sigmas.assign(sigmas, sigmas + n_steps + 1);
+  const size_t n = n_steps, D = w->d.D, C = w->cfg.timestep_channels;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = (off + bytes + 255) & ~size_t(255);
+    return o;
+  };
+  const size_t o_t = take(n * 4), o_f = take(n * C * 4), o_h = take(n * D * 4), o_e = take(n * D * 4);
+  const size_t o_s = take(n * D * 2), o_m = take(n * w->ada_rows * 4);
+  int prev = 0;
+  cudaGetDevice(&prev);
+  cudaSetDevice(w->device);
+  cudaError_t e = cudaMalloc(&m->base, off);
+  if (e == cudaSuccess) e = cudaMemcpy(m->base + o_t, sigmas, n * 4, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) e = gemm_set_attributes();
+  if (e == cudaSuccess) e = attention_set_attributes();
+  if (e == cudaSuccess) e = small_kernels_set_attributes();
+  cudaSetDevice(prev);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    if (m->base) cudaFree(m->base);
+    delete m;
+    return e == cudaErrorMemoryAllocation ? AF_ERR_OOM : cuda_fail(e);
+  }
+  m->t_dev = reinterpret_cast<float*>(m->base + o_t);
+  m->feat = reinterpret_cast<float*>(m->base + o_f);
+  m->h1 = reinterpret_cast<float*>(m->base + o_h);
+  m->temb = reinterpret_cast<float*>(m->base + o_e);
+  m->silu = reinterpret_cast<uint16_t*>(m->base + o_s);
+  m->mods = reinterpret_cast<float*>(m->base + o_m);
+  m->graphs.assign(n, nullptr);
+  m->graph_launches.assign(n, std::array<int64_t, AF_NUM_KERNEL_CLASSES>{0, 0, 0, 0});
+  *out = m;
+  return AF_OK;
+}
+
+void af_sampler_destroy(af_sampler* m) {
+  if (!m) return;
+  for (cudaGraphExec_t g : m->graphs)
+    if (g) cudaGraphExecDestroy(g);
+  if (m->base) cudaFree(m->base);
+  delete m;
+}
+
+af_status af_sampler_prepare(af_sampler* m, void* stream) {
+  if (!m) return AF_ERR_INVALID_ARG;
+  const af_weights* w = m->w;
+  af_scratch* s = m->s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int n = m->n_steps, D = w->d.D, C = w->cfg.timestep_channels;
+  {
+    LaunchScope ls(s, KC_OTHER, 2.0 * D * (C + D), st, 2 * ((n + 7) / 8) + 1);
+    AF_CUDA(launch_timestep_mlp(m->t_dev, n, w->ptr("time_step_proj.linear_1.weight"),
+                                w->ptr("time_step_proj.linear_1.bias"), w->ptr("time_step_proj.linear_2.weight"),
+                                w->ptr("time_step_proj.linear_2.bias"), C, D, m->feat, m->h1, m->temb, st));
+  }
+  {
+    LaunchScope ls(s, KC_OTHER, 6.0 * n * D, st);
+    AF_CUDA(launch_silu_bf16(m->temb, n * D, m->silu, st));
+  }
+  // every modulation of every step: mods[i, r] = W_ada[r] . silu(temb_i), one weight pass
+  GemmParams gp = gemm_base(s, n, static_cast<int>(w->ada_rows), D, EPI_STORE_F32, n);
+  gp.out_f32 = m->mods;
+  gp.ldo = static_cast<int>(w->ada_rows);
+  return run_gemm(s, gp, m->silu, ada_base(w), static_cast<int>(w->ada_rows), st);
+}
+
+af_status af_sampler_step(af_sampler* m, int step, void* stream) {
+  if (!m || step < 0 || step >= m->n_steps) return AF_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const float* premods = m->mods + static_cast<size_t>(step) * m->w->ada_rows;
+  auto enqueue = [&]() {
+    return denoise_step_impl(m->w, m->s, m->latents, m->text, m->Bi, m->H, m->W, m->L, m->guidance,
+                             m->sigmas[step], m->sigmas[step + 1], st, premods);
+  };
+  if (!m->use_graphs) return enqueue();
+  if (!st) return AF_ERR_INVALID_ARG;  // the legacy default stream cannot be captured
+  if (!m->graphs[step]) {
+    int64_t before[AF_NUM_KERNEL_CLASSES];
+    for (int i = 0; i < AF_NUM_KERNEL_CLASSES; ++i) before[i] = m->s->launches[i];
+    const bool prof = m->s->profiling;
+    m->s->profiling = false;  // no event records inside a graph
+    AF_CUDA(cudaStreamBeginCapture(st, cudaStreamCaptureModeThreadLocal));
+    const af_status qs = enqueue();
+    cudaGraph_t g = nullptr;
+    const cudaError_t ce = cudaStreamEndCapture(st, &g);
+    m->s->profiling = prof;
+    for (int i = 0; i < AF_NUM_KERNEL_CLASSES; ++i) {
+      m->graph_launches[step][i] = m->s->launches[i] - before[i];
+      m->s->launches[i] = before[i];
+    }
+    if (qs != AF_OK) {
+      if (g) cudaGraphDestroy(g);
+      return qs;
+    }
+    AF_CUDA(ce);
+    cudaGraphExec_t exec = nullptr;
+    const cudaError_t ie = cudaGraphInstantiate(&exec, g, 0);
+    cudaGraphDestroy(g);
+    AF_CUDA(ie);
+    m->graphs[step] = exec;
+  }
+  AF_CUDA(cudaGraphLaunch(m->graphs[step], st));
+  for (int i = 0; i < AF_NUM_KERNEL_CLASSES; ++i) m->s->launches[i] += m->graph_launches[step][i];
   return AF_OK;
 }
 

@@ -969,6 +969,21 @@ __global__ void attn_small_simt(const uint16_t* __restrict__ q, const uint16_t* 
   for (int d = 0; d < HD; ++d) dst[d] = static_cast<uint16_t>(pack_bf16(o[d] / l, 0.f) & 0xFFFFu);
 }
 
+cudaError_t attention_set_attributes() {
+  static uint64_t done = 0;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if ((done >> dev) & 1u) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(attn_hd256_online, cudaFuncAttributeMaxDynamicSharedMemorySize, AT_SMEM);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(attn_hd256_qknorm, cudaFuncAttributeMaxDynamicSharedMemorySize, QKN_SMEM);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(attn_hd256_qknorm_pair, cudaFuncAttributeMaxDynamicSharedMemorySize, AP_SMEM);
+  if (e != cudaSuccess) return e;
+  done |= uint64_t(1) << dev;
+  return cudaSuccess;
+}
+
 cudaError_t launch_attention(const AttnParams& p, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                              cudaStream_t stream) {
   if (p.N <= 0 || p.B <= 0 || p.H <= 0) return cudaSuccess;
@@ -979,15 +994,9 @@ cudaError_t launch_attention(const AttnParams& p, const uint16_t* q, const uint1
     if (!encode_tmap_3d(&tq, q, AT_HD, p.N, bh, rb, sb, 64, AT_BM, 1)) return cudaErrorInvalidValue;
     if (!encode_tmap_3d(&tk, k, AT_HD, p.N, bh, rb, sb, 64, AT_BN, 1)) return cudaErrorInvalidValue;
     if (!encode_tmap_3d(&tv, v, AT_HD, p.N, bh, rb, sb, 64, AT_BN, 1)) return cudaErrorInvalidValue;
-    static bool attr = false;
-    if (!attr) {
-      cudaError_t e = cudaFuncSetAttribute(attn_hd256_online, cudaFuncAttributeMaxDynamicSharedMemorySize, AT_SMEM);
+    {
+      cudaError_t e = attention_set_attributes();
       if (e != cudaSuccess) return e;
-      e = cudaFuncSetAttribute(attn_hd256_qknorm, cudaFuncAttributeMaxDynamicSharedMemorySize, QKN_SMEM);
-      if (e != cudaSuccess) return e;
-      e = cudaFuncSetAttribute(attn_hd256_qknorm_pair, cudaFuncAttributeMaxDynamicSharedMemorySize, AP_SMEM);
-      if (e != cudaSuccess) return e;
-      attr = true;
     }
     if (p.qk_normalized && p.N >= 256) {
       CUtensorMap tv2;  // V halves: 128 keys x 64 columns per box

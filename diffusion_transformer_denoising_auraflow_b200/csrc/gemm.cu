@@ -246,8 +246,19 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tbas
 #pragma unroll
       for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(ra[j]);
       if (!row_ok) continue;
-      uint16_t* dst = p.out + orow * p.ldo + col;
       const int n = min(32, p.N - col);
+      if (p.mode == EPI_STORE_F32) {
+        float* df = p.out_f32 + orow * p.ldo + col;
+        if (n == 32) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            reinterpret_cast<float4*>(df)[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+        } else {
+          for (int j = 0; j < n; ++j) df[j] = v[j];
+        }
+        continue;
+      }
+      uint16_t* dst = p.out + orow * p.ldo + col;
       if (p.mode == EPI_GATE_RES) {
         const float* g = p.gate + static_cast<size_t>(b) * p.gate_stride + col;
         if (n == 32) {
@@ -595,6 +606,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
 
 // ----------------------------------------------------------------- host launch
 
+// Opt the kernels into their dynamic shared memory, once per device (a plain
+// host call, never made while a stream is being captured after this ran).
+cudaError_t gemm_set_attributes() {
+  static uint64_t done = 0;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if ((done >> dev) & 1u) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(gemm_bf16_tcgen05, cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM_SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(gemm_bf16_tcgen05_pair, cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM2_SMEM);
+  if (e != cudaSuccess) return e;
+  done |= uint64_t(1) << dev;
+  return cudaSuccess;
+}
+
 cudaError_t launch_gemm(const GemmParams& p_in, const void* A, const void* W, int W_rows, cudaStream_t stream,
                         int num_sms) {
   GemmParams p = p_in;
@@ -605,14 +631,9 @@ cudaError_t launch_gemm(const GemmParams& p_in, const void* A, const void* W, in
   const bool pair = p.M >= 1024 && num_sms >= 2;
   if (!encode_tmap_2d(&tb, W, p.K, W_rows, static_cast<uint64_t>(p.K) * 2, GEMM_BK, pair ? 128 : GEMM_BN))
     return cudaErrorInvalidValue;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_bf16_tcgen05, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         GEMM_SMEM_BYTES);
+  {
+    cudaError_t e = gemm_set_attributes();
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(gemm_bf16_tcgen05_pair, cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM2_SMEM);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
   }
   p.num_n_tiles = p.mode == EPI_SWIGLU ? (p.N + 127) / 128 : (p.N + GEMM_BN - 1) / GEMM_BN;
   p.group_n = p.num_n_tiles < 16 ? p.num_n_tiles : 16;

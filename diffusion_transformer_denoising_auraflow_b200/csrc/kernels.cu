@@ -95,10 +95,94 @@ __global__ void __launch_bounds__(256) ln_modulate_kernel(const uint16_t* __rest
   }
 }
 
+// Wide-row variant (D = 3072): a CTA serves rows of one sample; (1 + scale)
+// and shift are staged once in shared memory (instead of every row re-reading
+// 24 KB of them from L2 after its reduction); each warp walks
+// LN_ROWS_PER_WARP rows, keeping the row packed as bf16 pairs in registers.
+constexpr int LN_ROWS_PER_WARP = 2;
+constexpr int LN_WARPS = 8;
+
+template <int VPL>
+__global__ void __launch_bounds__(256) ln_modulate_rows_kernel(const uint16_t* __restrict__ x,
+                                                               const float* __restrict__ shift,
+                                                               const float* __restrict__ scale, int mod_stride,
+                                                               uint16_t* __restrict__ y, int rows_per_batch, int D,
+                                                               float eps) {
+  extern __shared__ float mod_s[];  // [0, D): 1 + scale, [D, 2D): shift
+  const int b = blockIdx.y;
+  const float* sc = scale + static_cast<size_t>(b) * mod_stride;
+  const float* sh = shift + static_cast<size_t>(b) * mod_stride;
+  for (int i = threadIdx.x; i < D; i += blockDim.x) {
+    mod_s[i] = 1.0f + sc[i];
+    mod_s[D + i] = sh[i];
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r0 = (blockIdx.x * LN_WARPS + warp) * LN_ROWS_PER_WARP;
+  const size_t base = static_cast<size_t>(b) * rows_per_batch;
+  for (int k = 0; k < LN_ROWS_PER_WARP; ++k) {
+    const int r = r0 + k;
+    if (r >= rows_per_batch) break;  // uniform across the warp
+    uint4 cur[VPL];
+    const uint4* xr = reinterpret_cast<const uint4*>(x + (base + r) * D);
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) cur[i] = xr[i * 32 + lane];
+    // rows stay packed as bf16 pairs; each pass unpacks on the fly
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const uint32_t w[4] = {cur[i].x, cur[i].y, cur[i].z, cur[i].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) s += bf16_lo(w[e]) + bf16_hi(w[e]);
+    }
+    const float mean = warp_sum(s) / D;
+    float ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const uint32_t w[4] = {cur[i].x, cur[i].y, cur[i].z, cur[i].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float d0 = bf16_lo(w[e]) - mean, d1 = bf16_hi(w[e]) - mean;
+        ss += d0 * d0 + d1 * d1;
+      }
+    }
+    const float rstd = rsqrtf(warp_sum(ss) / D + eps);
+    uint4* yr = reinterpret_cast<uint4*>(y + (base + r) * D);
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const int vi = i * 32 + lane;
+      const float4 a0 = *reinterpret_cast<const float4*>(mod_s + vi * 8);
+      const float4 a1 = *reinterpret_cast<const float4*>(mod_s + vi * 8 + 4);
+      const float4 h0 = *reinterpret_cast<const float4*>(mod_s + D + vi * 8);
+      const float4 h1 = *reinterpret_cast<const float4*>(mod_s + D + vi * 8 + 4);
+      const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float hv[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+      const uint32_t w[4] = {cur[i].x, cur[i].y, cur[i].z, cur[i].w};
+      uint32_t o[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        o[e] = pack_bf16((bf16_lo(w[e]) - mean) * rstd * av[2 * e] + hv[2 * e],
+                         (bf16_hi(w[e]) - mean) * rstd * av[2 * e + 1] + hv[2 * e + 1]);
+      yr[vi] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+  }
+}
+
 cudaError_t launch_ln_modulate(const uint16_t* x, const float* shift, const float* scale, int mod_stride,
                                uint16_t* y, int rows, int rows_per_batch, int D, float eps, cudaStream_t s) {
   if (rows <= 0) return cudaSuccess;
   if (D % 8 != 0) return cudaErrorInvalidValue;
+  if (D == 3072 && rows % rows_per_batch == 0) {
+    cudaError_t e = small_kernels_set_attributes();
+    if (e != cudaSuccess) return e;
+    const int nb = rows / rows_per_batch;
+    const int rows_per_block = LN_WARPS * LN_ROWS_PER_WARP;
+    dim3 grid((rows_per_batch + rows_per_block - 1) / rows_per_block, nb);
+    const size_t smem = 2 * static_cast<size_t>(D) * sizeof(float);
+    ln_modulate_rows_kernel<12><<<grid, 32 * LN_WARPS, smem, s>>>(x, shift, scale, mod_stride, y, rows_per_batch, D,
+                                                                  eps);
+    return cudaGetLastError();
+  }
   const int nvec = D / 8;
   const int vpl = (nvec + 31) / 32;
   const int blocks = (rows + 7) / 8;
@@ -175,14 +259,36 @@ __global__ void __launch_bounds__(256) gemv_rows_kernel(const float* __restrict_
 }
 
 template <int VPL>
+static cudaError_t gemv_attr() {
+  return cudaFuncSetAttribute(gemv_rows_kernel<VPL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              GEMV_MAX_B * VPL * 256 * static_cast<int>(sizeof(float)));
+}
+
+// Shared-memory opt-ins of this file's kernels, once per device.
+cudaError_t small_kernels_set_attributes() {
+  static uint64_t done = 0;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if ((done >> dev) & 1u) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(ln_modulate_rows_kernel<12>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       2 * 3072 * static_cast<int>(sizeof(float)));
+  if (e == cudaSuccess) e = gemv_attr<1>();
+  if (e == cudaSuccess) e = gemv_attr<2>();
+  if (e == cudaSuccess) e = gemv_attr<4>();
+  if (e == cudaSuccess) e = gemv_attr<8>();
+  if (e == cudaSuccess) e = gemv_attr<12>();
+  if (e == cudaSuccess) e = gemv_attr<16>();
+  if (e != cudaSuccess) return e;
+  done |= uint64_t(1) << dev;
+  return cudaSuccess;
+}
+
+template <int VPL>
 static cudaError_t gemv_launch(const float* x, int nb, int K, const uint16_t* W, const uint16_t* bias, int rows,
                                int pre, int post, float* out, int out_stride, cudaStream_t s, int blocks) {
   const size_t smem = static_cast<size_t>(nb) * K * sizeof(float);
-  if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(gemv_rows_kernel<VPL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-  }
+  cudaError_t e = small_kernels_set_attributes();
+  if (e != cudaSuccess) return e;
   gemv_rows_kernel<VPL><<<blocks, 256, smem, s>>>(x, nb, K, W, bias, rows, pre, post, out, out_stride);
   return cudaGetLastError();
 }
@@ -457,6 +563,20 @@ __global__ void fill_kernel(float* __restrict__ dst, int n, float value) {
 
 cudaError_t launch_fill(float* dst, int n, float value, cudaStream_t s) {
   fill_kernel<<<(n + 255) / 256, 256, 0, s>>>(dst, n, value);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ SiLU, fp32 -> bf16 (GEMM operand)
+__global__ void silu_bf16_kernel(const float* __restrict__ x, int n, uint16_t* __restrict__ y) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) {
+    const float a = x[i];
+    y[i] = static_cast<uint16_t>(pack_bf16(a / (1.0f + __expf(-a)), 0.f) & 0xFFFFu);
+  }
+}
+
+cudaError_t launch_silu_bf16(const float* x, int n, uint16_t* y, cudaStream_t s) {
+  silu_bf16_kernel<<<(n + 255) / 256, 256, 0, s>>>(x, n, y);
   return cudaGetLastError();
 }
 

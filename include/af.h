@@ -215,6 +215,29 @@ af_status af_euler_cfg_step(float* latents, const float* velocity, int Bi, int C
 af_status af_denoise_step(const af_weights* w, af_scratch* s, float* latents, const uint16_t* text_emb, int Bi,
                           int H, int W, int L, float guidance, float sigma, float sigma_next, void* stream);
 
+/* ---- the sampling loop -----------------------------------------------------
+ * The pipeline's denoising loop ([ARCH] §在 AuraFlowPipeline 中的实际调用,
+ * [DEEP] §2.3: 25 flow-match Euler steps with CFG) as a reusable plan.  Every
+ * adaLN-Zero and pre-final modulation depends only on the step's sigma, so
+ * af_sampler_prepare computes them for all steps at once (one tensor-core
+ * GEMM reading the modulation weights once); af_sampler_step then runs step
+ * i exactly like af_denoise_step(sigma_i -> sigma_{i+1}) with those values.
+ * With use_graphs != 0 each step is captured into a CUDA graph on first use
+ * and replayed afterwards (needs a non-NULL stream; nothing may be captured
+ * on the stream around these calls).
+ *   latents:  device float[Bi, C, H, W], updated in place by every step
+ *   text_emb: device bf16[2 Bi, L, joint_attention_dim] (uncond rows first)
+ *   sigmas:   host float[n_steps + 1] (e.g. from af_sigma_schedule)
+ * Both device buffers are bound to the sampler: change their contents, not
+ * their addresses.  The scratch must fit a 2 Bi batch of this size. */
+typedef struct af_sampler af_sampler;
+af_status af_sampler_create(const af_weights* w, af_scratch* s, float* latents, const uint16_t* text_emb, int Bi,
+                            int H, int W, int L, int n_steps, const float* sigmas, float guidance, int use_graphs,
+                            af_sampler** out);
+af_status af_sampler_prepare(af_sampler* smp, void* stream);
+af_status af_sampler_step(af_sampler* smp, int step, void* stream);
+void af_sampler_destroy(af_sampler* smp);
+
 /* Host-side sigma schedule of the flow-match Euler sampler ([DEEP] §2.3:
  * num_train_timesteps 1000, shift 1.73, 25 steps): n_steps + 1 values
  * sigma_i = k s_i / (1 + (k - 1) s_i) with s = linspace(1, 1/num_train,
