@@ -319,21 +319,43 @@ def merge_heads(x):
     return x.transpose(0, 2, 1, 3).reshape(B, N, H * hd)
 
 
-def attention(q, k, v, scale=None):
-    """softmax(q k^T * scale) v per (batch, head); non-causal, no mask, no dropout.
+def attention(q, k, v, scale=None, key_mask=None):
+    """softmax(q k^T * scale) v per (batch, head); non-causal, no dropout.
 
     [ARCH §注意力处理器与 QKV 融合]: F.scaled_dot_product_attention with
     dropout_p 0, is_causal False and an explicit scale.  READING: scale is
     head_dim^-1/2.  q, k, v: [B, H, N, hd].
+
+    key_mask: optional bool [B, N_k], False = the key takes no part (its
+    logit is -inf), like a boolean SDPA attn_mask broadcast over heads and
+    queries.  The model's forward takes no mask ([ARCH §前向传播流程]); this
+    is the padded-prompt extension (the pipeline pads prompts to a common
+    length and builds an attention mask, [PIPE §AuraFlowPipeline 核心参数详解],
+    [ARCH §在 AuraFlowPipeline 中的实际调用]).
     """
     q, k, v = _f(q), _f(k), _f(v)
     if scale is None:
         scale = 1.0 / math.sqrt(q.shape[-1])
     s = (q @ np.swapaxes(k, -1, -2)) * scale
+    if key_mask is not None:
+        s = np.where(np.asarray(key_mask, bool)[:, None, None, :], s, -np.inf)
     s = s - s.max(axis=-1, keepdims=True)
     p = np.exp(s)
     p = p / p.sum(axis=-1, keepdims=True)
     return p @ v
+
+
+def text_key_mask(text_len, n_registers: int, L: int, n_image: int):
+    """Key mask [B, R + L + Ni] of the sequence [registers; text; image] when
+    sample b's prompt has text_len[b] real tokens and L - text_len[b] padding
+    tokens at its end.  Registers and image tokens are always attended.
+    (Padded-prompt extension; see ``attention``.)"""
+    tl = np.asarray(text_len, dtype=np.int64)
+    B = tl.shape[0]
+    m = np.ones((B, n_registers + L + n_image), dtype=bool)
+    for b in range(B):
+        m[b, n_registers + tl[b]:n_registers + L] = False
+    return m
 
 
 def qkv_normed(y, wq, wk, wv, heads: int, eps: float):
@@ -361,7 +383,7 @@ def feed_forward(y, w1, w2, w3):
 # c10. Blocks
 # --------------------------------------------------------------------------
 
-def single_block_mod(x, mod, w, prefix, heads, eps):
+def single_block_mod(x, mod, w, prefix, heads, eps, key_mask=None):
     """AuraFlowSingleTransformerBlock given its six modulation vectors.
 
     [ARCH §单 DiT 块]: adaLN-Zero DiT block on one (concatenated) sequence,
@@ -374,7 +396,7 @@ def single_block_mod(x, mod, w, prefix, heads, eps):
     y = modulate(x, mod["shift_msa"], mod["scale_msa"], eps)
     q, k, v = qkv_normed(y, w[prefix + "attn.to_q.weight"], w[prefix + "attn.to_k.weight"],
                          w[prefix + "attn.to_v.weight"], heads, eps)
-    o = merge_heads(attention(q, k, v))
+    o = merge_heads(attention(q, k, v, key_mask=key_mask))
     x = x + mod["gate_msa"][:, None, :] * (o @ _f(w[prefix + "attn.to_out.0.weight"]).T)
     y = modulate(x, mod["shift_mlp"], mod["scale_mlp"], eps)
     f = feed_forward(y, w[prefix + "ff.linear_1.weight"], w[prefix + "ff.linear_2.weight"],
@@ -382,12 +404,12 @@ def single_block_mod(x, mod, w, prefix, heads, eps):
     return x + mod["gate_mlp"][:, None, :] * f
 
 
-def single_block(x, temb, w, prefix, cfg: Config):
+def single_block(x, temb, w, prefix, cfg: Config, key_mask=None):
     mod = ada_ln_zero(temb, w[prefix + "norm1.linear.weight"])
-    return single_block_mod(x, mod, w, prefix, cfg.num_attention_heads, cfg.ln_eps)
+    return single_block_mod(x, mod, w, prefix, cfg.num_attention_heads, cfg.ln_eps, key_mask)
 
 
-def joint_block_mod(img, txt, mod_i, mod_t, w, prefix, heads, eps):
+def joint_block_mod(img, txt, mod_i, mod_t, w, prefix, heads, eps, key_mask=None):
     """AuraFlowJointTransformerBlock given both streams' modulation vectors.
 
     [ARCH §联合注意力块]: two residual streams (image, text), each with its
@@ -410,7 +432,7 @@ def joint_block_mod(img, txt, mod_i, mod_t, w, prefix, heads, eps):
     q = np.concatenate([qt, qi], axis=2)
     k = np.concatenate([kt, ki], axis=2)
     v = np.concatenate([vt, vi], axis=2)
-    o = merge_heads(attention(q, k, v))
+    o = merge_heads(attention(q, k, v, key_mask=key_mask))
     ot, oi = o[:, :nt], o[:, nt:]
     img = img + mod_i["gate_msa"][:, None, :] * (oi @ _f(w[prefix + "attn.to_out.0.weight"]).T)
     txt = txt + mod_t["gate_msa"][:, None, :] * (ot @ _f(w[prefix + "attn.to_add_out.weight"]).T)
@@ -425,17 +447,17 @@ def joint_block_mod(img, txt, mod_i, mod_t, w, prefix, heads, eps):
     return txt, img
 
 
-def joint_block(img, txt, temb, w, prefix, cfg: Config):
+def joint_block(img, txt, temb, w, prefix, cfg: Config, key_mask=None):
     mod_i = ada_ln_zero(temb, w[prefix + "norm1.linear.weight"])
     mod_t = ada_ln_zero(temb, w[prefix + "norm1_context.linear.weight"])
-    return joint_block_mod(img, txt, mod_i, mod_t, w, prefix, cfg.num_attention_heads, cfg.ln_eps)
+    return joint_block_mod(img, txt, mod_i, mod_t, w, prefix, cfg.num_attention_heads, cfg.ln_eps, key_mask)
 
 
 # --------------------------------------------------------------------------
 # Sampled-row evaluation of a block (same definition, fewer outputs)
 # --------------------------------------------------------------------------
 
-def single_block_rows(x, temb, w, prefix, cfg: Config, rows):
+def single_block_rows(x, temb, w, prefix, cfg: Config, rows, key_mask=None):
     """Rows ``rows`` (indices into the sequence) of single_block's output.
 
     Same formula as ``single_block``: K and V need every token, while the
@@ -450,7 +472,7 @@ def single_block_rows(x, temb, w, prefix, cfg: Config, rows):
     v = split_heads(y @ _f(w[prefix + "attn.to_v.weight"]).T, heads)
     yr = y[:, rows]
     q = layer_norm(split_heads(yr @ _f(w[prefix + "attn.to_q.weight"]).T, heads), eps)
-    o = merge_heads(attention(q, k, v))
+    o = merge_heads(attention(q, k, v, key_mask=key_mask))
     xr = x[:, rows] + mod["gate_msa"][:, None, :] * (o @ _f(w[prefix + "attn.to_out.0.weight"]).T)
     y2 = modulate(xr, mod["shift_mlp"], mod["scale_mlp"], eps)
     f = feed_forward(y2, w[prefix + "ff.linear_1.weight"], w[prefix + "ff.linear_2.weight"],
@@ -458,7 +480,7 @@ def single_block_rows(x, temb, w, prefix, cfg: Config, rows):
     return xr + mod["gate_mlp"][:, None, :] * f
 
 
-def joint_block_rows(img, txt, temb, w, prefix, cfg: Config, img_rows, txt_rows):
+def joint_block_rows(img, txt, temb, w, prefix, cfg: Config, img_rows, txt_rows, key_mask=None):
     """Rows of joint_block's outputs: (txt[:, txt_rows], img[:, img_rows])."""
     img, txt = _f(img), _f(txt)
     heads, eps = cfg.num_attention_heads, cfg.ln_eps
@@ -477,8 +499,8 @@ def joint_block_rows(img, txt, temb, w, prefix, cfg: Config, img_rows, txt_rows)
     v = np.concatenate([vt, vi], axis=2)
     qi = layer_norm(split_heads(yi[:, img_rows] @ _f(w[prefix + "attn.to_q.weight"]).T, heads), eps)
     qt = layer_norm(split_heads(yt[:, txt_rows] @ _f(w[prefix + "attn.add_q_proj.weight"]).T, heads), eps)
-    oi = merge_heads(attention(qi, k, v))
-    ot = merge_heads(attention(qt, k, v))
+    oi = merge_heads(attention(qi, k, v, key_mask=key_mask))
+    ot = merge_heads(attention(qt, k, v, key_mask=key_mask))
     xi = img[:, img_rows] + mi["gate_msa"][:, None, :] * (oi @ _f(w[prefix + "attn.to_out.0.weight"]).T)
     xt = txt[:, txt_rows] + mt["gate_msa"][:, None, :] * (ot @ _f(w[prefix + "attn.to_add_out.weight"]).T)
     y2i = modulate(xi, mi["shift_mlp"], mi["scale_mlp"], eps)
@@ -539,23 +561,28 @@ def output_stage(x_img, temb, w, cfg: Config, H: int, W: int):
     return unpatchify(o, p, cfg.out_channels, H // p, W // p)
 
 
-def transformer_forward(latents, text_emb, t, w, cfg: Config):
+def transformer_forward(latents, text_emb, t, w, cfg: Config, text_len=None):
     """AuraFlowTransformer2DModel.forward -> velocity [B, C_out, H, W].
 
     [ARCH §前向传播流程]: embed; num_mmdit_layers joint blocks updating both
     streams; cat(text, image); num_single_dit_layers single blocks; keep the
     image part combined[:, encoder_seq_len:]; pre-final; proj_out;
     unpatchify.  ``t`` is the model time in [0, 1] (timestep / 1000).
+    ``text_len`` (optional, [B]): real prompt tokens per sample; the rest of
+    the L text tokens are padding that no attention reads (``text_key_mask``).
     """
     latents = _f(latents)
     H, W = latents.shape[2], latents.shape[3]
     img, txt, temb = embed(latents, text_emb, t, w, cfg)
-    for i in range(cfg.num_mmdit_layers):
-        txt, img = joint_block(img, txt, temb, w, f"joint_transformer_blocks.{i}.", cfg)
     nt = txt.shape[1]
+    mask = None
+    if text_len is not None:
+        mask = text_key_mask(text_len, cfg.num_register_tokens, nt - cfg.num_register_tokens, img.shape[1])
+    for i in range(cfg.num_mmdit_layers):
+        txt, img = joint_block(img, txt, temb, w, f"joint_transformer_blocks.{i}.", cfg, mask)
     x = np.concatenate([txt, img], axis=1)
     for i in range(cfg.num_single_dit_layers):
-        x = single_block(x, temb, w, f"single_transformer_blocks.{i}.", cfg)
+        x = single_block(x, temb, w, f"single_transformer_blocks.{i}.", cfg, mask)
     return output_stage(x[:, nt:], temb, w, cfg, H, W)
 
 
