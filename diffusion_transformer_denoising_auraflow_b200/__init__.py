@@ -69,13 +69,13 @@ _SIGS = {
     "af_timestep_embed": [_P, _P, _P, _I, _P, _P],
     "af_timestep_embed_noalloc": [_P, _P, _I, _P, _P],
     "af_patch_embed": [_P, _P, _P, _I, _I, _I, _P, _P],
-    "af_joint_block": [_P, _P, _I, _P, _P, _P, _I, _I, _I, _P],
-    "af_single_block": [_P, _P, _I, _P, _P, _I, _I, _P],
-    "af_transformer_forward": [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P],
+    "af_joint_block": [_P, _P, _I, _P, _P, _P, _I, _I, _I, _P, _P],
+    "af_single_block": [_P, _P, _I, _P, _P, _I, _I, _I, _P, _P],
+    "af_transformer_forward": [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P],
     "af_euler_cfg_step": [_P, _P, _I, _I, _I, _I, _F, _F, _F, _P],
-    "af_denoise_step": [_P, _P, _P, _P, _I, _I, _I, _I, _F, _F, _F, _P],
+    "af_denoise_step": [_P, _P, _P, _P, _I, _I, _I, _I, _P, _F, _F, _F, _P],
     "af_sigma_schedule": [_I, _F, _I, _P],
-    "af_sampler_create": [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _F, _I, _P],
+    "af_sampler_create": [_P, _P, _P, _P, _I, _I, _I, _I, _P, _I, _P, _F, _I, _P],
     "af_sampler_prepare": [_P, _P],
     "af_sampler_step": [_P, _I, _P],
     "af_sampler_destroy": [_P],
@@ -84,7 +84,7 @@ _SIGS = {
     "af_profile_end": [_P, _P, _P, _P, _P],
     "af_ln_modulate": [_P, _P, _P, _I, _P, _I, _I, _I, _F, _P],
     "af_linear": [_P, _P, _P, _I, _I, _I, _P],
-    "af_attention": [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P],
+    "af_attention": [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _I, _I, _P],
     "af_status_string": [_I],
     "af_last_error": [],
 }
@@ -125,6 +125,15 @@ def _stream(stream):
     if isinstance(stream, torch.cuda.Stream):
         return ctypes.c_void_p(stream.cuda_stream)
     return ctypes.c_void_p(int(stream))
+
+
+def _lens(t, n: int, name: str):
+    """Optional per-sample lengths: None, or a CUDA int32 tensor of n entries."""
+    if t is None:
+        return ctypes.c_void_p(0)
+    if t.dim() != 1 or t.shape[0] != n:
+        raise ValueError(f"{name} must hold {n} entries")
+    return _dev(t, torch.int32, name)
 
 
 def _dev(t: torch.Tensor, dtype, name: str):
@@ -251,26 +260,30 @@ def patch_embed(w: Weights, s: Scratch, latents, img, stream=None):
                               _dev(img, torch.bfloat16, "img"), _stream(stream)), "af_patch_embed")
 
 
-def joint_block(w: Weights, s: Scratch, layer: int, img, txt, temb, stream=None):
+def joint_block(w: Weights, s: Scratch, layer: int, img, txt, temb, text_len=None, stream=None):
+    """text_len: optional CUDA int32 [B], real prompt tokens (padded prompts)."""
     B, Ni, _ = img.shape
     Nt = txt.shape[1]
     _check(lib.af_joint_block(w.handle, s.handle, layer, _dev(img, torch.bfloat16, "img"),
                               _dev(txt, torch.bfloat16, "txt"), _dev(temb, torch.float32, "temb"),
-                              B, Ni, Nt, _stream(stream)), "af_joint_block")
+                              B, Ni, Nt, _lens(text_len, B, "text_len"), _stream(stream)), "af_joint_block")
 
 
-def single_block(w: Weights, s: Scratch, layer: int, x, temb, stream=None):
+def single_block(w: Weights, s: Scratch, layer: int, x, temb, n_text: int = 0, text_len=None, stream=None):
+    """x = [text; image] per sample; with text_len the first n_text rows are the text stream."""
     B, N, _ = x.shape
     _check(lib.af_single_block(w.handle, s.handle, layer, _dev(x, torch.bfloat16, "x"),
-                               _dev(temb, torch.float32, "temb"), B, N, _stream(stream)), "af_single_block")
+                               _dev(temb, torch.float32, "temb"), B, N, int(n_text), _lens(text_len, B, "text_len"),
+                               _stream(stream)), "af_single_block")
 
 
-def transformer_forward(w: Weights, s: Scratch, latents, text_emb, t, velocity, stream=None):
+def transformer_forward(w: Weights, s: Scratch, latents, text_emb, t, velocity, text_len=None, stream=None):
     B, C, H, W = latents.shape
     L = text_emb.shape[1]
     _check(lib.af_transformer_forward(w.handle, s.handle, _dev(latents, torch.float32, "latents"),
                                       _dev(text_emb, torch.bfloat16, "text_emb"), _dev(t, torch.float32, "t"),
-                                      B, H, W, L, _dev(velocity, torch.float32, "velocity"), _stream(stream)),
+                                      B, H, W, L, _lens(text_len, B, "text_len"),
+                                      _dev(velocity, torch.float32, "velocity"), _stream(stream)),
            "af_transformer_forward")
 
 
@@ -284,14 +297,15 @@ def euler_cfg_step(latents, velocity, guidance: float, sigma: float, sigma_next:
 
 
 def denoise_step(w: Weights, s: Scratch, latents, text_emb, guidance: float, sigma: float, sigma_next: float,
-                 stream=None):
+                 stream=None, text_len=None):
     """One sampling step: CFG batch [uncond; text] forward at t = sigma, guidance, Euler to sigma_next."""
     Bi, C, H, W = latents.shape
     if text_emb.shape[0] != 2 * Bi:
         raise ValueError("text_emb must hold 2*Bi rows (uncond first)")
     L = text_emb.shape[1]
     _check(lib.af_denoise_step(w.handle, s.handle, _dev(latents, torch.float32, "latents"),
-                               _dev(text_emb, torch.bfloat16, "text_emb"), Bi, H, W, L, float(guidance), float(sigma),
+                               _dev(text_emb, torch.bfloat16, "text_emb"), Bi, H, W, L,
+                               _lens(text_len, 2 * Bi, "text_len"), float(guidance), float(sigma),
                                float(sigma_next), _stream(stream)), "af_denoise_step")
 
 
@@ -299,7 +313,8 @@ class Sampler:
     """The denoising loop as a plan (af_sampler): modulations of every step
     precomputed by prepare(), steps optionally replayed as CUDA graphs."""
 
-    def __init__(self, w: Weights, s: Scratch, latents, text_emb, sigmas, guidance: float, use_graphs: bool = True):
+    def __init__(self, w: Weights, s: Scratch, latents, text_emb, sigmas, guidance: float, use_graphs: bool = True,
+                 text_len=None):
         Bi, C, H, W = latents.shape
         L = text_emb.shape[1]
         if text_emb.shape[0] != 2 * Bi:
@@ -308,10 +323,11 @@ class Sampler:
         sig = (ctypes.c_float * len(sigmas))(*[float(x) for x in sigmas])
         h = ctypes.c_void_p()
         _check(lib.af_sampler_create(w.handle, s.handle, _dev(latents, torch.float32, "latents"),
-                                     _dev(text_emb, torch.bfloat16, "text_emb"), Bi, H, W, L, self.n_steps, sig,
+                                     _dev(text_emb, torch.bfloat16, "text_emb"), Bi, H, W, L,
+                                     _lens(text_len, 2 * Bi, "text_len"), self.n_steps, sig,
                                      float(guidance), 1 if use_graphs else 0, ctypes.byref(h)), "af_sampler_create")
         self.handle = h
-        self._keep = (w, s, latents, text_emb)
+        self._keep = (w, s, latents, text_emb, text_len)
 
     def prepare(self, stream=None):
         _check(lib.af_sampler_prepare(self.handle, _stream(stream)), "af_sampler_prepare")
@@ -352,8 +368,11 @@ def linear(A, W, C, stream=None):
                          M, N, K, _stream(stream)), "af_linear")
 
 
-def attention(q, k, v, o, qk_normalized: bool = False, stream=None):
+def attention(q, k, v, o, qk_normalized: bool = False, key_len=None, key_base: int = 0, key_end: int = 0,
+              stream=None):
+    """key_len: optional CUDA int32 [B]; keys [key_base + key_len[b], key_end) of sample b are masked."""
     B, H, N, hd = q.shape
     _check(lib.af_attention(_dev(q, torch.bfloat16, "q"), _dev(k, torch.bfloat16, "k"), _dev(v, torch.bfloat16, "v"),
-                            _dev(o, torch.bfloat16, "o"), B, H, N, hd, 1 if qk_normalized else 0, _stream(stream)),
+                            _dev(o, torch.bfloat16, "o"), B, H, N, hd, 1 if qk_normalized else 0,
+                            _lens(key_len, B, "key_len"), int(key_base), int(key_end), _stream(stream)),
            "af_attention")

@@ -66,6 +66,11 @@ struct AttnParams {
   int qk_normalized; // nonzero: every q, k row has L2 norm <= sqrt(hd) (per-head LayerNorm output)
   const uint16_t* q; // [B, H, N, hd] (read directly by the QK-normalised kernel)
   int* err;
+  // optional key mask: for sample b the keys [key_base + key_len[b], key_end)
+  // take no part in the softmax (key_len == nullptr: none); key_len[b] is
+  // clamped to [0, key_end - key_base]
+  const int* key_len = nullptr;
+  int key_base = 0, key_end = 0;
 };
 cudaError_t launch_attention(const AttnParams& p, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                              cudaStream_t stream);

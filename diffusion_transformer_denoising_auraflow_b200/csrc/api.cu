@@ -311,8 +311,25 @@ af_status swiglu(const af_weights* w, af_scratch* s, const uint16_t* y, int M, c
   return run_gemm(s, p, y, w12, 2 * d.F, st);
 }
 
+// Padding of the text part: for sample b the keys [base + len[b], end) are
+// masked (len == nullptr: no mask).
+struct KeyMask {
+  const int* len = nullptr;
+  int base = 0, end = 0;
+};
+
+KeyMask text_mask(const af_weights* w, const int* text_len, int Nt) {
+  KeyMask m;
+  if (text_len) {
+    m.len = text_len;
+    m.base = w->cfg.num_register_tokens;
+    m.end = Nt;
+  }
+  return m;
+}
+
 af_status attention(const af_weights* w, af_scratch* s, int B, int N, uint16_t* out_a, uint16_t* out_b, int split,
-                    cudaStream_t st) {
+                    const KeyMask& km, cudaStream_t st) {
   const Derived& d = w->d;
   AttnParams p;
   p.B = B;
@@ -326,6 +343,9 @@ af_status attention(const af_weights* w, af_scratch* s, int B, int N, uint16_t* 
   p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(d.hd));
   p.qk_normalized = 1;  // q and k come from the QK-norm epilogue of the QKV GEMM
   p.err = s->err;
+  p.key_len = km.len;
+  p.key_base = km.base;
+  p.key_end = km.end;
   LaunchScope ls(s, KC_ATTN, 4.0 * B * d.H * static_cast<double>(N) * N * d.hd, st);
   p.q = s->q;
   cudaError_t e = launch_attention(p, s->q, s->k, s->v, st);
@@ -350,7 +370,7 @@ af_status ln_mod(af_scratch* s, const uint16_t* x, const float* shift, const flo
 // [unit_row, +6D) per sample, sample stride mod_stride).
 af_status joint_block_impl(const af_weights* w, af_scratch* s, int layer, uint16_t* img, uint16_t* txt,
                            const float* mi, const float* mt, int mod_stride, int B, int Ni, int Nt,
-                           cudaStream_t st) {
+                           const KeyMask& km, cudaStream_t st) {
   const Derived& d = w->d;
   const int D = d.D;
   const float eps = w->cfg.ln_eps;
@@ -367,7 +387,7 @@ af_status joint_block_impl(const af_weights* w, af_scratch* s, int layer, uint16
   AF_TRY(ln_mod(s, txt, mt + 0 * D, mt + 1 * D, mod_stride, y_txt, B * Nt, Nt, D, eps, st));
   AF_TRY(qkv(w, s, y_txt, B, Nt, w->ptr(pre + "attn.add_q_proj.weight"), 0, N, st));
   AF_TRY(qkv(w, s, y_img, B, Ni, w->ptr(pre + "attn.to_q.weight"), Nt, N, st));
-  AF_TRY(attention(w, s, B, N, o_txt, o_img, Nt, st));
+  AF_TRY(attention(w, s, B, N, o_txt, o_img, Nt, km, st));
   AF_TRY(gated_residual(s, o_img, B, Ni, D, w->ptr(pre + "attn.to_out.0.weight"), D, img, mi + 2 * D, mod_stride, st));
   AF_TRY(gated_residual(s, o_txt, B, Nt, D, w->ptr(pre + "attn.to_add_out.weight"), D, txt, mt + 2 * D, mod_stride,
                         st));
@@ -383,14 +403,14 @@ af_status joint_block_impl(const af_weights* w, af_scratch* s, int layer, uint16
 }
 
 af_status single_block_impl(const af_weights* w, af_scratch* s, int layer, uint16_t* x, const float* m,
-                            int mod_stride, int B, int N, cudaStream_t st) {
+                            int mod_stride, int B, int N, const KeyMask& km, cudaStream_t st) {
   const Derived& d = w->d;
   const int D = d.D;
   const float eps = w->cfg.ln_eps;
   const std::string pre = "single_transformer_blocks." + std::to_string(layer) + ".";
   AF_TRY(ln_mod(s, x, m + 0 * D, m + 1 * D, mod_stride, s->y, B * N, N, D, eps, st));
   AF_TRY(qkv(w, s, s->y, B, N, w->ptr(pre + "attn.to_q.weight"), 0, N, st));
-  AF_TRY(attention(w, s, B, N, s->o, s->o, 0, st));
+  AF_TRY(attention(w, s, B, N, s->o, s->o, 0, km, st));
   AF_TRY(gated_residual(s, s->o, B, N, D, w->ptr(pre + "attn.to_out.0.weight"), D, x, m + 2 * D, mod_stride, st));
   AF_TRY(ln_mod(s, x, m + 3 * D, m + 4 * D, mod_stride, s->y, B * N, N, D, eps, st));
   AF_TRY(swiglu(w, s, s->y, B * N, w->ptr(pre + "ff.linear_1.weight"), s->h, st));
@@ -700,9 +720,10 @@ af_status af_patch_embed(const af_weights* w, af_scratch* s, const float* latent
 }
 
 af_status af_joint_block(const af_weights* w, af_scratch* s, int layer, uint16_t* img, uint16_t* txt,
-                         const float* temb, int B, int Ni, int Nt, void* stream) {
+                         const float* temb, int B, int Ni, int Nt, const int* text_len, void* stream) {
   AF_TRY(check_scratch(w, s));
   if (!img || !txt || !temb || B <= 0 || Ni <= 0 || Nt <= 0) return AF_ERR_INVALID_ARG;
+  if (text_len && Nt < w->cfg.num_register_tokens) return AF_ERR_SHAPE;
   if (layer < 0 || layer >= w->cfg.num_mmdit_layers) return AF_ERR_INVALID_ARG;
   if (B > s->max_b || Ni + Nt > s->max_n || Ni > s->max_n) return AF_ERR_SHAPE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -716,13 +737,14 @@ af_status af_joint_block(const af_weights* w, af_scratch* s, int layer, uint16_t
   }
   const float* mi = s->mods;
   const float* mt = s->mods + 6 * D;
-  return joint_block_impl(w, s, layer, img, txt, mi, mt, 12 * D, B, Ni, Nt, st);
+  return joint_block_impl(w, s, layer, img, txt, mi, mt, 12 * D, B, Ni, Nt, text_mask(w, text_len, Nt), st);
 }
 
 af_status af_single_block(const af_weights* w, af_scratch* s, int layer, uint16_t* x, const float* temb, int B,
-                          int N, void* stream) {
+                          int N, int Nt, const int* text_len, void* stream) {
   AF_TRY(check_scratch(w, s));
   if (!x || !temb || B <= 0 || N <= 0) return AF_ERR_INVALID_ARG;
+  if (text_len && (Nt < w->cfg.num_register_tokens || Nt > N)) return AF_ERR_SHAPE;
   if (layer < 0 || layer >= w->cfg.num_single_dit_layers) return AF_ERR_INVALID_ARG;
   if (B > s->max_b || N > s->max_n) return AF_ERR_SHAPE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -732,7 +754,7 @@ af_status af_single_block(const af_weights* w, af_scratch* s, int layer, uint16_
     LaunchScope ls(s, KC_OTHER, 2.0 * 6 * D * D, st, (B + 7) / 8);
     AF_CUDA(launch_modulation(temb, B, D, ada_base(w) + r * D, 6 * D, s->mods, st));
   }
-  return single_block_impl(w, s, layer, x, s->mods, 6 * D, B, N, st);
+  return single_block_impl(w, s, layer, x, s->mods, 6 * D, B, N, text_mask(w, text_len, Nt), st);
 }
 
 // premods != nullptr: every adaLN / pre-final modulation of this step was
@@ -740,8 +762,8 @@ af_status af_single_block(const af_weights* w, af_scratch* s, int layer, uint16_
 // premods[b * pre_stride + r]); the timestep MLP and the modulation GEMV are
 // skipped and `t` is not read.
 static af_status forward_impl(const af_weights* w, af_scratch* s, const float* latents, const uint16_t* text_emb,
-                              const float* t, int B, int H, int W, int L, float* velocity, cudaStream_t st,
-                              const float* premods = nullptr, int pre_stride = 0) {
+                              const float* t, int B, int H, int W, int L, const int* text_len, float* velocity,
+                              cudaStream_t st, const float* premods = nullptr, int pre_stride = 0) {
   AF_TRY(check_scratch(w, s));
   if (!latents || !text_emb || !t || !velocity || B <= 0 || H <= 0 || W <= 0 || L < 0) return AF_ERR_INVALID_ARG;
   const af_config& c = w->cfg;
@@ -756,6 +778,7 @@ static af_status forward_impl(const af_weights* w, af_scratch* s, const float* l
   const size_t R_ada = w->ada_rows;
   const float* mods = premods ? premods : s->mods;
   const int mstride = premods ? pre_stride : static_cast<int>(R_ada);
+  const KeyMask km = text_mask(w, text_len, Nt);
 
   // embedding stage
   if (!premods) {
@@ -789,7 +812,7 @@ static af_status forward_impl(const af_weights* w, af_scratch* s, const float* l
   for (int i = 0; i < c.num_mmdit_layers; ++i) {
     const float* mi = mods + w->unit_row[2 * i];
     const float* mt = mods + w->unit_row[2 * i + 1];
-    AF_TRY(joint_block_impl(w, s, i, s->img, s->txt, mi, mt, mstride, B, Ni, Nt, st));
+    AF_TRY(joint_block_impl(w, s, i, s->img, s->txt, mi, mt, mstride, B, Ni, Nt, km, st));
   }
   // x = cat(text, image) per sample
   AF_CUDA(cudaMemcpy2DAsync(s->x, static_cast<size_t>(N) * D * 2, s->txt, static_cast<size_t>(Nt) * D * 2,
@@ -799,7 +822,7 @@ static af_status forward_impl(const af_weights* w, af_scratch* s, const float* l
                             cudaMemcpyDeviceToDevice, st));
   for (int i = 0; i < c.num_single_dit_layers; ++i) {
     const float* m = mods + w->unit_row[2 * c.num_mmdit_layers + i];
-    AF_TRY(single_block_impl(w, s, i, s->x, m, mstride, B, N, st));
+    AF_TRY(single_block_impl(w, s, i, s->x, m, mstride, B, N, km, st));
   }
   // pre-final (scale first, then shift), proj_out, unpatchify on the image rows
   const float* pf = mods + w->pf_row;
@@ -810,13 +833,14 @@ static af_status forward_impl(const af_weights* w, af_scratch* s, const float* l
 }
 
 af_status af_transformer_forward(const af_weights* w, af_scratch* s, const float* latents, const uint16_t* text_emb,
-                                 const float* t, int B, int H, int W, int L, float* velocity, void* stream) {
-  return forward_impl(w, s, latents, text_emb, t, B, H, W, L, velocity, static_cast<cudaStream_t>(stream));
+                                 const float* t, int B, int H, int W, int L, const int* text_len, float* velocity,
+                                 void* stream) {
+  return forward_impl(w, s, latents, text_emb, t, B, H, W, L, text_len, velocity, static_cast<cudaStream_t>(stream));
 }
 
 static af_status denoise_step_impl(const af_weights* w, af_scratch* s, float* latents, const uint16_t* text_emb,
-                                   int Bi, int H, int W, int L, float guidance, float sigma, float sigma_next,
-                                   cudaStream_t st, const float* premods = nullptr) {
+                                   int Bi, int H, int W, int L, const int* text_len, float guidance, float sigma,
+                                   float sigma_next, cudaStream_t st, const float* premods = nullptr) {
   const int B = 2 * Bi;
   const size_t per = static_cast<size_t>(w->cfg.in_channels) * H * W;
   // CFG batch [uncond; text] shares the latents
@@ -826,7 +850,7 @@ static af_status denoise_step_impl(const af_weights* w, af_scratch* s, float* la
     LaunchScope ls(s, KC_OTHER, 4.0 * B, st);
     AF_CUDA(launch_fill(s->tvec, B, sigma, st));
   }
-  AF_TRY(forward_impl(w, s, s->lat2, text_emb, s->tvec, B, H, W, L, s->vel, st, premods, 0));
+  AF_TRY(forward_impl(w, s, s->lat2, text_emb, s->tvec, B, H, W, L, text_len, s->vel, st, premods, 0));
   LaunchScope ls(s, KC_OTHER, 16.0 * per * Bi, st);
   AF_CUDA(launch_euler_cfg(latents, s->vel, Bi, static_cast<int64_t>(per), guidance, sigma, sigma_next, st));
   return AF_OK;
@@ -844,9 +868,10 @@ static af_status check_step_args(const af_weights* w, af_scratch* s, const float
 }
 
 af_status af_denoise_step(const af_weights* w, af_scratch* s, float* latents, const uint16_t* text_emb, int Bi, int H,
-                          int W, int L, float guidance, float sigma, float sigma_next, void* stream) {
+                          int W, int L, const int* text_len, float guidance, float sigma, float sigma_next,
+                          void* stream) {
   AF_TRY(check_step_args(w, s, latents, text_emb, Bi, H, W, L));
-  return denoise_step_impl(w, s, latents, text_emb, Bi, H, W, L, guidance, sigma, sigma_next,
+  return denoise_step_impl(w, s, latents, text_emb, Bi, H, W, L, text_len, guidance, sigma, sigma_next,
                            static_cast<cudaStream_t>(stream));
 }
 
@@ -858,6 +883,7 @@ struct af_sampler {
   af_scratch* s = nullptr;
   float* latents = nullptr;
   const uint16_t* text = nullptr;
+  const int* text_len = nullptr;
   int Bi = 0, H = 0, W = 0, L = 0, n_steps = 0;
   float guidance = 1.f;
   bool use_graphs = false;
@@ -872,8 +898,8 @@ struct af_sampler {
 extern "C" {
 
 af_status af_sampler_create(const af_weights* w, af_scratch* s, float* latents, const uint16_t* text_emb, int Bi,
-                            int H, int W, int L, int n_steps, const float* sigmas, float guidance, int use_graphs,
-                            af_sampler** out) {
+                            int H, int W, int L, const int* text_len, int n_steps, const float* sigmas,
+                            float guidance, int use_graphs, af_sampler** out) {
   if (!out) return AF_ERR_INVALID_ARG;
   *out = nullptr;
   AF_TRY(check_step_args(w, s, latents, text_emb, Bi, H, W, L));
@@ -883,6 +909,7 @@ af_status af_sampler_create(const af_weights* w, af_scratch* s, float* latents, 
   m->s = s;
   m->latents = latents;
   m->text = text_emb;
+  m->text_len = text_len;
   m->Bi = Bi;
   m->H = H;
   m->W = W;
@@ -963,7 +990,7 @@ af_status af_sampler_step(af_sampler* m, int step, void* stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const float* premods = m->mods + static_cast<size_t>(step) * m->w->ada_rows;
   auto enqueue = [&]() {
-    return denoise_step_impl(m->w, m->s, m->latents, m->text, m->Bi, m->H, m->W, m->L, m->guidance,
+    return denoise_step_impl(m->w, m->s, m->latents, m->text, m->Bi, m->H, m->W, m->L, m->text_len, m->guidance,
                              m->sigmas[step], m->sigmas[step + 1], st, premods);
   };
   if (!m->use_graphs) return enqueue();
@@ -1084,8 +1111,9 @@ af_status af_linear(const uint16_t* A, const uint16_t* W, uint16_t* C, int M, in
 }
 
 af_status af_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* o, int B, int H, int N,
-                       int hd, int qk_normalized, void* stream) {
+                       int hd, int qk_normalized, const int* key_len, int key_base, int key_end, void* stream) {
   if (!q || !k || !v || !o || B <= 0 || H <= 0 || N <= 0) return AF_ERR_INVALID_ARG;
+  if (key_len && (key_base < 1 || key_end < key_base || key_end > N)) return AF_ERR_INVALID_ARG;
   if (!(hd == 256 || hd == 8 || hd == 16 || hd == 32 || hd == 64)) return AF_ERR_UNSUPPORTED;
   AttnParams p;
   p.B = B;
@@ -1100,6 +1128,9 @@ af_status af_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, 
   p.qk_normalized = qk_normalized ? 1 : 0;
   p.q = q;
   p.err = nullptr;
+  p.key_len = key_len;
+  p.key_base = key_base;
+  p.key_end = key_end;
   AF_CUDA(launch_attention(p, q, k, v, static_cast<cudaStream_t>(stream)));
   return AF_OK;
 }

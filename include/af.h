@@ -170,16 +170,23 @@ af_status af_patch_embed(const af_weights* w, af_scratch* s, const float* latent
  *   img:  device bf16[B, Ni, D] in/out (image stream).
  *   txt:  device bf16[B, Nt, D] in/out (text stream incl. registers).
  *   temb: device float[B, D].
- *   layer in [0, num_mmdit_layers). */
+ *   layer in [0, num_mmdit_layers).
+ *   text_len: NULL, or device int[B]: real prompt tokens of each sample
+ *   (see "Padded prompts" below); text rows [num_register_tokens +
+ *   text_len[b], Nt) are then masked as attention keys. */
 af_status af_joint_block(const af_weights* w, af_scratch* s, int layer, uint16_t* img, uint16_t* txt,
-                         const float* temb, int B, int Ni, int Nt, void* stream);
+                         const float* temb, int B, int Ni, int Nt, const int* text_len, void* stream);
 
 /* One AuraFlowSingleTransformerBlock ([ARCH] §单 DiT 块) in place on the
  * concatenated sequence x = [text; image]:
  *   x: device bf16[B, N, D] in/out; temb: device float[B, D];
- *   layer in [0, num_single_dit_layers). */
+ *   layer in [0, num_single_dit_layers).
+ *   Nt, text_len: the first Nt rows of x are the text stream (registers
+ *   included); with text_len != NULL (device int[B]) rows
+ *   [num_register_tokens + text_len[b], Nt) are masked as attention keys.
+ *   Nt is ignored when text_len is NULL. */
 af_status af_single_block(const af_weights* w, af_scratch* s, int layer, uint16_t* x, const float* temb,
-                          int B, int N, void* stream);
+                          int B, int N, int Nt, const int* text_len, void* stream);
 
 /* The whole AuraFlowTransformer2DModel forward ([ARCH] §前向传播流程):
  * patch embed, timestep embed, context_embedder (bias-free 2048 -> D) with
@@ -189,10 +196,21 @@ af_status af_single_block(const af_weights* w, af_scratch* s, int layer, uint16_
  *   latents:  device float[B, C_in, H, W]
  *   text_emb: device bf16[B, L, joint_attention_dim]
  *   t:        device float[B] (timestep / 1000)
- *   velocity: device float[B, C_out, H, W] (output) */
+ *   text_len: NULL (every text token is real, the model's own behaviour) or
+ *             device int[B], see "Padded prompts"
+ *   velocity: device float[B, C_out, H, W] (output)
+ *
+ * Padded prompts.  The pipeline pads every prompt of a batch to one length
+ * and builds an attention mask ([PIPE] §AuraFlowPipeline 核心参数详解,
+ * [ARCH] §在 AuraFlowPipeline 中的实际调用), but the transformer forward
+ * itself takes no mask ([ARCH] §前向传播流程).  As an extension, text_len[b]
+ * gives the real length of sample b's prompt: its last L - text_len[b] text
+ * tokens then take no part as attention keys in any block (boolean key mask,
+ * like an SDPA attn_mask); register tokens and image tokens always do.
+ * Values are clamped to [0, L]. */
 af_status af_transformer_forward(const af_weights* w, af_scratch* s, const float* latents,
                                  const uint16_t* text_emb, const float* t, int B, int H, int W, int L,
-                                 float* velocity, void* stream);
+                                 const int* text_len, float* velocity, void* stream);
 
 /* Classifier-free guidance combine and flow-match Euler step ([PIPE]
  * §AuraFlowPipeline 核心参数详解 (CFG formula), [ARCH] §在 AuraFlowPipeline
@@ -211,9 +229,11 @@ af_status af_euler_cfg_step(float* latents, const float* velocity, int Bi, int C
  * updates the latents in place with sigma_next.
  *   latents:  device float[Bi, C_in, H, W] in/out
  *   text_emb: device bf16[2 Bi, L, joint_attention_dim], uncond rows first.
+ *   text_len: NULL or device int[2 Bi] (padded prompts, as for the forward).
  * Needs a scratch created with max_batch >= 2 Bi. */
 af_status af_denoise_step(const af_weights* w, af_scratch* s, float* latents, const uint16_t* text_emb, int Bi,
-                          int H, int W, int L, float guidance, float sigma, float sigma_next, void* stream);
+                          int H, int W, int L, const int* text_len, float guidance, float sigma, float sigma_next,
+                          void* stream);
 
 /* ---- the sampling loop -----------------------------------------------------
  * The pipeline's denoising loop ([ARCH] §在 AuraFlowPipeline 中的实际调用,
@@ -227,13 +247,14 @@ af_status af_denoise_step(const af_weights* w, af_scratch* s, float* latents, co
  * on the stream around these calls).
  *   latents:  device float[Bi, C, H, W], updated in place by every step
  *   text_emb: device bf16[2 Bi, L, joint_attention_dim] (uncond rows first)
+ *   text_len: NULL or device int[2 Bi] (padded prompts)
  *   sigmas:   host float[n_steps + 1] (e.g. from af_sigma_schedule)
- * Both device buffers are bound to the sampler: change their contents, not
+ * The device buffers are bound to the sampler: change their contents, not
  * their addresses.  The scratch must fit a 2 Bi batch of this size. */
 typedef struct af_sampler af_sampler;
 af_status af_sampler_create(const af_weights* w, af_scratch* s, float* latents, const uint16_t* text_emb, int Bi,
-                            int H, int W, int L, int n_steps, const float* sigmas, float guidance, int use_graphs,
-                            af_sampler** out);
+                            int H, int W, int L, const int* text_len, int n_steps, const float* sigmas,
+                            float guidance, int use_graphs, af_sampler** out);
 af_status af_sampler_prepare(af_sampler* smp, void* stream);
 af_status af_sampler_step(af_sampler* smp, int step, void* stream);
 void af_sampler_destroy(af_sampler* smp);
@@ -280,9 +301,14 @@ af_status af_linear(const uint16_t* A, const uint16_t* W, uint16_t* C, int M, in
  *   qk_normalized: nonzero promises that every q and k row has L2 norm at
  *   most sqrt(hd) (up to bf16 rounding), as the per-head LayerNorm (QK-norm)
  *   guarantees; the kernel then uses a fixed softmax shift instead of a
- *   running maximum.  Pass 0 for arbitrary inputs. */
+ *   running maximum.  Pass 0 for arbitrary inputs.
+ *   key_len: NULL, or device int[B]: for sample b the keys
+ *   [key_base + key_len[b], key_end) are masked (key_len[b] clamped to
+ *   [0, key_end - key_base]); needs 1 <= key_base <= key_end <= N so that
+ *   every row keeps at least one key. */
 af_status af_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* o, int B,
-                       int H, int N, int hd, int qk_normalized, void* stream);
+                       int H, int N, int hd, int qk_normalized, const int* key_len, int key_base, int key_end,
+                       void* stream);
 
 const char* af_status_string(af_status st);
 /* Text of the last CUDA error seen by this thread's calls ("" if none). */

@@ -124,3 +124,50 @@ def test_real_width_forward_small_latent(af):
     af.transformer_forward(w, s, to_f32(lat), to_bf16(text), to_f32(tt), vel)
     s.sync()
     assert O.rel_l2(to_np(vel), ref) < STACK_TOL
+
+
+def test_tiny_forward_padded_prompts_match_oracle(af):
+    """Per-sample prompt lengths 3 and 8 of L = 8 (the first sample's last five
+    text tokens are padding): GPU forward with text_len vs the oracle's masked
+    forward, and the padding's values do not reach the velocity."""
+    cfg = tiny_config()
+    w = af.Weights(af_config(cfg))
+    drawn = draw_weights(cfg, 21)
+    upload(w, drawn)
+    s = af.Scratch(w, 2, 64, 8)
+    lat = synth.latents(21, (2, 4, 16, 16))
+    text = synth.text_embeddings(22, (2, 8, cfg.joint_attention_dim))
+    t = np.array([0.8, 0.3], np.float32)
+    lens = [3, 8]
+    tl = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    vel = torch.empty(2, 4, 16, 16, device="cuda")
+    af.transformer_forward(w, s, to_f32(lat), to_bf16(text), to_f32(t), vel, text_len=tl)
+    s.sync()
+    ref = O.transformer_forward(lat, text, t, drawn, cfg, text_len=lens)
+    assert O.rel_l2(to_np(vel), ref) < STACK_TOL
+    junk = text.copy()
+    junk[0, 3:] = 7.0
+    vel2 = torch.empty_like(vel)
+    af.transformer_forward(w, s, to_f32(lat), to_bf16(junk), to_f32(t), vel2, text_len=tl)
+    s.sync()
+    assert torch.equal(vel, vel2)
+
+
+def test_real_width_padded_prompts_match_oracle(af):
+    """D = 3072 (12 x 256 heads), 1 joint + 2 single blocks, 64 image tokens,
+    L = 40 text tokens with real lengths 17 and 40."""
+    cfg = O.Config(num_mmdit_layers=1, num_single_dit_layers=2, pos_embed_max_size=64 * 64)
+    w = af.Weights(af_config(cfg))
+    drawn = draw_weights(cfg, 23)
+    upload(w, drawn)
+    s = af.Scratch(w, 2, 64, 40)
+    lat = synth.latents(23, (2, 4, 16, 16))
+    text = synth.text_embeddings(24, (2, 40, cfg.joint_attention_dim))
+    t = np.array([1.0, 0.5], np.float32)
+    lens = [17, 40]
+    vel = torch.empty(2, 4, 16, 16, device="cuda")
+    af.transformer_forward(w, s, to_f32(lat), to_bf16(text), to_f32(t), vel,
+                           text_len=torch.tensor(lens, dtype=torch.int32, device="cuda"))
+    s.sync()
+    ref = O.transformer_forward(lat, text, t, drawn, cfg, text_len=lens)
+    assert O.rel_l2(to_np(vel), ref) < STACK_TOL

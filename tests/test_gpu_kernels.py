@@ -196,3 +196,51 @@ def test_euler_cfg_step_matches_oracle(af):
     af.euler_cfg_step(xt, to_f32(v), 3.5, 0.6, 0.6)    # sigma' = sigma: no-op, bit-exact
     torch.cuda.synchronize()
     assert np.array_equal(to_np(xt), x.astype(np.float64))
+
+
+# ---------------------------------------------------------------- attention with a key mask (padded prompts)
+
+MASK_CASES = [  # B, H, N, hd, key_base, key_end, key_len per sample
+    (2, 2, 1000, 256, 8, 400, [5, 300]),      # CTA-pair kernel: masked range spans several key tiles
+    (2, 1, 4360, 256, 8, 264, [0, 256]),      # the model's shape: 8 registers + 256 text tokens
+    (2, 2, 200, 256, 8, 100, [0, 50]),        # one-CTA kernels (N < 256)
+    (2, 2, 33, 16, 2, 20, [3, 18]),           # small heads (SIMT)
+]
+
+
+@pytest.mark.parametrize("qkn", [False, True])
+@pytest.mark.parametrize("B,H,N,hd,base,end,lens", MASK_CASES)
+def test_attention_key_mask_matches_oracle(af, B, H, N, hd, base, end, lens, qkn):
+    q = synth.normal(401, f"mq{N}", (B, H, N, hd), 1.0)
+    k = synth.normal(402, f"mk{N}", (B, H, N, hd), 1.0)
+    v = synth.normal(403, f"mv{N}", (B, H, N, hd), 1.0)
+    qn = synth.bf16_round(O.layer_norm(q, 1e-6).astype(np.float32))
+    kn = synth.bf16_round(O.layer_norm(k, 1e-6).astype(np.float32))
+    mask = np.ones((B, N), bool)
+    for b, n in enumerate(lens):
+        mask[b, base + n:end] = False
+    o = torch.empty(B, N, H * hd, dtype=torch.bfloat16, device="cuda")
+    kl = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    af.attention(to_bf16(qn), to_bf16(kn), to_bf16(v), o, qk_normalized=qkn, key_len=kl, key_base=base, key_end=end)
+    torch.cuda.synchronize()
+    ref = O.merge_heads(O.attention(qn, kn, v, key_mask=mask))
+    assert O.rel_l2(to_np(o), ref) < 1e-2
+    # masked keys carry no weight: changing them leaves the output bit-identical
+    k2 = kn.copy()
+    v2 = v.copy()
+    k2[~mask[:, None, :, None].repeat(H, 1).repeat(hd, 3)] = 0.5
+    v2[~mask[:, None, :, None].repeat(H, 1).repeat(hd, 3)] = 100.0
+    o2 = torch.empty_like(o)
+    af.attention(to_bf16(qn), to_bf16(k2), to_bf16(v2), o2, qk_normalized=qkn, key_len=kl, key_base=base, key_end=end)
+    torch.cuda.synchronize()
+    assert torch.equal(o, o2)
+
+
+def test_attention_rejects_bad_mask(af):
+    q = torch.zeros(1, 1, 64, 256, dtype=torch.bfloat16, device="cuda")
+    o = torch.empty(1, 64, 256, dtype=torch.bfloat16, device="cuda")
+    kl = torch.zeros(1, dtype=torch.int32, device="cuda")
+    with pytest.raises(af.AFError):          # key_base 0 could mask every key
+        af.attention(q, q, q, o, key_len=kl, key_base=0, key_end=10)
+    with pytest.raises(af.AFError):          # end beyond N
+        af.attention(q, q, q, o, key_len=kl, key_base=1, key_end=65)

@@ -155,3 +155,26 @@ def test_sampler_rejects_bad_args(af):
     with pytest.raises(af.AFError):          # step out of range
         smp.step(2, torch.cuda.Stream())
     smp.close()
+
+
+def test_sampler_padded_prompts_match_oracle(af):
+    cfg = tiny_config()
+    n = 3
+    w, s, drawn, x0, text = _setup(af, cfg, 83, 1, 16, 16, 8)
+    lens = [2, 6]                      # uncond prompt 2 tokens, text prompt 6 of 8
+    sig = af.sigma_schedule(n)
+    xt, tt = to_f32(x0), to_bf16(text)
+    stream = torch.cuda.Stream()
+    smp = af.Sampler(w, s, xt, tt, sig, 3.5, use_graphs=True,
+                     text_len=torch.tensor(lens, dtype=torch.int32, device="cuda"))
+    with torch.cuda.stream(stream):
+        smp.prepare(stream)
+        for i in range(n):
+            smp.step(i, stream)
+    stream.synchronize()
+    x = x0.astype(np.float64)
+    for i in range(n):
+        v = O.transformer_forward(np.concatenate([x, x]), text, np.full(2, sig[i]), drawn, cfg, text_len=lens)
+        x = O.euler_cfg_step(x, v, 3.5, sig[i], sig[i + 1])
+    assert O.rel_l2(to_np(xt) - x0, x - x0) < STACK_TOL
+    smp.close()
