@@ -77,7 +77,8 @@ cudaError_t launch_attention(const AttnParams& p, const uint16_t* q, const uint1
 
 // Small kernels (kernels.cu)
 cudaError_t launch_ln_modulate(const uint16_t* x, const float* shift, const float* scale, int mod_stride,
-                               uint16_t* y, int rows, int rows_per_batch, int D, float eps, cudaStream_t s);
+                               uint16_t* y, int rows, int rows_per_batch, int D, float eps, cudaStream_t s,
+                               int* err = nullptr);
 cudaError_t launch_timestep_mlp(const float* t, int B, const uint16_t* w1, const uint16_t* b1, const uint16_t* w2,
                                 const uint16_t* b2, int C, int D, float* feat, float* h1, float* temb, cudaStream_t s);
 cudaError_t launch_modulation(const float* temb, int B, int D, const uint16_t* w, int rows, float* out,

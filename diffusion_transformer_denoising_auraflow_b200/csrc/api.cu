@@ -356,7 +356,7 @@ af_status attention(const af_weights* w, af_scratch* s, int B, int N, uint16_t* 
 af_status ln_mod(af_scratch* s, const uint16_t* x, const float* shift, const float* scale, int mod_stride, uint16_t* y,
                  int rows, int rows_per_batch, int D, float eps, cudaStream_t st) {
   LaunchScope ls(s, KC_LN, 4.0 * rows * D, st);
-  cudaError_t e = launch_ln_modulate(x, shift, scale, mod_stride, y, rows, rows_per_batch, D, eps, st);
+  cudaError_t e = launch_ln_modulate(x, shift, scale, mod_stride, y, rows, rows_per_batch, D, eps, st, s->err);
   return e == cudaSuccess ? AF_OK : cuda_fail(e);
 }
 

@@ -661,34 +661,29 @@ __global__ void __launch_bounds__(QKN_THREADS, 1)
 // (sample, head), 128 per CTA, and walks the keys in tiles of 128 with
 // tcgen05.mma.cta_group::2 issued by the leader CTA:
 //   S = Q K^T   M = 256, N = 128, K = 256: each CTA supplies its 128 Q rows
-//               (shared memory) and half of the K tile (64 keys); each CTA's
-//               TMEM receives its 128 x 128 block of S.
-//   O += P V    M = 256, N = 256, K = 128: P is read from TMEM (each CTA's
-//               128 rows), V from shared memory (each CTA holds half of the
-//               tile, 128 head-dim columns); each CTA's TMEM accumulates its
-//               128 x 256 block of O.
+//               and half of the K tile (64 keys); each CTA's TMEM receives
+//               its 128 x 128 block of S.
+//   O += P V    M = 256, N = 256, K = 128: each CTA supplies its 128 rows of
+//               P and half of the V tile (128 head-dim columns); each CTA's
+//               TMEM accumulates its 128 x 256 block of O.
 // Per SM that is 64 KB of K/V per 128 keys instead of 128 KB, and every MMA
-// has N >= 128 (full tensor-core rate).  TMEM per CTA: O [0, 256), S
-// [256, 384), P0 [384, 448), P1 [448, 512) (bf16 pairs, one row per lane).
-// Shared memory per CTA: Q 64 KB, K and V halves double-buffered (4 x 32 KB).
+// has N >= 128 (full tensor-core rate).  TMEM per CTA: O [0, 256), S0
+// [256, 384), S1 [384, 512).  Shared memory per CTA: Q 64 KB, K and V halves
+// double-buffered (4 x 32 KB), one P buffer (128 x 128 bf16, 32 KB).
 // Softmax (fixed shift, as for attn_hd256_qknorm): warpgroup g of each CTA
 // owns keys [64 g, 64 g + 64) of every S tile; their partial row sums are
-// added at the end.  The softmax warps release S as soon as they have loaded
-// it and write P_j into TMEM buffer j & 1; the leader issues S_{j+1} as soon
-// as S_j is released and PV_j once P_j is written, so the tensor core
-// computes S_{j+1} and PV_j while the softmax of tile j+1 runs, and no
-// softmax ever waits for a PV product.  P buffer j & 1 is free again when
-// S_j completes: S_j is issued after PV_{j-2}, and a tcgen05.commit tracks
-// every earlier MMA of the issuing thread.  Barriers that gather both CTAs
-// live in the leader (TMA completions, S/P handshakes); commits are
-// multicast to both CTAs.  The follower's softmax warps arrive directly on
-// the leader's S/P barriers (CTA-scope release; a cluster-scope release there
-// costs ~1.2k cycles).
+// added at the end.  The leader issues S_0, S_1, then per tile PV_j followed
+// by S_{j+2}, so the tensor core computes the next scores while the softmax
+// warps publish P_{j+1}.  Barriers that gather both CTAs live in the leader
+// (TMA completions, S/P handshakes); commits are multicast to both CTAs.
+// The follower's softmax warps arrive directly on the leader's S/P barriers
+// (CTA-scope release; a cluster-scope release there costs ~1.2k cycles).
 constexpr int AP_BN = 128;
 constexpr uint32_t AP_Q_BYTES = 128 * AT_HD * 2;      // 64 KB
 constexpr uint32_t AP_KH_BYTES = 64 * AT_HD * 2;      // 32 KB: 64 keys x 256
 constexpr uint32_t AP_VH_BYTES = AP_BN * 128 * 2;     // 32 KB: 128 keys x 128 columns
-constexpr int AP_SMEM = AP_Q_BYTES + 2 * AP_KH_BYTES + 2 * AP_VH_BYTES + 2 * 128 * 4 + 256 + 1024;
+constexpr uint32_t AP_P_BYTES = 128 * AP_BN * 2;      // 32 KB
+constexpr int AP_SMEM = AP_Q_BYTES + 2 * AP_KH_BYTES + 2 * AP_VH_BYTES + AP_P_BYTES + 2 * 128 * 4 + 256 + 1024;
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
     attn_hd256_qknorm_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -698,20 +693,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
   uint8_t* sQ = smem;
   uint8_t* sK = sQ + AP_Q_BYTES;          // 2 buffers
   uint8_t* sV = sK + 2 * AP_KH_BYTES;     // 2 buffers
-  float* xsum = reinterpret_cast<float*>(sV + 2 * AP_VH_BYTES);  // [wg 2][row 128]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + 2 * AP_VH_BYTES + 2 * 128 * 4);
+  uint8_t* sP = sV + 2 * AP_VH_BYTES;
+  float* xsum = reinterpret_cast<float*>(sP + AP_P_BYTES);  // [wg 2][row 128]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + AP_P_BYTES + 2 * 128 * 4);
   uint64_t* q_full = bars + 0;     // leader: both CTAs' Q loads
   uint64_t* k_full = bars + 1;     // [2] leader: both K halves
   uint64_t* v_full = bars + 3;     // [2] leader: both V halves
   uint64_t* k_empty = bars + 5;    // [2] both CTAs (multicast commit)
   uint64_t* v_empty = bars + 7;    // [2] both CTAs
-  uint64_t* s_full = bars + 9;     // both CTAs
-  uint64_t* s_empty = bars + 10;   // leader: 16 softmax warps of both CTAs
-  uint64_t* p_full = bars + 11;    // [2] leader: 16 softmax warps of both CTAs
-  uint64_t* o_full = bars + 13;    // both CTAs: after the last PV
-  uint64_t* mma_done = bars + 14;  // leader
-  uint64_t* lbar = bars + 15;      // per CTA: 8 softmax warps
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  uint64_t* s_full = bars + 9;     // [2] both CTAs
+  uint64_t* s_empty = bars + 11;   // [2] leader: 16 softmax warps of both CTAs
+  uint64_t* p_full = bars + 13;    // leader: 16 softmax warps of both CTAs
+  uint64_t* pv_done = bars + 14;   // both CTAs
+  uint64_t* mma_done = bars + 15;  // leader
+  uint64_t* lbar = bars + 16;      // per CTA: 8 softmax warps
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -733,11 +729,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
       mbar_init(smem_u32(&v_full[i]), 1);
       mbar_init(smem_u32(&k_empty[i]), 1);
       mbar_init(smem_u32(&v_empty[i]), 1);
-      mbar_init(smem_u32(&p_full[i]), 2 * AT_SOFTMAX_WARPS);
+      mbar_init(smem_u32(&s_full[i]), 1);
+      mbar_init(smem_u32(&s_empty[i]), 2 * AT_SOFTMAX_WARPS);
     }
-    mbar_init(smem_u32(s_full), 1);
-    mbar_init(smem_u32(s_empty), 2 * AT_SOFTMAX_WARPS);
-    mbar_init(smem_u32(o_full), 1);
+    mbar_init(smem_u32(p_full), 2 * AT_SOFTMAX_WARPS);
+    mbar_init(smem_u32(pv_done), 1);
     mbar_init(smem_u32(mma_done), 1);
     mbar_init(smem_u32(lbar), AT_SOFTMAX_WARPS);
     *abort_flag = 0;
@@ -759,7 +755,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
   const uint32_t tmem = *tmem_slot;
   const uint32_t tO = tmem;
   const uint32_t tS = tmem + 256;
-  const uint32_t tP = tmem + 384;
   volatile int never = 0;
 
   if (warp == 0 || warp == AT_V_WARP) {
@@ -808,10 +803,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
       const uint32_t idesc_qk = make_idesc_bf16(256, AP_BN, false, false);
       const uint32_t idesc_pv = make_idesc_bf16(256, AT_HD, false, true);
       const uint32_t qaddr = smem_u32(sQ);
+      const uint32_t paddr = smem_u32(sP);
       bool ok = mbar_wait(smem_u32(q_full), 0, p.err, abort_flag);
       auto issue_s = [&](int j) -> bool {
         const int s = j & 1;
-        if (!mbar_wait(smem_u32(&k_full[s]), (j >> 1) & 1, p.err, abort_flag)) return false;
+        const uint32_t ph = (j >> 1) & 1;
+        if (!mbar_wait(smem_u32(&k_full[s]), ph, p.err, abort_flag)) return false;
+        if (!mbar_wait(smem_u32(&s_empty[s]), ph ^ 1u, p.err, abort_flag)) return false;
         tc_fence_after();
         const uint32_t kaddr = smem_u32(sK + s * AP_KH_BYTES);
 #pragma unroll
@@ -819,31 +817,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
           const uint32_t c = kk >> 2, off = (kk & 3) * 32;
           const uint64_t ad = make_sdesc(qaddr + c * (128 * 128) + off, 16, 1024, SWZ_128B);
           const uint64_t bd = make_sdesc(kaddr + c * (64 * 128) + off, 16, 1024, SWZ_128B);
-          mma_bf16_ss_pair(tS, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
+          mma_bf16_ss_pair(tS + s * AP_BN, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
         }
-        mma_commit_pair(smem_u32(s_full), 0x3);
+        mma_commit_pair(smem_u32(&s_full[s]), 0x3);
         mma_commit_pair(smem_u32(&k_empty[s]), 0x3);
         return true;
       };
       if (ok) ok = issue_s(0);
+      if (ok && nkv > 1) ok = issue_s(1);
       for (int j = 0; j < nkv && ok; ++j) {
         const int s = j & 1;
-        if (j + 1 < nkv) {  // S_{j+1} as soon as the softmax warps hold S_j in registers
-          if (!mbar_wait(smem_u32(s_empty), j & 1, p.err, abort_flag)) { ok = false; break; }
-          if (!issue_s(j + 1)) { ok = false; break; }
-        }
-        if (!mbar_wait(smem_u32(&p_full[s]), (j >> 1) & 1, p.err, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(smem_u32(p_full), j & 1, p.err, abort_flag)) { ok = false; break; }
         if (!mbar_wait(smem_u32(&v_full[s]), (j >> 1) & 1, p.err, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t vaddr = smem_u32(sV + s * AP_VH_BYTES);
 #pragma unroll
         for (int kk = 0; kk < AP_BN / 16; ++kk) {
+          const uint32_t c = kk >> 2, off = (kk & 3) * 32;
+          const uint64_t ad = make_sdesc(paddr + c * (128 * 128) + off, 16, 1024, SWZ_128B);
           const uint64_t bd = make_sdesc(vaddr + kk * (16 * 128), AP_BN * 128, 1024, SWZ_128B);
-          mma_bf16_ts_pair(tO, tP + 64 * s + 8 * kk, bd, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+          mma_bf16_ss_pair(tO, ad, bd, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
         }
+        mma_commit_pair(smem_u32(pv_done), 0x3);
         mma_commit_pair(smem_u32(&v_empty[s]), 0x3);
+        if (j + 2 < nkv && !issue_s(j + 2)) { ok = false; break; }
       }
-      if (ok) mma_commit_pair(smem_u32(o_full), 0x3);
       mma_commit_pair(smem_u32(mma_done), 0x1);
       mbar_wait(smem_u32(mma_done), 0, nullptr, &never, 100000000ull);
     }
@@ -861,19 +859,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
     const uint32_t p_full_l = mapa_shared(smem_u32(p_full), 0);
     float l = 0.f;
     bool ok = true;
+    uint8_t* prow = sP + wg * (128 * 128) + row * 128;
     for (int j = 0; j < nkv; ++j) {
       const int s = j & 1;
-      const bool got = mbar_wait(smem_u32(s_full), j & 1, p.err, abort_flag);
+      const bool got = mbar_wait(smem_u32(&s_full[s]), (j >> 1) & 1, p.err, abort_flag);
       __syncwarp();
       if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
       tc_fence_after();
       uint32_t r0[32], r1[32];
-      tmem_ld32(tS + 64 * wg + lane_off, r0);
-      tmem_ld32(tS + 64 * wg + 32 + lane_off, r1);
+      tmem_ld32(tS + s * AP_BN + 64 * wg + lane_off, r0);
+      tmem_ld32(tS + s * AP_BN + 64 * wg + 32 + lane_off, r1);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(s_empty_l);
+      if (lane == 0) mbar_arrive_cluster(s_empty_l + s * 8);
       const int kbase = kv_tile(j) * AP_BN + 64 * wg;
       const int kvalid = p.N - kbase, mlo = klo - kbase, mhi = khi - kbase;
       const bool partial = kvalid < 64 || (mlo < mhi && mlo < 64 && mhi > 0);
@@ -897,20 +896,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
         pk[16 + i] = pack_bf16(e2, e3);
       }
       l += rs;
-      // P_j into TMEM buffer j & 1 (keys [64 wg, +64) -> columns [32 wg, +32)); PV_{j-2},
-      // the last reader of that buffer, completed before S_j did
-      tmem_st32(tP + 64 * s + 32 * wg + lane_off, pk);
-      tmem_wait_st();
+      // the P buffer is free once PV_{j-1} has completed
+      if (j >= 1) {
+        const bool g2 = mbar_wait(smem_u32(pv_done), (j - 1) & 1, p.err, abort_flag);
+        __syncwarp();
+        if (!__all_sync(0xffffffffu, g2)) { ok = false; break; }
+      }
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        uint4 v = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+        *reinterpret_cast<uint4*>(prow + ((q ^ (row & 7)) << 4)) = v;
+      }
+      fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(p_full_l + s * 8);
+      if (lane == 0) mbar_arrive_cluster(p_full_l);
     }
     if (ok) {
       xsum[wg * 128 + row] = l;
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(lbar));
       const bool g3 = mbar_wait(smem_u32(lbar), 0, p.err, abort_flag) &&
-                      mbar_wait(smem_u32(o_full), 0, p.err, abort_flag);
+                      mbar_wait(smem_u32(pv_done), (nkv - 1) & 1, p.err, abort_flag);
       __syncwarp();
       if (__all_sync(0xffffffffu, g3)) {
         tc_fence_after();

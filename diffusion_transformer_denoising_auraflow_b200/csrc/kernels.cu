@@ -95,92 +95,147 @@ __global__ void __launch_bounds__(256) ln_modulate_kernel(const uint16_t* __rest
   }
 }
 
-// Wide-row variant (D = 3072): a CTA serves rows of one sample; (1 + scale)
-// and shift are staged once in shared memory (instead of every row re-reading
-// 24 KB of them from L2 after its reduction); each warp walks
-// LN_ROWS_PER_WARP rows, keeping the row packed as bf16 pairs in registers.
-constexpr int LN_ROWS_PER_WARP = 2;
-constexpr int LN_WARPS = 8;
+// Wide rows (D = 3072), HBM-bound: rows are streamed into shared memory by
+// bulk copies (4 stages of 8 rows = 192 KB in flight per SM, not limited by
+// registers); 8 consumer warps each normalise one row of a stage from shared
+// memory, with (1 + scale) and shift of the CTA's sample staged once.
+// Grid (CTAs per sample, samples); one CTA per SM.
+constexpr int LNB_D = 3072;
+constexpr int LNB_ROWS = 8;
+constexpr int LNB_STAGES = 4;
+constexpr uint32_t LNB_ROW_BYTES = LNB_D * 2;
+constexpr int LNB_THREADS = 32 * (LNB_ROWS + 1);
+constexpr int LNB_SMEM = LNB_STAGES * LNB_ROWS * LNB_ROW_BYTES + 2 * LNB_D * 4 + 128 + 128;
 
-template <int VPL>
-__global__ void __launch_bounds__(256) ln_modulate_rows_kernel(const uint16_t* __restrict__ x,
-                                                               const float* __restrict__ shift,
-                                                               const float* __restrict__ scale, int mod_stride,
-                                                               uint16_t* __restrict__ y, int rows_per_batch, int D,
-                                                               float eps) {
-  extern __shared__ float mod_s[];  // [0, D): 1 + scale, [D, 2D): shift
+__global__ void __launch_bounds__(LNB_THREADS, 1) ln_modulate_bulk_kernel(const uint16_t* __restrict__ x,
+                                                                         const float* __restrict__ shift,
+                                                                         const float* __restrict__ scale,
+                                                                         int mod_stride, uint16_t* __restrict__ y,
+                                                                         int rows_per_batch, float eps, int* err) {
+  extern __shared__ uint8_t lnb_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(lnb_raw) + 127) & ~uintptr_t(127));
+  uint8_t* rowbuf = smem;                                                       // [stage][row] x 6 KB
+  float* mod_s = reinterpret_cast<float*>(smem + LNB_STAGES * LNB_ROWS * LNB_ROW_BYTES);  // 1 + scale | shift
+  uint64_t* full = reinterpret_cast<uint64_t*>(mod_s + 2 * LNB_D);
+  uint64_t* empty = full + LNB_STAGES;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + LNB_STAGES);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.y;
+  const int nchunks = (rows_per_batch + LNB_ROWS - 1) / LNB_ROWS;
+  const size_t row0 = static_cast<size_t>(b) * rows_per_batch;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < LNB_STAGES; ++i) {
+      mbar_init(smem_u32(&full[i]), 1);
+      mbar_init(smem_u32(&empty[i]), LNB_ROWS);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
   const float* sc = scale + static_cast<size_t>(b) * mod_stride;
   const float* sh = shift + static_cast<size_t>(b) * mod_stride;
-  for (int i = threadIdx.x; i < D; i += blockDim.x) {
+  for (int i = threadIdx.x; i < LNB_D; i += blockDim.x) {
     mod_s[i] = 1.0f + sc[i];
-    mod_s[D + i] = sh[i];
+    mod_s[LNB_D + i] = sh[i];
   }
   __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int r0 = (blockIdx.x * LN_WARPS + warp) * LN_ROWS_PER_WARP;
-  const size_t base = static_cast<size_t>(b) * rows_per_batch;
-  for (int k = 0; k < LN_ROWS_PER_WARP; ++k) {
-    const int r = r0 + k;
-    if (r >= rows_per_batch) break;  // uniform across the warp
-    uint4 cur[VPL];
-    const uint4* xr = reinterpret_cast<const uint4*>(x + (base + r) * D);
-#pragma unroll
-    for (int i = 0; i < VPL; ++i) cur[i] = xr[i * 32 + lane];
-    // rows stay packed as bf16 pairs; each pass unpacks on the fly
-    float s = 0.f;
-#pragma unroll
-    for (int i = 0; i < VPL; ++i) {
-      const uint32_t w[4] = {cur[i].x, cur[i].y, cur[i].z, cur[i].w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) s += bf16_lo(w[e]) + bf16_hi(w[e]);
-    }
-    const float mean = warp_sum(s) / D;
-    float ss = 0.f;
-#pragma unroll
-    for (int i = 0; i < VPL; ++i) {
-      const uint32_t w[4] = {cur[i].x, cur[i].y, cur[i].z, cur[i].w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float d0 = bf16_lo(w[e]) - mean, d1 = bf16_hi(w[e]) - mean;
-        ss += d0 * d0 + d1 * d1;
+
+  if (warp == LNB_ROWS) {
+    // producer: one elected thread streams chunks of 8 rows
+    if (lane == 0) {
+      bool ok = true, issued = false;
+      int k = 0;
+      for (int c = blockIdx.x; c < nchunks; c += gridDim.x, ++k) {
+        const int st = k % LNB_STAGES;
+        const uint32_t ph = (k / LNB_STAGES) & 1;
+        if (!mbar_wait(smem_u32(&empty[st]), ph ^ 1u, err, abort_flag)) { ok = false; break; }
+        const int n = min(LNB_ROWS, rows_per_batch - c * LNB_ROWS);
+        mbar_arrive_expect_tx(smem_u32(&full[st]), n * LNB_ROW_BYTES);
+        for (int r = 0; r < n; ++r)
+          bulk_load(smem_u32(rowbuf + (st * LNB_ROWS + r) * LNB_ROW_BYTES),
+                    x + (row0 + static_cast<size_t>(c) * LNB_ROWS + r) * LNB_D, LNB_ROW_BYTES,
+                    smem_u32(&full[st]));
+        issued = true;
+      }
+      if (!ok && issued) {  // let copies already in flight land before the CTA exits
+        const uint64_t t0 = globaltimer();
+        while (globaltimer() - t0 < 200000ull) {
+        }
       }
     }
-    const float rstd = rsqrtf(warp_sum(ss) / D + eps);
-    uint4* yr = reinterpret_cast<uint4*>(y + (base + r) * D);
+    return;
+  }
+  // consumers: warp w normalises row w of every stage
+  constexpr int VPL = LNB_D / 256;
+  int k = 0;
+  for (int c = blockIdx.x; c < nchunks; c += gridDim.x, ++k) {
+    const int st = k % LNB_STAGES;
+    const uint32_t ph = (k / LNB_STAGES) & 1;
+    const bool got = mbar_wait(smem_u32(&full[st]), ph, err, abort_flag);
+    if (!__all_sync(0xffffffffu, got)) break;
+    const int r = c * LNB_ROWS + warp;
+    if (r < rows_per_batch) {
+      const uint4* xr = reinterpret_cast<const uint4*>(rowbuf + (st * LNB_ROWS + warp) * LNB_ROW_BYTES);
+      uint4 cur[VPL];
 #pragma unroll
-    for (int i = 0; i < VPL; ++i) {
-      const int vi = i * 32 + lane;
-      const float4 a0 = *reinterpret_cast<const float4*>(mod_s + vi * 8);
-      const float4 a1 = *reinterpret_cast<const float4*>(mod_s + vi * 8 + 4);
-      const float4 h0 = *reinterpret_cast<const float4*>(mod_s + D + vi * 8);
-      const float4 h1 = *reinterpret_cast<const float4*>(mod_s + D + vi * 8 + 4);
-      const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-      const float hv[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
-      const uint32_t w[4] = {cur[i].x, cur[i].y, cur[i].z, cur[i].w};
-      uint32_t o[4];
+      for (int i = 0; i < VPL; ++i) cur[i] = xr[i * 32 + lane];
+      float s = 0.f;
 #pragma unroll
-      for (int e = 0; e < 4; ++e)
-        o[e] = pack_bf16((bf16_lo(w[e]) - mean) * rstd * av[2 * e] + hv[2 * e],
-                         (bf16_hi(w[e]) - mean) * rstd * av[2 * e + 1] + hv[2 * e + 1]);
-      yr[vi] = make_uint4(o[0], o[1], o[2], o[3]);
+      for (int i = 0; i < VPL; ++i) {
+        const uint32_t w[4] = {cur[i].x, cur[i].y, cur[i].z, cur[i].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) s += bf16_lo(w[e]) + bf16_hi(w[e]);
+      }
+      const float mean = warp_sum(s) * (1.0f / LNB_D);
+      float ss = 0.f;
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) {
+        const uint32_t w[4] = {cur[i].x, cur[i].y, cur[i].z, cur[i].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float d0 = bf16_lo(w[e]) - mean, d1 = bf16_hi(w[e]) - mean;
+          ss += d0 * d0 + d1 * d1;
+        }
+      }
+      const float rstd = rsqrtf(warp_sum(ss) * (1.0f / LNB_D) + eps);
+      uint4* yr = reinterpret_cast<uint4*>(y + (row0 + r) * LNB_D);
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) {
+        const int vi = i * 32 + lane;
+        const float4 a0 = *reinterpret_cast<const float4*>(mod_s + vi * 8);
+        const float4 a1 = *reinterpret_cast<const float4*>(mod_s + vi * 8 + 4);
+        const float4 h0 = *reinterpret_cast<const float4*>(mod_s + LNB_D + vi * 8);
+        const float4 h1 = *reinterpret_cast<const float4*>(mod_s + LNB_D + vi * 8 + 4);
+        const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+        const float hv[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+        const uint32_t w[4] = {cur[i].x, cur[i].y, cur[i].z, cur[i].w};
+        uint32_t o[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          o[e] = pack_bf16((bf16_lo(w[e]) - mean) * rstd * av[2 * e] + hv[2 * e],
+                           (bf16_hi(w[e]) - mean) * rstd * av[2 * e + 1] + hv[2 * e + 1]);
+        yr[vi] = make_uint4(o[0], o[1], o[2], o[3]);
+      }
     }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(&empty[st]));
   }
 }
 
 cudaError_t launch_ln_modulate(const uint16_t* x, const float* shift, const float* scale, int mod_stride,
-                               uint16_t* y, int rows, int rows_per_batch, int D, float eps, cudaStream_t s) {
+                               uint16_t* y, int rows, int rows_per_batch, int D, float eps, cudaStream_t s,
+                               int* err) {
   if (rows <= 0) return cudaSuccess;
   if (D % 8 != 0) return cudaErrorInvalidValue;
-  if (D == 3072 && rows % rows_per_batch == 0) {
+  if (D == LNB_D && rows % rows_per_batch == 0 && (reinterpret_cast<uintptr_t>(x) & 15) == 0) {
     cudaError_t e = small_kernels_set_attributes();
     if (e != cudaSuccess) return e;
     const int nb = rows / rows_per_batch;
-    const int rows_per_block = LN_WARPS * LN_ROWS_PER_WARP;
-    dim3 grid((rows_per_batch + rows_per_block - 1) / rows_per_block, nb);
-    const size_t smem = 2 * static_cast<size_t>(D) * sizeof(float);
-    ln_modulate_rows_kernel<12><<<grid, 32 * LN_WARPS, smem, s>>>(x, shift, scale, mod_stride, y, rows_per_batch, D,
-                                                                  eps);
+    static int sms = 0;
+    if (!sms) sms = device_sm_count();
+    const int nchunks = (rows_per_batch + LNB_ROWS - 1) / LNB_ROWS;
+    const int per = max(1, min(nchunks, (sms + nb - 1) / nb));
+    ln_modulate_bulk_kernel<<<dim3(per, nb), LNB_THREADS, LNB_SMEM, s>>>(x, shift, scale, mod_stride, y,
+                                                                         rows_per_batch, eps, err);
     return cudaGetLastError();
   }
   const int nvec = D / 8;
@@ -270,8 +325,7 @@ cudaError_t small_kernels_set_attributes() {
   int dev = 0;
   cudaGetDevice(&dev);
   if ((done >> dev) & 1u) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(ln_modulate_rows_kernel<12>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       2 * 3072 * static_cast<int>(sizeof(float)));
+  cudaError_t e = cudaFuncSetAttribute(ln_modulate_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, LNB_SMEM);
   if (e == cudaSuccess) e = gemv_attr<1>();
   if (e == cudaSuccess) e = gemv_attr<2>();
   if (e == cudaSuccess) e = gemv_attr<4>();
