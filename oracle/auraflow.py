@@ -358,32 +358,103 @@ def text_key_mask(text_len, n_registers: int, L: int, n_image: int):
     return m
 
 
-def qkv_normed(y, wq, wk, wv, heads: int, eps: float):
+def _w8(w, fp8):
+    """The weight as the GEMM sees it: as is, or per-output-row e4m3."""
+    return fake_quant_rows(w) if fp8 else _f(w)
+
+
+def qkv_normed(y, wq, wk, wv, heads: int, eps: float, fp8: bool = False):
     """Bias-free Q/K/V projections, then per-head LayerNorm of Q and K (not V).
 
     [ARCH §模型概述] QK Norm and no bias; [ARCH §注意力处理器与 QKV 融合]
     norm_q/norm_k (image) and norm_added_q/norm_added_k (text).
     READING: the QK-norm is the same affine-free fp32 LayerNorm, eps 1e-6.
+    fp8: activations and weights pass through per-row e4m3 (8-bit variant).
     """
-    q = split_heads(y @ _f(wq).T, heads)
-    k = split_heads(y @ _f(wk).T, heads)
-    v = split_heads(y @ _f(wv).T, heads)
+    if fp8:
+        y = fake_quant_rows(y)
+    q = split_heads(y @ _w8(wq, fp8).T, heads)
+    k = split_heads(y @ _w8(wk, fp8).T, heads)
+    v = split_heads(y @ _w8(wv, fp8).T, heads)
     return layer_norm(q, eps), layer_norm(k, eps), v
 
 
-def feed_forward(y, w1, w2, w3):
+def feed_forward(y, w1, w2, w3, fp8: bool = False):
     """out_projection(silu(linear_1 y) * linear_2 y), all bias-free.
 
     [ARCH §FeedForward], [PIPE §深入源码] (SiLU-gated FFN).
     """
-    return (silu(y @ _f(w1).T) * (y @ _f(w2).T)) @ _f(w3).T
+    if fp8:   # 8-bit variant: the up-projections' inputs; the down-projection stays as is
+        y = fake_quant_rows(y)
+    return (silu(y @ _w8(w1, fp8).T) * (y @ _w8(w2, fp8).T)) @ _f(w3).T
+
+
+# --------------------------------------------------------------------------
+# 8-bit variant (extension): e4m3 weights and activations for the QKV and
+# FFN up-projections
+# --------------------------------------------------------------------------
+# The pipeline guide loads the transformer with 8-bit weights
+# ([PIPE] bitsandbytes quantisation sections).  The variant here is the
+# tensor-core-native form of that idea: the inputs of the two GEMMs whose
+# activations come straight out of the LayerNorm+modulate step (the fused
+# QKV projections and the FFN up-projections) are rounded to the e4m3 format,
+# each activation row (token) and each weight row (output channel) with its
+# own fp32 scale, and the product is rescaled by both scales.
+# READING: per-row absolute-maximum scaling, amax -> 448 (the largest finite
+# e4m3 value); the output projections and FFN down-projections stay bf16.
+
+E4M3_MAX = 448.0
+
+
+def e4m3_round(x):
+    """Nearest value of the 8-bit e4m3 format (1 sign bit, 4 exponent bits
+    with bias 7, 3 mantissa bits, no infinities, largest finite 448, smallest
+    subnormal 2^-9), ties to even, saturating at +-448.
+
+    Normal binade [2^e, 2^(e+1)) for e >= -6 holds 8 values spaced 2^(e-3);
+    below 2^-6 the spacing is the subnormal step 2^-9.
+    """
+    x = _f(x)
+    a = np.abs(x)
+    with np.errstate(divide="ignore"):
+        e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    e = np.maximum(e, -6.0)
+    step = np.exp2(e - 3.0)
+    q = np.round(a / step) * step          # np.round: half to even
+    q = np.minimum(q, E4M3_MAX)
+    return np.copysign(q, x)
+
+
+def quantize_rows_e4m3(x):
+    """Per-row e4m3 quantisation in the kernel's precision: with a = max |x|
+    over the row (fp32), inv = 448 / a and s = a / 448 (fp32 divisions; 1
+    for an all-zero row), the codes are e4m3(fp32(x * inv)).  Returns
+    (codes as float64 values, s as float32)."""
+    x32 = np.asarray(x, dtype=np.float64).astype(np.float32)
+    amax = np.max(np.abs(x32), axis=-1)
+    nz = amax > 0
+    safe = np.where(nz, amax, np.float32(1.0)).astype(np.float32)
+    inv = np.where(nz, np.float32(E4M3_MAX) / safe, np.float32(1.0)).astype(np.float32)
+    scale = np.where(nz, safe / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
+    y = (x32 * inv[..., None]).astype(np.float32)
+    return e4m3_round(y.astype(np.float64)), scale
+
+
+def dequantize_rows(codes, scale):
+    return _f(codes) * np.asarray(scale, dtype=np.float64)[..., None]
+
+
+def fake_quant_rows(x):
+    """x -> e4m3 codes x per-row scale, as the 8-bit GEMMs see it."""
+    q, s = quantize_rows_e4m3(x)
+    return dequantize_rows(q, s)
 
 
 # --------------------------------------------------------------------------
 # c10. Blocks
 # --------------------------------------------------------------------------
 
-def single_block_mod(x, mod, w, prefix, heads, eps, key_mask=None):
+def single_block_mod(x, mod, w, prefix, heads, eps, key_mask=None, fp8=False):
     """AuraFlowSingleTransformerBlock given its six modulation vectors.
 
     [ARCH §单 DiT 块]: adaLN-Zero DiT block on one (concatenated) sequence,
@@ -395,21 +466,21 @@ def single_block_mod(x, mod, w, prefix, heads, eps, key_mask=None):
     x = _f(x)
     y = modulate(x, mod["shift_msa"], mod["scale_msa"], eps)
     q, k, v = qkv_normed(y, w[prefix + "attn.to_q.weight"], w[prefix + "attn.to_k.weight"],
-                         w[prefix + "attn.to_v.weight"], heads, eps)
+                         w[prefix + "attn.to_v.weight"], heads, eps, fp8)
     o = merge_heads(attention(q, k, v, key_mask=key_mask))
     x = x + mod["gate_msa"][:, None, :] * (o @ _f(w[prefix + "attn.to_out.0.weight"]).T)
     y = modulate(x, mod["shift_mlp"], mod["scale_mlp"], eps)
     f = feed_forward(y, w[prefix + "ff.linear_1.weight"], w[prefix + "ff.linear_2.weight"],
-                     w[prefix + "ff.out_projection.weight"])
+                     w[prefix + "ff.out_projection.weight"], fp8)
     return x + mod["gate_mlp"][:, None, :] * f
 
 
-def single_block(x, temb, w, prefix, cfg: Config, key_mask=None):
+def single_block(x, temb, w, prefix, cfg: Config, key_mask=None, fp8=False):
     mod = ada_ln_zero(temb, w[prefix + "norm1.linear.weight"])
-    return single_block_mod(x, mod, w, prefix, cfg.num_attention_heads, cfg.ln_eps, key_mask)
+    return single_block_mod(x, mod, w, prefix, cfg.num_attention_heads, cfg.ln_eps, key_mask, fp8)
 
 
-def joint_block_mod(img, txt, mod_i, mod_t, w, prefix, heads, eps, key_mask=None):
+def joint_block_mod(img, txt, mod_i, mod_t, w, prefix, heads, eps, key_mask=None, fp8=False):
     """AuraFlowJointTransformerBlock given both streams' modulation vectors.
 
     [ARCH §联合注意力块]: two residual streams (image, text), each with its
@@ -426,9 +497,9 @@ def joint_block_mod(img, txt, mod_i, mod_t, w, prefix, heads, eps, key_mask=None
     yi = modulate(img, mod_i["shift_msa"], mod_i["scale_msa"], eps)
     yt = modulate(txt, mod_t["shift_msa"], mod_t["scale_msa"], eps)
     qi, ki, vi = qkv_normed(yi, w[prefix + "attn.to_q.weight"], w[prefix + "attn.to_k.weight"],
-                            w[prefix + "attn.to_v.weight"], heads, eps)
+                            w[prefix + "attn.to_v.weight"], heads, eps, fp8)
     qt, kt, vt = qkv_normed(yt, w[prefix + "attn.add_q_proj.weight"], w[prefix + "attn.add_k_proj.weight"],
-                            w[prefix + "attn.add_v_proj.weight"], heads, eps)
+                            w[prefix + "attn.add_v_proj.weight"], heads, eps, fp8)
     q = np.concatenate([qt, qi], axis=2)
     k = np.concatenate([kt, ki], axis=2)
     v = np.concatenate([vt, vi], axis=2)
@@ -440,17 +511,17 @@ def joint_block_mod(img, txt, mod_i, mod_t, w, prefix, heads, eps, key_mask=None
     yt = modulate(txt, mod_t["shift_mlp"], mod_t["scale_mlp"], eps)
     img = img + mod_i["gate_mlp"][:, None, :] * feed_forward(
         yi, w[prefix + "ff.linear_1.weight"], w[prefix + "ff.linear_2.weight"],
-        w[prefix + "ff.out_projection.weight"])
+        w[prefix + "ff.out_projection.weight"], fp8)
     txt = txt + mod_t["gate_mlp"][:, None, :] * feed_forward(
         yt, w[prefix + "ff_context.linear_1.weight"], w[prefix + "ff_context.linear_2.weight"],
-        w[prefix + "ff_context.out_projection.weight"])
+        w[prefix + "ff_context.out_projection.weight"], fp8)
     return txt, img
 
 
-def joint_block(img, txt, temb, w, prefix, cfg: Config, key_mask=None):
+def joint_block(img, txt, temb, w, prefix, cfg: Config, key_mask=None, fp8=False):
     mod_i = ada_ln_zero(temb, w[prefix + "norm1.linear.weight"])
     mod_t = ada_ln_zero(temb, w[prefix + "norm1_context.linear.weight"])
-    return joint_block_mod(img, txt, mod_i, mod_t, w, prefix, cfg.num_attention_heads, cfg.ln_eps, key_mask)
+    return joint_block_mod(img, txt, mod_i, mod_t, w, prefix, cfg.num_attention_heads, cfg.ln_eps, key_mask, fp8)
 
 
 # --------------------------------------------------------------------------
@@ -561,7 +632,7 @@ def output_stage(x_img, temb, w, cfg: Config, H: int, W: int):
     return unpatchify(o, p, cfg.out_channels, H // p, W // p)
 
 
-def transformer_forward(latents, text_emb, t, w, cfg: Config, text_len=None):
+def transformer_forward(latents, text_emb, t, w, cfg: Config, text_len=None, fp8=False):
     """AuraFlowTransformer2DModel.forward -> velocity [B, C_out, H, W].
 
     [ARCH §前向传播流程]: embed; num_mmdit_layers joint blocks updating both
@@ -570,6 +641,7 @@ def transformer_forward(latents, text_emb, t, w, cfg: Config, text_len=None):
     unpatchify.  ``t`` is the model time in [0, 1] (timestep / 1000).
     ``text_len`` (optional, [B]): real prompt tokens per sample; the rest of
     the L text tokens are padding that no attention reads (``text_key_mask``).
+    ``fp8``: the 8-bit variant of the QKV and FFN up-projections.
     """
     latents = _f(latents)
     H, W = latents.shape[2], latents.shape[3]
@@ -579,10 +651,10 @@ def transformer_forward(latents, text_emb, t, w, cfg: Config, text_len=None):
     if text_len is not None:
         mask = text_key_mask(text_len, cfg.num_register_tokens, nt - cfg.num_register_tokens, img.shape[1])
     for i in range(cfg.num_mmdit_layers):
-        txt, img = joint_block(img, txt, temb, w, f"joint_transformer_blocks.{i}.", cfg, mask)
+        txt, img = joint_block(img, txt, temb, w, f"joint_transformer_blocks.{i}.", cfg, mask, fp8)
     x = np.concatenate([txt, img], axis=1)
     for i in range(cfg.num_single_dit_layers):
-        x = single_block(x, temb, w, f"single_transformer_blocks.{i}.", cfg, mask)
+        x = single_block(x, temb, w, f"single_transformer_blocks.{i}.", cfg, mask, fp8)
     return output_stage(x[:, nt:], temb, w, cfg, H, W)
 
 
