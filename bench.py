@@ -56,6 +56,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--seed", type=int, default=4)
+    ap.add_argument("--fp8", action="store_true",
+                    help="8-bit variant: e4m3 QKV and FFN up-projections (af_weights_quantize_fp8)")
     ap.add_argument("--direct", action="store_true",
                     help="time the per-step entry point (af_denoise_step) instead of the sampler plan")
     ap.add_argument("--case", default="step", choices=["step", "single_block"],
@@ -253,6 +255,9 @@ def run_af(args, rank, world, local_rank):
     cfg = af.Config.default(pos_embed_max_size=G * G)
     w = af.Weights(cfg, local_rank)
     make_weights(af, torch, w, args.seed, device)
+    if args.fp8:
+        w.quantize_fp8()
+        torch.cuda.synchronize()
     s = af.Scratch(w, 2, Ni, L)
     stream = torch.cuda.Stream(device)
     torch.cuda.set_stream(stream)   # graphs cannot be captured on the legacy default stream
@@ -369,10 +374,18 @@ def run_af(args, rank, world, local_rank):
                 traffic = float(tr["bytes_per_launch"])
         except (OSError, ValueError, KeyError):
             traffic = None
-    roofline = {"bound": "tensor", "kernel": "gemm_bf16_tcgen05_pair (M >= 1024) / gemm_bf16_tcgen05",
+    peak = pk["bf16_tflops_sustained"]
+    peak_note = f"{pk['source']} (sustained cuBLAS bf16)"
+    if args.fp8:
+        # e4m3 GEMMs (QKV, FFN up) run at twice the bf16 rate nominally; weight the peak by their FLOP share
+        D, F = model_dims()[:2]
+        f8 = (3.0 * D * D + 2.0 * D * F) / (4.0 * D * D + 3.0 * D * F)
+        peak = 1.0 / (f8 / (2.0 * peak) + (1.0 - f8) / peak)
+        peak_note += f"; {f8:.0%} of GEMM FLOPs e4m3 at 2x (nominal ratio), FLOP-weighted"
+    roofline = {"bound": "tensor", "kernel": "gemm_tcgen05_pair (M >= 1024) / gemm_tcgen05",
                 "achieved": gemm_tflops,
-                "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s", "frac": gemm_tflops / pk["bf16_tflops_sustained"],
-                "traffic": traffic, "peak_source": f"{pk['source']} (sustained cuBLAS bf16)",
+                "peak": peak, "unit": "TFLOP/s", "frac": gemm_tflops / peak,
+                "traffic": None if args.fp8 else traffic, "peak_source": peak_note,
                 "flops_per_launch": gemm_flops_launch, "ms_per_launch": gemm_ms_launch}
     step_ms_classes = [x / n_prof for x in ms]
 
@@ -410,7 +423,8 @@ def run_af(args, rank, world, local_rank):
         line = {
             "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": t_max / args.steps * 1000.0, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": "e4m3 (QKV, FFN up) + bf16" if args.fp8 else "bf16",
             "data": "synthetic (seeded random weights ~N(0,0.02^2), positions ~N(0,0.1^2); latents, text ~N(0,1))",
             "config": {"workload": wl["name"], "cfg_batch": 2, "tokens": 8 + L + Ni, "global_batch": 2 * world,
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",

@@ -85,6 +85,10 @@ _SIGS = {
     "af_ln_modulate": [_P, _P, _P, _I, _P, _I, _I, _I, _F, _P],
     "af_linear": [_P, _P, _P, _I, _I, _I, _P],
     "af_attention": [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _I, _I, _P],
+    "af_weights_quantize_fp8": [_P, _I, _P],
+    "af_quantize_rows_e4m3": [_P, _I, _I, _P, _P, _P],
+    "af_ln_modulate_e4m3": [_P, _P, _P, _I, _P, _P, _I, _I, _I, _F, _P],
+    "af_linear_fp8": [_P, _P, _P, _P, _P, _I, _I, _I, _P],
     "af_status_string": [_I],
     "af_last_error": [],
 }
@@ -181,6 +185,12 @@ class Weights:
         _check(lib.af_weights_set(self.handle, self.find(name), ctypes.c_void_p(tensor.data_ptr()),
                                   1 if tensor.is_cuda else 0, _stream(stream) if tensor.is_cuda else None),
                f"af_weights_set({name})")
+
+    def quantize_fp8(self, enable: bool = True, stream=None):
+        """Switch the QKV and FFN up-projections to the 8-bit (e4m3) variant
+        (re-quantising the current weights), or back to bf16."""
+        _check(lib.af_weights_quantize_fp8(self.handle, 1 if enable else 0, _stream(stream)),
+               "af_weights_quantize_fp8")
 
     def nbytes(self) -> int:
         b = ctypes.c_size_t()
@@ -376,3 +386,29 @@ def attention(q, k, v, o, qk_normalized: bool = False, key_len=None, key_base: i
                             _dev(o, torch.bfloat16, "o"), B, H, N, hd, 1 if qk_normalized else 0,
                             _lens(key_len, B, "key_len"), int(key_base), int(key_end), _stream(stream)),
            "af_attention")
+
+
+def quantize_rows_e4m3(x, q, scale, stream=None):
+    """Per-row e4m3 codes of bf16 x [rows, cols] into uint8 q and float scale [rows]."""
+    rows, cols = x.shape
+    _check(lib.af_quantize_rows_e4m3(_dev(x, torch.bfloat16, "x"), rows, cols, _dev(q, torch.uint8, "q"),
+                                     _dev(scale, torch.float32, "scale"), _stream(stream)), "af_quantize_rows_e4m3")
+
+
+def ln_modulate_e4m3(x, shift, scale, mod_stride: int, y8, yscale, eps: float, stream=None):
+    B, N, D = x.shape
+    _check(lib.af_ln_modulate_e4m3(_dev(x, torch.bfloat16, "x"), ctypes.c_void_p(shift.data_ptr()),
+                                   ctypes.c_void_p(scale.data_ptr()), mod_stride, _dev(y8, torch.uint8, "y8"),
+                                   _dev(yscale, torch.float32, "yscale"), B, N, D, float(eps), _stream(stream)),
+           "af_ln_modulate_e4m3")
+
+
+def linear_fp8(A8, a_scale, W8, w_scale, C, stream=None):
+    """C = diag(a_scale) (A8 W8^T) diag(w_scale) with e4m3 codes A8 [M, K], W8 [N, K]."""
+    M, K = A8.shape
+    N = W8.shape[0]
+    if w_scale.numel() < (N + 255) // 256 * 256:
+        raise ValueError("w_scale must hold ceil(N / 256) * 256 entries")
+    _check(lib.af_linear_fp8(_dev(A8, torch.uint8, "A8"), _dev(a_scale, torch.float32, "a_scale"),
+                             _dev(W8, torch.uint8, "W8"), _dev(w_scale, torch.float32, "w_scale"),
+                             _dev(C, torch.bfloat16, "C"), M, N, K, _stream(stream)), "af_linear_fp8")

@@ -34,6 +34,11 @@ struct GemmParams {
   float eps;
   int num_m_tiles, num_n_tiles, num_tiles, group_n;
   int* err;                // device error word
+  // 8-bit GEMM (A and W in e4m3) when w_scale != nullptr: acc[m, n] is
+  // rescaled by a_scale[m] * w_scale[weight row of n]; w_scale must be
+  // readable 32 rows past every weight row the GEMM touches (pad to 256)
+  const float* a_scale = nullptr;
+  const float* w_scale = nullptr;
 };
 
 constexpr int GEMM_BM = 128;
@@ -45,7 +50,7 @@ constexpr int GEMM_SMEM_BYTES = GEMM_STAGES * (GEMM_BM + GEMM_BN) * GEMM_BK * 2 
 
 // Host helpers (gemm.cu)
 bool encode_tmap_2d(CUtensorMap* map, const void* ptr, uint64_t inner, uint64_t outer, uint64_t row_bytes,
-                    uint32_t box_inner, uint32_t box_outer);
+                    uint32_t box_inner, uint32_t box_outer, bool bytes = false);
 bool encode_tmap_3d(CUtensorMap* map, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1_bytes,
                     uint64_t s2_bytes, uint32_t b0, uint32_t b1, uint32_t b2);
 cudaError_t launch_gemm(const GemmParams& p_in, const void* A, const void* W, int W_rows, cudaStream_t stream,
@@ -78,7 +83,9 @@ cudaError_t launch_attention(const AttnParams& p, const uint16_t* q, const uint1
 // Small kernels (kernels.cu)
 cudaError_t launch_ln_modulate(const uint16_t* x, const float* shift, const float* scale, int mod_stride,
                                uint16_t* y, int rows, int rows_per_batch, int D, float eps, cudaStream_t s,
-                               int* err = nullptr);
+                               int* err = nullptr, uint8_t* y8 = nullptr, float* yscale = nullptr);
+// y8 != nullptr: write e4m3 codes + per-row scales (y8 [rows, D], yscale [rows]) instead of bf16 y
+cudaError_t launch_quantize_rows_e4m3(const uint16_t* x, int rows, int K, uint8_t* q, float* scale, cudaStream_t s);
 cudaError_t launch_timestep_mlp(const float* t, int B, const uint16_t* w1, const uint16_t* b1, const uint16_t* w2,
                                 const uint16_t* b2, int C, int D, float* feat, float* h1, float* temb, cudaStream_t s);
 cudaError_t launch_modulation(const float* temb, int B, int D, const uint16_t* w, int rows, float* out,

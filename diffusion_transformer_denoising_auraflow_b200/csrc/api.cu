@@ -89,6 +89,15 @@ struct af_weights {
   size_t ada_rows = 0;
   std::vector<size_t> unit_row;  // first row of unit u (joint i: 2i img, 2i+1 txt; single j: 2J + j)
   size_t pf_row = 0;             // first row of norm_out
+  // 8-bit variant: e4m3 copies of the fused QKV and FFN up-projection
+  // weights with one fp32 scale per row (af_weights_quantize_fp8).  Each
+  // region starts at a multiple of 256 rows of the 8-bit pack, so every
+  // scale a 256-column tile can touch exists.
+  bool fp8 = false;
+  uint8_t* fp8_codes = nullptr;  // [fp8_rows, D]
+  float* fp8_scales = nullptr;   // [fp8_rows]
+  size_t fp8_rows = 0;
+  std::unordered_map<std::string, size_t> fp8_row;  // region's first tensor name -> first row
 
   const uint16_t* ptr(const std::string& n) const {
     auto it = index.find(n);
@@ -105,6 +114,8 @@ struct af_scratch {
   int* err;
   float *temb, *h1, *mods, *tfeat;
   uint16_t *y, *q, *k, *v, *o, *h;
+  uint8_t* y8;    // 8-bit variant: e4m3 codes of y, one fp32 scale per row in yscale
+  float* yscale;
   uint16_t *img, *txt, *x;
   float *lat2, *vel, *tvec;  // denoise step: CFG-duplicated latents, velocity, model times
   int sms;
@@ -273,9 +284,26 @@ af_status run_gemm(af_scratch* s, const GemmParams& p, const void* A, const void
   return AF_OK;
 }
 
+// A GEMM operand: bf16 (scale == nullptr) or e4m3 codes with one fp32 scale per row.
+struct Operand {
+  const void* ptr;
+  const float* scale;
+};
+
+// The weight region starting at tensor `name` as the GEMM reads it.
+Operand weight_op(const af_weights* w, const std::string& name) {
+  if (w->fp8) {
+    auto it = w->fp8_row.find(name);
+    if (it != w->fp8_row.end())
+      return {w->fp8_codes + it->second * static_cast<size_t>(w->d.D), w->fp8_scales + it->second};
+  }
+  return {w->ptr(name), nullptr};
+}
+
 // QKV projection of one stream with per-head LayerNorm of Q and K.
-af_status qkv(const af_weights* w, af_scratch* s, const uint16_t* y, int B, int rows, const uint16_t* wqkv,
-              int row_off, int n_total, cudaStream_t st) {
+af_status qkv(const af_weights* w, af_scratch* s, Operand y, int B, int rows, Operand wqkv, int row_off,
+              int n_total, cudaStream_t st) {
+  if ((y.scale != nullptr) != (wqkv.scale != nullptr)) return AF_ERR_UNSUPPORTED;
   const Derived& d = w->d;
   GemmParams p = gemm_base(s, B * rows, 3 * d.D, d.D, EPI_QKV, rows);
   p.q = s->q;
@@ -287,7 +315,9 @@ af_status qkv(const af_weights* w, af_scratch* s, const uint16_t* y, int B, int 
   p.qkv_row_off = row_off;
   p.D = d.D;
   p.eps = w->cfg.ln_eps;
-  return run_gemm(s, p, y, wqkv, 3 * d.D, st);
+  p.a_scale = y.scale;
+  p.w_scale = wqkv.scale;
+  return run_gemm(s, p, y.ptr, wqkv.ptr, 3 * d.D, st);
 }
 
 // x += gate[b] * (A W^T)
@@ -302,13 +332,15 @@ af_status gated_residual(af_scratch* s, const uint16_t* A, int B, int rows, int 
 }
 
 // h = silu(y W1^T) * (y W2^T), W1 and W2 interleaved in 128-row groups ([2F, D])
-af_status swiglu(const af_weights* w, af_scratch* s, const uint16_t* y, int M, const uint16_t* w12,
-                 uint16_t* h, cudaStream_t st) {
+af_status swiglu(const af_weights* w, af_scratch* s, Operand y, int M, Operand w12, uint16_t* h, cudaStream_t st) {
+  if ((y.scale != nullptr) != (w12.scale != nullptr)) return AF_ERR_UNSUPPORTED;
   const Derived& d = w->d;
   GemmParams p = gemm_base(s, M, d.F, d.D, EPI_SWIGLU, M);
   p.out = h;
   p.ldo = d.F;
-  return run_gemm(s, p, y, w12, 2 * d.F, st);
+  p.a_scale = y.scale;
+  p.w_scale = w12.scale;
+  return run_gemm(s, p, y.ptr, w12.ptr, 2 * d.F, st);
 }
 
 // Padding of the text part: for sample b the keys [base + len[b], end) are
@@ -353,10 +385,13 @@ af_status attention(const af_weights* w, af_scratch* s, int B, int N, uint16_t* 
   return AF_OK;
 }
 
+// LayerNorm + modulate of `rows` rows into y (bf16), or into e4m3 codes y8 +
+// row scales ys when y8 != nullptr.
 af_status ln_mod(af_scratch* s, const uint16_t* x, const float* shift, const float* scale, int mod_stride, uint16_t* y,
-                 int rows, int rows_per_batch, int D, float eps, cudaStream_t st) {
-  LaunchScope ls(s, KC_LN, 4.0 * rows * D, st);
-  cudaError_t e = launch_ln_modulate(x, shift, scale, mod_stride, y, rows, rows_per_batch, D, eps, st, s->err);
+                 int rows, int rows_per_batch, int D, float eps, cudaStream_t st, uint8_t* y8 = nullptr,
+                 float* ys = nullptr) {
+  LaunchScope ls(s, KC_LN, (y8 ? 3.0 : 4.0) * rows * D, st);
+  cudaError_t e = launch_ln_modulate(x, shift, scale, mod_stride, y, rows, rows_per_batch, D, eps, st, s->err, y8, ys);
   return e == cudaSuccess ? AF_OK : cuda_fail(e);
 }
 
@@ -382,19 +417,27 @@ af_status joint_block_impl(const af_weights* w, af_scratch* s, int layer, uint16
   uint16_t* o_txt = s->o + static_cast<size_t>(B) * Ni * D;
   uint16_t* h_img = s->h;
   uint16_t* h_txt = s->h + static_cast<size_t>(B) * Ni * d.F;
+  // 8-bit variant: the LayerNorm outputs feeding QKV and FFN-up become e4m3 + row scales
+  const bool f8 = w->fp8;
+  uint8_t* q8_img = f8 ? s->y8 : nullptr;
+  uint8_t* q8_txt = f8 ? s->y8 + static_cast<size_t>(B) * Ni * D : nullptr;
+  float* ys_img = f8 ? s->yscale : nullptr;
+  float* ys_txt = f8 ? s->yscale + static_cast<size_t>(B) * Ni : nullptr;
+  const Operand a_img = f8 ? Operand{q8_img, ys_img} : Operand{y_img, nullptr};
+  const Operand a_txt = f8 ? Operand{q8_txt, ys_txt} : Operand{y_txt, nullptr};
 
-  AF_TRY(ln_mod(s, img, mi + 0 * D, mi + 1 * D, mod_stride, y_img, B * Ni, Ni, D, eps, st));
-  AF_TRY(ln_mod(s, txt, mt + 0 * D, mt + 1 * D, mod_stride, y_txt, B * Nt, Nt, D, eps, st));
-  AF_TRY(qkv(w, s, y_txt, B, Nt, w->ptr(pre + "attn.add_q_proj.weight"), 0, N, st));
-  AF_TRY(qkv(w, s, y_img, B, Ni, w->ptr(pre + "attn.to_q.weight"), Nt, N, st));
+  AF_TRY(ln_mod(s, img, mi + 0 * D, mi + 1 * D, mod_stride, y_img, B * Ni, Ni, D, eps, st, q8_img, ys_img));
+  AF_TRY(ln_mod(s, txt, mt + 0 * D, mt + 1 * D, mod_stride, y_txt, B * Nt, Nt, D, eps, st, q8_txt, ys_txt));
+  AF_TRY(qkv(w, s, a_txt, B, Nt, weight_op(w, pre + "attn.add_q_proj.weight"), 0, N, st));
+  AF_TRY(qkv(w, s, a_img, B, Ni, weight_op(w, pre + "attn.to_q.weight"), Nt, N, st));
   AF_TRY(attention(w, s, B, N, o_txt, o_img, Nt, km, st));
   AF_TRY(gated_residual(s, o_img, B, Ni, D, w->ptr(pre + "attn.to_out.0.weight"), D, img, mi + 2 * D, mod_stride, st));
   AF_TRY(gated_residual(s, o_txt, B, Nt, D, w->ptr(pre + "attn.to_add_out.weight"), D, txt, mt + 2 * D, mod_stride,
                         st));
-  AF_TRY(ln_mod(s, img, mi + 3 * D, mi + 4 * D, mod_stride, y_img, B * Ni, Ni, D, eps, st));
-  AF_TRY(ln_mod(s, txt, mt + 3 * D, mt + 4 * D, mod_stride, y_txt, B * Nt, Nt, D, eps, st));
-  AF_TRY(swiglu(w, s, y_img, B * Ni, w->ptr(pre + "ff.linear_1.weight"), h_img, st));
-  AF_TRY(swiglu(w, s, y_txt, B * Nt, w->ptr(pre + "ff_context.linear_1.weight"), h_txt, st));
+  AF_TRY(ln_mod(s, img, mi + 3 * D, mi + 4 * D, mod_stride, y_img, B * Ni, Ni, D, eps, st, q8_img, ys_img));
+  AF_TRY(ln_mod(s, txt, mt + 3 * D, mt + 4 * D, mod_stride, y_txt, B * Nt, Nt, D, eps, st, q8_txt, ys_txt));
+  AF_TRY(swiglu(w, s, a_img, B * Ni, weight_op(w, pre + "ff.linear_1.weight"), h_img, st));
+  AF_TRY(swiglu(w, s, a_txt, B * Nt, weight_op(w, pre + "ff_context.linear_1.weight"), h_txt, st));
   AF_TRY(gated_residual(s, h_img, B, Ni, d.F, w->ptr(pre + "ff.out_projection.weight"), D, img, mi + 5 * D,
                         mod_stride, st));
   AF_TRY(gated_residual(s, h_txt, B, Nt, d.F, w->ptr(pre + "ff_context.out_projection.weight"), D, txt, mt + 5 * D,
@@ -408,12 +451,16 @@ af_status single_block_impl(const af_weights* w, af_scratch* s, int layer, uint1
   const int D = d.D;
   const float eps = w->cfg.ln_eps;
   const std::string pre = "single_transformer_blocks." + std::to_string(layer) + ".";
-  AF_TRY(ln_mod(s, x, m + 0 * D, m + 1 * D, mod_stride, s->y, B * N, N, D, eps, st));
-  AF_TRY(qkv(w, s, s->y, B, N, w->ptr(pre + "attn.to_q.weight"), 0, N, st));
+  const bool f8 = w->fp8;
+  uint8_t* q8 = f8 ? s->y8 : nullptr;
+  float* ys = f8 ? s->yscale : nullptr;
+  const Operand a = f8 ? Operand{q8, ys} : Operand{s->y, nullptr};
+  AF_TRY(ln_mod(s, x, m + 0 * D, m + 1 * D, mod_stride, s->y, B * N, N, D, eps, st, q8, ys));
+  AF_TRY(qkv(w, s, a, B, N, weight_op(w, pre + "attn.to_q.weight"), 0, N, st));
   AF_TRY(attention(w, s, B, N, s->o, s->o, 0, km, st));
   AF_TRY(gated_residual(s, s->o, B, N, D, w->ptr(pre + "attn.to_out.0.weight"), D, x, m + 2 * D, mod_stride, st));
-  AF_TRY(ln_mod(s, x, m + 3 * D, m + 4 * D, mod_stride, s->y, B * N, N, D, eps, st));
-  AF_TRY(swiglu(w, s, s->y, B * N, w->ptr(pre + "ff.linear_1.weight"), s->h, st));
+  AF_TRY(ln_mod(s, x, m + 3 * D, m + 4 * D, mod_stride, s->y, B * N, N, D, eps, st, q8, ys));
+  AF_TRY(swiglu(w, s, a, B * N, weight_op(w, pre + "ff.linear_1.weight"), s->h, st));
   AF_TRY(gated_residual(s, s->h, B, N, d.F, w->ptr(pre + "ff.out_projection.weight"), D, x, m + 5 * D, mod_stride,
                         st));
   return AF_OK;
@@ -528,6 +575,8 @@ af_status af_weights_create(const af_config* cfg, int device, af_weights** out) 
 void af_weights_destroy(af_weights* w) {
   if (!w) return;
   if (w->base) cudaFree(w->base);
+  if (w->fp8_codes) cudaFree(w->fp8_codes);
+  if (w->fp8_scales) cudaFree(w->fp8_scales);
   delete w;
 }
 
@@ -586,6 +635,71 @@ af_status af_weights_set(af_weights* w, int id, const uint16_t* src, int src_is_
   return AF_OK;
 }
 
+af_status af_weights_quantize_fp8(af_weights* w, int enable, void* stream) {
+  if (!w) return AF_ERR_INVALID_ARG;
+  if (!enable) {
+    if (w->fp8_codes) cudaFree(w->fp8_codes);
+    if (w->fp8_scales) cudaFree(w->fp8_scales);
+    w->fp8_codes = nullptr;
+    w->fp8_scales = nullptr;
+    w->fp8_rows = 0;
+    w->fp8_row.clear();
+    w->fp8 = false;
+    return AF_OK;
+  }
+  const af_config& c = w->cfg;
+  const int D = w->d.D;
+  const size_t qkv_rows = 3 * static_cast<size_t>(D), up_rows = 2 * static_cast<size_t>(w->d.F);
+  std::vector<std::pair<std::string, size_t>> regions;
+  for (int i = 0; i < c.num_mmdit_layers; ++i) {
+    const std::string b = "joint_transformer_blocks." + std::to_string(i) + ".";
+    regions.push_back({b + "attn.to_q.weight", qkv_rows});
+    regions.push_back({b + "attn.add_q_proj.weight", qkv_rows});
+    regions.push_back({b + "ff.linear_1.weight", up_rows});
+    regions.push_back({b + "ff_context.linear_1.weight", up_rows});
+  }
+  for (int i = 0; i < c.num_single_dit_layers; ++i) {
+    const std::string b = "single_transformer_blocks." + std::to_string(i) + ".";
+    regions.push_back({b + "attn.to_q.weight", qkv_rows});
+    regions.push_back({b + "ff.linear_1.weight", up_rows});
+  }
+  std::unordered_map<std::string, size_t> first;
+  size_t rows = 0;
+  for (auto& r : regions) {
+    first[r.first] = rows;
+    rows += (r.second + 255) / 256 * 256;
+  }
+  int prev = 0;
+  cudaGetDevice(&prev);
+  cudaSetDevice(w->device);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaSuccess;
+  if (!w->fp8_codes) {
+    e = cudaMalloc(&w->fp8_codes, rows * D);
+    if (e == cudaSuccess) e = cudaMalloc(&w->fp8_scales, rows * sizeof(float));
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      if (w->fp8_codes) cudaFree(w->fp8_codes);
+      w->fp8_codes = nullptr;
+      w->fp8_scales = nullptr;
+      cudaSetDevice(prev);
+      return AF_ERR_OOM;
+    }
+    w->fp8_rows = rows;
+    e = cudaMemsetAsync(w->fp8_scales, 0, rows * sizeof(float), st);  // padding rows
+  }
+  for (size_t i = 0; i < regions.size() && e == cudaSuccess; ++i) {
+    const size_t r0 = first[regions[i].first];
+    e = launch_quantize_rows_e4m3(w->ptr(regions[i].first), static_cast<int>(regions[i].second), D,
+                                  w->fp8_codes + r0 * D, w->fp8_scales + r0, st);
+  }
+  cudaSetDevice(prev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  w->fp8_row = first;
+  w->fp8 = true;
+  return AF_OK;
+}
+
 af_status af_weights_bytes(const af_weights* w, size_t* bytes) {
   if (!w || !bytes) return AF_ERR_INVALID_ARG;
   *bytes = w->bytes;
@@ -627,6 +741,8 @@ af_status af_scratch_create(const af_weights* w, int max_batch, int max_img_toke
   const size_t o_img = take(B * s->max_ni * D * 2);
   const size_t o_txt = take(B * s->max_nt * D * 2);
   const size_t o_x = take(rowsN * D * 2);
+  const size_t o_y8 = take(rowsN * D);
+  const size_t o_ys = take(rowsN * 4);
   const int cmax = w->cfg.in_channels > w->cfg.out_channels ? w->cfg.in_channels : w->cfg.out_channels;
   const size_t lat_elems = B * static_cast<size_t>(cmax) * s->max_ni * w->cfg.patch_size * w->cfg.patch_size;
   const size_t o_lat2 = take(lat_elems * 4);
@@ -665,6 +781,8 @@ af_status af_scratch_create(const af_weights* w, int max_batch, int max_img_toke
   s->img = reinterpret_cast<uint16_t*>(s->base + o_img);
   s->txt = reinterpret_cast<uint16_t*>(s->base + o_txt);
   s->x = reinterpret_cast<uint16_t*>(s->base + o_x);
+  s->y8 = s->base + o_y8;
+  s->yscale = reinterpret_cast<float*>(s->base + o_ys);
   s->lat2 = reinterpret_cast<float*>(s->base + o_lat2);
   s->vel = reinterpret_cast<float*>(s->base + o_vel);
   s->tvec = reinterpret_cast<float*>(s->base + o_tvec);
@@ -1087,6 +1205,46 @@ af_status af_ln_modulate(const uint16_t* x, const float* shift, const float* sca
   if (!x || !shift || !scale || !y || B <= 0 || N <= 0 || D <= 0 || mod_stride < 0) return AF_ERR_INVALID_ARG;
   if (D % 8 != 0 || D > 4096) return AF_ERR_UNSUPPORTED;
   AF_CUDA(launch_ln_modulate(x, shift, scale, mod_stride, y, B * N, N, D, eps, static_cast<cudaStream_t>(stream)));
+  return AF_OK;
+}
+
+af_status af_ln_modulate_e4m3(const uint16_t* x, const float* shift, const float* scale, int mod_stride, uint8_t* y8,
+                              float* yscale, int B, int N, int D, float eps, void* stream) {
+  if (!x || !shift || !scale || !y8 || !yscale || B <= 0 || N <= 0 || D <= 0 || mod_stride < 0)
+    return AF_ERR_INVALID_ARG;
+  if (D % 8 != 0 || D > 4096) return AF_ERR_UNSUPPORTED;
+  AF_CUDA(launch_ln_modulate(x, shift, scale, mod_stride, nullptr, B * N, N, D, eps, static_cast<cudaStream_t>(stream),
+                             nullptr, y8, yscale));
+  return AF_OK;
+}
+
+af_status af_quantize_rows_e4m3(const uint16_t* x, int rows, int cols, uint8_t* q, float* scale, void* stream) {
+  if (!x || !q || !scale || rows <= 0 || cols <= 0) return AF_ERR_INVALID_ARG;
+  if (cols % 8 != 0) return AF_ERR_UNSUPPORTED;
+  AF_CUDA(launch_quantize_rows_e4m3(x, rows, cols, q, scale, static_cast<cudaStream_t>(stream)));
+  return AF_OK;
+}
+
+af_status af_linear_fp8(const uint8_t* A, const float* a_scale, const uint8_t* W, const float* w_scale, uint16_t* C,
+                        int M, int N, int K, void* stream) {
+  if (!A || !a_scale || !W || !w_scale || !C || M <= 0 || N <= 0 || K <= 0) return AF_ERR_INVALID_ARG;
+  if (K % 16 != 0 || N % 8 != 0) return AF_ERR_UNSUPPORTED;
+  GemmParams p;
+  memset(&p, 0, sizeof(p));
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.mode = EPI_STORE;
+  p.rows_per_batch = M;
+  p.out_rows_per_batch = M;
+  p.out = C;
+  p.ldo = N;
+  p.err = nullptr;
+  p.a_scale = a_scale;
+  p.w_scale = w_scale;
+  static int sms = 0;
+  if (!sms) sms = device_sm_count();
+  AF_CUDA(launch_gemm(p, A, W, N, static_cast<cudaStream_t>(stream), sms));
   return AF_OK;
 }
 

@@ -46,14 +46,15 @@ static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
 }
 
 bool encode_tmap_2d(CUtensorMap* map, const void* ptr, uint64_t inner, uint64_t outer, uint64_t row_bytes,
-                    uint32_t box_inner, uint32_t box_outer) {
+                    uint32_t box_inner, uint32_t box_outer, bool bytes) {
   auto enc = get_encode();
   if (!enc) return false;
   cuuint64_t dims[2] = {inner, outer};
   cuuint64_t strides[1] = {row_bytes};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+  CUresult r = enc(map, bytes ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                   const_cast<void*>(ptr), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -124,11 +125,34 @@ __device__ __forceinline__ void store_bf16_n(uint16_t* dst, const float* v, int 
   }
 }
 
+// 32 accumulator columns of this thread's row as floats.  For the 8-bit
+// GEMM (p.w_scale set) the fp32 sums of e4m3 products are rescaled by the
+// row's activation scale a_s and the scales of weight rows [wrow, wrow + 32).
+__device__ __forceinline__ void acc_load32(const GemmParams& p, uint32_t taddr, float a_s, int wrow, float (&v)[32]) {
+  uint32_t r[32];
+  tmem_ld32(taddr, r);
+  tmem_wait_ld();
+  if (p.w_scale) {
+    const float4* ws = reinterpret_cast<const float4*>(p.w_scale + wrow);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float4 w4 = ws[i];
+      v[4 * i + 0] = __uint_as_float(r[4 * i + 0]) * (a_s * w4.x);
+      v[4 * i + 1] = __uint_as_float(r[4 * i + 1]) * (a_s * w4.y);
+      v[4 * i + 2] = __uint_as_float(r[4 * i + 2]) * (a_s * w4.z);
+      v[4 * i + 3] = __uint_as_float(r[4 * i + 3]) * (a_s * w4.w);
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+  }
+}
+
 // QK-norm epilogue for one output row: columns [c0, c0 + width) of the tile
 // hold (256 / hd) heads of Q, K or V.  Q and K are LayerNorm-ed over each
 // head's hd values (two passes over TMEM: mean, then variance), V is stored as is.
 __device__ __forceinline__ void epilogue_qkv(const GemmParams& p, uint32_t tbase, int n0, bool row_ok, int b,
-                                             int n_in) {
+                                             int n_in, float a_s) {
   const int hd = p.hd;
   const int tok = p.qkv_row_off + n_in;
   if (hd >= 32) {
@@ -141,34 +165,30 @@ __device__ __forceinline__ void epilogue_qkv(const GemmParams& p, uint32_t tbase
       uint16_t* base = which == 0 ? p.q : (which == 1 ? p.k : p.v);
       uint16_t* dst = base + ((static_cast<size_t>(b) * p.heads + head) * p.n_total + tok) * hd;
       float mean = 0.f, rstd = 1.f;
-      uint32_t r[32];
+      float v[32];
       if (which < 2) {
         float s = 0.f;
         for (int c = 0; c < chunks; ++c) {
-          tmem_ld32(tbase + h0 + c * 32, r);
-          tmem_wait_ld();
+          acc_load32(p, tbase + h0 + c * 32, a_s, col + c * 32, v);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) s += __uint_as_float(r[j]);
+          for (int j = 0; j < 32; ++j) s += v[j];
         }
         mean = s / hd;
         float ss = 0.f;
         for (int c = 0; c < chunks; ++c) {
-          tmem_ld32(tbase + h0 + c * 32, r);
-          tmem_wait_ld();
+          acc_load32(p, tbase + h0 + c * 32, a_s, col + c * 32, v);
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
-            const float d = __uint_as_float(r[j]) - mean;
+            const float d = v[j] - mean;
             ss += d * d;
           }
         }
         rstd = rsqrtf(ss / hd + p.eps);
       }
       for (int c = 0; c < chunks; ++c) {
-        tmem_ld32(tbase + h0 + c * 32, r);
-        tmem_wait_ld();
-        float v[32];
+        acc_load32(p, tbase + h0 + c * 32, a_s, col + c * 32, v);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = (__uint_as_float(r[j]) - mean) * rstd;
+        for (int j = 0; j < 32; ++j) v[j] = (v[j] - mean) * rstd;
         if (row_ok) store_bf16x32(dst + c * 32, v);
       }
     }
@@ -176,9 +196,8 @@ __device__ __forceinline__ void epilogue_qkv(const GemmParams& p, uint32_t tbase
     // small heads (hd in {8, 16}): each 32-column chunk holds 32 / hd heads
     for (int c = 0; c < GEMM_BN / 32; ++c) {
       if (n0 + c * 32 >= p.N) break;
-      uint32_t r[32];
-      tmem_ld32(tbase + c * 32, r);
-      tmem_wait_ld();
+      float r[32];
+      acc_load32(p, tbase + c * 32, a_s, n0 + c * 32, r);
       for (int s0 = 0; s0 < 32; s0 += hd) {
         const int col = n0 + c * 32 + s0;
         if (col >= p.N) break;
@@ -190,16 +209,16 @@ __device__ __forceinline__ void epilogue_qkv(const GemmParams& p, uint32_t tbase
         float mean = 0.f, rstd = 1.f;
         if (which < 2) {
           float s = 0.f;
-          for (int j = 0; j < hd; ++j) s += __uint_as_float(r[s0 + j]);
+          for (int j = 0; j < hd; ++j) s += r[s0 + j];
           mean = s / hd;
           float ss = 0.f;
           for (int j = 0; j < hd; ++j) {
-            const float d = __uint_as_float(r[s0 + j]) - mean;
+            const float d = r[s0 + j] - mean;
             ss += d * d;
           }
           rstd = rsqrtf(ss / hd + p.eps);
         }
-        for (int j = 0; j < hd; ++j) v[j] = (__uint_as_float(r[s0 + j]) - mean) * rstd;
+        for (int j = 0; j < hd; ++j) v[j] = (r[s0 + j] - mean) * rstd;
         if (row_ok)
           for (int j = 0; j < hd; ++j) dst[j] = static_cast<uint16_t>(pack_bf16(v[j], 0.f) & 0xFFFFu);
       }
@@ -216,20 +235,20 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tbas
   const int b = r / p.rows_per_batch;
   const int n_in = r - b * p.rows_per_batch;
   const size_t orow = static_cast<size_t>(b) * p.out_rows_per_batch + p.out_row_off + n_in;
+  const float a_s = (p.a_scale && row_ok) ? p.a_scale[r] : 1.0f;
 
   if (p.mode == EPI_QKV) {
-    epilogue_qkv(p, tbase, nb * GEMM_BN, row_ok, b, n_in);
+    epilogue_qkv(p, tbase, nb * GEMM_BN, row_ok, b, n_in, a_s);
   } else if (p.mode == EPI_SWIGLU) {
     const int col0 = nb * 128;
 #pragma unroll 1
     for (int c = 0; c < 4; ++c) {
-      uint32_t ra[32], rb[32];
-      tmem_ld32(tbase + c * 32, ra);
-      tmem_ld32(tbase + 128 + c * 32, rb);
-      tmem_wait_ld();
-      float v[32];
+      // weight rows of the interleaved pair: W1 at nb*256 + [0, 128), W2 at nb*256 + 128 + [0, 128)
+      float va[32], v[32];
+      acc_load32(p, tbase + c * 32, a_s, nb * 256 + c * 32, va);
+      acc_load32(p, tbase + 128 + c * 32, a_s, nb * 256 + 128 + c * 32, v);
 #pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] = silu_f(__uint_as_float(ra[j])) * __uint_as_float(rb[j]);
+      for (int j = 0; j < 32; ++j) v[j] = silu_f(va[j]) * v[j];
       const int col = col0 + c * 32;
       if (row_ok && col < p.N) store_bf16_n(p.out + orow * p.ldo + col, v, p.N - col);
     }
@@ -239,12 +258,8 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tbas
     for (int c = 0; c < GEMM_BN / 32; ++c) {
       const int col = col0 + c * 32;
       if (col >= p.N) break;  // uniform across the warp
-      uint32_t ra[32];
-      tmem_ld32(tbase + c * 32, ra);
-      tmem_wait_ld();
       float v[32];
-#pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(ra[j]);
+      acc_load32(p, tbase + c * 32, a_s, col, v);
       if (!row_ok) continue;
       const int n = min(32, p.N - col);
       if (p.mode == EPI_STORE_F32) {
@@ -287,9 +302,14 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tbas
 }
 
 
+// FP8 = false: bf16 operands, 64 K elements (128 bytes) per stage, kind::f16.
+// FP8 = true:  e4m3 operands, 128 K elements (128 bytes) per stage,
+//              kind::f8f6f4; the epilogue applies the row / column scales.
+template <bool FP8>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
-    gemm_bf16_tcgen05(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                      const GemmParams p) {
+    gemm_tcgen05(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                 const GemmParams p) {
+  constexpr int KB = FP8 ? 2 * GEMM_BK : GEMM_BK;  // K elements per stage
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -331,7 +351,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int num_k = (p.K + GEMM_BK - 1) / GEMM_BK;
+  const int num_k = (p.K + KB - 1) / KB;
   volatile int never = 0;
 
   if (warp == 0) {
@@ -354,8 +374,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
           const uint32_t a_dst = smem_u32(sA + stage * A_STAGE_BYTES);
           const uint32_t b_dst = smem_u32(sB + stage * B_STAGE_BYTES);
-          tma_load_2d(a_dst, &tmA, fb, kb * GEMM_BK, mb * GEMM_BM);
-          tma_load_2d(b_dst, &tmB, fb, kb * GEMM_BK, wrow);
+          tma_load_2d(a_dst, &tmA, fb, kb * KB, mb * GEMM_BM);
+          tma_load_2d(b_dst, &tmB, fb, kb * KB, wrow);
           if (++stage == GEMM_STAGES) {
             stage = 0;
             phase ^= 1u;
@@ -370,7 +390,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t idesc = make_idesc_bf16(GEMM_BM, GEMM_BN, false, false);
+      const uint32_t idesc =
+          FP8 ? make_idesc_e4m3(GEMM_BM, GEMM_BN, false, false) : make_idesc_bf16(GEMM_BM, GEMM_BN, false, false);
       int stage = 0;
       uint32_t phase = 0, acc = 0, acc_phase = 0;
       bool ok = true;
@@ -387,8 +408,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           const uint64_t adesc = make_sdesc(smem_u32(sA + stage * A_STAGE_BYTES), 16, 1024, SWZ_128B);
           const uint64_t bdesc = make_sdesc(smem_u32(sB + stage * B_STAGE_BYTES), 16, 1024, SWZ_128B);
 #pragma unroll
-          for (int k = 0; k < GEMM_BK / 16; ++k)
-            mma_bf16_ss(d, adesc + 2 * k, bdesc + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+          for (int k = 0; k < 4; ++k) {  // 32 bytes of K per instruction
+            if constexpr (FP8)
+              mma_e4m3_ss(d, adesc + 2 * k, bdesc + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+            else
+              mma_bf16_ss(d, adesc + 2 * k, bdesc + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+          }
           mma_commit(smem_u32(&empty[stage]));
           if (++stage == GEMM_STAGES) {
             stage = 0;
@@ -448,9 +473,11 @@ constexpr uint32_t G2_A_BYTES = 128 * GEMM_BK * 2;  // 16 KB
 constexpr uint32_t G2_B_BYTES = 128 * GEMM_BK * 2;  // 16 KB
 constexpr int GEMM2_SMEM = G2_STAGES * (G2_A_BYTES + G2_B_BYTES) + 1024 + 1024;
 
+template <bool FP8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
-    gemm_bf16_tcgen05_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                           const GemmParams p) {
+    gemm_tcgen05_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                      const GemmParams p) {
+  constexpr int KB = FP8 ? 2 * GEMM_BK : GEMM_BK;  // K elements per stage (128 bytes per row)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -497,7 +524,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
   cluster_sync();  // the partner's barriers exist before anything signals them
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int num_k = (p.K + GEMM_BK - 1) / GEMM_BK;
+  const int num_k = (p.K + KB - 1) / KB;
   volatile int never = 0;
 
   if (warp == 0) {
@@ -518,8 +545,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
           const uint32_t fb_local = smem_u32(&full[stage]);
           if (leader) mbar_arrive_expect_tx(fb_local, 2 * (G2_A_BYTES + G2_B_BYTES));
           const uint32_t fb = mapa_shared(fb_local, 0);
-          tma_load_2d_pair(smem_u32(sA + stage * G2_A_BYTES), &tmA, fb, kb * GEMM_BK, arow);
-          tma_load_2d_pair(smem_u32(sB + stage * G2_B_BYTES), &tmB, fb, kb * GEMM_BK, wrow);
+          tma_load_2d_pair(smem_u32(sA + stage * G2_A_BYTES), &tmA, fb, kb * KB, arow);
+          tma_load_2d_pair(smem_u32(sB + stage * G2_B_BYTES), &tmB, fb, kb * KB, wrow);
           issued = true;
           if (++stage == G2_STAGES) {
             stage = 0;
@@ -535,7 +562,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     }
   } else if (warp == 1) {
     if (lane == 0 && leader) {
-      const uint32_t idesc = make_idesc_bf16(256, GEMM_BN, false, false);
+      const uint32_t idesc = FP8 ? make_idesc_e4m3(256, GEMM_BN, false, false) : make_idesc_bf16(256, GEMM_BN, false, false);
       int stage = 0;
       uint32_t phase = 0, acc = 0, acc_phase = 0;
       bool ok = true;
@@ -552,8 +579,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
           const uint64_t adesc = make_sdesc(smem_u32(sA + stage * G2_A_BYTES), 16, 1024, SWZ_128B);
           const uint64_t bdesc = make_sdesc(smem_u32(sB + stage * G2_B_BYTES), 16, 1024, SWZ_128B);
 #pragma unroll
-          for (int k = 0; k < GEMM_BK / 16; ++k)
-            mma_bf16_ss_pair(d, adesc + 2 * k, bdesc + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+          for (int k = 0; k < 4; ++k) {  // 32 bytes of K per instruction
+            if constexpr (FP8)
+              mma_e4m3_ss_pair(d, adesc + 2 * k, bdesc + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+            else
+              mma_bf16_ss_pair(d, adesc + 2 * k, bdesc + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+          }
           mma_commit_pair(smem_u32(&empty[stage]), 0x3);
           if (++stage == G2_STAGES) {
             stage = 0;
@@ -613,9 +644,13 @@ cudaError_t gemm_set_attributes() {
   int dev = 0;
   cudaGetDevice(&dev);
   if ((done >> dev) & 1u) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(gemm_bf16_tcgen05, cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM_SMEM_BYTES);
-  if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(gemm_bf16_tcgen05_pair, cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM2_SMEM);
+  cudaError_t e = cudaFuncSetAttribute(gemm_tcgen05<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM_SMEM_BYTES);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(gemm_tcgen05<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM_SMEM_BYTES);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(gemm_tcgen05_pair<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM2_SMEM);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(gemm_tcgen05_pair<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM2_SMEM);
   if (e != cudaSuccess) return e;
   done |= uint64_t(1) << dev;
   return cudaSuccess;
@@ -625,11 +660,16 @@ cudaError_t launch_gemm(const GemmParams& p_in, const void* A, const void* W, in
                         int num_sms) {
   GemmParams p = p_in;
   if (p.M <= 0 || p.N <= 0) return cudaSuccess;
-  if (p.K <= 0 || (p.K % 8) != 0) return cudaErrorInvalidValue;
+  const bool fp8 = p.w_scale != nullptr;
+  const int esz = fp8 ? 1 : 2;
+  const int kb = fp8 ? 2 * GEMM_BK : GEMM_BK;  // 128-byte K boxes either way
+  if (p.K <= 0 || (p.K * esz) % 16 != 0) return cudaErrorInvalidValue;
+  if (fp8 && !p.a_scale) return cudaErrorInvalidValue;
   CUtensorMap ta, tb;
-  if (!encode_tmap_2d(&ta, A, p.K, p.M, static_cast<uint64_t>(p.K) * 2, GEMM_BK, GEMM_BM)) return cudaErrorInvalidValue;
+  if (!encode_tmap_2d(&ta, A, p.K, p.M, static_cast<uint64_t>(p.K) * esz, kb, GEMM_BM, fp8))
+    return cudaErrorInvalidValue;
   const bool pair = p.M >= 1024 && num_sms >= 2;
-  if (!encode_tmap_2d(&tb, W, p.K, W_rows, static_cast<uint64_t>(p.K) * 2, GEMM_BK, pair ? 128 : GEMM_BN))
+  if (!encode_tmap_2d(&tb, W, p.K, W_rows, static_cast<uint64_t>(p.K) * esz, kb, pair ? 128 : GEMM_BN, fp8))
     return cudaErrorInvalidValue;
   {
     cudaError_t e = gemm_set_attributes();
@@ -643,13 +683,19 @@ cudaError_t launch_gemm(const GemmParams& p_in, const void* A, const void* W, in
     p.num_tiles = p.num_m_tiles * p.num_n_tiles;
     const int pairs = num_sms / 2;
     const int grid = 2 * (p.num_tiles < pairs ? p.num_tiles : pairs);
-    gemm_bf16_tcgen05_pair<<<grid, GEMM_THREADS, GEMM2_SMEM, stream>>>(ta, tb, p);
+    if (fp8)
+      gemm_tcgen05_pair<true><<<grid, GEMM_THREADS, GEMM2_SMEM, stream>>>(ta, tb, p);
+    else
+      gemm_tcgen05_pair<false><<<grid, GEMM_THREADS, GEMM2_SMEM, stream>>>(ta, tb, p);
     return cudaGetLastError();
   }
   p.num_m_tiles = (p.M + GEMM_BM - 1) / GEMM_BM;
   p.num_tiles = p.num_m_tiles * p.num_n_tiles;
   const int grid = p.num_tiles < num_sms ? p.num_tiles : num_sms;
-  gemm_bf16_tcgen05<<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, stream>>>(ta, tb, p);
+  if (fp8)
+    gemm_tcgen05<true><<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, stream>>>(ta, tb, p);
+  else
+    gemm_tcgen05<false><<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, stream>>>(ta, tb, p);
   return cudaGetLastError();
 }
 

@@ -26,13 +26,24 @@ __device__ __forceinline__ float warp_sum(float v) {
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
 }
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Per-row e4m3 scaling (the 8-bit GEMM inputs): a = max |row|, codes
+// e4m3(x * (448 / a)), scale a / 448 (1 and zeros for an all-zero row).
+__device__ __forceinline__ float e4m3_inv_scale(float amax) { return amax > 0.f ? 448.0f / amax : 1.0f; }
+__device__ __forceinline__ float e4m3_scale(float amax) { return amax > 0.f ? amax / 448.0f : 1.0f; }
 
 // ------------------------------------------------------------------ LN + modulate
-template <int VPL>  // 8-element vectors per lane
+template <int VPL, bool OUT8>  // 8-element vectors per lane; OUT8: e4m3 codes + row scale
 __global__ void __launch_bounds__(256) ln_modulate_kernel(const uint16_t* __restrict__ x,
                                                           const float* __restrict__ shift,
                                                           const float* __restrict__ scale, int mod_stride,
-                                                          uint16_t* __restrict__ y, int rows, int rows_per_batch,
+                                                          uint16_t* __restrict__ y, uint8_t* __restrict__ y8,
+                                                          float* __restrict__ yscale, int rows, int rows_per_batch,
                                                           int D, float eps) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
@@ -71,7 +82,7 @@ __global__ void __launch_bounds__(256) ln_modulate_kernel(const uint16_t* __rest
   const int b = warp / rows_per_batch;
   const float* sh = shift + static_cast<size_t>(b) * mod_stride;
   const float* sc = scale + static_cast<size_t>(b) * mod_stride;
-  uint4* yr = reinterpret_cast<uint4*>(y + static_cast<size_t>(warp) * D);
+  float amax = 0.f;
 #pragma unroll
   for (int i = 0; i < VPL; ++i) {
     const int vi = i * 32 + lane;
@@ -82,15 +93,38 @@ __global__ void __launch_bounds__(256) ln_modulate_kernel(const uint16_t* __rest
       const float4 h1 = *reinterpret_cast<const float4*>(sh + vi * 8 + 4);
       const float scv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
       const float shv[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
-      float o[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) o[e] = (v[i][e] - mean) * rstd * (1.0f + scv[e]) + shv[e];
-      uint4 u;
-      u.x = pack_bf16(o[0], o[1]);
-      u.y = pack_bf16(o[2], o[3]);
-      u.z = pack_bf16(o[4], o[5]);
-      u.w = pack_bf16(o[6], o[7]);
-      yr[vi] = u;
+      for (int e = 0; e < 8; ++e) {
+        v[i][e] = (v[i][e] - mean) * rstd * (1.0f + scv[e]) + shv[e];  // the row's output, in place
+        amax = fmaxf(amax, fabsf(v[i][e]));
+      }
+    }
+  }
+  if constexpr (OUT8) {
+    amax = warp_max(amax);
+    const float inv = e4m3_inv_scale(amax);
+    uint2* yr = reinterpret_cast<uint2*>(y8 + static_cast<size_t>(warp) * D);
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const int vi = i * 32 + lane;
+      if (vi < nvec)
+        yr[vi] = make_uint2(pack_e4m3x4(v[i][0] * inv, v[i][1] * inv, v[i][2] * inv, v[i][3] * inv),
+                            pack_e4m3x4(v[i][4] * inv, v[i][5] * inv, v[i][6] * inv, v[i][7] * inv));
+    }
+    if (lane == 0) yscale[warp] = e4m3_scale(amax);
+  } else {
+    uint4* yr = reinterpret_cast<uint4*>(y + static_cast<size_t>(warp) * D);
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const int vi = i * 32 + lane;
+      if (vi < nvec) {
+        uint4 u;
+        u.x = pack_bf16(v[i][0], v[i][1]);
+        u.y = pack_bf16(v[i][2], v[i][3]);
+        u.z = pack_bf16(v[i][4], v[i][5]);
+        u.w = pack_bf16(v[i][6], v[i][7]);
+        yr[vi] = u;
+      }
     }
   }
 }
@@ -107,10 +141,13 @@ constexpr uint32_t LNB_ROW_BYTES = LNB_D * 2;
 constexpr int LNB_THREADS = 32 * (LNB_ROWS + 1);
 constexpr int LNB_SMEM = LNB_STAGES * LNB_ROWS * LNB_ROW_BYTES + 2 * LNB_D * 4 + 128 + 128;
 
+template <bool OUT8>
 __global__ void __launch_bounds__(LNB_THREADS, 1) ln_modulate_bulk_kernel(const uint16_t* __restrict__ x,
                                                                          const float* __restrict__ shift,
                                                                          const float* __restrict__ scale,
                                                                          int mod_stride, uint16_t* __restrict__ y,
+                                                                         uint8_t* __restrict__ y8,
+                                                                         float* __restrict__ yscale,
                                                                          int rows_per_batch, float eps, int* err) {
   extern __shared__ uint8_t lnb_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(lnb_raw) + 127) & ~uintptr_t(127));
@@ -197,9 +234,8 @@ __global__ void __launch_bounds__(LNB_THREADS, 1) ln_modulate_bulk_kernel(const 
         }
       }
       const float rstd = rsqrtf(warp_sum(ss) * (1.0f / LNB_D) + eps);
-      uint4* yr = reinterpret_cast<uint4*>(y + (row0 + r) * LNB_D);
-#pragma unroll
-      for (int i = 0; i < VPL; ++i) {
+      // output element 2e (+1) of vector i: (x - mean) rstd (1 + scale) + shift
+      auto out8 = [&](int i, float (&o)[8]) {
         const int vi = i * 32 + lane;
         const float4 a0 = *reinterpret_cast<const float4*>(mod_s + vi * 8);
         const float4 a1 = *reinterpret_cast<const float4*>(mod_s + vi * 8 + 4);
@@ -208,12 +244,41 @@ __global__ void __launch_bounds__(LNB_THREADS, 1) ln_modulate_bulk_kernel(const 
         const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
         const float hv[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
         const uint32_t w[4] = {cur[i].x, cur[i].y, cur[i].z, cur[i].w};
-        uint32_t o[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-          o[e] = pack_bf16((bf16_lo(w[e]) - mean) * rstd * av[2 * e] + hv[2 * e],
-                           (bf16_hi(w[e]) - mean) * rstd * av[2 * e + 1] + hv[2 * e + 1]);
-        yr[vi] = make_uint4(o[0], o[1], o[2], o[3]);
+        for (int e = 0; e < 4; ++e) {
+          o[2 * e] = (bf16_lo(w[e]) - mean) * rstd * av[2 * e] + hv[2 * e];
+          o[2 * e + 1] = (bf16_hi(w[e]) - mean) * rstd * av[2 * e + 1] + hv[2 * e + 1];
+        }
+      };
+      if constexpr (OUT8) {
+        float amax = 0.f;
+#pragma unroll
+        for (int i = 0; i < VPL; ++i) {
+          float o[8];
+          out8(i, o);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(o[e]));
+        }
+        amax = warp_max(amax);
+        const float inv = e4m3_inv_scale(amax);
+        uint2* yr = reinterpret_cast<uint2*>(y8 + (row0 + r) * LNB_D);
+#pragma unroll
+        for (int i = 0; i < VPL; ++i) {
+          float o[8];
+          out8(i, o);
+          yr[i * 32 + lane] = make_uint2(pack_e4m3x4(o[0] * inv, o[1] * inv, o[2] * inv, o[3] * inv),
+                                         pack_e4m3x4(o[4] * inv, o[5] * inv, o[6] * inv, o[7] * inv));
+        }
+        if (lane == 0) yscale[row0 + r] = e4m3_scale(amax);
+      } else {
+        uint4* yr = reinterpret_cast<uint4*>(y + (row0 + r) * LNB_D);
+#pragma unroll
+        for (int i = 0; i < VPL; ++i) {
+          float o[8];
+          out8(i, o);
+          yr[i * 32 + lane] = make_uint4(pack_bf16(o[0], o[1]), pack_bf16(o[2], o[3]), pack_bf16(o[4], o[5]),
+                                         pack_bf16(o[6], o[7]));
+        }
       }
     }
     __syncwarp();
@@ -223,9 +288,11 @@ __global__ void __launch_bounds__(LNB_THREADS, 1) ln_modulate_bulk_kernel(const 
 
 cudaError_t launch_ln_modulate(const uint16_t* x, const float* shift, const float* scale, int mod_stride,
                                uint16_t* y, int rows, int rows_per_batch, int D, float eps, cudaStream_t s,
-                               int* err) {
+                               int* err, uint8_t* y8, float* yscale) {
   if (rows <= 0) return cudaSuccess;
   if (D % 8 != 0) return cudaErrorInvalidValue;
+  const bool out8 = y8 != nullptr;
+  if (out8 && !yscale) return cudaErrorInvalidValue;
   if (D == LNB_D && rows % rows_per_batch == 0 && (reinterpret_cast<uintptr_t>(x) & 15) == 0) {
     cudaError_t e = small_kernels_set_attributes();
     if (e != cudaSuccess) return e;
@@ -234,18 +301,26 @@ cudaError_t launch_ln_modulate(const uint16_t* x, const float* shift, const floa
     if (!sms) sms = device_sm_count();
     const int nchunks = (rows_per_batch + LNB_ROWS - 1) / LNB_ROWS;
     const int per = max(1, min(nchunks, (sms + nb - 1) / nb));
-    ln_modulate_bulk_kernel<<<dim3(per, nb), LNB_THREADS, LNB_SMEM, s>>>(x, shift, scale, mod_stride, y,
-                                                                         rows_per_batch, eps, err);
+    if (out8)
+      ln_modulate_bulk_kernel<true><<<dim3(per, nb), LNB_THREADS, LNB_SMEM, s>>>(x, shift, scale, mod_stride, y, y8,
+                                                                               yscale, rows_per_batch, eps, err);
+    else
+      ln_modulate_bulk_kernel<false><<<dim3(per, nb), LNB_THREADS, LNB_SMEM, s>>>(x, shift, scale, mod_stride, y, y8,
+                                                                                yscale, rows_per_batch, eps, err);
     return cudaGetLastError();
   }
   const int nvec = D / 8;
   const int vpl = (nvec + 31) / 32;
   const int blocks = (rows + 7) / 8;
-#define AF_LN_CASE(N)                                                                                    \
-  if (vpl <= N) {                                                                                        \
-    ln_modulate_kernel<N><<<blocks, 256, 0, s>>>(x, shift, scale, mod_stride, y, rows, rows_per_batch, D, \
-                                                 eps);                                                   \
-    return cudaGetLastError();                                                                           \
+#define AF_LN_CASE(N)                                                                                        \
+  if (vpl <= N) {                                                                                            \
+    if (out8)                                                                                                \
+      ln_modulate_kernel<N, true><<<blocks, 256, 0, s>>>(x, shift, scale, mod_stride, y, y8, yscale, rows,    \
+                                                         rows_per_batch, D, eps);                            \
+    else                                                                                                     \
+      ln_modulate_kernel<N, false><<<blocks, 256, 0, s>>>(x, shift, scale, mod_stride, y, y8, yscale, rows,   \
+                                                          rows_per_batch, D, eps);                           \
+    return cudaGetLastError();                                                                               \
   }
   AF_LN_CASE(1)
   AF_LN_CASE(2)
@@ -255,6 +330,41 @@ cudaError_t launch_ln_modulate(const uint16_t* x, const float* shift, const floa
   AF_LN_CASE(16)
 #undef AF_LN_CASE
   return cudaErrorInvalidValue;
+}
+
+// ------------------------------------------------------------------ per-row e4m3 quantisation
+// One warp per row of a bf16 [rows, K] matrix (K a multiple of 8): codes
+// e4m3(x * 448 / amax) into q [rows, K] and the row scale amax / 448.
+__global__ void __launch_bounds__(256) quantize_rows_e4m3_kernel(const uint16_t* __restrict__ x, int rows, int K,
+                                                                 uint8_t* __restrict__ q, float* __restrict__ scale) {
+  const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<size_t>(row) * K);
+  const int nvec = K >> 3;
+  float amax = 0.f;
+  for (int vi = lane; vi < nvec; vi += 32) {
+    const uint4 u = xr[vi];
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(w[e])), fabsf(bf16_hi(w[e]))));
+  }
+  amax = warp_max(amax);
+  const float inv = e4m3_inv_scale(amax);
+  uint2* qr = reinterpret_cast<uint2*>(q + static_cast<size_t>(row) * K);
+  for (int vi = lane; vi < nvec; vi += 32) {
+    const uint4 u = xr[vi];
+    qr[vi] = make_uint2(pack_e4m3x4(bf16_lo(u.x) * inv, bf16_hi(u.x) * inv, bf16_lo(u.y) * inv, bf16_hi(u.y) * inv),
+                        pack_e4m3x4(bf16_lo(u.z) * inv, bf16_hi(u.z) * inv, bf16_lo(u.w) * inv, bf16_hi(u.w) * inv));
+  }
+  if (lane == 0) scale[row] = e4m3_scale(amax);
+}
+
+cudaError_t launch_quantize_rows_e4m3(const uint16_t* x, int rows, int K, uint8_t* q, float* scale, cudaStream_t s) {
+  if (rows <= 0) return cudaSuccess;
+  if (K <= 0 || K % 8 != 0) return cudaErrorInvalidValue;
+  quantize_rows_e4m3_kernel<<<(rows + 7) / 8, 256, 0, s>>>(x, rows, K, q, scale);
+  return cudaGetLastError();
 }
 
 // ------------------------------------------------------------------ batched GEMV
@@ -325,7 +435,10 @@ cudaError_t small_kernels_set_attributes() {
   int dev = 0;
   cudaGetDevice(&dev);
   if ((done >> dev) & 1u) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(ln_modulate_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, LNB_SMEM);
+  cudaError_t e =
+      cudaFuncSetAttribute(ln_modulate_bulk_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, LNB_SMEM);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(ln_modulate_bulk_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, LNB_SMEM);
   if (e == cudaSuccess) e = gemv_attr<1>();
   if (e == cudaSuccess) e = gemv_attr<2>();
   if (e == cudaSuccess) e = gemv_attr<4>();

@@ -259,6 +259,42 @@ af_status af_sampler_prepare(af_sampler* smp, void* stream);
 af_status af_sampler_step(af_sampler* smp, int step, void* stream);
 void af_sampler_destroy(af_sampler* smp);
 
+/* ---- 8-bit variant ----------------------------------------------------------
+ * The pipeline guide loads the transformer with 8-bit weights ([PIPE]
+ * bitsandbytes sections).  This is the tensor-core form of that idea: the
+ * fused QKV projections and the FFN up-projections (the GEMMs whose inputs
+ * come straight out of LayerNorm + modulate) run with e4m3 operands on
+ * tcgen05 kind::f8f6f4 MMAs, each activation row (token) and each weight row
+ * (output channel) scaled by its own fp32 factor amax / 448; the output
+ * projections, FFN down-projections and attention stay bf16.
+ *
+ * af_weights_quantize_fp8(w, 1, stream) quantises the current bf16 values
+ * of those weights into a second device pack (about 46% of the bf16 pack)
+ * and switches every later forward, block and sampler step on `w` to the
+ * 8-bit GEMMs; call it again after changing weights.  enable = 0 frees the
+ * pack and returns to bf16.  Create samplers after switching. */
+af_status af_weights_quantize_fp8(af_weights* w, int enable, void* stream);
+
+/* Per-row e4m3 quantisation: for each row of x (device bf16 [rows, cols],
+ * cols % 8 == 0) with a = max |x|: q = e4m3(x * (448 / a)) (round to nearest
+ * even, saturating), scale = a / 448 (1 and zero codes for an all-zero row).
+ *   q: device uint8 [rows, cols]; scale: device float [rows]. */
+af_status af_quantize_rows_e4m3(const uint16_t* x, int rows, int cols, uint8_t* q, float* scale, void* stream);
+
+/* af_ln_modulate with e4m3 output: y8 = per-row quantised LayerNorm+modulate
+ * output (device uint8 [B*N, D]) and yscale its row scales (device float
+ * [B*N]), with the rule of af_quantize_rows_e4m3. */
+af_status af_ln_modulate_e4m3(const uint16_t* x, const float* shift, const float* scale, int mod_stride,
+                              uint8_t* y8, float* yscale, int B, int N, int D, float eps, void* stream);
+
+/* C[m, n] = a_scale[m] * w_scale[n] * sum_k A[m, k] W[n, k] with e4m3
+ * operands on the tensor cores (fp32 accumulate, bf16 out).
+ *   A: device uint8 [M, K]; W: device uint8 [N, K]; C: device bf16 [M, N];
+ *   a_scale: device float [M]; w_scale: device float, readable for
+ *   ceil(N / 256) * 256 entries.  K % 16 == 0, N % 8 == 0. */
+af_status af_linear_fp8(const uint8_t* A, const float* a_scale, const uint8_t* W, const float* w_scale, uint16_t* C,
+                        int M, int N, int K, void* stream);
+
 /* Host-side sigma schedule of the flow-match Euler sampler ([DEEP] §2.3:
  * num_train_timesteps 1000, shift 1.73, 25 steps): n_steps + 1 values
  * sigma_i = k s_i / (1 + (k - 1) s_i) with s = linspace(1, 1/num_train,

@@ -67,3 +67,19 @@ def to_np(t):
 def upload(weights_obj, w: dict):
     for name, arr in w.items():
         weights_obj.set(name, to_bf16(arr))
+
+
+def e4m3_lut():
+    """Value of each of the 256 e4m3 codes (sign, 4 exponent bits with bias 7,
+    3 mantissa bits; 0x7F / 0xFF NaN), from the format definition."""
+    out = np.empty(256)
+    for c in range(256):
+        s = -1.0 if c & 0x80 else 1.0
+        e, m = (c >> 3) & 0xF, c & 0x7
+        if e == 0xF and m == 0x7:
+            out[c] = np.nan
+        elif e == 0:
+            out[c] = s * m * 2.0 ** -9
+        else:
+            out[c] = s * (1.0 + m / 8.0) * 2.0 ** (e - 7)
+    return out

@@ -1,0 +1,166 @@
+"""GPU parity of the 8-bit (e4m3) variant against the oracle.
+
+Quantised codes are an integer decision taken in fp32 on both sides (the
+oracle's quantiser follows the kernel's fp32 steps), so the weight and
+activation quantiser is compared bit for bit.  Where the kernel's fp32
+LayerNorm output differs from the oracle's fp64 one in the last bits, a code
+may move by one step: at most 1% of codes, never by more than one step.
+The 8-bit GEMM is compared with the exact product of the GPU's own codes
+(bf16 output rounding, 3e-3); blocks and the forward with the oracle's
+8-bit variant at the block (2e-2) and stack (5e-2) tolerances.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import synth
+from helpers import af_config, draw_weights, e4m3_lut, tiny_config, to_bf16, to_f32, to_np, upload
+
+pytestmark = pytest.mark.gpu
+LUT = e4m3_lut()
+
+
+@pytest.fixture(scope="module")
+def af():
+    import diffusion_transformer_denoising_auraflow_b200 as m
+    return m
+
+
+def _codes(t):
+    return LUT[t.cpu().numpy().astype(np.int64)]
+
+
+@pytest.mark.parametrize("rows,cols", [(37, 3072), (300, 520), (5, 8), (64, 96)])
+def test_quantize_rows_bit_exact(af, rows, cols):
+    x = synth.normal(701, f"q{rows}_{cols}", (rows, cols), 1.0)
+    x[1] *= 1e-4
+    x[2] = 0.0
+    x[3, 5] = 300.0          # one outlier row
+    x = synth.bf16_round(x.astype(np.float32))
+    q = torch.empty(rows, cols, dtype=torch.uint8, device="cuda")
+    s = torch.empty(rows, dtype=torch.float32, device="cuda")
+    af.quantize_rows_e4m3(to_bf16(x), q, s)
+    torch.cuda.synchronize()
+    ref_q, ref_s = O.quantize_rows_e4m3(x)
+    assert np.array_equal(s.cpu().numpy(), ref_s)
+    assert np.array_equal(_codes(q), ref_q)
+
+
+@pytest.mark.parametrize("B,N,D", [(2, 300, 3072), (2, 37, 32), (1, 9, 256)])
+def test_ln_modulate_e4m3_matches_oracle(af, B, N, D):
+    x = synth.bf16_round((synth.normal(711, f"lx{N}_{D}", (B, N, D), 1.0) * 3 + 0.5).astype(np.float32))
+    mods = synth.normal(712, f"lm{D}", (B, 6 * D), 0.5, "f32")
+    y8 = torch.empty(B * N, D, dtype=torch.uint8, device="cuda")
+    ys = torch.empty(B * N, dtype=torch.float32, device="cuda")
+    md = to_f32(mods)
+    af.ln_modulate_e4m3(to_bf16(x), md[:, 3 * D:], md[:, 4 * D:], 6 * D, y8, ys, 1e-6)
+    torch.cuda.synchronize()
+    y = O.modulate(x, mods[:, 3 * D:4 * D], mods[:, 4 * D:5 * D], 1e-6).reshape(B * N, D)
+    ref_q, ref_s = O.quantize_rows_e4m3(y)
+    got_s = ys.cpu().numpy()
+    assert np.allclose(got_s, ref_s, rtol=1e-5)
+    got_q = _codes(y8)
+    same = np.mean(got_q == ref_q)
+    assert same > 0.99
+    # a differing code is a neighbour: within one e4m3 step (2^-3 relative, or the subnormal step)
+    diff = np.abs(got_q - ref_q)
+    assert np.all(diff <= np.maximum(np.abs(ref_q) * 2.0 ** -3, 2.0 ** -9) * (1 + 1e-9))
+    deq = got_q * got_s[:, None]
+    assert O.rel_l2(deq, y) < 4e-2          # the e4m3 rounding itself
+
+
+@pytest.mark.parametrize("M,N,K", [(300, 520, 256), (64, 96, 32), (129, 256, 528),
+                                   # M >= 1024 runs on CTA pairs
+                                   (1100, 776, 528), (4096, 3072, 3072), (2304, 16, 64)])
+def test_linear_fp8_matches_exact_product_of_codes(af, M, N, K):
+    A = synth.bf16_round(synth.normal(721, f"fa{M}_{K}", (M, K), 1.0).astype(np.float32))
+    W = synth.bf16_round(synth.normal(722, f"fw{N}_{K}", (N, K), 0.02).astype(np.float32))
+    a8 = torch.empty(M, K, dtype=torch.uint8, device="cuda")
+    w8 = torch.empty(N, K, dtype=torch.uint8, device="cuda")
+    sa = torch.empty(M, dtype=torch.float32, device="cuda")
+    sw = torch.zeros((N + 255) // 256 * 256, dtype=torch.float32, device="cuda")
+    af.quantize_rows_e4m3(to_bf16(A), a8, sa)
+    af.quantize_rows_e4m3(to_bf16(W), w8, sw[:N])
+    C = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    af.linear_fp8(a8, sa, w8, sw, C)
+    torch.cuda.synchronize()
+    ref = (_codes(a8) * sa.cpu().numpy()[:, None].astype(np.float64)) @ \
+          (_codes(w8) * sw[:N].cpu().numpy()[:, None].astype(np.float64)).T
+    assert O.rel_l2(to_np(C), ref) < 3e-3
+    # and the 8-bit product stays near the bf16 one
+    assert O.rel_l2(to_np(C), A.astype(np.float64) @ W.astype(np.float64).T) < 1e-1
+
+
+def _block_case(af, cfg, seed, names):
+    w = af.Weights(af_config(cfg))
+    drawn = draw_weights(cfg, seed, names)
+    upload(w, drawn)
+    w.quantize_fp8()
+    return w, drawn
+
+
+def test_single_block_fp8_matches_oracle(af):
+    """Real width (D = 3072, F = 8192), B = 2, 300 tokens."""
+    from helpers import block_names
+    cfg = O.Config(num_mmdit_layers=0, num_single_dit_layers=1, pos_embed_max_size=64 * 64)
+    pre = "single_transformer_blocks.0."
+    w, drawn = _block_case(af, cfg, 731, block_names(cfg, "single", 0))
+    s = af.Scratch(w, 2, 512, 64)
+    x = synth.activations(732, "f8x", (2, 300, 3072))
+    temb = synth.conditioning(733, (2, 3072))
+    xt = to_bf16(x)
+    af.single_block(w, s, 0, xt, to_f32(temb))
+    s.sync()
+    ref8 = O.single_block(x, temb, drawn, pre, cfg, fp8=True)
+    got = to_np(xt)
+    assert O.rel_l2(got - x, ref8 - x) < 2e-2
+    # the variant differs from the bf16 block by the e4m3 rounding, visibly but not grossly
+    ref16 = O.single_block(x, temb, drawn, pre, cfg)
+    err16 = O.rel_l2(got - x, ref16 - x)
+    assert 1e-3 < err16 < 0.15
+
+
+def test_joint_block_fp8_matches_oracle(af):
+    from helpers import block_names
+    cfg = O.Config(num_mmdit_layers=1, num_single_dit_layers=0, pos_embed_max_size=64 * 64)
+    pre = "joint_transformer_blocks.0."
+    w, drawn = _block_case(af, cfg, 741, block_names(cfg, "joint", 0))
+    s = af.Scratch(w, 2, 256, 40)
+    img = synth.activations(742, "f8i", (2, 256, 3072))
+    txt = synth.activations(743, "f8t", (2, 48, 3072))
+    temb = synth.conditioning(744, (2, 3072))
+    it, tt = to_bf16(img), to_bf16(txt)
+    af.joint_block(w, s, 0, it, tt, to_f32(temb))
+    s.sync()
+    rt, ri = O.joint_block(img, txt, temb, drawn, pre, cfg, fp8=True)
+    assert O.rel_l2(to_np(it) - img, ri - img) < 2e-2
+    assert O.rel_l2(to_np(tt) - txt, rt - txt) < 2e-2
+
+
+def test_tiny_forward_fp8_matches_oracle(af):
+    cfg = tiny_config()
+    w = af.Weights(af_config(cfg))
+    drawn = draw_weights(cfg, 751)
+    upload(w, drawn)
+    w.quantize_fp8()
+    s = af.Scratch(w, 2, 64, 8)
+    lat = synth.latents(752, (2, 4, 16, 16))
+    text = synth.text_embeddings(753, (2, 8, cfg.joint_attention_dim))
+    t = np.array([0.8, 0.3], np.float32)
+    vel = torch.empty(2, 4, 16, 16, device="cuda")
+    af.transformer_forward(w, s, to_f32(lat), to_bf16(text), to_f32(t), vel)
+    s.sync()
+    ref = O.transformer_forward(lat, text, t, drawn, cfg, fp8=True)
+    assert O.rel_l2(to_np(vel), ref) < 5e-2
+    # switching back restores the bf16 path bit for bit
+    w.quantize_fp8(False)
+    vel16 = torch.empty_like(vel)
+    af.transformer_forward(w, s, to_f32(lat), to_bf16(text), to_f32(t), vel16)
+    w2 = af.Weights(af_config(cfg))
+    upload(w2, drawn)
+    s2 = af.Scratch(w2, 2, 64, 8)
+    vel16b = torch.empty_like(vel)
+    af.transformer_forward(w2, s2, to_f32(lat), to_bf16(text), to_f32(t), vel16b)
+    s2.sync()
+    assert torch.equal(vel16, vel16b)
