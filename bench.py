@@ -459,6 +459,8 @@ def run_single_block_case(args):
     cfg = af.Config.default(num_mmdit_layers=0, num_single_dit_layers=1, pos_embed_max_size=G * G)
     w = af.Weights(cfg, 0)
     make_weights(af, torch, w, args.seed, torch.device("cuda", 0))
+    if args.fp8:
+        w.quantize_fp8()
     s = af.Scratch(w, 2, Ni, L)
     gen = torch.Generator(device="cuda")
     gen.manual_seed(args.seed)
@@ -476,7 +478,7 @@ def run_single_block_case(args):
     ms = e0.elapsed_time(e1) / args.steps
     D, F = 3072, 8192
     flops = 2 * (2.0 * N * (4 * D * D + 3 * D * F) + 4.0 * N * N * D)
-    print(json.dumps({"case": "single_block", "tokens": N, "ms_per_block": ms,
+    print(json.dumps({"case": "single_block", "fp8": bool(args.fp8), "tokens": N, "ms_per_block": ms,
                       "tflops": flops / (ms * 1e-3) / 1e12}), flush=True)
     return 0
 
