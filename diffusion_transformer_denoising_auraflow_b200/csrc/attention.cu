@@ -1,6 +1,7 @@
 // attention.cu -- joint / self attention of the AuraFlow blocks on sm_100a.
 //
-//   O = softmax(Q K^T * hd^-1/2) V   per (sample, head); non-causal, no mask
+//   O = softmax(Q K^T * hd^-1/2) V   per (sample, head); non-causal, with an
+//   optional per-sample masked key range (padded prompts)
 //
 // ("Diffusers 中的 AuraFlowTransformer2DModel架构解析与源码级使用指南",
 // §注意力处理器与 QKV 融合: text and image tokens are concatenated and
@@ -181,8 +182,8 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
 #pragma unroll
         for (int kk = 0; kk < AT_HD / 16; ++kk) {
           const uint32_t c = kk >> 2, off = (kk & 3) * 32;
-          const uint64_t ad = make_sdesc(qaddr + c * (AT_BM * 128) + off, 16, 1024, SWZ_128B);
-          const uint64_t bd = make_sdesc(kaddr + c * (AT_BN * 128) + off, 16, 1024, SWZ_128B);
+          const uint64_t ad = make_sdesc(qaddr, 16, 1024, SWZ_128B) + static_cast<uint64_t>((c * (AT_BM * 128) + off) >> 4);
+          const uint64_t bd = make_sdesc(kaddr, 16, 1024, SWZ_128B) + static_cast<uint64_t>((c * (AT_BN * 128) + off) >> 4);
           mma_bf16_ss(tS + s * AT_BN, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
         }
         mma_commit(smem_u32(&s_full[s]));
@@ -199,8 +200,8 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
         const uint32_t vaddr = smem_u32(sV + s * AT_KV_BYTES);
 #pragma unroll
         for (int kk = 0; kk < AT_BN / 16; ++kk) {
-          const uint64_t ad = make_sdesc(paddr + kk * 32, 16, 1024, SWZ_128B);
-          const uint64_t bd = make_sdesc(vaddr + kk * (16 * 128), AT_BN * 128, 1024, SWZ_128B);
+          const uint64_t ad = make_sdesc(paddr, 16, 1024, SWZ_128B) + static_cast<uint64_t>((kk * 32) >> 4);
+          const uint64_t bd = make_sdesc(vaddr, AT_BN * 128, 1024, SWZ_128B) + static_cast<uint64_t>((kk * (16 * 128)) >> 4);
           mma_bf16_ss(tO, ad, bd, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(smem_u32(o_done));
@@ -490,7 +491,7 @@ __global__ void __launch_bounds__(QKN_THREADS, 1)
 #pragma unroll
         for (int kk = 0; kk < AT_HD / 16; ++kk) {
           const uint32_t c = kk >> 2, off = (kk & 3) * 32;
-          const uint64_t bd = make_sdesc(kaddr + c * (AT_BN * 128) + off, 16, 1024, SWZ_128B);
+          const uint64_t bd = make_sdesc(kaddr, 16, 1024, SWZ_128B) + static_cast<uint64_t>((c * (AT_BN * 128) + off) >> 4);
           mma_bf16_ts(tS + s * AT_BN, tQ + kk * 8, bd, idesc_qk, kk > 0 ? 1u : 0u);
         }
         mma_commit(smem_u32(&s_full[s]));
@@ -509,8 +510,8 @@ __global__ void __launch_bounds__(QKN_THREADS, 1)
         const uint32_t vaddr = smem_u32(sV + vb * AT_KV_BYTES);
 #pragma unroll
         for (int kk = 0; kk < AT_BN / 16; ++kk) {
-          const uint64_t ad = make_sdesc(paddr + kk * 32, 16, 1024, SWZ_128B);
-          const uint64_t bd = make_sdesc(vaddr + kk * (16 * 128), AT_BN * 128, 1024, SWZ_128B);
+          const uint64_t ad = make_sdesc(paddr, 16, 1024, SWZ_128B) + static_cast<uint64_t>((kk * 32) >> 4);
+          const uint64_t bd = make_sdesc(vaddr, AT_BN * 128, 1024, SWZ_128B) + static_cast<uint64_t>((kk * (16 * 128)) >> 4);
           mma_bf16_ss(tO, ad, bd, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(smem_u32(&pv_done[s]));
@@ -815,8 +816,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
 #pragma unroll
         for (int kk = 0; kk < AT_HD / 16; ++kk) {
           const uint32_t c = kk >> 2, off = (kk & 3) * 32;
-          const uint64_t ad = make_sdesc(qaddr + c * (128 * 128) + off, 16, 1024, SWZ_128B);
-          const uint64_t bd = make_sdesc(kaddr + c * (64 * 128) + off, 16, 1024, SWZ_128B);
+          const uint64_t ad = make_sdesc(qaddr, 16, 1024, SWZ_128B) + static_cast<uint64_t>((c * (128 * 128) + off) >> 4);
+          const uint64_t bd = make_sdesc(kaddr, 16, 1024, SWZ_128B) + static_cast<uint64_t>((c * (64 * 128) + off) >> 4);
           mma_bf16_ss_pair(tS + s * AP_BN, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
         }
         mma_commit_pair(smem_u32(&s_full[s]), 0x3);
@@ -834,8 +835,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
 #pragma unroll
         for (int kk = 0; kk < AP_BN / 16; ++kk) {
           const uint32_t c = kk >> 2, off = (kk & 3) * 32;
-          const uint64_t ad = make_sdesc(paddr + c * (128 * 128) + off, 16, 1024, SWZ_128B);
-          const uint64_t bd = make_sdesc(vaddr + kk * (16 * 128), AP_BN * 128, 1024, SWZ_128B);
+          const uint64_t ad = make_sdesc(paddr, 16, 1024, SWZ_128B) + static_cast<uint64_t>((c * (128 * 128) + off) >> 4);
+          const uint64_t bd = make_sdesc(vaddr, AP_BN * 128, 1024, SWZ_128B) + static_cast<uint64_t>((kk * (16 * 128)) >> 4);
           mma_bf16_ss_pair(tO, ad, bd, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit_pair(smem_u32(pv_done), 0x3);
