@@ -168,23 +168,23 @@ __device__ __forceinline__ void epilogue_qkv(const GemmParams& p, uint32_t tbase
       float mean = 0.f, rstd = 1.f;
       float v[32];
       if (which < 2) {
-        float s = 0.f;
+        // one pass over TMEM: sums of (x - k) and (x - k)^2 with the shift k =
+        // the head's first value, so E[x^2] - mean^2 does not cancel when the
+        // mean is large against the spread
+        float k = 0.f, s1 = 0.f, s2 = 0.f;
         for (int c = 0; c < chunks; ++c) {
           acc_load32(p, tbase + h0 + c * 32, a_s, col + c * 32, v);
-#pragma unroll
-          for (int j = 0; j < 32; ++j) s += v[j];
-        }
-        mean = s / hd;
-        float ss = 0.f;
-        for (int c = 0; c < chunks; ++c) {
-          acc_load32(p, tbase + h0 + c * 32, a_s, col + c * 32, v);
+          if (c == 0) k = v[0];
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
-            const float d = v[j] - mean;
-            ss += d * d;
+            const float d = v[j] - k;
+            s1 += d;
+            s2 += d * d;
           }
         }
-        rstd = rsqrtf(ss / hd + p.eps);
+        const float m1 = s1 / hd;
+        mean = k + m1;
+        rstd = rsqrtf(fmaxf(s2 / hd - m1 * m1, 0.f) + p.eps);
       }
       for (int c = 0; c < chunks; ++c) {
         acc_load32(p, tbase + h0 + c * 32, a_s, col + c * 32, v);
