@@ -1,21 +1,25 @@
 #!/usr/bin/env python
 """Denoise-step throughput of the AuraFlow forward on B200.
 
-One step = one pass of the sampling loop body on the 1024 x 1024 workload:
-the latent [1, 4, 128, 128] is duplicated into a CFG batch of 2, the full
+One step = one step of the 25-step, shift-1.73 sampling loop on the
+1024 x 1024 workload, run through the sampler plan (af_sampler: every step's
+modulations from one GEMM per 25-step run, each step a CUDA graph): the
+latent [1, 4, 128, 128] is duplicated into a CFG batch of 2, the full
 AuraFlowTransformer2DModel forward (patch embed, 4 joint + 32 single blocks,
 pre-final, unpatchify; D = 3072, 12 x 256 heads, FFN 8192, 256 text tokens +
 8 registers) runs on it, and the guidance combine + flow-match Euler update
-moves the latent to the next sigma of the 25-step, shift-1.73 schedule.
+moves the latent to the next sigma.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl af|reference]
-                    [--workload 1024|1536] [--no-cpu-baseline]
+                    [--workload 1024|1536] [--fp8] [--direct] [--no-cpu-baseline]
+                    [--no-e2e] [--case single_block]
 
 Prints one JSON line (rank 0).  Under torchrun every rank runs its own
 independent replica (weak scaling, no collective on the data path); the
 elapsed time is the max over ranks.  ``--impl reference`` times the fp64 CPU
-oracle (the reference arm of this build) on a bounded sample of the same
-workload.
+oracle on a bounded sample of the same workload.  ``--fp8`` times the 8-bit
+variant (e4m3 QKV and FFN up-projections), ``--direct`` the per-step entry
+point without the plan.
 """
 from __future__ import annotations
 

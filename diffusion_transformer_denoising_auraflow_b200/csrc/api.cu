@@ -539,7 +539,7 @@ af_status af_weights_create(const af_config* cfg, int device, af_weights** out) 
   *out = nullptr;
   Derived d;
   AF_TRY(derive(cfg, &d));
-  // kernel coverage of this build
+  // shapes the kernels cover
   if (d.D % 32 != 0 || d.F % 128 != 0 || cfg->joint_attention_dim % 8 != 0) return AF_ERR_UNSUPPORTED;
   if (!(d.hd == 256 || d.hd == 8 || d.hd == 16 || d.hd == 32 || d.hd == 64)) return AF_ERR_UNSUPPORTED;
   if (cfg->patch_size * cfg->patch_size * cfg->in_channels > 64) return AF_ERR_UNSUPPORTED;

@@ -43,7 +43,7 @@ typedef enum {
   AF_OK = 0,
   AF_ERR_INVALID_ARG = 1,  /* null handle/pointer, bad enum, negative size */
   AF_ERR_SHAPE = 2,        /* sizes inconsistent with the model or over capacity */
-  AF_ERR_UNSUPPORTED = 3,  /* configuration this build does not implement */
+  AF_ERR_UNSUPPORTED = 3,  /* configuration the kernels do not cover */
   AF_ERR_OOM = 4,          /* device allocation failed in a *_create call */
   AF_ERR_CUDA = 5,         /* CUDA runtime error (see af_last_error) */
   AF_ERR_TIMEOUT = 6,      /* a bounded device-side wait expired (from af_sync) */

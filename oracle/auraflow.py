@@ -8,8 +8,9 @@ legs of ``bench.py`` may import it.  It shares no code with the CUDA library.
 Everything is numpy float64.  Inputs arrive as float32 arrays holding
 bf16-exact (or fp32) values and are upcast once; no intermediate result is
 rounded.  Library primitives used as single steps: ``@`` (matmul), ``exp``,
-``sqrt``, ``cos``/``sin``.  Nothing is blocked, fused or reordered beyond what
-the definitions below state.
+``sqrt``, ``cos``/``sin`` (and ``log2``/``exp2``/``floor``/``round`` for the
+e4m3 rounding of the 8-bit variant).  Nothing is blocked, fused or reordered
+beyond what the definitions below state.
 
 Pages cited (title, then section):
 
