@@ -83,3 +83,18 @@ def e4m3_lut():
         else:
             out[c] = s * (1.0 + m / 8.0) * 2.0 ** (e - 7)
     return out
+
+
+def device_weights(af_module, w, seed: int, device="cuda"):
+    """Fill every tensor of the pack with seeded N(0, std^2) values drawn on
+    the device (the full 6.8 B-parameter model in seconds); the stds are the
+    synthetic-input recipe's."""
+    import zlib
+    import torch
+    for name, shape in w.tensors():
+        g = torch.Generator(device=device)
+        g.manual_seed((seed * 1000003 + zlib.crc32(name.encode())) % (2 ** 63))
+        t = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+        t.mul_(synth.weight_std(name))
+        w.set(name, t.to(torch.bfloat16).contiguous())
+    torch.cuda.synchronize()

@@ -148,3 +148,22 @@ def test_joint_block_full_size_sampled_rows(af, joint_setup):
     tr = [0, 7, 8, 128, 255]
     rt, ri = O.joint_block_rows(img, txt, temb, drawn, "joint_transformer_blocks.0.", cfg, ir, tr)
     assert O.rel_l2(gi[:, ir], ri) < BLOCK_TOL and O.rel_l2(gt[:, tr], rt) < BLOCK_TOL
+
+
+def test_single_block_1536_workload_sampled_rows(af, single_setup):
+    """The 1536^2 shape: B = 2, 8 registers + 256 text + 9216 image tokens
+    (9480 rows: 37 full 256-row GEMM tiles and a ragged tail, 75 key tiles of
+    the pair attention)."""
+    cfg, w, _, drawn = single_setup
+    s = af.Scratch(w, 2, 9216, 256)
+    N = 9480
+    x = synth.activations(15, "x1536", (2, N, 3072))
+    temb = synth.conditioning(15, (2, 3072))
+    xt = to_bf16(x)
+    af.single_block(w, s, 0, xt, to_f32(temb))
+    s.sync()
+    got = to_np(xt)
+    rows = [0, 7, 8, 263, 264, 4095, 4096, 7777, 9215, 9216, 9472, 9479]
+    ref = O.single_block_rows(x, temb, drawn, "single_transformer_blocks.0.", cfg, rows)
+    assert O.rel_l2(got[:, rows], ref) < BLOCK_TOL
+    s.close()

@@ -171,3 +171,59 @@ def test_real_width_padded_prompts_match_oracle(af):
     s.sync()
     ref = O.transformer_forward(lat, text, t, drawn, cfg, text_len=lens)
     assert O.rel_l2(to_np(vel), ref) < STACK_TOL
+
+
+@pytest.fixture(scope="module")
+def full_model(af):
+    """The full model (4 joint + 32 single blocks, D = 3072) with device-drawn
+    weights, position grid 96 x 96 (room for the 1536^2 latent)."""
+    from helpers import device_weights
+    cfg = af.Config.default(pos_embed_max_size=96 * 96)
+    w = af.Weights(cfg)
+    device_weights(af, w, 31)
+    s = af.Scratch(w, 2, 96 * 96, 256)
+    yield w, s
+    s.close()
+    w.close()
+
+
+@pytest.mark.parametrize("side", [128, 192])
+def test_full_size_forward_batch_independence(af, full_model, side):
+    """The 1024^2 and 1536^2 workloads (latent 4 x side x side, 256 text
+    tokens, CFG batch 2) in the launch configuration the bench times: each
+    sample of the batch equals its own B = 1 forward bit for bit (every
+    kernel is row- or (sample, head)-local), and the output is finite."""
+    w, s = full_model
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(side)
+    lat = torch.randn(2, 4, side, side, generator=gen, device="cuda")
+    text = torch.randn(2, 256, 2048, generator=gen, device="cuda").to(torch.bfloat16)
+    t = torch.tensor([1.0, 0.37], device="cuda")
+    both = torch.empty(2, 4, side, side, device="cuda")
+    af.transformer_forward(w, s, lat, text, t, both)
+    s.sync()
+    assert torch.isfinite(both).all()
+    for b in range(2):
+        one = torch.empty(1, 4, side, side, device="cuda")
+        af.transformer_forward(w, s, lat[b:b + 1].contiguous(), text[b:b + 1].contiguous(),
+                               t[b:b + 1].contiguous(), one)
+        s.sync()
+        assert torch.equal(both[b:b + 1], one)
+
+
+def test_full_size_guidance_one_is_the_text_half(af, full_model):
+    """At the 1024^2 workload a denoise step with guidance 1 moves the latent
+    by (sigma' - sigma) times the text-conditioned velocity alone."""
+    w, s = full_model
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(7)
+    lat = torch.randn(1, 4, 128, 128, generator=gen, device="cuda")
+    text = torch.randn(2, 256, 2048, generator=gen, device="cuda").to(torch.bfloat16)
+    sig, sig_next = 0.8, 0.75
+    x = lat.clone()
+    af.denoise_step(w, s, x, text, 1.0, sig, sig_next)
+    v = torch.empty(1, 4, 128, 128, device="cuda")
+    af.transformer_forward(w, s, lat, text[1:2].contiguous(), torch.tensor([sig], device="cuda"), v)
+    s.sync()
+    ref = lat + (sig_next - sig) * v
+    assert torch.allclose(x, ref, rtol=1e-5, atol=1e-6)
