@@ -131,34 +131,15 @@ __global__ void __launch_bounds__(256) ln_modulate_kernel(const uint16_t* __rest
 
 // Wide rows (D = 3072), HBM-bound: rows are streamed into shared memory by
 // bulk copies (4 stages of 8 rows = 192 KB in flight per SM, not limited by
-// registers).  The 8 consumer warps split the columns of a stage (warp w:
-// columns [384 w, +384)), so each lane keeps the (1 + scale) and shift of
-// its 12 columns in registers instead of re-reading 24 KB of them per row;
-// the per-row sums (mean, then squared deviations, then the e4m3 maximum)
-// are combined across warps through shared memory with named barriers.
+// registers); 8 consumer warps each normalise one row of a stage from shared
+// memory, with (1 + scale) and shift of the CTA's sample staged once.
 // Grid (CTAs per sample, samples); one CTA per SM.
 constexpr int LNB_D = 3072;
 constexpr int LNB_ROWS = 8;
 constexpr int LNB_STAGES = 4;
 constexpr uint32_t LNB_ROW_BYTES = LNB_D * 2;
 constexpr int LNB_THREADS = 32 * (LNB_ROWS + 1);
-constexpr int LNB_SMEM = LNB_STAGES * LNB_ROWS * LNB_ROW_BYTES + 2 * LNB_D * 4 + 3 * LNB_ROWS * 8 * 4 + 128 + 128;
-
-// Named barrier 1 over the 8 consumer warps (the producer warp never joins).
-__device__ __forceinline__ void consumers_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
-// The same barrier, returning whether v holds in every consumer thread.
-__device__ __forceinline__ bool consumers_all(bool v) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.and.pred q, 1, 256, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"(static_cast<uint32_t>(v))
-      : "memory");
-  return r != 0;
-}
+constexpr int LNB_SMEM = LNB_STAGES * LNB_ROWS * LNB_ROW_BYTES + 2 * LNB_D * 4 + 128 + 128;
 
 template <bool OUT8>
 __global__ void __launch_bounds__(LNB_THREADS, 1) ln_modulate_bulk_kernel(const uint16_t* __restrict__ x,
@@ -172,7 +153,7 @@ __global__ void __launch_bounds__(LNB_THREADS, 1) ln_modulate_bulk_kernel(const 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(lnb_raw) + 127) & ~uintptr_t(127));
   uint8_t* rowbuf = smem;                                                       // [stage][row] x 6 KB
   float* mod_s = reinterpret_cast<float*>(smem + LNB_STAGES * LNB_ROWS * LNB_ROW_BYTES);  // 1 + scale | shift
-  uint64_t* full = reinterpret_cast<uint64_t*>(mod_s + 2 * LNB_D + 3 * LNB_ROWS * 8);  // after the partial sums
+  uint64_t* full = reinterpret_cast<uint64_t*>(mod_s + 2 * LNB_D);
   uint64_t* empty = full + LNB_STAGES;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + LNB_STAGES);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -220,127 +201,83 @@ __global__ void __launch_bounds__(LNB_THREADS, 1) ln_modulate_bulk_kernel(const 
     }
     return;
   }
-  // consumers: warp w owns columns [384 w, 384 w + 384) of every row, so its
-  // (1 + scale) and shift stay in registers (lane: 3 vectors of 4 columns);
-  // the row statistics are summed across the 8 warps through shared memory
-  constexpr int VPT = 3;                            // 4-column vectors per lane
-  float* red = mod_s + 2 * LNB_D;                   // [3][LNB_ROWS][8] partial sums
-  float av[VPT][4], hv[VPT][4];
-#pragma unroll
-  for (int i = 0; i < VPT; ++i) {
-    const int col = 4 * (warp * 96 + i * 32 + lane);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      av[i][e] = mod_s[col + e];
-      hv[i][e] = mod_s[LNB_D + col + e];
-    }
-  }
+  // consumers: warp w normalises row w of every stage
+  constexpr int VPL = LNB_D / 256;
   int k = 0;
   for (int c = blockIdx.x; c < nchunks; c += gridDim.x, ++k) {
     const int st = k % LNB_STAGES;
     const uint32_t ph = (k / LNB_STAGES) & 1;
     const bool got = mbar_wait(smem_u32(&full[st]), ph, err, abort_flag);
-    if (!consumers_all(got)) break;  // uniform across the 8 consumer warps (a barrier)
-    const int nvalid = min(LNB_ROWS, rows_per_batch - c * LNB_ROWS);
-    // this lane's 12 values of each of the 8 rows, packed bf16
-    uint2 cur[LNB_ROWS][VPT];
+    if (!__all_sync(0xffffffffu, got)) break;
+    const int r = c * LNB_ROWS + warp;
+    if (r < rows_per_batch) {
+      const uint4* xr = reinterpret_cast<const uint4*>(rowbuf + (st * LNB_ROWS + warp) * LNB_ROW_BYTES);
+      uint4 cur[VPL];
 #pragma unroll
-    for (int r = 0; r < LNB_ROWS; ++r) {
-      const uint2* xr = reinterpret_cast<const uint2*>(rowbuf + (st * LNB_ROWS + r) * LNB_ROW_BYTES);
+      for (int i = 0; i < VPL; ++i) cur[i] = xr[i * 32 + lane];
+      float s = 0.f;
 #pragma unroll
-      for (int i = 0; i < VPT; ++i) cur[r][i] = xr[warp * 96 + i * 32 + lane];
-    }
-    // pass 1: row sums
+      for (int i = 0; i < VPL; ++i) {
+        const uint32_t w[4] = {cur[i].x, cur[i].y, cur[i].z, cur[i].w};
 #pragma unroll
-    for (int r = 0; r < LNB_ROWS; ++r) {
-      float s1 = 0.f;
-#pragma unroll
-      for (int i = 0; i < VPT; ++i)
-        s1 += (bf16_lo(cur[r][i].x) + bf16_hi(cur[r][i].x)) + (bf16_lo(cur[r][i].y) + bf16_hi(cur[r][i].y));
-      s1 = warp_sum(s1);
-      if (lane == 0) red[r * 8 + warp] = s1;
-    }
-    consumers_sync();
-    float mean[LNB_ROWS];
-#pragma unroll
-    for (int r = 0; r < LNB_ROWS; ++r) {
-      float t = 0.f;
-#pragma unroll
-      for (int w = 0; w < 8; ++w) t += red[r * 8 + w];
-      mean[r] = t * (1.0f / LNB_D);
-    }
-    // pass 2: sums of squared deviations
-#pragma unroll
-    for (int r = 0; r < LNB_ROWS; ++r) {
-      float s2 = 0.f;
-#pragma unroll
-      for (int i = 0; i < VPT; ++i) {
-        const float d0 = bf16_lo(cur[r][i].x) - mean[r], d1 = bf16_hi(cur[r][i].x) - mean[r];
-        const float d2 = bf16_lo(cur[r][i].y) - mean[r], d3 = bf16_hi(cur[r][i].y) - mean[r];
-        s2 += (d0 * d0 + d1 * d1) + (d2 * d2 + d3 * d3);
+        for (int e = 0; e < 4; ++e) s += bf16_lo(w[e]) + bf16_hi(w[e]);
       }
-      s2 = warp_sum(s2);
-      if (lane == 0) red[LNB_ROWS * 8 + r * 8 + warp] = s2;
-    }
-    consumers_sync();
-    float rstd[LNB_ROWS];
+      const float mean = warp_sum(s) * (1.0f / LNB_D);
+      float ss = 0.f;
 #pragma unroll
-    for (int r = 0; r < LNB_ROWS; ++r) {
-      float t = 0.f;
+      for (int i = 0; i < VPL; ++i) {
+        const uint32_t w[4] = {cur[i].x, cur[i].y, cur[i].z, cur[i].w};
 #pragma unroll
-      for (int w = 0; w < 8; ++w) t += red[LNB_ROWS * 8 + r * 8 + w];
-      rstd[r] = rsqrtf(t * (1.0f / LNB_D) + eps);
-    }
-    // output element e of vector i of row r: (x - mean) rstd (1 + scale) + shift
-    auto out4 = [&](int r, int i, float (&o)[4]) {
-      const float xv[4] = {bf16_lo(cur[r][i].x), bf16_hi(cur[r][i].x), bf16_lo(cur[r][i].y), bf16_hi(cur[r][i].y)};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) o[e] = (xv[e] - mean[r]) * rstd[r] * av[i][e] + hv[i][e];
-    };
-    if constexpr (OUT8) {
-      // pass 3: row maxima of |output| for the e4m3 scale
-#pragma unroll
-      for (int r = 0; r < LNB_ROWS; ++r) {
-        float m = 0.f;
-#pragma unroll
-        for (int i = 0; i < VPT; ++i) {
-          float o[4];
-          out4(r, i, o);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) m = fmaxf(m, fabsf(o[e]));
+        for (int e = 0; e < 4; ++e) {
+          const float d0 = bf16_lo(w[e]) - mean, d1 = bf16_hi(w[e]) - mean;
+          ss += d0 * d0 + d1 * d1;
         }
-        m = warp_max(m);
-        if (lane == 0) red[2 * LNB_ROWS * 8 + r * 8 + warp] = m;
       }
-      consumers_sync();
+      const float rstd = rsqrtf(warp_sum(ss) * (1.0f / LNB_D) + eps);
+      // output element 2e (+1) of vector i: (x - mean) rstd (1 + scale) + shift
+      auto out8 = [&](int i, float (&o)[8]) {
+        const int vi = i * 32 + lane;
+        const float4 a0 = *reinterpret_cast<const float4*>(mod_s + vi * 8);
+        const float4 a1 = *reinterpret_cast<const float4*>(mod_s + vi * 8 + 4);
+        const float4 h0 = *reinterpret_cast<const float4*>(mod_s + LNB_D + vi * 8);
+        const float4 h1 = *reinterpret_cast<const float4*>(mod_s + LNB_D + vi * 8 + 4);
+        const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+        const float hv[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+        const uint32_t w[4] = {cur[i].x, cur[i].y, cur[i].z, cur[i].w};
 #pragma unroll
-      for (int r = 0; r < LNB_ROWS; ++r) {
+        for (int e = 0; e < 4; ++e) {
+          o[2 * e] = (bf16_lo(w[e]) - mean) * rstd * av[2 * e] + hv[2 * e];
+          o[2 * e + 1] = (bf16_hi(w[e]) - mean) * rstd * av[2 * e + 1] + hv[2 * e + 1];
+        }
+      };
+      if constexpr (OUT8) {
         float amax = 0.f;
 #pragma unroll
-        for (int w = 0; w < 8; ++w) amax = fmaxf(amax, red[2 * LNB_ROWS * 8 + r * 8 + w]);
-        if (r < nvalid) {
-          const float inv = e4m3_inv_scale(amax);
-          uint32_t* yr = reinterpret_cast<uint32_t*>(y8 + (row0 + static_cast<size_t>(c) * LNB_ROWS + r) * LNB_D);
+        for (int i = 0; i < VPL; ++i) {
+          float o[8];
+          out8(i, o);
 #pragma unroll
-          for (int i = 0; i < VPT; ++i) {
-            float o[4];
-            out4(r, i, o);
-            yr[warp * 96 + i * 32 + lane] = pack_e4m3x4(o[0] * inv, o[1] * inv, o[2] * inv, o[3] * inv);
-          }
-          if (warp == 0 && lane == 0) yscale[row0 + static_cast<size_t>(c) * LNB_ROWS + r] = e4m3_scale(amax);
+          for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(o[e]));
         }
-      }
-    } else {
+        amax = warp_max(amax);
+        const float inv = e4m3_inv_scale(amax);
+        uint2* yr = reinterpret_cast<uint2*>(y8 + (row0 + r) * LNB_D);
 #pragma unroll
-      for (int r = 0; r < LNB_ROWS; ++r) {
-        if (r < nvalid) {
-          uint2* yr = reinterpret_cast<uint2*>(y + (row0 + static_cast<size_t>(c) * LNB_ROWS + r) * LNB_D);
+        for (int i = 0; i < VPL; ++i) {
+          float o[8];
+          out8(i, o);
+          yr[i * 32 + lane] = make_uint2(pack_e4m3x4(o[0] * inv, o[1] * inv, o[2] * inv, o[3] * inv),
+                                         pack_e4m3x4(o[4] * inv, o[5] * inv, o[6] * inv, o[7] * inv));
+        }
+        if (lane == 0) yscale[row0 + r] = e4m3_scale(amax);
+      } else {
+        uint4* yr = reinterpret_cast<uint4*>(y + (row0 + r) * LNB_D);
 #pragma unroll
-          for (int i = 0; i < VPT; ++i) {
-            float o[4];
-            out4(r, i, o);
-            yr[warp * 96 + i * 32 + lane] = make_uint2(pack_bf16(o[0], o[1]), pack_bf16(o[2], o[3]));
-          }
+        for (int i = 0; i < VPL; ++i) {
+          float o[8];
+          out8(i, o);
+          yr[i * 32 + lane] = make_uint4(pack_bf16(o[0], o[1]), pack_bf16(o[2], o[3]), pack_bf16(o[4], o[5]),
+                                         pack_bf16(o[6], o[7]));
         }
       }
     }
