@@ -364,6 +364,11 @@ def _w8(w, fp8):
     return fake_quant_rows(w) if fp8 else _f(w)
 
 
+def _a8(x, fp8):
+    """A GEMM's activation input as the GEMM sees it: as is, or per-token e4m3."""
+    return fake_quant_rows(x) if fp8 else _f(x)
+
+
 def qkv_normed(y, wq, wk, wv, heads: int, eps: float, fp8: bool = False):
     """Bias-free Q/K/V projections, then per-head LayerNorm of Q and K (not V).
 
@@ -385,9 +390,9 @@ def feed_forward(y, w1, w2, w3, fp8: bool = False):
 
     [ARCH §FeedForward], [PIPE §深入源码] (SiLU-gated FFN).
     """
-    if fp8:   # 8-bit variant: the up-projections' inputs; the down-projection stays as is
-        y = fake_quant_rows(y)
-    return (silu(y @ _w8(w1, fp8).T) * (y @ _w8(w2, fp8).T)) @ _f(w3).T
+    y = _a8(y, fp8)
+    h = silu(y @ _w8(w1, fp8).T) * (y @ _w8(w2, fp8).T)
+    return _a8(h, fp8) @ _w8(w3, fp8).T
 
 
 # --------------------------------------------------------------------------
@@ -396,13 +401,13 @@ def feed_forward(y, w1, w2, w3, fp8: bool = False):
 # --------------------------------------------------------------------------
 # The pipeline guide loads the transformer with 8-bit weights
 # ([PIPE] bitsandbytes quantisation sections).  The variant here is the
-# tensor-core-native form of that idea: the inputs of the two GEMMs whose
-# activations come straight out of the LayerNorm+modulate step (the fused
-# QKV projections and the FFN up-projections) are rounded to the e4m3 format,
-# each activation row (token) and each weight row (output channel) with its
-# own fp32 scale, and the product is rescaled by both scales.
+# tensor-core-native form of that idea: the operands of every projection in
+# the blocks (fused QKV, output projection, FFN up and down) are rounded to
+# the e4m3 format, each activation row (token) and each weight row (output
+# channel) with its own fp32 scale, and the product is rescaled by both.
 # READING: per-row absolute-maximum scaling, amax -> 448 (the largest finite
-# e4m3 value); the output projections and FFN down-projections stay bf16.
+# e4m3 value); the attention itself, the LayerNorms, the modulations and the
+# embedding / output stages stay as in the bf16 path.
 
 E4M3_MAX = 448.0
 
@@ -469,7 +474,7 @@ def single_block_mod(x, mod, w, prefix, heads, eps, key_mask=None, fp8=False):
     q, k, v = qkv_normed(y, w[prefix + "attn.to_q.weight"], w[prefix + "attn.to_k.weight"],
                          w[prefix + "attn.to_v.weight"], heads, eps, fp8)
     o = merge_heads(attention(q, k, v, key_mask=key_mask))
-    x = x + mod["gate_msa"][:, None, :] * (o @ _f(w[prefix + "attn.to_out.0.weight"]).T)
+    x = x + mod["gate_msa"][:, None, :] * (_a8(o, fp8) @ _w8(w[prefix + "attn.to_out.0.weight"], fp8).T)
     y = modulate(x, mod["shift_mlp"], mod["scale_mlp"], eps)
     f = feed_forward(y, w[prefix + "ff.linear_1.weight"], w[prefix + "ff.linear_2.weight"],
                      w[prefix + "ff.out_projection.weight"], fp8)
@@ -506,8 +511,8 @@ def joint_block_mod(img, txt, mod_i, mod_t, w, prefix, heads, eps, key_mask=None
     v = np.concatenate([vt, vi], axis=2)
     o = merge_heads(attention(q, k, v, key_mask=key_mask))
     ot, oi = o[:, :nt], o[:, nt:]
-    img = img + mod_i["gate_msa"][:, None, :] * (oi @ _f(w[prefix + "attn.to_out.0.weight"]).T)
-    txt = txt + mod_t["gate_msa"][:, None, :] * (ot @ _f(w[prefix + "attn.to_add_out.weight"]).T)
+    img = img + mod_i["gate_msa"][:, None, :] * (_a8(oi, fp8) @ _w8(w[prefix + "attn.to_out.0.weight"], fp8).T)
+    txt = txt + mod_t["gate_msa"][:, None, :] * (_a8(ot, fp8) @ _w8(w[prefix + "attn.to_add_out.weight"], fp8).T)
     yi = modulate(img, mod_i["shift_mlp"], mod_i["scale_mlp"], eps)
     yt = modulate(txt, mod_t["shift_mlp"], mod_t["scale_mlp"], eps)
     img = img + mod_i["gate_mlp"][:, None, :] * feed_forward(
@@ -642,7 +647,7 @@ def transformer_forward(latents, text_emb, t, w, cfg: Config, text_len=None, fp8
     unpatchify.  ``t`` is the model time in [0, 1] (timestep / 1000).
     ``text_len`` (optional, [B]): real prompt tokens per sample; the rest of
     the L text tokens are padding that no attention reads (``text_key_mask``).
-    ``fp8``: the 8-bit variant of the QKV and FFN up-projections.
+    ``fp8``: the 8-bit variant (e4m3 operands for every projection in the blocks).
     """
     latents = _f(latents)
     H, W = latents.shape[2], latents.shape[3]
