@@ -89,15 +89,18 @@ struct af_weights {
   size_t ada_rows = 0;
   std::vector<size_t> unit_row;  // first row of unit u (joint i: 2i img, 2i+1 txt; single j: 2J + j)
   size_t pf_row = 0;             // first row of norm_out
-  // 8-bit variant: e4m3 copies of the fused QKV and FFN up-projection
-  // weights with one fp32 scale per row (af_weights_quantize_fp8).  Each
-  // region starts at a multiple of 256 rows of the 8-bit pack, so every
-  // scale a 256-column tile can touch exists.
+  // 8-bit variant: e4m3 copies of every block projection's weight (fused
+  // QKV, output projection, FFN up pair, FFN down) with one fp32 scale per
+  // row (af_weights_quantize_fp8).  Each region's scales start at a multiple
+  // of 256 rows, so every scale a 256-column tile can touch exists.
+  struct Fp8Region {
+    size_t code_off;   // bytes into fp8_codes
+    size_t scale_off;  // entries into fp8_scales
+  };
   bool fp8 = false;
-  uint8_t* fp8_codes = nullptr;  // [fp8_rows, D]
-  float* fp8_scales = nullptr;   // [fp8_rows]
-  size_t fp8_rows = 0;
-  std::unordered_map<std::string, size_t> fp8_row;  // region's first tensor name -> first row
+  uint8_t* fp8_codes = nullptr;
+  float* fp8_scales = nullptr;
+  std::unordered_map<std::string, Fp8Region> fp8_region;  // region's first tensor name -> offsets
 
   const uint16_t* ptr(const std::string& n) const {
     auto it = index.find(n);
@@ -293,9 +296,9 @@ struct Operand {
 // The weight region starting at tensor `name` as the GEMM reads it.
 Operand weight_op(const af_weights* w, const std::string& name) {
   if (w->fp8) {
-    auto it = w->fp8_row.find(name);
-    if (it != w->fp8_row.end())
-      return {w->fp8_codes + it->second * static_cast<size_t>(w->d.D), w->fp8_scales + it->second};
+    auto it = w->fp8_region.find(name);
+    if (it != w->fp8_region.end())
+      return {w->fp8_codes + it->second.code_off, w->fp8_scales + it->second.scale_off};
   }
   return {w->ptr(name), nullptr};
 }
@@ -321,14 +324,25 @@ af_status qkv(const af_weights* w, af_scratch* s, Operand y, int B, int rows, Op
 }
 
 // x += gate[b] * (A W^T)
-af_status gated_residual(af_scratch* s, const uint16_t* A, int B, int rows, int K, const uint16_t* W, int N,
-                         uint16_t* x, const float* gate, int gate_stride, cudaStream_t st) {
+af_status gated_residual(af_scratch* s, Operand A, int B, int rows, int K, Operand W, int N, uint16_t* x,
+                         const float* gate, int gate_stride, cudaStream_t st) {
+  if ((A.scale != nullptr) != (W.scale != nullptr)) return AF_ERR_UNSUPPORTED;
   GemmParams p = gemm_base(s, B * rows, N, K, EPI_GATE_RES, rows);
   p.out = x;
   p.ldo = N;
   p.gate = gate;
   p.gate_stride = gate_stride;
-  return run_gemm(s, p, A, W, N, st);
+  p.a_scale = A.scale;
+  p.w_scale = W.scale;
+  return run_gemm(s, p, A.ptr, W.ptr, N, st);
+}
+
+// The 8-bit variant's per-token quantisation of a bf16 activation [rows, K]
+// (attention output, SwiGLU product) into e4m3 codes + row scales.
+af_status quantize_act(af_scratch* s, const uint16_t* x, int rows, int K, uint8_t* q, float* scale, cudaStream_t st) {
+  LaunchScope ls(s, KC_LN, 3.0 * rows * K, st);
+  cudaError_t e = launch_quantize_rows_e4m3(x, rows, K, q, scale, st);
+  return e == cudaSuccess ? AF_OK : cuda_fail(e);
 }
 
 // h = silu(y W1^T) * (y W2^T), W1 and W2 interleaved in 128-row groups ([2F, D])
@@ -431,17 +445,34 @@ af_status joint_block_impl(const af_weights* w, af_scratch* s, int layer, uint16
   AF_TRY(qkv(w, s, a_txt, B, Nt, weight_op(w, pre + "attn.add_q_proj.weight"), 0, N, st));
   AF_TRY(qkv(w, s, a_img, B, Ni, weight_op(w, pre + "attn.to_q.weight"), Nt, N, st));
   AF_TRY(attention(w, s, B, N, o_txt, o_img, Nt, km, st));
-  AF_TRY(gated_residual(s, o_img, B, Ni, D, w->ptr(pre + "attn.to_out.0.weight"), D, img, mi + 2 * D, mod_stride, st));
-  AF_TRY(gated_residual(s, o_txt, B, Nt, D, w->ptr(pre + "attn.to_add_out.weight"), D, txt, mt + 2 * D, mod_stride,
-                        st));
+  // 8-bit variant: the attention output and the SwiGLU product are quantised
+  // per token (into the same e4m3 buffer, free again once QKV / FFN-up ran)
+  Operand oa_img{o_img, nullptr}, oa_txt{o_txt, nullptr}, ha_img{h_img, nullptr}, ha_txt{h_txt, nullptr};
+  if (f8) {
+    AF_TRY(quantize_act(s, o_img, B * Ni, D, q8_img, ys_img, st));
+    AF_TRY(quantize_act(s, o_txt, B * Nt, D, q8_txt, ys_txt, st));
+    oa_img = {q8_img, ys_img};
+    oa_txt = {q8_txt, ys_txt};
+  }
+  AF_TRY(gated_residual(s, oa_img, B, Ni, D, weight_op(w, pre + "attn.to_out.0.weight"), D, img, mi + 2 * D,
+                        mod_stride, st));
+  AF_TRY(gated_residual(s, oa_txt, B, Nt, D, weight_op(w, pre + "attn.to_add_out.weight"), D, txt, mt + 2 * D,
+                        mod_stride, st));
   AF_TRY(ln_mod(s, img, mi + 3 * D, mi + 4 * D, mod_stride, y_img, B * Ni, Ni, D, eps, st, q8_img, ys_img));
   AF_TRY(ln_mod(s, txt, mt + 3 * D, mt + 4 * D, mod_stride, y_txt, B * Nt, Nt, D, eps, st, q8_txt, ys_txt));
   AF_TRY(swiglu(w, s, a_img, B * Ni, weight_op(w, pre + "ff.linear_1.weight"), h_img, st));
   AF_TRY(swiglu(w, s, a_txt, B * Nt, weight_op(w, pre + "ff_context.linear_1.weight"), h_txt, st));
-  AF_TRY(gated_residual(s, h_img, B, Ni, d.F, w->ptr(pre + "ff.out_projection.weight"), D, img, mi + 5 * D,
+  if (f8) {
+    uint8_t* h8_txt = s->y8 + static_cast<size_t>(B) * Ni * d.F;
+    AF_TRY(quantize_act(s, h_img, B * Ni, d.F, s->y8, ys_img, st));
+    AF_TRY(quantize_act(s, h_txt, B * Nt, d.F, h8_txt, ys_txt, st));
+    ha_img = {s->y8, ys_img};
+    ha_txt = {h8_txt, ys_txt};
+  }
+  AF_TRY(gated_residual(s, ha_img, B, Ni, d.F, weight_op(w, pre + "ff.out_projection.weight"), D, img, mi + 5 * D,
                         mod_stride, st));
-  AF_TRY(gated_residual(s, h_txt, B, Nt, d.F, w->ptr(pre + "ff_context.out_projection.weight"), D, txt, mt + 5 * D,
-                        mod_stride, st));
+  AF_TRY(gated_residual(s, ha_txt, B, Nt, d.F, weight_op(w, pre + "ff_context.out_projection.weight"), D, txt,
+                        mt + 5 * D, mod_stride, st));
   return AF_OK;
 }
 
@@ -458,10 +489,19 @@ af_status single_block_impl(const af_weights* w, af_scratch* s, int layer, uint1
   AF_TRY(ln_mod(s, x, m + 0 * D, m + 1 * D, mod_stride, s->y, B * N, N, D, eps, st, q8, ys));
   AF_TRY(qkv(w, s, a, B, N, weight_op(w, pre + "attn.to_q.weight"), 0, N, st));
   AF_TRY(attention(w, s, B, N, s->o, s->o, 0, km, st));
-  AF_TRY(gated_residual(s, s->o, B, N, D, w->ptr(pre + "attn.to_out.0.weight"), D, x, m + 2 * D, mod_stride, st));
+  Operand oa{s->o, nullptr}, ha{s->h, nullptr};
+  if (f8) {  // per-token e4m3 of the attention output (the QKV input codes are dead by now)
+    AF_TRY(quantize_act(s, s->o, B * N, D, q8, ys, st));
+    oa = {q8, ys};
+  }
+  AF_TRY(gated_residual(s, oa, B, N, D, weight_op(w, pre + "attn.to_out.0.weight"), D, x, m + 2 * D, mod_stride, st));
   AF_TRY(ln_mod(s, x, m + 3 * D, m + 4 * D, mod_stride, s->y, B * N, N, D, eps, st, q8, ys));
   AF_TRY(swiglu(w, s, a, B * N, weight_op(w, pre + "ff.linear_1.weight"), s->h, st));
-  AF_TRY(gated_residual(s, s->h, B, N, d.F, w->ptr(pre + "ff.out_projection.weight"), D, x, m + 5 * D, mod_stride,
+  if (f8) {  // per-token e4m3 of the SwiGLU product (rows of F codes)
+    AF_TRY(quantize_act(s, s->h, B * N, d.F, q8, ys, st));
+    ha = {q8, ys};
+  }
+  AF_TRY(gated_residual(s, ha, B, N, d.F, weight_op(w, pre + "ff.out_projection.weight"), D, x, m + 5 * D, mod_stride,
                         st));
   return AF_OK;
 }
@@ -642,32 +682,41 @@ af_status af_weights_quantize_fp8(af_weights* w, int enable, void* stream) {
     if (w->fp8_scales) cudaFree(w->fp8_scales);
     w->fp8_codes = nullptr;
     w->fp8_scales = nullptr;
-    w->fp8_rows = 0;
-    w->fp8_row.clear();
+    w->fp8_region.clear();
     w->fp8 = false;
     return AF_OK;
   }
   const af_config& c = w->cfg;
-  const int D = w->d.D;
-  const size_t qkv_rows = 3 * static_cast<size_t>(D), up_rows = 2 * static_cast<size_t>(w->d.F);
-  std::vector<std::pair<std::string, size_t>> regions;
+  const size_t D = w->d.D, F = w->d.F;
+  struct Region {
+    std::string name;
+    size_t rows, cols;
+  };
+  std::vector<Region> regions;
   for (int i = 0; i < c.num_mmdit_layers; ++i) {
     const std::string b = "joint_transformer_blocks." + std::to_string(i) + ".";
-    regions.push_back({b + "attn.to_q.weight", qkv_rows});
-    regions.push_back({b + "attn.add_q_proj.weight", qkv_rows});
-    regions.push_back({b + "ff.linear_1.weight", up_rows});
-    regions.push_back({b + "ff_context.linear_1.weight", up_rows});
+    regions.push_back({b + "attn.to_q.weight", 3 * D, D});
+    regions.push_back({b + "attn.add_q_proj.weight", 3 * D, D});
+    regions.push_back({b + "attn.to_out.0.weight", D, D});
+    regions.push_back({b + "attn.to_add_out.weight", D, D});
+    regions.push_back({b + "ff.linear_1.weight", 2 * F, D});
+    regions.push_back({b + "ff_context.linear_1.weight", 2 * F, D});
+    regions.push_back({b + "ff.out_projection.weight", D, F});
+    regions.push_back({b + "ff_context.out_projection.weight", D, F});
   }
   for (int i = 0; i < c.num_single_dit_layers; ++i) {
     const std::string b = "single_transformer_blocks." + std::to_string(i) + ".";
-    regions.push_back({b + "attn.to_q.weight", qkv_rows});
-    regions.push_back({b + "ff.linear_1.weight", up_rows});
+    regions.push_back({b + "attn.to_q.weight", 3 * D, D});
+    regions.push_back({b + "attn.to_out.0.weight", D, D});
+    regions.push_back({b + "ff.linear_1.weight", 2 * F, D});
+    regions.push_back({b + "ff.out_projection.weight", D, F});
   }
-  std::unordered_map<std::string, size_t> first;
-  size_t rows = 0;
+  std::unordered_map<std::string, af_weights::Fp8Region> where;
+  size_t code_bytes = 0, scale_rows = 0;
   for (auto& r : regions) {
-    first[r.first] = rows;
-    rows += (r.second + 255) / 256 * 256;
+    where[r.name] = {code_bytes, scale_rows};
+    code_bytes = (code_bytes + r.rows * r.cols + 255) & ~size_t(255);
+    scale_rows += (r.rows + 255) / 256 * 256;
   }
   int prev = 0;
   cudaGetDevice(&prev);
@@ -675,8 +724,8 @@ af_status af_weights_quantize_fp8(af_weights* w, int enable, void* stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaSuccess;
   if (!w->fp8_codes) {
-    e = cudaMalloc(&w->fp8_codes, rows * D);
-    if (e == cudaSuccess) e = cudaMalloc(&w->fp8_scales, rows * sizeof(float));
+    e = cudaMalloc(&w->fp8_codes, code_bytes);
+    if (e == cudaSuccess) e = cudaMalloc(&w->fp8_scales, scale_rows * sizeof(float));
     if (e != cudaSuccess) {
       cudaGetLastError();
       if (w->fp8_codes) cudaFree(w->fp8_codes);
@@ -685,17 +734,17 @@ af_status af_weights_quantize_fp8(af_weights* w, int enable, void* stream) {
       cudaSetDevice(prev);
       return AF_ERR_OOM;
     }
-    w->fp8_rows = rows;
-    e = cudaMemsetAsync(w->fp8_scales, 0, rows * sizeof(float), st);  // padding rows
+    e = cudaMemsetAsync(w->fp8_scales, 0, scale_rows * sizeof(float), st);  // padding rows
   }
   for (size_t i = 0; i < regions.size() && e == cudaSuccess; ++i) {
-    const size_t r0 = first[regions[i].first];
-    e = launch_quantize_rows_e4m3(w->ptr(regions[i].first), static_cast<int>(regions[i].second), D,
-                                  w->fp8_codes + r0 * D, w->fp8_scales + r0, st);
+    const auto& r = regions[i];
+    const auto& at = where[r.name];
+    e = launch_quantize_rows_e4m3(w->ptr(r.name), static_cast<int>(r.rows), static_cast<int>(r.cols),
+                                  w->fp8_codes + at.code_off, w->fp8_scales + at.scale_off, st);
   }
   cudaSetDevice(prev);
   if (e != cudaSuccess) return cuda_fail(e);
-  w->fp8_row = first;
+  w->fp8_region = where;
   w->fp8 = true;
   return AF_OK;
 }
@@ -741,7 +790,7 @@ af_status af_scratch_create(const af_weights* w, int max_batch, int max_img_toke
   const size_t o_img = take(B * s->max_ni * D * 2);
   const size_t o_txt = take(B * s->max_nt * D * 2);
   const size_t o_x = take(rowsN * D * 2);
-  const size_t o_y8 = take(rowsN * D);
+  const size_t o_y8 = take(rowsN * (D > F ? D : F));  // e4m3 codes of y, O or h (8-bit variant)
   const size_t o_ys = take(rowsN * 4);
   const int cmax = w->cfg.in_channels > w->cfg.out_channels ? w->cfg.in_channels : w->cfg.out_channels;
   const size_t lat_elems = B * static_cast<size_t>(cmax) * s->max_ni * w->cfg.patch_size * w->cfg.patch_size;

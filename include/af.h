@@ -261,18 +261,20 @@ void af_sampler_destroy(af_sampler* smp);
 
 /* ---- 8-bit variant ----------------------------------------------------------
  * The pipeline guide loads the transformer with 8-bit weights ([PIPE]
- * bitsandbytes sections).  This is the tensor-core form of that idea: the
- * fused QKV projections and the FFN up-projections (the GEMMs whose inputs
- * come straight out of LayerNorm + modulate) run with e4m3 operands on
- * tcgen05 kind::f8f6f4 MMAs, each activation row (token) and each weight row
- * (output channel) scaled by its own fp32 factor amax / 448; the output
- * projections, FFN down-projections and attention stay bf16.
+ * bitsandbytes sections).  This is the tensor-core form of that idea: every
+ * projection of the blocks (fused QKV, output projection, FFN up pair, FFN
+ * down) runs with e4m3 operands on tcgen05 kind::f8f6f4 MMAs, each
+ * activation row (token) and each weight row (output channel) scaled by its
+ * own fp32 factor amax / 448.  The LayerNorm+modulate kernel emits e4m3
+ * directly; the attention output and the SwiGLU product are quantised per
+ * token by a separate pass.  Attention, the LayerNorms, the modulations and
+ * the embedding / output stages stay as in the bf16 path.
  *
  * af_weights_quantize_fp8(w, 1, stream) quantises the current bf16 values
- * of those weights into a second device pack (about 46% of the bf16 pack)
- * and switches every later forward, block and sampler step on `w` to the
- * 8-bit GEMMs; call it again after changing weights.  enable = 0 frees the
- * pack and returns to bf16.  Create samplers after switching. */
+ * of those weights into a second device pack (about a third of the bf16
+ * pack) and switches every later forward, block and sampler step on `w` to
+ * the 8-bit GEMMs; call it again after changing weights.  enable = 0 frees
+ * the pack and returns to bf16.  Create samplers after switching. */
 af_status af_weights_quantize_fp8(af_weights* w, int enable, void* stream);
 
 /* Per-row e4m3 quantisation: for each row of x (device bf16 [rows, cols],

@@ -118,7 +118,7 @@ def test_single_block_fp8_matches_oracle(af):
     # the variant differs from the bf16 block by the e4m3 rounding, visibly but not grossly
     ref16 = O.single_block(x, temb, drawn, pre, cfg)
     err16 = O.rel_l2(got - x, ref16 - x)
-    assert 1e-3 < err16 < 0.15
+    assert 1e-3 < err16 < 0.2
 
 
 def test_joint_block_fp8_matches_oracle(af):
