@@ -369,6 +369,20 @@ def _a8(x, fp8):
     return fake_quant_rows(x) if fp8 else _f(x)
 
 
+def round_bf16(x):
+    """fp32 value of x, then rounded to bf16 (8 significant bits) to nearest even."""
+    b = np.asarray(x, dtype=np.float64).astype(np.float32).view(np.uint32).astype(np.uint64)
+    b = (b + 0x7FFF + ((b >> 16) & 1)) & 0xFFFF0000
+    return b.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+def _a8_stored(x, fp8):
+    """Like _a8 for an activation the kernel path stores as bf16 before it is
+    quantised (the attention output, the SwiGLU product): the per-token e4m3
+    decision is taken on the bf16 value, in the kernel's precision."""
+    return fake_quant_rows(round_bf16(x)) if fp8 else _f(x)
+
+
 def qkv_normed(y, wq, wk, wv, heads: int, eps: float, fp8: bool = False):
     """Bias-free Q/K/V projections, then per-head LayerNorm of Q and K (not V).
 
@@ -392,7 +406,7 @@ def feed_forward(y, w1, w2, w3, fp8: bool = False):
     """
     y = _a8(y, fp8)
     h = silu(y @ _w8(w1, fp8).T) * (y @ _w8(w2, fp8).T)
-    return _a8(h, fp8) @ _w8(w3, fp8).T
+    return _a8_stored(h, fp8) @ _w8(w3, fp8).T
 
 
 # --------------------------------------------------------------------------
@@ -474,7 +488,7 @@ def single_block_mod(x, mod, w, prefix, heads, eps, key_mask=None, fp8=False):
     q, k, v = qkv_normed(y, w[prefix + "attn.to_q.weight"], w[prefix + "attn.to_k.weight"],
                          w[prefix + "attn.to_v.weight"], heads, eps, fp8)
     o = merge_heads(attention(q, k, v, key_mask=key_mask))
-    x = x + mod["gate_msa"][:, None, :] * (_a8(o, fp8) @ _w8(w[prefix + "attn.to_out.0.weight"], fp8).T)
+    x = x + mod["gate_msa"][:, None, :] * (_a8_stored(o, fp8) @ _w8(w[prefix + "attn.to_out.0.weight"], fp8).T)
     y = modulate(x, mod["shift_mlp"], mod["scale_mlp"], eps)
     f = feed_forward(y, w[prefix + "ff.linear_1.weight"], w[prefix + "ff.linear_2.weight"],
                      w[prefix + "ff.out_projection.weight"], fp8)
@@ -511,8 +525,8 @@ def joint_block_mod(img, txt, mod_i, mod_t, w, prefix, heads, eps, key_mask=None
     v = np.concatenate([vt, vi], axis=2)
     o = merge_heads(attention(q, k, v, key_mask=key_mask))
     ot, oi = o[:, :nt], o[:, nt:]
-    img = img + mod_i["gate_msa"][:, None, :] * (_a8(oi, fp8) @ _w8(w[prefix + "attn.to_out.0.weight"], fp8).T)
-    txt = txt + mod_t["gate_msa"][:, None, :] * (_a8(ot, fp8) @ _w8(w[prefix + "attn.to_add_out.weight"], fp8).T)
+    img = img + mod_i["gate_msa"][:, None, :] * (_a8_stored(oi, fp8) @ _w8(w[prefix + "attn.to_out.0.weight"], fp8).T)
+    txt = txt + mod_t["gate_msa"][:, None, :] * (_a8_stored(ot, fp8) @ _w8(w[prefix + "attn.to_add_out.weight"], fp8).T)
     yi = modulate(img, mod_i["shift_mlp"], mod_i["scale_mlp"], eps)
     yt = modulate(txt, mod_t["shift_mlp"], mod_t["scale_mlp"], eps)
     img = img + mod_i["gate_mlp"][:, None, :] * feed_forward(

@@ -112,3 +112,20 @@ def test_fp8_forward_is_close_to_bf16_forward():
     assert np.array_equal(O.transformer_forward(lat, text, t, w, cfg, fp8=False), ref)
     err = O.rel_l2(O.transformer_forward(lat, text, t, w, cfg, fp8=True), ref)
     assert 1e-8 < err < 5e-2      # nonzero, yet small
+
+
+def test_round_bf16_matches_the_format():
+    # bf16 keeps the top 16 bits of the fp32 pattern; ties go to the even pattern
+    x = np.array([1.0, 1.0 + 2.0 ** -8, 1.0 + 2.0 ** -7, 1.0 + 3 * 2.0 ** -8, -2.5, 3.0e38, 1e-40])
+    got = O.round_bf16(x)
+    assert got[0] == 1.0
+    assert got[1] == 1.0                    # halfway between 1 and 1 + 2^-7: even (1.0)
+    assert got[2] == 1.0 + 2.0 ** -7        # representable
+    assert got[3] == 1.0 + 2.0 ** -6        # halfway between 1 + 2^-7 (odd) and 1 + 2^-6 (even)
+    assert got[4] == -2.5
+    # every value is a bf16 (low 16 bits of its fp32 pattern are zero)
+    bits = got.astype(np.float32).view(np.uint32)
+    assert np.all((bits & 0xFFFF) == 0)
+    r = np.random.default_rng(5).normal(size=1000)
+    g = O.round_bf16(r)
+    assert np.all(np.abs(g - r) <= 2.0 ** -8 * np.abs(r))
