@@ -360,9 +360,54 @@ __global__ void __launch_bounds__(256) quantize_rows_e4m3_kernel(const uint16_t*
   if (lane == 0) scale[row] = e4m3_scale(amax);
 }
 
+// Wide rows (K a multiple of 1024, up to 8192: the attention output and the
+// SwiGLU product): one CTA per row, each thread keeps 32 consecutive values
+// in registers, so the row is read from HBM once; the row maximum is reduced
+// across the CTA's warps through shared memory.
+__global__ void __launch_bounds__(256) quantize_wide_rows_e4m3_kernel(const uint16_t* __restrict__ x, int K,
+                                                                      uint8_t* __restrict__ q,
+                                                                      float* __restrict__ scale) {
+  __shared__ float wmax[8];
+  const size_t row = blockIdx.x;
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const uint4* xr = reinterpret_cast<const uint4*>(x + row * K) + 4 * t;
+  uint4 u[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) u[i] = xr[i];
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t w[4] = {u[i].x, u[i].y, u[i].z, u[i].w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(w[e])), fabsf(bf16_hi(w[e]))));
+  }
+  amax = warp_max(amax);
+  if (lane == 0) wmax[warp] = amax;
+  __syncthreads();
+  amax = wmax[0];
+  for (int i = 1; i < static_cast<int>(blockDim.x >> 5); ++i) amax = fmaxf(amax, wmax[i]);
+  const float inv = e4m3_inv_scale(amax);
+  uint32_t c[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    c[2 * i] = pack_e4m3x4(bf16_lo(u[i].x) * inv, bf16_hi(u[i].x) * inv, bf16_lo(u[i].y) * inv, bf16_hi(u[i].y) * inv);
+    c[2 * i + 1] =
+        pack_e4m3x4(bf16_lo(u[i].z) * inv, bf16_hi(u[i].z) * inv, bf16_lo(u[i].w) * inv, bf16_hi(u[i].w) * inv);
+  }
+  uint4* qr = reinterpret_cast<uint4*>(q + row * K) + 2 * t;
+  qr[0] = make_uint4(c[0], c[1], c[2], c[3]);
+  qr[1] = make_uint4(c[4], c[5], c[6], c[7]);
+  if (t == 0) scale[row] = e4m3_scale(amax);
+}
+
 cudaError_t launch_quantize_rows_e4m3(const uint16_t* x, int rows, int K, uint8_t* q, float* scale, cudaStream_t s) {
   if (rows <= 0) return cudaSuccess;
   if (K <= 0 || K % 8 != 0) return cudaErrorInvalidValue;
+  const bool aligned = ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(q)) & 15) == 0;
+  if (K % 1024 == 0 && K <= 8192 && aligned) {  // 32 values per thread, 1 to 8 warps
+    quantize_wide_rows_e4m3_kernel<<<rows, K / 32, 0, s>>>(x, K, q, scale);
+    return cudaGetLastError();
+  }
   quantize_rows_e4m3_kernel<<<(rows + 7) / 8, 256, 0, s>>>(x, rows, K, q, scale);
   return cudaGetLastError();
 }
