@@ -18,7 +18,7 @@ Prints one JSON line (rank 0).  Under torchrun every rank runs its own
 independent replica (weak scaling, no collective on the data path); the
 elapsed time is the max over ranks.  ``--impl reference`` times the fp64 CPU
 oracle on a bounded sample of the same workload.  ``--fp8`` times the 8-bit
-variant (e4m3 QKV and FFN up-projections), ``--direct`` the per-step entry
+variant (e4m3 operands for every block projection), ``--direct`` the per-step entry
 point without the plan.
 """
 from __future__ import annotations
@@ -61,7 +61,7 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--seed", type=int, default=4)
     ap.add_argument("--fp8", action="store_true",
-                    help="8-bit variant: e4m3 QKV and FFN up-projections (af_weights_quantize_fp8)")
+                    help="8-bit variant: e4m3 operands for every block projection (af_weights_quantize_fp8)")
     ap.add_argument("--direct", action="store_true",
                     help="time the per-step entry point (af_denoise_step) instead of the sampler plan")
     ap.add_argument("--case", default="step", choices=["step", "single_block"],

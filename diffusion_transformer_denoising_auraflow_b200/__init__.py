@@ -187,7 +187,7 @@ class Weights:
                f"af_weights_set({name})")
 
     def quantize_fp8(self, enable: bool = True, stream=None):
-        """Switch the QKV and FFN up-projections to the 8-bit (e4m3) variant
+        """Switch every block projection to the 8-bit (e4m3) variant
         (re-quantising the current weights), or back to bf16."""
         _check(lib.af_weights_quantize_fp8(self.handle, 1 if enable else 0, _stream(stream)),
                "af_weights_quantize_fp8")
