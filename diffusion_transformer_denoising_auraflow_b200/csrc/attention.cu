@@ -661,54 +661,76 @@ __global__ void __launch_bounds__(QKN_THREADS, 1)
 // attn_hd256_qknorm_pair: a cluster of two CTAs takes 256 query rows of one
 // (sample, head), 128 per CTA, and walks the keys in tiles of 128 with
 // tcgen05.mma.cta_group::2 issued by the leader CTA:
-//   S = Q K^T   M = 256, N = 128, K = 256: each CTA supplies its 128 Q rows
-//               and half of the K tile (64 keys); each CTA's TMEM receives
-//               its 128 x 128 block of S.
+//   S = Q K^T   M = 256, N = 128, K = 256: A (Q) is read from each CTA's
+//               TMEM (its 128 rows), B is half of the K tile (64 keys) from
+//               each CTA's shared memory; each CTA's TMEM receives its
+//               128 x 128 block of S.
 //   O += P V    M = 256, N = 256, K = 128: each CTA supplies its 128 rows of
-//               P and half of the V tile (128 head-dim columns); each CTA's
-//               TMEM accumulates its 128 x 256 block of O.
+//               P and half of the V tile (128 head-dim columns) from shared
+//               memory; each CTA's TMEM accumulates its 128 x 256 block of O.
 // Per SM that is 64 KB of K/V per 128 keys instead of 128 KB, and every MMA
-// has N >= 128 (full tensor-core rate).  TMEM per CTA: O [0, 256), S0
-// [256, 384), S1 [384, 512).  Shared memory per CTA: Q 64 KB, K and V halves
-// double-buffered (4 x 32 KB), one P buffer (128 x 128 bf16, 32 KB).
+// has N >= 128 (full tensor-core rate).  TMEM per CTA: O [0, 256), S
+// [256, 384), Q [384, 512).  Shared memory per CTA: two P buffers (128 x 128
+// bf16, 32 KB each), K and V halves double-buffered (4 x 32 KB).  The Q tile
+// lands in the two P buffers and the softmax warps move it to TMEM before
+// the first P is written; each thread copies exactly the rows of the P slots
+// it later overwrites, so no barrier separates the two uses.
+// With Q in TMEM the S products read only K from shared memory (a third of
+// the operand bytes per cycle), which leaves bandwidth for the softmax
+// warps' P stores; with two P buffers P_{j+1} is written while PV_j still
+// reads P_j, so the softmax of one tile no longer waits for the previous
+// tile's PV.
 // Softmax (fixed shift, as for attn_hd256_qknorm): warpgroup g of each CTA
 // owns keys [64 g, 64 g + 64) of every S tile; their partial row sums are
-// added at the end.  The leader issues S_0, S_1, then per tile PV_j followed
-// by S_{j+2}, so the tensor core computes the next scores while the softmax
-// warps publish P_{j+1}.  Barriers that gather both CTAs live in the leader
-// (TMA completions, S/P handshakes); commits are multicast to both CTAs.
-// The follower's softmax warps arrive directly on the leader's S/P barriers
-// (CTA-scope release; a cluster-scope release there costs ~1.2k cycles).
+// added at the end.  The leader issues S_{j+1} as soon as both CTAs' softmax
+// warps have read S_j out of TMEM, then PV_j once P_j is published, so the
+// tensor core computes the next scores while the softmax warps work.
+// Barriers that gather both CTAs live in the leader (TMA completions, S/P
+// handshakes); commits are multicast to both CTAs.  The follower's softmax
+// warps arrive directly on the leader's S/P barriers (CTA-scope release; a
+// cluster-scope release there costs ~1.2k cycles).
+// D (+)= A * B over the CTA pair with A in TMEM: each CTA's 128 rows of A are
+// read from its own TMEM at a_tmem (two consecutive K elements per 32-bit
+// column), B split along N between the two CTAs' shared memory.
+__device__ __forceinline__ void mma_bf16_ts_pair(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                                 uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 constexpr int AP_BN = 128;
-constexpr uint32_t AP_Q_BYTES = 128 * AT_HD * 2;      // 64 KB
 constexpr uint32_t AP_KH_BYTES = 64 * AT_HD * 2;      // 32 KB: 64 keys x 256
 constexpr uint32_t AP_VH_BYTES = AP_BN * 128 * 2;     // 32 KB: 128 keys x 128 columns
-constexpr uint32_t AP_P_BYTES = 128 * AP_BN * 2;      // 32 KB
-constexpr int AP_SMEM = AP_Q_BYTES + 2 * AP_KH_BYTES + 2 * AP_VH_BYTES + AP_P_BYTES + 2 * 128 * 4 + 256 + 1024;
+constexpr uint32_t AP_P_BYTES = 128 * AP_BN * 2;      // 32 KB (two of them hold the 64 KB Q tile first)
+constexpr int AP_SMEM = 2 * AP_P_BYTES + 2 * AP_KH_BYTES + 2 * AP_VH_BYTES + 2 * 128 * 4 + 256 + 1024;
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
     attn_hd256_qknorm_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                            const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;
-  uint8_t* sK = sQ + AP_Q_BYTES;          // 2 buffers
+  uint8_t* sP = smem;                     // 2 buffers; the Q tile first
+  uint8_t* sK = sP + 2 * AP_P_BYTES;      // 2 buffers
   uint8_t* sV = sK + 2 * AP_KH_BYTES;     // 2 buffers
-  uint8_t* sP = sV + 2 * AP_VH_BYTES;
-  float* xsum = reinterpret_cast<float*>(sP + AP_P_BYTES);  // [wg 2][row 128]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + AP_P_BYTES + 2 * 128 * 4);
-  uint64_t* q_full = bars + 0;     // leader: both CTAs' Q loads
+  float* xsum = reinterpret_cast<float*>(sV + 2 * AP_VH_BYTES);  // [wg 2][row 128]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + 2 * AP_VH_BYTES + 2 * 128 * 4);
+  uint64_t* q_smem = bars + 0;     // per CTA: this CTA's Q tile has landed
   uint64_t* k_full = bars + 1;     // [2] leader: both K halves
   uint64_t* v_full = bars + 3;     // [2] leader: both V halves
   uint64_t* k_empty = bars + 5;    // [2] both CTAs (multicast commit)
   uint64_t* v_empty = bars + 7;    // [2] both CTAs
-  uint64_t* s_full = bars + 9;     // [2] both CTAs
-  uint64_t* s_empty = bars + 11;   // [2] leader: 16 softmax warps of both CTAs
-  uint64_t* p_full = bars + 13;    // leader: 16 softmax warps of both CTAs
-  uint64_t* pv_done = bars + 14;   // both CTAs
-  uint64_t* mma_done = bars + 15;  // leader
-  uint64_t* lbar = bars + 16;      // per CTA: 8 softmax warps
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
+  uint64_t* s_full = bars + 9;     // both CTAs
+  uint64_t* s_empty = bars + 10;   // leader: 16 softmax warps of both CTAs
+  uint64_t* p_full = bars + 11;    // [2] leader: 16 softmax warps of both CTAs
+  uint64_t* pv_done = bars + 13;   // [2] both CTAs
+  uint64_t* q_tmem = bars + 15;    // leader: 16 softmax warps have moved Q to TMEM
+  uint64_t* mma_done = bars + 16;  // leader
+  uint64_t* lbar = bars + 17;      // per CTA: 8 softmax warps
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -724,17 +746,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
   auto kv_tile = [&](int j) { const int t = j + kv0; return t < nkv ? t : t - nkv; };
 
   if (threadIdx.x == 0) {
-    mbar_init(smem_u32(q_full), 1);
+    mbar_init(smem_u32(q_smem), 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&k_full[i]), 1);
       mbar_init(smem_u32(&v_full[i]), 1);
       mbar_init(smem_u32(&k_empty[i]), 1);
       mbar_init(smem_u32(&v_empty[i]), 1);
-      mbar_init(smem_u32(&s_full[i]), 1);
-      mbar_init(smem_u32(&s_empty[i]), 2 * AT_SOFTMAX_WARPS);
+      mbar_init(smem_u32(&p_full[i]), 2 * AT_SOFTMAX_WARPS);
+      mbar_init(smem_u32(&pv_done[i]), 1);
     }
-    mbar_init(smem_u32(p_full), 2 * AT_SOFTMAX_WARPS);
-    mbar_init(smem_u32(pv_done), 1);
+    mbar_init(smem_u32(s_full), 1);
+    mbar_init(smem_u32(s_empty), 2 * AT_SOFTMAX_WARPS);
+    mbar_init(smem_u32(q_tmem), 2 * AT_SOFTMAX_WARPS);
     mbar_init(smem_u32(mma_done), 1);
     mbar_init(smem_u32(lbar), AT_SOFTMAX_WARPS);
     *abort_flag = 0;
@@ -756,11 +779,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
   const uint32_t tmem = *tmem_slot;
   const uint32_t tO = tmem;
   const uint32_t tS = tmem + 256;
+  const uint32_t tQ = tmem + 384;
   volatile int never = 0;
 
   if (warp == 0 || warp == AT_V_WARP) {
-    // warp 0: Q then the K halves (keys [64 rank, +64) of each tile);
-    // last warp: the V halves (head-dim columns [128 rank, +128)).
+    // warp 0: this CTA's Q tile, then the K halves (keys [64 rank, +64) of
+    // each tile); last warp: the V halves (head-dim columns [128 rank, +128)).
     if (lane == 0) {
       const bool is_k = warp == 0;
       uint64_t* full = is_k ? k_full : v_full;
@@ -769,10 +793,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
       uint8_t* buf = is_k ? sK : sV;
       bool ok = true, issued = false;
       if (is_k) {
-        const uint32_t qb = mapa_shared(smem_u32(q_full), 0);
-        if (leader) mbar_arrive_expect_tx(smem_u32(q_full), 2 * AP_Q_BYTES);
+        mbar_arrive_expect_tx(smem_u32(q_smem), 2 * AP_P_BYTES);
         for (int c = 0; c < 4; ++c)
-          tma_load_3d_pair(smem_u32(sQ + c * (128 * 128)), &tmQ, qb, c * 64, q0, bh);
+          tma_load_3d(smem_u32(sP + c * (128 * 128)), &tmQ, smem_u32(q_smem), c * 64, q0, bh);
         issued = true;
       }
       for (int j = 0; j < nkv; ++j) {
@@ -803,45 +826,44 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
     if (lane == 0 && leader) {
       const uint32_t idesc_qk = make_idesc_bf16(256, AP_BN, false, false);
       const uint32_t idesc_pv = make_idesc_bf16(256, AT_HD, false, true);
-      const uint32_t qaddr = smem_u32(sQ);
-      const uint32_t paddr = smem_u32(sP);
-      bool ok = mbar_wait(smem_u32(q_full), 0, p.err, abort_flag);
+      bool ok = mbar_wait(smem_u32(q_tmem), 0, p.err, abort_flag);
+      // S_j into the single S buffer: the K half of tile j has landed and the
+      // softmax warps of both CTAs have read S_{j-1}.
       auto issue_s = [&](int j) -> bool {
         const int s = j & 1;
-        const uint32_t ph = (j >> 1) & 1;
-        if (!mbar_wait(smem_u32(&k_full[s]), ph, p.err, abort_flag)) return false;
-        if (!mbar_wait(smem_u32(&s_empty[s]), ph ^ 1u, p.err, abort_flag)) return false;
+        if (!mbar_wait(smem_u32(&k_full[s]), (j >> 1) & 1, p.err, abort_flag)) return false;
+        if (j > 0 && !mbar_wait(smem_u32(s_empty), (j - 1) & 1, p.err, abort_flag)) return false;
         tc_fence_after();
         const uint32_t kaddr = smem_u32(sK + s * AP_KH_BYTES);
+        const uint64_t kdesc = make_sdesc(kaddr, 16, 1024, SWZ_128B);
 #pragma unroll
         for (int kk = 0; kk < AT_HD / 16; ++kk) {
           const uint32_t c = kk >> 2, off = (kk & 3) * 32;
-          const uint64_t ad = make_sdesc(qaddr, 16, 1024, SWZ_128B) + static_cast<uint64_t>((c * (128 * 128) + off) >> 4);
-          const uint64_t bd = make_sdesc(kaddr, 16, 1024, SWZ_128B) + static_cast<uint64_t>((c * (64 * 128) + off) >> 4);
-          mma_bf16_ss_pair(tS + s * AP_BN, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
+          const uint64_t bd = kdesc + static_cast<uint64_t>((c * (64 * 128) + off) >> 4);
+          mma_bf16_ts_pair(tS, tQ + kk * 8, bd, idesc_qk, kk > 0 ? 1u : 0u);
         }
-        mma_commit_pair(smem_u32(&s_full[s]), 0x3);
+        mma_commit_pair(smem_u32(s_full), 0x3);
         mma_commit_pair(smem_u32(&k_empty[s]), 0x3);
         return true;
       };
       if (ok) ok = issue_s(0);
-      if (ok && nkv > 1) ok = issue_s(1);
       for (int j = 0; j < nkv && ok; ++j) {
         const int s = j & 1;
-        if (!mbar_wait(smem_u32(p_full), j & 1, p.err, abort_flag)) { ok = false; break; }
+        if (j + 1 < nkv && !issue_s(j + 1)) { ok = false; break; }
+        if (!mbar_wait(smem_u32(&p_full[s]), (j >> 1) & 1, p.err, abort_flag)) { ok = false; break; }
         if (!mbar_wait(smem_u32(&v_full[s]), (j >> 1) & 1, p.err, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t vaddr = smem_u32(sV + s * AP_VH_BYTES);
+        const uint64_t pdesc = make_sdesc(smem_u32(sP + s * AP_P_BYTES), 16, 1024, SWZ_128B);
+        const uint64_t vdesc = make_sdesc(smem_u32(sV + s * AP_VH_BYTES), AP_BN * 128, 1024, SWZ_128B);
 #pragma unroll
         for (int kk = 0; kk < AP_BN / 16; ++kk) {
           const uint32_t c = kk >> 2, off = (kk & 3) * 32;
-          const uint64_t ad = make_sdesc(paddr, 16, 1024, SWZ_128B) + static_cast<uint64_t>((c * (128 * 128) + off) >> 4);
-          const uint64_t bd = make_sdesc(vaddr, AP_BN * 128, 1024, SWZ_128B) + static_cast<uint64_t>((kk * (16 * 128)) >> 4);
+          const uint64_t ad = pdesc + static_cast<uint64_t>((c * (128 * 128) + off) >> 4);
+          const uint64_t bd = vdesc + static_cast<uint64_t>((kk * (16 * 128)) >> 4);
           mma_bf16_ss_pair(tO, ad, bd, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
         }
-        mma_commit_pair(smem_u32(pv_done), 0x3);
+        mma_commit_pair(smem_u32(&pv_done[s]), 0x3);
         mma_commit_pair(smem_u32(&v_empty[s]), 0x3);
-        if (j + 2 < nkv && !issue_s(j + 2)) { ok = false; break; }
       }
       mma_commit_pair(smem_u32(mma_done), 0x1);
       mbar_wait(smem_u32(mma_done), 0, nullptr, &never, 100000000ull);
@@ -860,20 +882,47 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
     const uint32_t p_full_l = mapa_shared(smem_u32(p_full), 0);
     float l = 0.f;
     bool ok = true;
-    uint8_t* prow = sP + wg * (128 * 128) + row * 128;
-    for (int j = 0; j < nkv; ++j) {
+    {
+      // This thread's Q row, 64-column chunks wg and wg + 2 (the P slots
+      // (buffer 0, group wg) and (buffer 1, group wg) that it overwrites
+      // later), from shared memory into TMEM columns [32 chunk, +32).
+      const bool got = mbar_wait(smem_u32(q_smem), 0, p.err, abort_flag);
+      __syncwarp();
+      if (!__all_sync(0xffffffffu, got)) {
+        ok = false;
+      } else {
+        for (int cc = wg; cc < 4; cc += 2) {
+          const uint8_t* qrow = sP + cc * (128 * 128) + row * 128;
+          uint32_t qv[32];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const uint4 u = *reinterpret_cast<const uint4*>(qrow + ((q ^ (row & 7)) << 4));
+            qv[4 * q] = u.x;
+            qv[4 * q + 1] = u.y;
+            qv[4 * q + 2] = u.z;
+            qv[4 * q + 3] = u.w;
+          }
+          tmem_st32(tQ + cc * 32 + lane_off, qv);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(q_tmem), 0));
+      }
+    }
+    for (int j = 0; j < nkv && ok; ++j) {
       const int s = j & 1;
-      const bool got = mbar_wait(smem_u32(&s_full[s]), (j >> 1) & 1, p.err, abort_flag);
+      const bool got = mbar_wait(smem_u32(s_full), j & 1, p.err, abort_flag);
       __syncwarp();
       if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
       tc_fence_after();
       uint32_t r0[32], r1[32];
-      tmem_ld32(tS + s * AP_BN + 64 * wg + lane_off, r0);
-      tmem_ld32(tS + s * AP_BN + 64 * wg + 32 + lane_off, r1);
+      tmem_ld32(tS + 64 * wg + lane_off, r0);
+      tmem_ld32(tS + 64 * wg + 32 + lane_off, r1);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(s_empty_l + s * 8);
+      if (lane == 0) mbar_arrive_cluster(s_empty_l);
       const int kbase = kv_tile(j) * AP_BN + 64 * wg;
       const int kvalid = p.N - kbase, mlo = klo - kbase, mhi = khi - kbase;
       const bool partial = kvalid < 64 || (mlo < mhi && mlo < 64 && mhi > 0);
@@ -897,12 +946,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
         pk[16 + i] = pack_bf16(e2, e3);
       }
       l += rs;
-      // the P buffer is free once PV_{j-1} has completed
-      if (j >= 1) {
-        const bool g2 = mbar_wait(smem_u32(pv_done), (j - 1) & 1, p.err, abort_flag);
+      // P buffer s is free once PV_{j-2} has completed
+      if (j >= 2) {
+        const bool g2 = mbar_wait(smem_u32(&pv_done[s]), ((j - 2) >> 1) & 1, p.err, abort_flag);
         __syncwarp();
         if (!__all_sync(0xffffffffu, g2)) { ok = false; break; }
       }
+      uint8_t* prow = sP + s * AP_P_BYTES + wg * (128 * 128) + row * 128;
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
         uint4 v = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
@@ -911,14 +961,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(p_full_l);
+      if (lane == 0) mbar_arrive_cluster(p_full_l + s * 8);
     }
     if (ok) {
       xsum[wg * 128 + row] = l;
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(lbar));
+      const int jl = nkv - 1;
       const bool g3 = mbar_wait(smem_u32(lbar), 0, p.err, abort_flag) &&
-                      mbar_wait(smem_u32(pv_done), (nkv - 1) & 1, p.err, abort_flag);
+                      mbar_wait(smem_u32(&pv_done[jl & 1]), (jl >> 1) & 1, p.err, abort_flag);
       __syncwarp();
       if (__all_sync(0xffffffffu, g3)) {
         tc_fence_after();
