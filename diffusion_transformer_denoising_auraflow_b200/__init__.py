@@ -150,6 +150,45 @@ def _dev(t: torch.Tensor, dtype, name: str):
     return ctypes.c_void_p(t.data_ptr())
 
 
+AF_ERR_SHAPE = 2
+
+
+def _need(ok: bool, where: str, detail: str):
+    """The library sees raw pointers only: a buffer whose size does not match
+    the call is reported here, as the library reports its own shape errors,
+    before anything is launched."""
+    if not ok:
+        raise AFError(AF_ERR_SHAPE, where, detail)
+
+
+def _need_shape(t, shape, name: str, where: str):
+    got = tuple(t.shape)
+    _need(got == tuple(shape), where, f"{name} must have shape {tuple(shape)}, got {got}")
+
+
+def _elems_from_start(t) -> int:
+    """Elements of t's storage from t's first element on (a view may reach
+    past its own shape into the storage it was cut from)."""
+    return t.untyped_storage().nbytes() // t.element_size() - t.storage_offset()
+
+
+def _dev_rows(t, dtype, name: str, rows: int, row_stride: int, row_len: int, where: str):
+    """A CUDA tensor or strided view read as `rows` rows of `row_len`
+    elements, `row_stride` elements apart, from its first element."""
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    need = (rows - 1) * row_stride + row_len if rows > 0 else 0
+    avail = _elems_from_start(t)
+    _need(need <= avail, where, f"{name} holds {avail} elements from its start, the call reads {need}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _width(w) -> int:
+    return w.cfg.derived()[0]
+
+
 class Weights:
     """Device-resident bf16 weight pack (af_weights)."""
 
@@ -182,7 +221,17 @@ class Weights:
         """Copy a bf16 tensor (host or device, contiguous, listed numel) into the pack."""
         if tensor.dtype != torch.bfloat16 or not tensor.is_contiguous():
             raise TypeError("weights must be contiguous bfloat16")
-        _check(lib.af_weights_set(self.handle, self.find(name), ctypes.c_void_p(tensor.data_ptr()),
+        idx = self.find(name)
+        buf = ctypes.create_string_buffer(256)
+        nd = ctypes.c_int()
+        shp = (ctypes.c_int64 * 2)()
+        _check(lib.af_weights_tensor_info(self.handle, idx, buf, 256, ctypes.byref(nd), shp), "af_weights_tensor_info")
+        numel = 1
+        for d in shp[: nd.value]:
+            numel *= d
+        _need(tensor.numel() == numel, f"af_weights_set({name})",
+              f"the pack holds {numel} elements, the tensor {tensor.numel()}")
+        _check(lib.af_weights_set(self.handle, idx, ctypes.c_void_p(tensor.data_ptr()),
                                   1 if tensor.is_cuda else 0, _stream(stream) if tensor.is_cuda else None),
                f"af_weights_set({name})")
 
@@ -252,12 +301,14 @@ class Scratch:
 
 
 def timestep_embed(w: Weights, s: Scratch, t, temb, stream=None):
+    _need_shape(temb, (t.numel(), _width(w)), "temb", "af_timestep_embed")
     _check(lib.af_timestep_embed(w.handle, s.handle, _dev(t, torch.float32, "t"), t.numel(),
                                  _dev(temb, torch.float32, "temb"), _stream(stream)), "af_timestep_embed")
 
 
 def timestep_embed_noalloc(w: Weights, t, temb, stream=None):
     """af_timestep_embed without a scratch handle: nothing is allocated (fixed device array)."""
+    _need_shape(temb, (t.numel(), _width(w)), "temb", "af_timestep_embed_noalloc")
     st = lib.af_timestep_embed_noalloc(w.handle, _dev(t, torch.float32, "t"), t.numel(),
                                        _dev(temb, torch.float32, "temb"), _stream(stream))
     if st != AF_OK:
@@ -266,14 +317,22 @@ def timestep_embed_noalloc(w: Weights, t, temb, stream=None):
 
 def patch_embed(w: Weights, s: Scratch, latents, img, stream=None):
     B, C, H, W = latents.shape
+    p = w.cfg.patch_size
+    _need(C == w.cfg.in_channels, "af_patch_embed", f"latents must have {w.cfg.in_channels} channels, got {C}")
+    if H % p == 0 and W % p == 0:   # otherwise the library rejects the latent size itself
+        _need_shape(img, (B, (H // p) * (W // p), _width(w)), "img", "af_patch_embed")
     _check(lib.af_patch_embed(w.handle, s.handle, _dev(latents, torch.float32, "latents"), B, H, W,
                               _dev(img, torch.bfloat16, "img"), _stream(stream)), "af_patch_embed")
 
 
 def joint_block(w: Weights, s: Scratch, layer: int, img, txt, temb, text_len=None, stream=None):
     """text_len: optional CUDA int32 [B], real prompt tokens (padded prompts)."""
-    B, Ni, _ = img.shape
+    B, Ni = img.shape[:2]
     Nt = txt.shape[1]
+    D = _width(w)
+    _need_shape(img, (B, Ni, D), "img", "af_joint_block")
+    _need_shape(txt, (B, Nt, D), "txt", "af_joint_block")
+    _need_shape(temb, (B, D), "temb", "af_joint_block")
     _check(lib.af_joint_block(w.handle, s.handle, layer, _dev(img, torch.bfloat16, "img"),
                               _dev(txt, torch.bfloat16, "txt"), _dev(temb, torch.float32, "temb"),
                               B, Ni, Nt, _lens(text_len, B, "text_len"), _stream(stream)), "af_joint_block")
@@ -281,7 +340,10 @@ def joint_block(w: Weights, s: Scratch, layer: int, img, txt, temb, text_len=Non
 
 def single_block(w: Weights, s: Scratch, layer: int, x, temb, n_text: int = 0, text_len=None, stream=None):
     """x = [text; image] per sample; with text_len the first n_text rows are the text stream."""
-    B, N, _ = x.shape
+    B, N = x.shape[:2]
+    D = _width(w)
+    _need_shape(x, (B, N, D), "x", "af_single_block")
+    _need_shape(temb, (B, D), "temb", "af_single_block")
     _check(lib.af_single_block(w.handle, s.handle, layer, _dev(x, torch.bfloat16, "x"),
                                _dev(temb, torch.float32, "temb"), B, N, int(n_text), _lens(text_len, B, "text_len"),
                                _stream(stream)), "af_single_block")
@@ -290,6 +352,11 @@ def single_block(w: Weights, s: Scratch, layer: int, x, temb, n_text: int = 0, t
 def transformer_forward(w: Weights, s: Scratch, latents, text_emb, t, velocity, text_len=None, stream=None):
     B, C, H, W = latents.shape
     L = text_emb.shape[1]
+    where = "af_transformer_forward"
+    _need(C == w.cfg.in_channels, where, f"latents must have {w.cfg.in_channels} channels, got {C}")
+    _need_shape(text_emb, (B, L, w.cfg.joint_attention_dim), "text_emb", where)
+    _need(t.numel() == B, where, f"t must hold {B} values, got {t.numel()}")
+    _need_shape(velocity, (B, w.cfg.out_channels, H, W), "velocity", where)
     _check(lib.af_transformer_forward(w.handle, s.handle, _dev(latents, torch.float32, "latents"),
                                       _dev(text_emb, torch.bfloat16, "text_emb"), _dev(t, torch.float32, "t"),
                                       B, H, W, L, _lens(text_len, B, "text_len"),
@@ -313,6 +380,8 @@ def denoise_step(w: Weights, s: Scratch, latents, text_emb, guidance: float, sig
     if text_emb.shape[0] != 2 * Bi:
         raise ValueError("text_emb must hold 2*Bi rows (uncond first)")
     L = text_emb.shape[1]
+    _need(C == w.cfg.in_channels, "af_denoise_step", f"latents must have {w.cfg.in_channels} channels, got {C}")
+    _need_shape(text_emb, (2 * Bi, L, w.cfg.joint_attention_dim), "text_emb", "af_denoise_step")
     _check(lib.af_denoise_step(w.handle, s.handle, _dev(latents, torch.float32, "latents"),
                                _dev(text_emb, torch.bfloat16, "text_emb"), Bi, H, W, L,
                                _lens(text_len, 2 * Bi, "text_len"), float(guidance), float(sigma),
@@ -329,6 +398,8 @@ class Sampler:
         L = text_emb.shape[1]
         if text_emb.shape[0] != 2 * Bi:
             raise ValueError("text_emb must hold 2*Bi rows (uncond first)")
+        _need(C == w.cfg.in_channels, "af_sampler_create", f"latents must have {w.cfg.in_channels} channels, got {C}")
+        _need_shape(text_emb, (2 * Bi, L, w.cfg.joint_attention_dim), "text_emb", "af_sampler_create")
         self.n_steps = len(sigmas) - 1
         sig = (ctypes.c_float * len(sigmas))(*[float(x) for x in sigmas])
         h = ctypes.c_void_p()
@@ -366,14 +437,19 @@ def sigma_schedule(n_steps: int, shift: float = 1.73, num_train_timesteps: int =
 
 def ln_modulate(x, shift, scale, mod_stride: int, y, eps: float, stream=None):
     B, N, D = x.shape
-    _check(lib.af_ln_modulate(_dev(x, torch.bfloat16, "x"), ctypes.c_void_p(shift.data_ptr()),
-                              ctypes.c_void_p(scale.data_ptr()), mod_stride, _dev(y, torch.bfloat16, "y"),
+    where = "af_ln_modulate"
+    _need_shape(y, (B, N, D), "y", where)
+    sh = _dev_rows(shift, torch.float32, "shift", B, mod_stride, D, where)
+    sc = _dev_rows(scale, torch.float32, "scale", B, mod_stride, D, where)
+    _check(lib.af_ln_modulate(_dev(x, torch.bfloat16, "x"), sh, sc, mod_stride, _dev(y, torch.bfloat16, "y"),
                               B, N, D, float(eps), _stream(stream)), "af_ln_modulate")
 
 
 def linear(A, W, C, stream=None):
     M, K = A.shape
     N = W.shape[0]
+    _need_shape(W, (N, K), "W", "af_linear")
+    _need_shape(C, (M, N), "C", "af_linear")
     _check(lib.af_linear(_dev(A, torch.bfloat16, "A"), _dev(W, torch.bfloat16, "W"), _dev(C, torch.bfloat16, "C"),
                          M, N, K, _stream(stream)), "af_linear")
 
@@ -382,6 +458,9 @@ def attention(q, k, v, o, qk_normalized: bool = False, key_len=None, key_base: i
               stream=None):
     """key_len: optional CUDA int32 [B]; keys [key_base + key_len[b], key_end) of sample b are masked."""
     B, H, N, hd = q.shape
+    _need_shape(k, (B, H, N, hd), "k", "af_attention")
+    _need_shape(v, (B, H, N, hd), "v", "af_attention")
+    _need_shape(o, (B, N, H * hd), "o", "af_attention")
     _check(lib.af_attention(_dev(q, torch.bfloat16, "q"), _dev(k, torch.bfloat16, "k"), _dev(v, torch.bfloat16, "v"),
                             _dev(o, torch.bfloat16, "o"), B, H, N, hd, 1 if qk_normalized else 0,
                             _lens(key_len, B, "key_len"), int(key_base), int(key_end), _stream(stream)),
@@ -391,14 +470,20 @@ def attention(q, k, v, o, qk_normalized: bool = False, key_len=None, key_base: i
 def quantize_rows_e4m3(x, q, scale, stream=None):
     """Per-row e4m3 codes of bf16 x [rows, cols] into uint8 q and float scale [rows]."""
     rows, cols = x.shape
+    _need_shape(q, (rows, cols), "q", "af_quantize_rows_e4m3")
+    _need(scale.numel() >= rows, "af_quantize_rows_e4m3", f"scale must hold {rows} values, got {scale.numel()}")
     _check(lib.af_quantize_rows_e4m3(_dev(x, torch.bfloat16, "x"), rows, cols, _dev(q, torch.uint8, "q"),
                                      _dev(scale, torch.float32, "scale"), _stream(stream)), "af_quantize_rows_e4m3")
 
 
 def ln_modulate_e4m3(x, shift, scale, mod_stride: int, y8, yscale, eps: float, stream=None):
     B, N, D = x.shape
-    _check(lib.af_ln_modulate_e4m3(_dev(x, torch.bfloat16, "x"), ctypes.c_void_p(shift.data_ptr()),
-                                   ctypes.c_void_p(scale.data_ptr()), mod_stride, _dev(y8, torch.uint8, "y8"),
+    where = "af_ln_modulate_e4m3"
+    _need(y8.numel() == B * N * D, where, f"y8 must hold {B * N * D} codes, got {y8.numel()}")
+    _need(yscale.numel() >= B * N, where, f"yscale must hold {B * N} values, got {yscale.numel()}")
+    sh = _dev_rows(shift, torch.float32, "shift", B, mod_stride, D, where)
+    sc = _dev_rows(scale, torch.float32, "scale", B, mod_stride, D, where)
+    _check(lib.af_ln_modulate_e4m3(_dev(x, torch.bfloat16, "x"), sh, sc, mod_stride, _dev(y8, torch.uint8, "y8"),
                                    _dev(yscale, torch.float32, "yscale"), B, N, D, float(eps), _stream(stream)),
            "af_ln_modulate_e4m3")
 
@@ -409,6 +494,9 @@ def linear_fp8(A8, a_scale, W8, w_scale, C, stream=None):
     N = W8.shape[0]
     if w_scale.numel() < (N + 255) // 256 * 256:
         raise ValueError("w_scale must hold ceil(N / 256) * 256 entries")
+    _need_shape(W8, (N, K), "W8", "af_linear_fp8")
+    _need_shape(C, (M, N), "C", "af_linear_fp8")
+    _need(a_scale.numel() >= M, "af_linear_fp8", f"a_scale must hold {M} values, got {a_scale.numel()}")
     _check(lib.af_linear_fp8(_dev(A8, torch.uint8, "A8"), _dev(a_scale, torch.float32, "a_scale"),
                              _dev(W8, torch.uint8, "W8"), _dev(w_scale, torch.float32, "w_scale"),
                              _dev(C, torch.bfloat16, "C"), M, N, K, _stream(stream)), "af_linear_fp8")
