@@ -337,13 +337,20 @@ def attention(q, k, v, scale=None, key_mask=None):
     q, k, v = _f(q), _f(k), _f(v)
     if scale is None:
         scale = 1.0 / math.sqrt(q.shape[-1])
-    s = (q @ np.swapaxes(k, -1, -2)) * scale
-    if key_mask is not None:
-        s = np.where(np.asarray(key_mask, bool)[:, None, None, :], s, -np.inf)
-    s = s - s.max(axis=-1, keepdims=True)
-    p = np.exp(s)
-    p = p / p.sum(axis=-1, keepdims=True)
-    return p @ v
+    B, H = q.shape[0], q.shape[1]
+    out = np.empty(q.shape[:-1] + (v.shape[-1],), dtype=F64)
+    # one (sample, head) at a time: the softmax of each is independent, and
+    # the N x N logits of one head stay small enough for the 9480-token workload
+    for b in range(B):
+        for h in range(H):
+            s = (q[b, h] @ k[b, h].T) * scale
+            if key_mask is not None:
+                s = np.where(np.asarray(key_mask, bool)[b][None, :], s, -np.inf)
+            s = s - s.max(axis=-1, keepdims=True)
+            p = np.exp(s)
+            p = p / p.sum(axis=-1, keepdims=True)
+            out[b, h] = p @ v[b, h]
+    return out
 
 
 def text_key_mask(text_len, n_registers: int, L: int, n_image: int):
