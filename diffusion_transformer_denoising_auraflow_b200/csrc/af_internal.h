@@ -103,6 +103,36 @@ cudaError_t attention_set_attributes();
 cudaError_t small_kernels_set_attributes();
 cudaError_t launch_euler_cfg(float* lat, const float* v, int Bi, int64_t per_sample, float g, float sigma,
                              float sigma_next, cudaStream_t s);
+cudaError_t launch_timestep_features(const float* t, int B, int C, float* feat, cudaStream_t s);
+
+// Weight-pack filling (init.cu).  interleave: 0 plain, 1 / 2 = linear_1 /
+// linear_2 rows of an FFN up pair stored in alternating 128-row groups.
+uint32_t crc32_ieee(const char* s);
+cudaError_t launch_init_normal(void* dst, bool f32, size_t numel, int cols, int interleave, uint32_t key,
+                               uint64_t seed, float stdv, cudaStream_t s);
+cudaError_t launch_convert_copy(const void* src, bool src_f32, void* dst, bool dst_f32, size_t numel, int cols,
+                                int interleave, cudaStream_t s);
+
+// The fp32 forward's kernels (fp32.cu).  mode: EPI_STORE (rows remapped per
+// sample) or EPI_GATE_RES (out[m, n] += gate[b, n] * acc).
+cudaError_t f32_gemm(const float* A, const float* W, int M, int N, int K, int mode, float* out, int ldo,
+                     int rows_per_batch, int out_rows_per_batch, int out_row_off, const float* gate, int gate_stride,
+                     cudaStream_t s);
+cudaError_t f32_ln_modulate(const float* x, const float* shift, const float* scale, int mod_stride, float* y,
+                            int rows, int rows_per_batch, int D, float eps, cudaStream_t s);
+cudaError_t f32_qkv_split(const float* t, int M, int rows_per_batch, int heads, int hd, float eps, float* q, float* k,
+                          float* v, int n_total, int row_off, cudaStream_t s);
+cudaError_t f32_swiglu(const float* t, int M, int F, float* h, cudaStream_t s);
+cudaError_t f32_attention(const float* q, const float* k, const float* v, int B, int H, int N, int hd, float scale,
+                          float* out_a, float* out_b, int split, int ldo, const int* key_len, int key_base,
+                          int key_end, cudaStream_t s);
+cudaError_t f32_gemv(const float* x, int B, int K, const float* W, const float* bias, int rows, int pre, int post,
+                     float* out, int out_stride, cudaStream_t s);
+cudaError_t f32_patch_embed(const float* lat, int B, int C, int H, int W, int p, const float* w_pe, const float* pos,
+                            int G, int D, float* out, cudaStream_t s);
+cudaError_t f32_output_stage(const float* x, int rows_per_batch, int row_off, int B, int hp, int wp, int D,
+                             const float* scale, const float* shift, int mod_stride, const float* w_out, int p, int C,
+                             float* vel, cudaStream_t s);
 
 }  // namespace af
 
@@ -114,5 +144,6 @@ const uint16_t* weights_tensor(const af_weights* w, const char* name);
 int weights_device(const af_weights* w);
 int weights_inner_dim(const af_weights* w);
 int weights_timestep_channels(const af_weights* w);
+bool weights_is_f32(const af_weights* w);
 void set_last_error(const std::string& msg);
 }  // namespace af

@@ -81,6 +81,8 @@ struct af_weights {
   af_config cfg;
   Derived d;
   int device;
+  bool f32 = false;  // AF_DTYPE_F32 pack: fp32 tensors, fp32 forward (fp32.cu)
+  size_t esz = 2;    // bytes per stored element
   uint8_t* base = nullptr;
   size_t bytes = 0;
   std::vector<TensorInfo> tensors;
@@ -106,6 +108,7 @@ struct af_weights {
     auto it = index.find(n);
     return it == index.end() ? nullptr : reinterpret_cast<const uint16_t*>(base + tensors[it->second].offset);
   }
+  const float* ptrf(const std::string& n) const { return reinterpret_cast<const float*>(ptr(n)); }
 };
 
 struct af_scratch {
@@ -119,7 +122,8 @@ struct af_scratch {
   uint16_t *y, *q, *k, *v, *o, *h;
   uint8_t* y8;    // 8-bit variant: e4m3 codes of y, one fp32 scale per row in yscale
   float* yscale;
-  uint16_t *img, *txt, *x;
+  uint16_t *img, *txt, *x;   // (fp32 pack: these activation buffers hold floats)
+  float* tmp;                // fp32 pack: GEMM outputs before QK-norm / SwiGLU, [B*N, max(3D, 2F)]
   float *lat2, *vel, *tvec;  // denoise step: CFG-duplicated latents, velocity, model times
   int sms;
   // launch accounting / profiling (kernel classes: GEMM, attention, LN, other)
@@ -148,7 +152,7 @@ void add_tensor(af_weights* w, size_t& off, const std::string& name, int64_t r, 
   t.offset = off;
   w->index[name] = static_cast<int>(w->tensors.size());
   w->tensors.push_back(t);
-  off += t.numel() * 2;
+  off += t.numel() * w->esz;
 }
 
 void mark_pair(af_weights* w, const std::string& w1, const std::string& w2) {
@@ -202,8 +206,10 @@ void build_layout(af_weights* w) {
     add_tensor(w, off, b + "ff_context.linear_1.weight", F, D);
     add_tensor(w, off, b + "ff_context.linear_2.weight", F, D, false);
     add_tensor(w, off, b + "ff_context.out_projection.weight", D, F);
-    mark_pair(w, b + "ff.linear_1.weight", b + "ff.linear_2.weight");
-    mark_pair(w, b + "ff_context.linear_1.weight", b + "ff_context.linear_2.weight");
+    if (!w->f32) {  // the fp32 forward multiplies by [linear_1; linear_2] as stored
+      mark_pair(w, b + "ff.linear_1.weight", b + "ff.linear_2.weight");
+      mark_pair(w, b + "ff_context.linear_1.weight", b + "ff_context.linear_2.weight");
+    }
   }
   for (int i = 0; i < c.num_single_dit_layers; ++i) {
     const std::string b = "single_transformer_blocks." + std::to_string(i) + ".";
@@ -214,7 +220,7 @@ void build_layout(af_weights* w) {
     add_tensor(w, off, b + "ff.linear_1.weight", F, D);
     add_tensor(w, off, b + "ff.linear_2.weight", F, D, false);
     add_tensor(w, off, b + "ff.out_projection.weight", D, F);
-    mark_pair(w, b + "ff.linear_1.weight", b + "ff.linear_2.weight");
+    if (!w->f32) mark_pair(w, b + "ff.linear_1.weight", b + "ff.linear_2.weight");
   }
   add_tensor(w, off, "pos_embed.proj.weight", D, p * p * c.in_channels);
   add_tensor(w, off, "pos_embed.pos_embed", c.pos_embed_max_size, D);
@@ -232,9 +238,24 @@ const uint16_t* ada_base(const af_weights* w) {
   return reinterpret_cast<const uint16_t*>(w->base + w->tensors[0].offset);
 }
 
+// Kernels launch on the current device, so it must be the pack's.
+af_status check_device(const af_weights* w) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    g_last_error = cudaGetErrorString(cudaGetLastError());
+    return AF_ERR_CUDA;
+  }
+  if (dev != w->device) {
+    g_last_error = "the current device (" + std::to_string(dev) + ") is not the weight pack's device (" +
+                   std::to_string(w->device) + ")";
+    return AF_ERR_INVALID_ARG;
+  }
+  return AF_OK;
+}
+
 af_status check_scratch(const af_weights* w, af_scratch* s) {
   if (!w || !s || s->w != w) return AF_ERR_INVALID_ARG;
-  return AF_OK;
+  return check_device(w);
 }
 
 enum { KC_GEMM = 0, KC_ATTN = 1, KC_LN = 2, KC_OTHER = 3 };
@@ -519,11 +540,177 @@ af_status check_dev_ptr(const void* p) {
 
 }  // namespace
 
+// ------------------------------------------------------------ the fp32 forward
+// Same sequence as forward_impl ([ARCH] §前向传播流程, §联合注意力块, §单 DiT 块)
+// on an fp32 pack, every step in fp32 (fp32.cu).  Activation buffers of the
+// scratch hold floats; s->tmp holds the [rows, 3D] QKV and [rows, 2F] FFN-up
+// products before the QK-norm split and the SwiGLU.
+namespace {
+
+struct F32Step {
+  af_scratch* s;
+  cudaStream_t st;
+};
+
+af_status f32_done(cudaError_t e) { return e == cudaSuccess ? AF_OK : cuda_fail(e); }
+
+af_status f32_gemm_op(F32Step& k, const float* A, const float* W, int M, int N, int K, int mode, float* out, int ldo,
+                      int rows_per_batch, int out_rows_per_batch = 0, int out_row_off = 0, const float* gate = nullptr,
+                      int gate_stride = 0) {
+  LaunchScope ls(k.s, KC_GEMM, 2.0 * M * N * K, k.st);
+  return f32_done(f32_gemm(A, W, M, N, K, mode, out, ldo, rows_per_batch,
+                           out_rows_per_batch > 0 ? out_rows_per_batch : rows_per_batch, out_row_off, gate,
+                           gate_stride, k.st));
+}
+
+af_status f32_ln_op(F32Step& k, const float* x, const float* shift, const float* scale, int mod_stride, float* y,
+                    int rows, int rows_per_batch, int D, float eps) {
+  LaunchScope ls(k.s, KC_LN, 8.0 * rows * D, k.st);
+  return f32_done(f32_ln_modulate(x, shift, scale, mod_stride, y, rows, rows_per_batch, D, eps, k.st));
+}
+
+// Q/K/V of one stream: [rows, 3D] product, per-head LayerNorm of Q and K, scatter
+af_status f32_qkv_op(const af_weights* w, F32Step& k, const float* y, int B, int rows, const float* wqkv, int row_off,
+                     int n_total) {
+  const Derived& d = w->d;
+  AF_TRY(f32_gemm_op(k, y, wqkv, B * rows, 3 * d.D, d.D, EPI_STORE, k.s->tmp, 3 * d.D, B * rows));
+  LaunchScope ls(k.s, KC_OTHER, 24.0 * B * rows * d.D, k.st);
+  return f32_done(f32_qkv_split(k.s->tmp, B * rows, rows, d.H, d.hd, w->cfg.ln_eps, reinterpret_cast<float*>(k.s->q),
+                                reinterpret_cast<float*>(k.s->k), reinterpret_cast<float*>(k.s->v), n_total, row_off,
+                                k.st));
+}
+
+// x += gate * (silu(y W1^T) * (y W2^T)) W3^T, with W1 and W2 stored one after the other
+af_status f32_ffn_op(const af_weights* w, F32Step& k, const float* y, int B, int rows, const float* w12,
+                     const float* w3, float* h, float* x, const float* gate, int gate_stride) {
+  const Derived& d = w->d;
+  const int M = B * rows;
+  AF_TRY(f32_gemm_op(k, y, w12, M, 2 * d.F, d.D, EPI_STORE, k.s->tmp, 2 * d.F, M));
+  {
+    LaunchScope ls(k.s, KC_OTHER, 12.0 * M * d.F, k.st);
+    AF_TRY(f32_done(f32_swiglu(k.s->tmp, M, d.F, h, k.st)));
+  }
+  return f32_gemm_op(k, h, w3, M, d.D, d.F, EPI_GATE_RES, x, d.D, rows, 0, 0, gate, gate_stride);
+}
+
+af_status f32_attention_op(const af_weights* w, F32Step& k, int B, int N, float* out_a, float* out_b, int split,
+                           const KeyMask& km) {
+  const Derived& d = w->d;
+  LaunchScope ls(k.s, KC_ATTN, 4.0 * B * d.H * static_cast<double>(N) * N * d.hd, k.st);
+  return f32_done(f32_attention(reinterpret_cast<const float*>(k.s->q), reinterpret_cast<const float*>(k.s->k),
+                                reinterpret_cast<const float*>(k.s->v), B, d.H, N, d.hd,
+                                1.0f / sqrtf(static_cast<float>(d.hd)), out_a, out_b, split, d.D, km.len, km.base,
+                                km.end, k.st));
+}
+
+af_status f32_timestep_mlp(const af_weights* w, F32Step& k, const float* t, int B, float* feat, float* h1,
+                           float* temb) {
+  const int C = w->cfg.timestep_channels, D = w->d.D;
+  LaunchScope ls(k.s, KC_OTHER, 4.0 * D * (C + D), k.st, 3);
+  AF_TRY(f32_done(launch_timestep_features(t, B, C, feat, k.st)));
+  AF_TRY(f32_done(f32_gemv(feat, B, C, w->ptrf("time_step_proj.linear_1.weight"),
+                           w->ptrf("time_step_proj.linear_1.bias"), D, 0, 1, h1, D, k.st)));
+  return f32_done(f32_gemv(h1, B, D, w->ptrf("time_step_proj.linear_2.weight"), w->ptrf("time_step_proj.linear_2.bias"),
+                           D, 0, 0, temb, D, k.st));
+}
+
+af_status f32_modulations(const af_weights* w, F32Step& k, const float* temb, int B, float* out) {
+  const int rows = static_cast<int>(w->ada_rows);
+  LaunchScope ls(k.s, KC_OTHER, 4.0 * rows * w->d.D, k.st);
+  return f32_done(f32_gemv(temb, B, w->d.D, reinterpret_cast<const float*>(w->base + w->tensors[0].offset), nullptr,
+                           rows, 1, 0, out, rows, k.st));
+}
+
+af_status f32_forward(const af_weights* w, af_scratch* s, const float* latents, const float* text_emb, const float* t,
+                      int B, int H, int W, int L, const KeyMask& km, float* velocity, cudaStream_t st,
+                      const float* premods, int pre_stride) {
+  const af_config& c = w->cfg;
+  const Derived& d = w->d;
+  const int p = c.patch_size, hp = H / p, wp = W / p, Ni = hp * wp;
+  const int R = c.num_register_tokens, Nt = R + L, N = Nt + Ni, D = d.D;
+  const float eps = c.ln_eps;
+  F32Step k{s, st};
+  float* img = reinterpret_cast<float*>(s->img);
+  float* txt = reinterpret_cast<float*>(s->txt);
+  float* x = reinterpret_cast<float*>(s->x);
+  float* y = reinterpret_cast<float*>(s->y);
+  float* o = reinterpret_cast<float*>(s->o);
+  float* h = reinterpret_cast<float*>(s->h);
+  const float* mods = premods ? premods : s->mods;
+  const int ms = premods ? pre_stride : static_cast<int>(w->ada_rows);
+  if (!premods) {
+    AF_TRY(f32_timestep_mlp(w, k, t, B, s->tfeat, s->h1, s->temb));
+    AF_TRY(f32_modulations(w, k, s->temb, B, s->mods));
+  }
+  {
+    LaunchScope ls(s, KC_OTHER, 8.0 * B * Ni * D, st);
+    AF_TRY(f32_done(f32_patch_embed(latents, B, c.in_channels, H, W, p, w->ptrf("pos_embed.proj.weight"),
+                                    w->ptrf("pos_embed.pos_embed"), d.G, D, img, st)));
+  }
+  for (int b = 0; b < B && R > 0; ++b)  // register tokens at the head of every sample's text stream
+    AF_CUDA(cudaMemcpyAsync(txt + static_cast<size_t>(b) * Nt * D, w->ptrf("register_tokens"),
+                            static_cast<size_t>(R) * D * 4, cudaMemcpyDeviceToDevice, st));
+  if (L > 0)
+    AF_TRY(f32_gemm_op(k, text_emb, w->ptrf("context_embedder.weight"), B * L, D, c.joint_attention_dim, EPI_STORE,
+                       txt, D, L, Nt, R));
+  for (int i = 0; i < c.num_mmdit_layers; ++i) {
+    const std::string pre = "joint_transformer_blocks." + std::to_string(i) + ".";
+    const float* mi = mods + w->unit_row[2 * i];
+    const float* mt = mods + w->unit_row[2 * i + 1];
+    float* yi = y;
+    float* yt = y + static_cast<size_t>(B) * Ni * D;
+    float* oi = o;
+    float* ot = o + static_cast<size_t>(B) * Ni * D;
+    float* hi = h;
+    float* ht = h + static_cast<size_t>(B) * Ni * d.F;
+    AF_TRY(f32_ln_op(k, img, mi + 0 * D, mi + 1 * D, ms, yi, B * Ni, Ni, D, eps));
+    AF_TRY(f32_ln_op(k, txt, mt + 0 * D, mt + 1 * D, ms, yt, B * Nt, Nt, D, eps));
+    AF_TRY(f32_qkv_op(w, k, yt, B, Nt, w->ptrf(pre + "attn.add_q_proj.weight"), 0, N));
+    AF_TRY(f32_qkv_op(w, k, yi, B, Ni, w->ptrf(pre + "attn.to_q.weight"), Nt, N));
+    AF_TRY(f32_attention_op(w, k, B, N, ot, oi, Nt, km));
+    AF_TRY(f32_gemm_op(k, oi, w->ptrf(pre + "attn.to_out.0.weight"), B * Ni, D, D, EPI_GATE_RES, img, D, Ni, 0, 0,
+                       mi + 2 * D, ms));
+    AF_TRY(f32_gemm_op(k, ot, w->ptrf(pre + "attn.to_add_out.weight"), B * Nt, D, D, EPI_GATE_RES, txt, D, Nt, 0, 0,
+                       mt + 2 * D, ms));
+    AF_TRY(f32_ln_op(k, img, mi + 3 * D, mi + 4 * D, ms, yi, B * Ni, Ni, D, eps));
+    AF_TRY(f32_ln_op(k, txt, mt + 3 * D, mt + 4 * D, ms, yt, B * Nt, Nt, D, eps));
+    AF_TRY(f32_ffn_op(w, k, yi, B, Ni, w->ptrf(pre + "ff.linear_1.weight"), w->ptrf(pre + "ff.out_projection.weight"),
+                      hi, img, mi + 5 * D, ms));
+    AF_TRY(f32_ffn_op(w, k, yt, B, Nt, w->ptrf(pre + "ff_context.linear_1.weight"),
+                      w->ptrf(pre + "ff_context.out_projection.weight"), ht, txt, mt + 5 * D, ms));
+  }
+  // x = cat(text, image) per sample
+  AF_CUDA(cudaMemcpy2DAsync(x, static_cast<size_t>(N) * D * 4, txt, static_cast<size_t>(Nt) * D * 4,
+                            static_cast<size_t>(Nt) * D * 4, B, cudaMemcpyDeviceToDevice, st));
+  AF_CUDA(cudaMemcpy2DAsync(x + static_cast<size_t>(Nt) * D, static_cast<size_t>(N) * D * 4, img,
+                            static_cast<size_t>(Ni) * D * 4, static_cast<size_t>(Ni) * D * 4, B,
+                            cudaMemcpyDeviceToDevice, st));
+  for (int i = 0; i < c.num_single_dit_layers; ++i) {
+    const std::string pre = "single_transformer_blocks." + std::to_string(i) + ".";
+    const float* m = mods + w->unit_row[2 * c.num_mmdit_layers + i];
+    AF_TRY(f32_ln_op(k, x, m + 0 * D, m + 1 * D, ms, y, B * N, N, D, eps));
+    AF_TRY(f32_qkv_op(w, k, y, B, N, w->ptrf(pre + "attn.to_q.weight"), 0, N));
+    AF_TRY(f32_attention_op(w, k, B, N, o, o, 0, km));
+    AF_TRY(f32_gemm_op(k, o, w->ptrf(pre + "attn.to_out.0.weight"), B * N, D, D, EPI_GATE_RES, x, D, N, 0, 0,
+                       m + 2 * D, ms));
+    AF_TRY(f32_ln_op(k, x, m + 3 * D, m + 4 * D, ms, y, B * N, N, D, eps));
+    AF_TRY(f32_ffn_op(w, k, y, B, N, w->ptrf(pre + "ff.linear_1.weight"), w->ptrf(pre + "ff.out_projection.weight"),
+                      h, x, m + 5 * D, ms));
+  }
+  const float* pf = mods + w->pf_row;  // pre-final: scale first, then shift
+  LaunchScope ls(s, KC_OTHER, 8.0 * B * Ni * D, st);
+  return f32_done(f32_output_stage(x, N, Nt, B, hp, wp, D, pf, pf + D, ms, w->ptrf("proj_out.weight"), p,
+                                   c.out_channels, velocity, st));
+}
+
+}  // namespace
+
 namespace af {
 const uint16_t* weights_tensor(const af_weights* w, const char* name) { return w->ptr(name); }
 int weights_device(const af_weights* w) { return w->device; }
 int weights_inner_dim(const af_weights* w) { return w->d.D; }
 int weights_timestep_channels(const af_weights* w) { return w->cfg.timestep_channels; }
+bool weights_is_f32(const af_weights* w) { return w->f32; }
 void set_last_error(const std::string& msg) { g_last_error = msg; }
 }  // namespace af
 
@@ -562,6 +749,7 @@ af_status af_config_default(af_config* c) {
   c->timestep_channels = 256;
   c->ffn_inner = 0;
   c->ln_eps = 1e-6f;
+  c->dtype = AF_DTYPE_BF16;
   return AF_OK;
 }
 
@@ -579,14 +767,23 @@ af_status af_weights_create(const af_config* cfg, int device, af_weights** out) 
   *out = nullptr;
   Derived d;
   AF_TRY(derive(cfg, &d));
+  if (cfg->dtype != AF_DTYPE_BF16 && cfg->dtype != AF_DTYPE_F32) return AF_ERR_INVALID_ARG;
   // shapes the kernels cover
-  if (d.D % 32 != 0 || d.F % 128 != 0 || cfg->joint_attention_dim % 8 != 0) return AF_ERR_UNSUPPORTED;
-  if (!(d.hd == 256 || d.hd == 8 || d.hd == 16 || d.hd == 32 || d.hd == 64)) return AF_ERR_UNSUPPORTED;
-  if (cfg->patch_size * cfg->patch_size * cfg->in_channels > 64) return AF_ERR_UNSUPPORTED;
+  if (cfg->dtype == AF_DTYPE_F32) {
+    if (!(d.hd == 8 || d.hd == 16 || d.hd == 32 || d.hd == 64)) return AF_ERR_UNSUPPORTED;
+  } else {
+    if (d.D % 32 != 0 || d.F % 128 != 0 || cfg->joint_attention_dim % 8 != 0) return AF_ERR_UNSUPPORTED;
+    if (!(d.hd == 256 || d.hd == 8 || d.hd == 16 || d.hd == 32 || d.hd == 64)) return AF_ERR_UNSUPPORTED;
+    if (cfg->patch_size * cfg->patch_size * cfg->in_channels > 64) return AF_ERR_UNSUPPORTED;
+    // the timestep / modulation GEMV reads rows of 16-byte vectors, at most 4096 wide
+    if (cfg->timestep_channels % 8 != 0 || cfg->timestep_channels > 4096 || d.D > 4096) return AF_ERR_UNSUPPORTED;
+  }
   af_weights* w = new af_weights();
   w->cfg = *cfg;
   w->d = d;
   w->device = device;
+  w->f32 = cfg->dtype == AF_DTYPE_F32;
+  w->esz = w->f32 ? 4 : 2;
   build_layout(w);
   int prev = 0;
   cudaGetDevice(&prev);
@@ -650,33 +847,99 @@ af_status af_weights_find(const af_weights* w, const char* name, int* id) {
   return AF_OK;
 }
 
-af_status af_weights_set(af_weights* w, int id, const uint16_t* src, int src_is_device, void* stream) {
+af_status af_weights_set(af_weights* w, int id, const void* src, int src_is_device, int src_dtype, void* stream) {
   if (!w || !src || id < 0 || id >= static_cast<int>(w->tensors.size())) return AF_ERR_INVALID_ARG;
+  if (src_dtype != AF_DTYPE_BF16 && src_dtype != AF_DTYPE_F32) return AF_ERR_INVALID_ARG;
+  AF_TRY(check_device(w));
   const TensorInfo& t = w->tensors[id];
-  const size_t bytes = t.numel() * 2;
+  const bool src_f32 = src_dtype == AF_DTYPE_F32;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (src_is_device) AF_TRY(check_dev_ptr(src));
+  uint8_t* dst = w->base + (t.interleave ? t.pair_base : t.offset);
+  const int cols = t.ndim == 2 ? static_cast<int>(t.shape[1]) : 1;
+  if (src_is_device && src_f32 != w->f32) {  // convert on the device, in the pack's layout
+    AF_CUDA(launch_convert_copy(src, src_f32, dst, w->f32, t.numel(), cols, t.interleave, st));
+    return AF_OK;
+  }
+  std::vector<uint8_t> conv;
+  if (!src_is_device && src_f32 != w->f32) {  // convert on the host, then copy
+    conv.resize(t.numel() * w->esz);
+    for (size_t i = 0; i < t.numel(); ++i) {
+      if (w->f32) {
+        const uint32_t u = static_cast<uint32_t>(static_cast<const uint16_t*>(src)[i]) << 16;
+        memcpy(conv.data() + 4 * i, &u, 4);
+      } else {
+        uint32_t u;
+        memcpy(&u, static_cast<const float*>(src) + i, 4);
+        const uint16_t b = static_cast<uint16_t>((u + 0x7FFFu + ((u >> 16) & 1u)) >> 16);  // nearest even
+        memcpy(conv.data() + 2 * i, &b, 2);
+      }
+    }
+    src = conv.data();
+  }
+  const size_t bytes = t.numel() * w->esz;
   if (t.interleave) {
     // 128-row groups of this half go to every other 128-row slot of the pair
-    const size_t group = static_cast<size_t>(128) * t.shape[1] * 2;
-    uint8_t* dst = w->base + t.pair_base + (t.interleave == 2 ? group : 0);
+    const size_t group = static_cast<size_t>(128) * t.shape[1] * w->esz;
+    uint8_t* d0 = dst + (t.interleave == 2 ? group : 0);
     const size_t groups = static_cast<size_t>(t.shape[0]) / 128;
     if (src_is_device)
-      AF_CUDA(cudaMemcpy2DAsync(dst, 2 * group, src, group, group, groups, cudaMemcpyDeviceToDevice, st));
+      AF_CUDA(cudaMemcpy2DAsync(d0, 2 * group, src, group, group, groups, cudaMemcpyDeviceToDevice, st));
     else
-      AF_CUDA(cudaMemcpy2D(dst, 2 * group, src, group, group, groups, cudaMemcpyHostToDevice));
+      AF_CUDA(cudaMemcpy2D(d0, 2 * group, src, group, group, groups, cudaMemcpyHostToDevice));
     return AF_OK;
   }
   if (src_is_device) {
-    AF_CUDA(cudaMemcpyAsync(w->base + t.offset, src, bytes, cudaMemcpyDeviceToDevice, st));
+    AF_CUDA(cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, st));
   } else {
-    AF_CUDA(cudaMemcpy(w->base + t.offset, src, bytes, cudaMemcpyHostToDevice));
+    AF_CUDA(cudaMemcpy(dst, src, bytes, cudaMemcpyHostToDevice));
+  }
+  return AF_OK;
+}
+
+af_status af_weights_get(const af_weights* w, int id, void* dst, int dst_is_device, void* stream) {
+  if (!w || !dst || id < 0 || id >= static_cast<int>(w->tensors.size())) return AF_ERR_INVALID_ARG;
+  AF_TRY(check_device(w));
+  if (dst_is_device) AF_TRY(check_dev_ptr(dst));
+  const TensorInfo& t = w->tensors[id];
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const cudaMemcpyKind kind = dst_is_device ? cudaMemcpyDeviceToDevice : cudaMemcpyDeviceToHost;
+  if (t.interleave) {
+    const size_t group = static_cast<size_t>(128) * t.shape[1] * w->esz;
+    const uint8_t* s0 = w->base + t.pair_base + (t.interleave == 2 ? group : 0);
+    const size_t groups = static_cast<size_t>(t.shape[0]) / 128;
+    if (dst_is_device)
+      AF_CUDA(cudaMemcpy2DAsync(dst, group, s0, 2 * group, group, groups, kind, st));
+    else
+      AF_CUDA(cudaMemcpy2D(dst, group, s0, 2 * group, group, groups, kind));
+    return AF_OK;
+  }
+  if (dst_is_device)
+    AF_CUDA(cudaMemcpyAsync(dst, w->base + t.offset, t.numel() * w->esz, kind, st));
+  else
+    AF_CUDA(cudaMemcpy(dst, w->base + t.offset, t.numel() * w->esz, kind));
+  return AF_OK;
+}
+
+af_status af_weights_init_random(af_weights* w, uint64_t seed, float std, void* stream) {
+  if (!w || !(std >= 0.f)) return AF_ERR_INVALID_ARG;
+  AF_TRY(check_device(w));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  for (const TensorInfo& t : w->tensors) {
+    // [ARCH] §Patch Embedding: positions ~N(0, 0.1^2); §Register Tokens: ~N(0, 0.02^2)
+    const bool pos = t.name == "pos_embed.pos_embed";
+    const float sd = pos ? 0.1f : (t.name == "register_tokens" ? 0.02f : std);
+    uint8_t* dst = w->base + (t.interleave ? t.pair_base : t.offset);
+    const int cols = t.ndim == 2 ? static_cast<int>(t.shape[1]) : 1;
+    AF_CUDA(launch_init_normal(dst, w->f32, t.numel(), cols, t.interleave, crc32_ieee(t.name.c_str()), seed, sd, st));
   }
   return AF_OK;
 }
 
 af_status af_weights_quantize_fp8(af_weights* w, int enable, void* stream) {
   if (!w) return AF_ERR_INVALID_ARG;
+  if (w->f32) return AF_ERR_UNSUPPORTED;
+  AF_TRY(check_device(w));
   if (!enable) {
     if (w->fp8_codes) cudaFree(w->fp8_codes);
     if (w->fp8_scales) cudaFree(w->fp8_scales);
@@ -759,6 +1022,7 @@ af_status af_scratch_create(const af_weights* w, int max_batch, int max_img_toke
                             af_scratch** out) {
   if (!w || !out || max_batch <= 0 || max_img_tokens <= 0 || max_text_len < 0) return AF_ERR_INVALID_ARG;
   *out = nullptr;
+  AF_TRY(check_device(w));
   const Derived& d = w->d;
   af_scratch* s = new af_scratch();
   s->w = w;
@@ -781,17 +1045,19 @@ af_status af_scratch_create(const af_weights* w, int max_batch, int max_img_toke
   const size_t o_h1 = take(B * D * 4);
   const size_t o_tfeat = take(B * w->cfg.timestep_channels * 4);
   const size_t o_mods = take(B * w->ada_rows * 4);
-  const size_t o_y = take(rowsN * D * 2);
-  const size_t o_q = take(rowsN * D * 2);
-  const size_t o_k = take(rowsN * D * 2);
-  const size_t o_v = take(rowsN * D * 2);
-  const size_t o_o = take(rowsN * D * 2);
-  const size_t o_h = take(rowsN * F * 2);
-  const size_t o_img = take(B * s->max_ni * D * 2);
-  const size_t o_txt = take(B * s->max_nt * D * 2);
-  const size_t o_x = take(rowsN * D * 2);
-  const size_t o_y8 = take(rowsN * (D > F ? D : F));  // e4m3 codes of y, O or h (8-bit variant)
-  const size_t o_ys = take(rowsN * 4);
+  const size_t es = w->esz;  // activations are stored like the weights: bf16, or fp32 for an fp32 pack
+  const size_t o_y = take(rowsN * D * es);
+  const size_t o_q = take(rowsN * D * es);
+  const size_t o_k = take(rowsN * D * es);
+  const size_t o_v = take(rowsN * D * es);
+  const size_t o_o = take(rowsN * D * es);
+  const size_t o_h = take(rowsN * F * es);
+  const size_t o_img = take(B * s->max_ni * D * es);
+  const size_t o_txt = take(B * s->max_nt * D * es);
+  const size_t o_x = take(rowsN * D * es);
+  const size_t o_y8 = take(w->f32 ? 0 : rowsN * (D > F ? D : F));  // e4m3 codes of y, O or h (8-bit variant)
+  const size_t o_ys = take(w->f32 ? 0 : rowsN * 4);
+  const size_t o_tmp = take(w->f32 ? rowsN * (3 * D > 2 * F ? 3 * D : 2 * F) * 4 : 0);
   const int cmax = w->cfg.in_channels > w->cfg.out_channels ? w->cfg.in_channels : w->cfg.out_channels;
   const size_t lat_elems = B * static_cast<size_t>(cmax) * s->max_ni * w->cfg.patch_size * w->cfg.patch_size;
   const size_t o_lat2 = take(lat_elems * 4);
@@ -831,6 +1097,7 @@ af_status af_scratch_create(const af_weights* w, int max_batch, int max_img_toke
   s->txt = reinterpret_cast<uint16_t*>(s->base + o_txt);
   s->x = reinterpret_cast<uint16_t*>(s->base + o_x);
   s->y8 = s->base + o_y8;
+  s->tmp = reinterpret_cast<float*>(s->base + o_tmp);
   s->yscale = reinterpret_cast<float*>(s->base + o_ys);
   s->lat2 = reinterpret_cast<float*>(s->base + o_lat2);
   s->vel = reinterpret_cast<float*>(s->base + o_vel);
@@ -864,6 +1131,10 @@ af_status af_timestep_embed(const af_weights* w, af_scratch* s, const float* t, 
   if (!t || !temb || B <= 0) return AF_ERR_INVALID_ARG;
   if (B > s->max_b) return AF_ERR_SHAPE;
   const Derived& d = w->d;
+  if (w->f32) {
+    F32Step k{s, static_cast<cudaStream_t>(stream)};
+    return f32_timestep_mlp(w, k, t, B, s->tfeat, s->h1, temb);
+  }
   LaunchScope ls(s, KC_OTHER, 2.0 * d.D * (w->cfg.timestep_channels + d.D), static_cast<cudaStream_t>(stream), 3);
   AF_CUDA(launch_timestep_mlp(t, B, w->ptr("time_step_proj.linear_1.weight"), w->ptr("time_step_proj.linear_1.bias"),
                               w->ptr("time_step_proj.linear_2.weight"), w->ptr("time_step_proj.linear_2.bias"),
@@ -875,6 +1146,7 @@ af_status af_patch_embed(const af_weights* w, af_scratch* s, const float* latent
                          uint16_t* img_tokens, void* stream) {
   AF_TRY(check_scratch(w, s));
   if (!latents || !img_tokens || B <= 0 || H <= 0 || W <= 0) return AF_ERR_INVALID_ARG;
+  if (w->f32) return AF_ERR_UNSUPPORTED;
   const int p = w->cfg.patch_size;
   if (H % p || W % p || H / p > w->d.G || W / p > w->d.G) return AF_ERR_SHAPE;
   const int Ni = (H / p) * (W / p);
@@ -890,6 +1162,7 @@ af_status af_joint_block(const af_weights* w, af_scratch* s, int layer, uint16_t
                          const float* temb, int B, int Ni, int Nt, const int* text_len, void* stream) {
   AF_TRY(check_scratch(w, s));
   if (!img || !txt || !temb || B <= 0 || Ni <= 0 || Nt <= 0) return AF_ERR_INVALID_ARG;
+  if (w->f32) return AF_ERR_UNSUPPORTED;
   if (text_len && Nt < w->cfg.num_register_tokens) return AF_ERR_SHAPE;
   if (layer < 0 || layer >= w->cfg.num_mmdit_layers) return AF_ERR_INVALID_ARG;
   if (B > s->max_b || Ni + Nt > s->max_n || Ni > s->max_n) return AF_ERR_SHAPE;
@@ -911,6 +1184,7 @@ af_status af_single_block(const af_weights* w, af_scratch* s, int layer, uint16_
                           int N, int Nt, const int* text_len, void* stream) {
   AF_TRY(check_scratch(w, s));
   if (!x || !temb || B <= 0 || N <= 0) return AF_ERR_INVALID_ARG;
+  if (w->f32) return AF_ERR_UNSUPPORTED;
   if (text_len && (Nt < w->cfg.num_register_tokens || Nt > N)) return AF_ERR_SHAPE;
   if (layer < 0 || layer >= w->cfg.num_single_dit_layers) return AF_ERR_INVALID_ARG;
   if (B > s->max_b || N > s->max_n) return AF_ERR_SHAPE;
@@ -928,7 +1202,7 @@ af_status af_single_block(const af_weights* w, af_scratch* s, int layer, uint16_
 // precomputed (rows in the adaLN unit order, element (b, r) at
 // premods[b * pre_stride + r]); the timestep MLP and the modulation GEMV are
 // skipped and `t` is not read.
-static af_status forward_impl(const af_weights* w, af_scratch* s, const float* latents, const uint16_t* text_emb,
+static af_status forward_impl(const af_weights* w, af_scratch* s, const float* latents, const void* text_emb,
                               const float* t, int B, int H, int W, int L, const int* text_len, float* velocity,
                               cudaStream_t st, const float* premods = nullptr, int pre_stride = 0) {
   AF_TRY(check_scratch(w, s));
@@ -946,6 +1220,9 @@ static af_status forward_impl(const af_weights* w, af_scratch* s, const float* l
   const float* mods = premods ? premods : s->mods;
   const int mstride = premods ? pre_stride : static_cast<int>(R_ada);
   const KeyMask km = text_mask(w, text_len, Nt);
+  if (w->f32)
+    return f32_forward(w, s, latents, static_cast<const float*>(text_emb), t, B, H, W, L, km, velocity, st, premods,
+                       pre_stride);
 
   // embedding stage
   if (!premods) {
@@ -973,7 +1250,7 @@ static af_status forward_impl(const af_weights* w, af_scratch* s, const float* l
     gp.ldo = D;
     gp.out_rows_per_batch = Nt;
     gp.out_row_off = R;
-    AF_TRY(run_gemm(s, gp, text_emb, w->ptr("context_embedder.weight"), D, st));
+    AF_TRY(run_gemm(s, gp, static_cast<const uint16_t*>(text_emb), w->ptr("context_embedder.weight"), D, st));
   }
   // joint blocks
   for (int i = 0; i < c.num_mmdit_layers; ++i) {
@@ -999,13 +1276,13 @@ static af_status forward_impl(const af_weights* w, af_scratch* s, const float* l
   return AF_OK;
 }
 
-af_status af_transformer_forward(const af_weights* w, af_scratch* s, const float* latents, const uint16_t* text_emb,
+af_status af_transformer_forward(const af_weights* w, af_scratch* s, const float* latents, const void* text_emb,
                                  const float* t, int B, int H, int W, int L, const int* text_len, float* velocity,
                                  void* stream) {
   return forward_impl(w, s, latents, text_emb, t, B, H, W, L, text_len, velocity, static_cast<cudaStream_t>(stream));
 }
 
-static af_status denoise_step_impl(const af_weights* w, af_scratch* s, float* latents, const uint16_t* text_emb,
+static af_status denoise_step_impl(const af_weights* w, af_scratch* s, float* latents, const void* text_emb,
                                    int Bi, int H, int W, int L, const int* text_len, float guidance, float sigma,
                                    float sigma_next, cudaStream_t st, const float* premods = nullptr) {
   const int B = 2 * Bi;
@@ -1023,7 +1300,7 @@ static af_status denoise_step_impl(const af_weights* w, af_scratch* s, float* la
   return AF_OK;
 }
 
-static af_status check_step_args(const af_weights* w, af_scratch* s, const float* latents, const uint16_t* text_emb,
+static af_status check_step_args(const af_weights* w, af_scratch* s, const float* latents, const void* text_emb,
                                  int Bi, int H, int W, int L) {
   AF_TRY(check_scratch(w, s));
   if (!latents || !text_emb || Bi <= 0 || H <= 0 || W <= 0 || L < 0) return AF_ERR_INVALID_ARG;
@@ -1034,7 +1311,7 @@ static af_status check_step_args(const af_weights* w, af_scratch* s, const float
   return AF_OK;
 }
 
-af_status af_denoise_step(const af_weights* w, af_scratch* s, float* latents, const uint16_t* text_emb, int Bi, int H,
+af_status af_denoise_step(const af_weights* w, af_scratch* s, float* latents, const void* text_emb, int Bi, int H,
                           int W, int L, const int* text_len, float guidance, float sigma, float sigma_next,
                           void* stream) {
   AF_TRY(check_step_args(w, s, latents, text_emb, Bi, H, W, L));
@@ -1049,7 +1326,7 @@ struct af_sampler {
   const af_weights* w = nullptr;
   af_scratch* s = nullptr;
   float* latents = nullptr;
-  const uint16_t* text = nullptr;
+  const void* text = nullptr;
   const int* text_len = nullptr;
   int Bi = 0, H = 0, W = 0, L = 0, n_steps = 0;
   float guidance = 1.f;
@@ -1064,7 +1341,7 @@ struct af_sampler {
 
 extern "C" {
 
-af_status af_sampler_create(const af_weights* w, af_scratch* s, float* latents, const uint16_t* text_emb, int Bi,
+af_status af_sampler_create(const af_weights* w, af_scratch* s, float* latents, const void* text_emb, int Bi,
                             int H, int W, int L, const int* text_len, int n_steps, const float* sigmas,
                             float guidance, int use_graphs, af_sampler** out) {
   if (!out) return AF_ERR_INVALID_ARG;
@@ -1135,6 +1412,12 @@ af_status af_sampler_prepare(af_sampler* m, void* stream) {
   af_scratch* s = m->s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int n = m->n_steps, D = w->d.D, C = w->cfg.timestep_channels;
+  AF_TRY(check_device(w));
+  if (w->f32) {  // every step's modulations by the fp32 GEMV, silu(temb) kept in fp32
+    F32Step k{s, st};
+    AF_TRY(f32_timestep_mlp(w, k, m->t_dev, n, m->feat, m->h1, m->temb));
+    return f32_modulations(w, k, m->temb, n, m->mods);
+  }
   {
     LaunchScope ls(s, KC_OTHER, 2.0 * D * (C + D), st, 2 * ((n + 7) / 8) + 1);
     AF_CUDA(launch_timestep_mlp(m->t_dev, n, w->ptr("time_step_proj.linear_1.weight"),

@@ -546,6 +546,11 @@ __global__ void timestep_features_kernel(const float* __restrict__ t, int B, int
   }
 }
 
+cudaError_t launch_timestep_features(const float* t, int B, int C, float* feat, cudaStream_t s) {
+  timestep_features_kernel<<<(B * C / 2 + 255) / 256, 256, 0, s>>>(t, B, C, feat);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_timestep_mlp(const float* t, int B, const uint16_t* w1, const uint16_t* b1, const uint16_t* w2,
                                 const uint16_t* b2, int C, int D, float* feat, float* h1, float* temb, cudaStream_t s) {
   timestep_features_kernel<<<(B * C / 2 + 255) / 256, 256, 0, s>>>(t, B, C, feat);

@@ -25,7 +25,11 @@
 //     other's intermediates; serialise them.
 //   * The first call on each device resolves the array's device address
 //     (cudaGetSymbolAddress, with that device made current); make that first
-//     call before any stream capture.
+//     call before any stream capture.  A lookup that fails is not cached:
+//     the next call tries again.
+//   * Like every entry point taking a weight pack, it launches on the
+//     current device, which must be the pack's (else AF_ERR_INVALID_ARG);
+//     fp32 packs are not covered (AF_ERR_UNSUPPORTED).
 #include <mutex>
 #include <string>
 
@@ -38,28 +42,31 @@ constexpr int kNoAllocFloats = 65536;
 static __device__ __align__(256) float g_noalloc_scratch[kNoAllocFloats];
 
 constexpr int kMaxDevices = 64;
-float* g_addr[kMaxDevices] = {};
-cudaError_t g_setup[kMaxDevices] = {};
-std::once_flag g_once[kMaxDevices];
+float* g_addr[kMaxDevices] = {};  // resolved device address per device, nullptr until a lookup succeeds
+std::mutex g_addr_mutex;
 
 // Device address of g_noalloc_scratch on `dev` (the host-side symbol is only
-// a stand-in and must never be handed to a kernel).
+// a stand-in and must never be handed to a kernel).  Only a successful
+// lookup is remembered.
 cudaError_t scratch_address(int dev, float** out) {
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::call_once(g_once[dev], [dev] {
+  std::lock_guard<std::mutex> lock(g_addr_mutex);
+  if (!g_addr[dev]) {
     int prev = 0;
     cudaError_t e = cudaGetDevice(&prev);
     if (e == cudaSuccess) e = cudaSetDevice(dev);
-    if (e == cudaSuccess) {
-      void* p = nullptr;
-      e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-      g_addr[dev] = static_cast<float*>(p);
-      cudaSetDevice(prev);
+    if (e != cudaSuccess) return e;
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    cudaSetDevice(prev);
+    if (e != cudaSuccess || !p) {
+      cudaGetLastError();  // leave no sticky error behind; the next call retries
+      return e != cudaSuccess ? e : cudaErrorInvalidSymbol;
     }
-    g_setup[dev] = e;
-  });
+    g_addr[dev] = static_cast<float*>(p);
+  }
   *out = g_addr[dev];
-  return g_setup[dev];
+  return cudaSuccess;
 }
 
 }  // namespace
@@ -68,6 +75,17 @@ extern "C" af_status af_timestep_embed_noalloc(const af_weights* w, const float*
                                                void* stream) {
   using namespace af;
   if (!w || !t || !temb || B <= 0) return AF_ERR_INVALID_ARG;
+  if (weights_is_f32(w)) return AF_ERR_UNSUPPORTED;
+  int cur = -1;
+  if (cudaGetDevice(&cur) != cudaSuccess) {
+    set_last_error(cudaGetErrorString(cudaGetLastError()));
+    return AF_ERR_CUDA;
+  }
+  if (cur != weights_device(w)) {
+    set_last_error("af_timestep_embed_noalloc: the current device (" + std::to_string(cur) +
+                   ") is not the weight pack's device (" + std::to_string(weights_device(w)) + ")");
+    return AF_ERR_INVALID_ARG;
+  }
   const int C = weights_timestep_channels(w);
   const int D = weights_inner_dim(w);
   if (static_cast<long long>(B) * (C + D) > kNoAllocFloats) {

@@ -13,8 +13,16 @@
  * Conventions shared by every call
  * --------------------------------
  *  - Tensors are caller-owned, contiguous, row-major.  "device" pointers
- *    must be CUDA device memory of the device the weight pack lives on.
+ *    must be CUDA device memory of the device the weight pack lives on, and
+ *    that device must be the current one when a call taking a weight pack
+ *    or scratch handle is made (else AF_ERR_INVALID_ARG, nothing launched).
  *    bf16 tensors are passed as uint16_t bit patterns.
+ *  - A weight pack stores bf16 (AF_DTYPE_BF16, the tensor-core path) or
+ *    fp32 (AF_DTYPE_F32, plain fp32 arithmetic end to end for small
+ *    configurations).  With an fp32 pack every activation a call takes or
+ *    returns as bf16 below is fp32 instead (text_emb, which is declared
+ *    const void*); the block-level, patch-embed and 8-bit calls take bf16
+ *    packs only and return AF_ERR_UNSUPPORTED for an fp32 pack.
  *  - Compute calls are asynchronous on `stream` (a cudaStream_t passed as
  *    void*; NULL = legacy default stream).  They return once all work is
  *    enqueued.
@@ -50,6 +58,11 @@ typedef enum {
   AF_ERR_NOT_FOUND = 7     /* unknown tensor name */
 } af_status;
 
+/* Storage / arithmetic type of a weight pack (af_config.dtype) and of the
+ * tensors handed to af_weights_set / af_weights_get. */
+#define AF_DTYPE_BF16 0
+#define AF_DTYPE_F32 1
+
 /* Model configuration: the constructor parameters of
  * AuraFlowTransformer2DModel ([ARCH] §构造参数详解).
  *   inner_dim D = num_attention_heads * attention_head_dim.
@@ -60,7 +73,11 @@ typedef enum {
  *   num_register_tokens: learned tokens at the head of the text sequence
  *                ([ARCH] §Register Tokens), 8 in the model.
  *   timestep_channels: sinusoidal timestep channels, 256 ([ARCH] §前向传播流程).
- *   ln_eps: epsilon of every LayerNorm (adaLN and QK-norm). */
+ *   ln_eps: epsilon of every LayerNorm (adaLN and QK-norm).
+ *   dtype: AF_DTYPE_BF16 (bf16 weights and activations, fp32 accumulation
+ *                and statistics, tcgen05 tensor cores) or AF_DTYPE_F32
+ *                (fp32 weights, activations and arithmetic, SIMT kernels;
+ *                head_dim 8, 16, 32 or 64). */
 typedef struct {
   int patch_size;
   int in_channels;
@@ -75,6 +92,7 @@ typedef struct {
   int timestep_channels;
   int ffn_inner;
   float ln_eps;
+  int dtype;
 } af_config;
 
 typedef struct af_weights af_weights; /* device-resident weight pack (bf16) */
@@ -82,7 +100,8 @@ typedef struct af_scratch af_scratch; /* device work buffers + error word */
 
 /* Fill *cfg with the page's defaults (patch 2, 4 -> 4 channels, 4 joint +
  * 32 single blocks, 12 heads x 256, joint_attention_dim 2048,
- * pos_embed_max_size 1024, 8 registers, 256 timestep channels, eps 1e-6). */
+ * pos_embed_max_size 1024, 8 registers, 256 timestep channels, eps 1e-6),
+ * dtype AF_DTYPE_BF16. */
 af_status af_config_default(af_config* cfg);
 
 /* Derived sizes: inner_dim D, FFN width F, position grid side G.
@@ -90,10 +109,15 @@ af_status af_config_default(af_config* cfg);
 af_status af_config_derive(const af_config* cfg, int* inner_dim, int* ffn_inner, int* grid_side);
 
 /* ---- weight pack --------------------------------------------------------
- * One device allocation holding every parameter in bf16.  Tensors are
+ * One device allocation holding every parameter in cfg->dtype.  Tensors are
  * addressed by the diffusers-style names listed by af_weights_tensor_info
  * (e.g. "single_transformer_blocks.3.attn.to_q.weight"), each with the
- * nn.Linear layout [out, in].  Freshly created packs are zero-filled. */
+ * nn.Linear layout [out, in].  Freshly created packs are zero-filled.
+ * AF_ERR_UNSUPPORTED for shapes the kernels do not cover: for bf16 packs
+ * D % 32, F % 128, joint_attention_dim % 8 or timestep_channels % 8 not 0,
+ * D or timestep_channels above 4096, head_dim not in {8, 16, 32, 64, 256},
+ * or p * p * in_channels above 64; for fp32 packs head_dim not in
+ * {8, 16, 32, 64}. */
 af_status af_weights_create(const af_config* cfg, int device, af_weights** out);
 void af_weights_destroy(af_weights* w);
 af_status af_weights_num_tensors(const af_weights* w, int* n);
@@ -102,18 +126,37 @@ af_status af_weights_num_tensors(const af_weights* w, int* n);
 af_status af_weights_tensor_info(const af_weights* w, int id, char* name, size_t name_cap,
                                  int* ndim, int64_t shape[2]);
 af_status af_weights_find(const af_weights* w, const char* name, int* id);
-/* Copy one tensor (bf16 bit patterns, numel elements as listed) into the
- * pack.  src_is_device != 0: src is device memory on the pack's device,
- * else host memory.  Asynchronous on `stream` for device sources; host
- * sources are copied synchronously. */
-af_status af_weights_set(af_weights* w, int id, const uint16_t* src, int src_is_device, void* stream);
+/* Copy one tensor (numel elements as listed) into the pack.  src_dtype:
+ * AF_DTYPE_BF16 (uint16_t bit patterns) or AF_DTYPE_F32 (float); the values
+ * are converted to the pack's dtype (fp32 -> bf16 rounds to nearest even).
+ * src_is_device != 0: src is device memory on the pack's device, else host
+ * memory.  Asynchronous on `stream` for device sources; host sources are
+ * copied synchronously. */
+af_status af_weights_set(af_weights* w, int id, const void* src, int src_is_device, int src_dtype, void* stream);
+/* Copy one tensor out of the pack, in the pack's dtype (numel elements,
+ * [out, in] row-major).  dst_is_device != 0: device memory on the pack's
+ * device (asynchronous on `stream`), else host memory (synchronous). */
+af_status af_weights_get(const af_weights* w, int id, void* dst, int dst_is_device, void* stream);
+/* Fill every tensor of the pack with seeded synthetic values, on the device:
+ * linear weights and biases ~N(0, std^2), the learned position table
+ * ~N(0, 0.1^2) and the register tokens ~N(0, 0.02^2), the scales of their
+ * random initialisation in [ARCH] §Patch Embedding and §Register Tokens.
+ * Element j of tensor `name` takes lane j % 4 of the Philox4x32-10 block
+ * j / 4 (Salmon et al., SC 2011) under key (seed mod 2^32, seed div 2^32)
+ * and counter (block mod 2^32, block div 2^32, CRC-32(name), 0); the four
+ * words become uniforms (x + 1/2) / 2^32 and the Box-Muller transform (in
+ * fp64) turns pairs into normals; the stored value is float32(z * std),
+ * rounded to bf16 (nearest even) in a bf16 pack.  Asynchronous on `stream`.
+ * An 8-bit copy made by af_weights_quantize_fp8 is not refreshed. */
+af_status af_weights_init_random(af_weights* w, uint64_t seed, float std, void* stream);
 /* Total bytes of the pack (for reporting). */
 af_status af_weights_bytes(const af_weights* w, size_t* bytes);
 
 /* ---- scratch ------------------------------------------------------------
  * Work buffers for batches up to max_batch with at most max_img_tokens
- * image tokens ((H/p)*(W/p)) and at most max_text_len text tokens (before
- * the registers are prepended). */
+ * image tokens ((H/p)*(W/p), so any latent shape, square or not, whose
+ * patch grid has that many tokens fits) and at most max_text_len text
+ * tokens (before the registers are prepended). */
 af_status af_scratch_create(const af_weights* w, int max_batch, int max_img_tokens, int max_text_len,
                             af_scratch** out);
 void af_scratch_destroy(af_scratch* s);
@@ -149,6 +192,8 @@ af_status af_timestep_embed(const af_weights* w, af_scratch* s, const float* t, 
  * any stream capture.
  *   t: device float[B]; temb: device float[B, D] (output). */
 af_status af_timestep_embed_noalloc(const af_weights* w, const float* t, int B, float* temb, void* stream);
+/* (AF_ERR_UNSUPPORTED for an fp32 pack; AF_ERR_INVALID_ARG when the current
+ * device is not the pack's.) */
 
 /* Patch embedding with centre-cropped learned positions ([ARCH] §Patch
  * Embedding): img[b, n] = W_pe patch(b, n) + PE[(r0 + n / wp) * G + c0 + n % wp]
@@ -194,7 +239,7 @@ af_status af_single_block(const af_weights* w, af_scratch* s, int layer, uint16_
  * [text; image], the single blocks, the image slice, the pre-final
  * modulation x * (1 + scale) + shift, proj_out (bias-free) and unpatchify.
  *   latents:  device float[B, C_in, H, W]
- *   text_emb: device bf16[B, L, joint_attention_dim]
+ *   text_emb: device bf16[B, L, joint_attention_dim] (fp32 for an fp32 pack)
  *   t:        device float[B] (timestep / 1000)
  *   text_len: NULL (every text token is real, the model's own behaviour) or
  *             device int[B], see "Padded prompts"
@@ -209,7 +254,7 @@ af_status af_single_block(const af_weights* w, af_scratch* s, int layer, uint16_
  * like an SDPA attn_mask); register tokens and image tokens always do.
  * Values are clamped to [0, L]. */
 af_status af_transformer_forward(const af_weights* w, af_scratch* s, const float* latents,
-                                 const uint16_t* text_emb, const float* t, int B, int H, int W, int L,
+                                 const void* text_emb, const float* t, int B, int H, int W, int L,
                                  const int* text_len, float* velocity, void* stream);
 
 /* Classifier-free guidance combine and flow-match Euler step ([PIPE]
@@ -228,10 +273,11 @@ af_status af_euler_cfg_step(float* latents, const float* velocity, int Bi, int C
  * runs at model time t = sigma on the 2 Bi batch, and af_euler_cfg_step
  * updates the latents in place with sigma_next.
  *   latents:  device float[Bi, C_in, H, W] in/out
- *   text_emb: device bf16[2 Bi, L, joint_attention_dim], uncond rows first.
+ *   text_emb: device bf16[2 Bi, L, joint_attention_dim], uncond rows first
+ *             (fp32 for an fp32 pack).
  *   text_len: NULL or device int[2 Bi] (padded prompts, as for the forward).
  * Needs a scratch created with max_batch >= 2 Bi. */
-af_status af_denoise_step(const af_weights* w, af_scratch* s, float* latents, const uint16_t* text_emb, int Bi,
+af_status af_denoise_step(const af_weights* w, af_scratch* s, float* latents, const void* text_emb, int Bi,
                           int H, int W, int L, const int* text_len, float guidance, float sigma, float sigma_next,
                           void* stream);
 
@@ -246,13 +292,14 @@ af_status af_denoise_step(const af_weights* w, af_scratch* s, float* latents, co
  * and replayed afterwards (needs a non-NULL stream; nothing may be captured
  * on the stream around these calls).
  *   latents:  device float[Bi, C, H, W], updated in place by every step
- *   text_emb: device bf16[2 Bi, L, joint_attention_dim] (uncond rows first)
+ *   text_emb: device bf16[2 Bi, L, joint_attention_dim] (uncond rows first;
+ *             fp32 for an fp32 pack)
  *   text_len: NULL or device int[2 Bi] (padded prompts)
  *   sigmas:   host float[n_steps + 1] (e.g. from af_sigma_schedule)
  * The device buffers are bound to the sampler: change their contents, not
  * their addresses.  The scratch must fit a 2 Bi batch of this size. */
 typedef struct af_sampler af_sampler;
-af_status af_sampler_create(const af_weights* w, af_scratch* s, float* latents, const uint16_t* text_emb, int Bi,
+af_status af_sampler_create(const af_weights* w, af_scratch* s, float* latents, const void* text_emb, int Bi,
                             int H, int W, int L, const int* text_len, int n_steps, const float* sigmas,
                             float guidance, int use_graphs, af_sampler** out);
 af_status af_sampler_prepare(af_sampler* smp, void* stream);

@@ -26,9 +26,11 @@ def full_config(**kw) -> O.Config:
     return O.Config(**c)
 
 
-def af_config(cfg: O.Config):
+def af_config(cfg: O.Config, dtype: int = 0):
+    """The library's configuration of an oracle configuration; dtype 1 makes
+    an fp32 weight pack (fp32 arithmetic end to end)."""
     import diffusion_transformer_denoising_auraflow_b200 as af
-    return af.Config.default(
+    return af.Config.default(dtype=dtype,
         patch_size=cfg.patch_size, in_channels=cfg.in_channels, out_channels=cfg.out_channels,
         num_mmdit_layers=cfg.num_mmdit_layers, num_single_dit_layers=cfg.num_single_dit_layers,
         attention_head_dim=cfg.attention_head_dim, num_attention_heads=cfg.num_attention_heads,
@@ -37,12 +39,12 @@ def af_config(cfg: O.Config):
         ffn_inner=0, ln_eps=cfg.ln_eps)
 
 
-def draw_weights(cfg: O.Config, seed: int, names=None) -> dict:
+def draw_weights(cfg: O.Config, seed: int, names=None, dtype: str = "bf16") -> dict:
     specs = O.weight_specs(cfg)
     if names is not None:
         keep = set(names)
         specs = [s for s in specs if s[0] in keep]
-    return synth.weights(seed, specs)
+    return synth.weights(seed, specs, dtype)
 
 
 def block_names(cfg: O.Config, kind: str, i: int):
@@ -65,8 +67,11 @@ def to_np(t):
 
 
 def upload(weights_obj, w: dict):
+    """Copy drawn arrays into the pack in its own dtype (bf16 or fp32)."""
+    import torch
+    conv = to_f32 if weights_obj.dtype == torch.float32 else to_bf16
     for name, arr in w.items():
-        weights_obj.set(name, to_bf16(arr))
+        weights_obj.set(name, conv(arr))
 
 
 def e4m3_lut():
@@ -86,15 +91,9 @@ def e4m3_lut():
 
 
 def device_weights(af_module, w, seed: int, device="cuda"):
-    """Fill every tensor of the pack with seeded N(0, std^2) values drawn on
-    the device (the full 6.8 B-parameter model in seconds); the stds are the
-    synthetic-input recipe's."""
-    import zlib
+    """Fill every tensor of the pack on the device with the synthetic-input
+    recipe (af_weights_init_random: the full 6.8 B-parameter model in well
+    under a second); the values equal synth.weights(seed, ...) drawn on the host."""
     import torch
-    for name, shape in w.tensors():
-        g = torch.Generator(device=device)
-        g.manual_seed((seed * 1000003 + zlib.crc32(name.encode())) % (2 ** 63))
-        t = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
-        t.mul_(synth.weight_std(name))
-        w.set(name, t.to(torch.bfloat16).contiguous())
+    w.init_random(seed, 0.02)
     torch.cuda.synchronize()

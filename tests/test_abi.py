@@ -45,7 +45,7 @@ def test_defaults_match_page_values():
     c = af.Config.default()
     o = O.Config()
     for f, _ in af.Config._fields_:
-        if f in ("ffn_inner",):
+        if f in ("ffn_inner", "dtype"):
             continue
         assert getattr(c, f) == pytest.approx(getattr(o, f)), f
 
@@ -63,6 +63,15 @@ def test_argument_errors_are_host_side():
     out = ctypes.c_void_p()
     bad = af.Config.default(attention_head_dim=96)
     assert L.af_weights_create(ctypes.byref(bad), 0, ctypes.byref(out)) == 3
+    # shapes the timestep / modulation GEMV cannot run are refused at creation
+    assert L.af_weights_create(ctypes.byref(af.Config.default(timestep_channels=260)), 0, ctypes.byref(out)) == 3
+    wide = af.Config.default(num_attention_heads=20)   # D = 5120 > 4096
+    assert L.af_weights_create(ctypes.byref(wide), 0, ctypes.byref(out)) == 3
+    f32_big_head = af.Config.default(dtype=af.AF_DTYPE_F32)   # the fp32 path covers head_dim <= 64
+    assert L.af_weights_create(ctypes.byref(f32_big_head), 0, ctypes.byref(out)) == 3
+    assert L.af_weights_create(ctypes.byref(af.Config.default(dtype=7)), 0, ctypes.byref(out)) == 1
+    assert L.af_weights_set(None, 0, None, 0, 0, None) == 1
+    assert L.af_weights_init_random(None, 1, 0.02, None) == 1
 
 
 def test_sigma_schedule_matches_oracle():

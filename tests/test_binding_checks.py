@@ -123,3 +123,13 @@ def test_strided_modulation_views_reach_their_storage():
     assert (B - 1) * 6 * D + D <= af._elems_from_start(md[:, 5 * D:])
     short = z(B - 1, 6 * D)
     assert (B - 1) * 6 * D + D > af._elems_from_start(short[:, 3 * D:])
+
+
+def test_device_mismatch_rule():
+    """Every tensor must be on the weight pack's device and that device must be
+    current (the library launches there); the first violation is named."""
+    assert af.device_mismatch([("x", 0), ("temb", 0)], 0, 0) is None
+    assert "temb is on cuda:1" in af.device_mismatch([("x", 0), ("temb", 1)], 0, 0)
+    assert "current device is cuda:1" in af.device_mismatch([("x", 0)], 1, 0)
+    assert af.device_mismatch([("x", 2)], 2, 2) is None
+    assert "x is on cuda:0" in af.device_mismatch([("x", 0)], 2, 2)

@@ -1,10 +1,13 @@
 """GPU parity of whole blocks against the fp64 oracle.
 
-The tolerance per block is relative L2 <= 2e-2 (bf16 path).  Small token
-counts with a ragged tail exercise several tiles; the full single-block and
-joint-block workloads (B = 2, 4096 image + 256 text tokens, D = 3072,
-F = 8192) are checked on sampled rows, which the oracle computes from all
-keys and values.
+The tolerance per block is relative L2 <= 2e-2 (bf16 path), asserted on the
+block's update (output minus input): the residual input passes through the
+block exactly, so comparing whole outputs would dilute the error of the
+update by the size of the input.  Small token counts with a ragged tail
+exercise several tiles; the full single-block and joint-block workloads
+(B = 2, 4096 image + 256 text tokens, D = 3072, F = 8192) and the 1536^2
+single block are checked on sampled rows, which the oracle computes from all
+keys and values.  Every achieved error is printed.
 """
 import numpy as np
 import pytest
@@ -60,8 +63,9 @@ def test_single_block_small(af, single_setup, N):
     temb = synth.conditioning(2, (2, 3072))
     got = _run_single(af, single_setup, x, temb)
     ref = O.single_block(x, temb, drawn, "single_transformer_blocks.0.", cfg)
-    err = O.rel_l2(got - x, ref - x)   # the block's update, the harder comparison
-    assert O.rel_l2(got, ref) < BLOCK_TOL and err < 5e-2, err
+    err = O.rel_l2(got - x, ref - x)
+    print(f"\nsingle block N={N}: update rel-L2 {err:.3e}, output {O.rel_l2(got, ref):.3e}")
+    assert err < BLOCK_TOL
 
 
 def test_single_block_zero_gates_identity(af, single_setup):
@@ -97,7 +101,9 @@ def test_single_block_full_size_sampled_rows(af, single_setup):
     got = _run_single(af, single_setup, x, temb)
     rows = [0, 1, 127, 128, 255, 256, 1000, 2047, 2048, 3333, 4223, 4224, 4351]
     ref = O.single_block_rows(x, temb, drawn, "single_transformer_blocks.0.", cfg, rows)
-    assert O.rel_l2(got[:, rows], ref) < BLOCK_TOL
+    err = O.rel_l2(got[:, rows] - x[:, rows], ref - x[:, rows])
+    print(f"\nsingle block 1024^2 workload, sampled rows: update rel-L2 {err:.3e}")
+    assert err < BLOCK_TOL
 
 
 def _run_joint(af, setup, img, txt, temb):
@@ -115,8 +121,9 @@ def test_joint_block_small(af, joint_setup):
     temb = synth.conditioning(6, (2, 3072))
     gt, gi = _run_joint(af, joint_setup, img, txt, temb)
     rt, ri = O.joint_block(img, txt, temb, drawn, "joint_transformer_blocks.0.", cfg)
-    assert O.rel_l2(gi, ri) < BLOCK_TOL and O.rel_l2(gt, rt) < BLOCK_TOL
-    assert O.rel_l2(gi - img, ri - img) < 5e-2 and O.rel_l2(gt - txt, rt - txt) < 5e-2
+    ei, et = O.rel_l2(gi - img, ri - img), O.rel_l2(gt - txt, rt - txt)
+    print(f"\njoint block small: update rel-L2 image {ei:.3e}, text {et:.3e}")
+    assert ei < BLOCK_TOL and et < BLOCK_TOL
 
 
 def test_joint_block_zero_gates_identity(af, joint_setup):
@@ -147,7 +154,10 @@ def test_joint_block_full_size_sampled_rows(af, joint_setup):
     ir = [0, 127, 128, 1500, 4095]
     tr = [0, 7, 8, 128, 255]
     rt, ri = O.joint_block_rows(img, txt, temb, drawn, "joint_transformer_blocks.0.", cfg, ir, tr)
-    assert O.rel_l2(gi[:, ir], ri) < BLOCK_TOL and O.rel_l2(gt[:, tr], rt) < BLOCK_TOL
+    ei = O.rel_l2(gi[:, ir] - img[:, ir], ri - img[:, ir])
+    et = O.rel_l2(gt[:, tr] - txt[:, tr], rt - txt[:, tr])
+    print(f"\njoint block workload, sampled rows: update rel-L2 image {ei:.3e}, text {et:.3e}")
+    assert ei < BLOCK_TOL and et < BLOCK_TOL
 
 
 def test_single_block_1536_workload_sampled_rows(af, single_setup):
@@ -165,5 +175,7 @@ def test_single_block_1536_workload_sampled_rows(af, single_setup):
     got = to_np(xt)
     rows = [0, 7, 8, 263, 264, 4095, 4096, 7777, 9215, 9216, 9472, 9479]
     ref = O.single_block_rows(x, temb, drawn, "single_transformer_blocks.0.", cfg, rows)
-    assert O.rel_l2(got[:, rows], ref) < BLOCK_TOL
+    err = O.rel_l2(got[:, rows] - x[:, rows], ref - x[:, rows])
+    print(f"\nsingle block 1536^2 workload, sampled rows: update rel-L2 {err:.3e}")
+    assert err < BLOCK_TOL
     s.close()

@@ -1,6 +1,16 @@
 """GPU parity of the whole forward (+ CFG / Euler step) against the oracle.
 
 Tolerance for the full stack on the bf16 path: relative L2 <= 5e-2.
+
+The tiny model is also run as the fp32 model its configuration states (an
+fp32 weight pack: fp32 weights, activations and arithmetic end to end).  Its
+bound, relative L2 <= 1e-4, comes from fp32 rounding: a dot product of
+length K accumulates about sqrt(K) u relative error (u = 2^-24, K <= 256 here,
+so ~1e-6 per step), and a dozen sequential steps with LayerNorm and softmax
+in between leave two orders of magnitude of margin below 1e-4; the achieved
+error is printed.  A latent update is a difference of two fp32 latents and is
+known only to 2^-24 |x| / |dx| relative; that floor is added to the bound of
+the step tests.
 """
 import numpy as np
 import pytest
@@ -13,6 +23,7 @@ from helpers import af_config, draw_weights, tiny_config, to_bf16, to_f32, to_np
 pytestmark = pytest.mark.gpu
 
 STACK_TOL = 5e-2
+F32_TOL = 1e-4
 
 
 @pytest.fixture(scope="module")
@@ -42,6 +53,97 @@ def test_tiny_forward_matches_oracle(af):
     cfg = tiny_config()
     *_, got, ref = _forward(af, cfg, 1, 1, 16, 16, 8, 0.5)
     assert O.rel_l2(got, ref) < STACK_TOL
+
+
+def _f32_floor(x_next, x):
+    """fp32 storage floor of a latent update x_next - x, relative."""
+    return 2.0 ** -24 * np.linalg.norm(x_next) / np.linalg.norm(np.asarray(x_next) - x)
+
+
+def _tiny_f32(af, seed, B, L=8):
+    cfg = tiny_config()
+    w = af.Weights(af_config(cfg, dtype=af.AF_DTYPE_F32))
+    drawn = draw_weights(cfg, seed, dtype="f32")
+    upload(w, drawn)
+    s = af.Scratch(w, B, 64, L)
+    text = synth.text_embeddings(seed, (B, L, cfg.joint_attention_dim), "f32")
+    return cfg, w, s, drawn, text
+
+
+def test_tiny_fp32_forward_matches_oracle(af):
+    """The tiny model as configured: fp32, batch 1, latent 4 x 16 x 16 (64 image
+    tokens), 8 text tokens, timestep 500 (t = 0.5)."""
+    cfg, w, s, drawn, text = _tiny_f32(af, 1, 1)
+    lat = synth.latents(1, (1, 4, 16, 16))
+    t = np.full((1,), 0.5, np.float32)
+    vel = torch.empty(1, 4, 16, 16, device="cuda")
+    af.transformer_forward(w, s, to_f32(lat), to_f32(text), to_f32(t), vel)
+    s.sync()
+    ref = O.transformer_forward(lat, text, t, drawn, cfg)
+    err = O.rel_l2(to_np(vel), ref)
+    print(f"\ntiny fp32 forward rel-L2 {err:.3e}")
+    assert err < F32_TOL
+
+
+def test_tiny_fp32_denoise_step_sampler_and_mask(af):
+    """fp32 tiny model: one CFG denoise step per call and two through the
+    sampler plan (CUDA graphs) against the oracle's loop, and padded prompts."""
+    cfg, w, s, drawn, text = _tiny_f32(af, 12, 2)
+    lat = synth.latents(12, (1, 4, 16, 16))
+    sig = [float(np.float32(x)) for x in O.sigma_schedule(25, 1.73)]
+    x = to_f32(lat)
+    af.denoise_step(w, s, x, to_f32(text), 3.5, sig[0], sig[1])
+    s.sync()
+    v = O.transformer_forward(np.concatenate([lat, lat]), text, np.full((2,), sig[0], np.float32), drawn, cfg)
+    ref = O.euler_cfg_step(lat, v, 3.5, sig[0], sig[1])
+    err = O.rel_l2(to_np(x) - lat, ref - lat)
+    floor = _f32_floor(ref, lat)
+    print(f"\ntiny fp32 denoise step rel-L2 {err:.3e} (fp32 storage floor {floor:.1e})")
+    assert err < F32_TOL + 4 * floor
+    # the sampler plan: modulations of every step precomputed, steps as graphs
+    xs = to_f32(lat)
+    st = torch.cuda.Stream()
+    smp = af.Sampler(w, s, xs, to_f32(text), sig[:3], 3.5, use_graphs=True)
+    smp.prepare(st)
+    smp.step(0, st)
+    smp.step(1, st)
+    st.synchronize()
+    ref = lat.astype(np.float64)
+    for i in range(2):
+        v = O.transformer_forward(np.concatenate([ref, ref]), text, np.full((2,), sig[i], np.float32), drawn, cfg)
+        ref = O.euler_cfg_step(ref, v, 3.5, sig[i], sig[i + 1])
+    err = O.rel_l2(to_np(xs) - lat, ref - lat)
+    floor = _f32_floor(ref, lat)
+    print(f"tiny fp32 sampler (2 steps) rel-L2 {err:.3e} (fp32 storage floor {floor:.1e})")
+    assert err < F32_TOL + 4 * floor
+    smp.close()
+    # padded prompts: real lengths 3 and 8
+    lens = [3, 8]
+    lat2 = synth.latents(13, (2, 4, 16, 16))
+    t = np.array([0.8, 0.3], np.float32)
+    vel = torch.empty(2, 4, 16, 16, device="cuda")
+    af.transformer_forward(w, s, to_f32(lat2), to_f32(text), to_f32(t), vel,
+                           text_len=torch.tensor(lens, dtype=torch.int32, device="cuda"))
+    s.sync()
+    ref = O.transformer_forward(lat2, text, t, drawn, cfg, text_len=lens)
+    err = O.rel_l2(to_np(vel), ref)
+    print(f"tiny fp32 padded-prompt forward rel-L2 {err:.3e}")
+    assert err < F32_TOL
+
+
+def test_fp32_pack_rejects_bf16_only_calls(af):
+    cfg, w, s, drawn, text = _tiny_f32(af, 14, 1)
+    with pytest.raises(af.AFError) as ei:
+        af.single_block(w, s, 0, torch.zeros(1, 10, 32, device="cuda", dtype=torch.bfloat16),
+                        torch.zeros(1, 32, device="cuda"))
+    assert ei.value.status == 3
+    with pytest.raises(af.AFError) as ei:
+        w.quantize_fp8()
+    assert ei.value.status == 3
+    with pytest.raises(TypeError):   # an fp32 pack takes fp32 text embeddings
+        af.transformer_forward(w, s, torch.zeros(1, 4, 16, 16, device="cuda"),
+                               torch.zeros(1, 8, 32, device="cuda", dtype=torch.bfloat16),
+                               torch.zeros(1, device="cuda"), torch.empty(1, 4, 16, 16, device="cuda"))
 
 
 def test_tiny_forward_cfg_euler_step(af):
