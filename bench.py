@@ -31,7 +31,6 @@ import subprocess
 import sys
 import threading
 import time
-import zlib
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
@@ -48,6 +47,7 @@ WORKLOADS = {
 GUIDANCE = 3.5
 N_SCHED = 25
 SHIFT = 1.73
+NOMINAL_BF16_TFLOPS = 2250.0   # B200 dense bf16 tensor-core peak (nominal, without sparsity)
 
 
 def parse():
@@ -59,14 +59,17 @@ def parse():
     ap.add_argument("--workload", default="1024", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-1536", action="store_true", help="skip the 1536x1536 sub-record of the default line")
     ap.add_argument("--seed", type=int, default=4)
     ap.add_argument("--fp8", action="store_true",
                     help="8-bit variant: e4m3 operands for every block projection (af_weights_quantize_fp8)")
     ap.add_argument("--direct", action="store_true",
                     help="time the per-step entry point (af_denoise_step) instead of the sampler plan")
-    ap.add_argument("--case", default="step", choices=["step", "single_block"],
-                    help="single_block: time one full-shape AuraFlowSingleTransformerBlock only "
-                         "(a small command for profiler captures)")
+    ap.add_argument("--case", default="step", choices=["step", "single_block", "small_model"],
+                    help="single_block: time one full-shape AuraFlowSingleTransformerBlock only; "
+                         "small_model: a 1-block model's forward + guidance/Euler step at the workload's "
+                         "shapes (every HBM-bound kernel, a few GB on the device); both are small "
+                         "commands for profiler captures")
     return ap.parse_args()
 
 
@@ -221,12 +224,16 @@ def run_reference(args, rank, world):
     value = 1.0 / step_s
     cores = blas_threads()
     sample = (f"one single DiT block of the workload (B=2, {N} tokens, D=3072) in the fp64 numpy oracle per "
-              f"timed step; a denoise step is taken as 36 such blocks (joint blocks cost the same FLOPs); "
+              f"timed unit; a denoise step is taken as 36 such blocks (joint blocks cost the same FLOPs); "
               f"{cpu_model()}")
+    # what ran: args.steps single blocks of ms_per_step each; value is the
+    # steps/s those blocks extrapolate to (36 blocks per denoise step)
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1000.0,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_block * 1000.0,
+            "timed_unit": "one single DiT block (1/36 of a denoise step); steps and ms_per_step count blocks",
+            "extrapolated_to_step": {"blocks_per_step": 36, "s_per_denoise_step": step_s, "steps_per_s": value},
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": wl["name"], "sample": "1 of 36 blocks per step"},
+            "data": "synthetic", "config": {"workload": wl["name"], "sample": "1 of 36 blocks per timed unit"},
             "cpu_baseline": {"value": value, "unit": "steps/s", "cores": cores, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -236,13 +243,10 @@ def run_reference(args, rank, world):
 # ----------------------------------------------------------------------------- CUDA arm
 
 def make_weights(af, torch, w, seed, device):
-    import synth
-    for name, shape in w.tensors():
-        g = torch.Generator(device=device)
-        g.manual_seed((seed * 1000003 + zlib.crc32(name.encode())) % (2 ** 63))
-        t = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
-        t.mul_(synth.weight_std(name))
-        w.set(name, t.to(torch.bfloat16).contiguous())
+    """Seeded synthetic weights filled on the device by the library
+    (af_weights_init_random: linear weights ~N(0, 0.02^2), positions
+    ~N(0, 0.1^2), registers ~N(0, 0.02^2))."""
+    w.init_random(seed, 0.02)
     torch.cuda.synchronize()
 
 
@@ -439,6 +443,8 @@ def run_af(args, rank, world, local_rank):
                        "l2": "no flush needed: each step streams 13.6 GB of weights (> 126 MB L2)"},
             "tflops": tflops, "tflops_frac_of_peak": tflops * 1e12 / (pk["bf16_tflops"] * 1e12),
             "tflops_peak_used": pk["bf16_tflops"], "peak_source": pk["source"] + " (burst cuBLAS bf16)",
+            "tflops_frac_of_nominal_peak": tflops / NOMINAL_BF16_TFLOPS,
+            "nominal_peak_tflops": NOMINAL_BF16_TFLOPS,
             "clocks": clocks, "gpu_launches": launches, "roofline": roofline,
             "kernel_ms_per_step": {"gemm": step_ms_classes[0], "attention": step_ms_classes[1],
                                    "ln_modulate": step_ms_classes[2], "other": step_ms_classes[3]},
@@ -446,13 +452,79 @@ def run_af(args, rank, world, local_rank):
             "e2e": e2e,
             "path": ("per-step calls (af_denoise_step)" if args.direct else
                      "af_sampler: modulations of all 25 steps in one GEMM per run (timed), steps as CUDA graphs"),
+            "plan_prepare": (None if args.direct else
+                             f"the 25-step modulation GEMM (af_sampler_prepare) is timed at every step whose index "
+                             f"is a multiple of 25: {(args.steps + N_SCHED - 1) // N_SCHED} time(s) in these "
+                             f"{args.steps} steps"),
             "per_step_path_steps_per_s": direct,
         }
     for plan in plans.values():
         plan.close()
     s.close()
     w.close()
+    if line is not None and world == 1 and args.workload == "1024" and not args.no_1536:
+        line["workloads"] = {"1536": measure_1536(args, af, torch, device, stream, pk)}
     return line
+
+
+def measure_1536(args, af, torch, device, stream, pk):
+    """The 1536 x 1536 workload (latent 4 x 192 x 192, 9216 image + 264 text
+    tokens, 96 x 96 position grid), timed like the main line through the
+    sampler plan (graphs captured untimed first), plus the per-kernel-class
+    split of one per-step-path step."""
+    wl = WORKLOADS["1536"]
+    H, W, L, G = wl["H"], wl["W"], wl["L"], wl["G"]
+    Ni = (H // 2) * (W // 2)
+    w = af.Weights(af.Config.default(pos_embed_max_size=G * G), device.index)
+    make_weights(af, torch, w, args.seed, device)
+    if args.fp8:
+        w.quantize_fp8()
+    s = af.Scratch(w, 2, Ni, L)
+    gen = torch.Generator(device=device)
+    gen.manual_seed(args.seed * 7919 + 1536)
+    lat0 = torch.randn(1, 4, H, W, generator=gen, device=device)
+    text = torch.randn(2, L, 2048, generator=gen, device=device).to(torch.bfloat16)
+    lat = lat0.clone()
+    sig = af.sigma_schedule(N_SCHED, SHIFT)
+    plan = af.Sampler(w, s, lat, text, sig, GUIDANCE, use_graphs=True)
+    plan.prepare(stream)
+    for i in range(N_SCHED):       # capture every step graph (untimed)
+        plan.step(i, stream)
+    lat.copy_(lat0)
+    steps = max(3, min(args.steps, 8))
+    plan.prepare(stream)
+    for i in range(2):
+        plan.step(i, stream)
+    s.sync(stream)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(device.index) as clk:
+        e0.record(stream)
+        for i in range(steps):
+            j = i % N_SCHED
+            if j == 0:
+                plan.prepare(stream)
+            plan.step(j, stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    t = e0.elapsed_time(e1) / 1000.0
+    s.profile_begin()
+    af.denoise_step(w, s, lat, text, GUIDANCE, sig[3], sig[4], stream)
+    ms, nl, work = s.profile_end(stream)
+    plan.close()
+    s.close()
+    w.close()
+    value = steps / t
+    tflops = step_flops(H, W, L) * value / 1e12
+    return {"workload": wl["name"], "tokens": 8 + L + Ni, "steps": steps, "value": value, "unit": "steps/s",
+            "ms_per_step": t / steps * 1000.0, "tflops": tflops,
+            "tflops_frac_of_peak": tflops / pk["bf16_tflops"], "tflops_frac_of_nominal_peak": tflops / NOMINAL_BF16_TFLOPS,
+            "kernel_ms_per_step": {"gemm": ms[0], "attention": ms[1], "ln_modulate": ms[2], "other": ms[3]},
+            "kernel_rates": {"gemm_tflops": work[0] / (ms[0] * 1e-3) / 1e12 if ms[0] > 0 else None,
+                             "attention_tflops": work[1] / (ms[1] * 1e-3) / 1e12 if ms[1] > 0 else None,
+                             "ln_modulate_gbs": work[2] / (ms[2] * 1e-3) / 1e9 if ms[2] > 0 else None},
+            "clocks": clk.summary(),
+            "note": "same timing as the main line (sampler plan, CUDA graphs, device events, prepare timed at "
+                    "step 0); kernel split from one per-step-path step under the event profiler"}
 
 
 def run_single_block_case(args):
@@ -491,6 +563,39 @@ def run_single_block_case(args):
     return 0
 
 
+def run_small_model_case(args):
+    """A model with one single DiT block at the workload's full shapes (CFG
+    batch 2, 8 + L + Ni tokens, D = 3072): every HBM-bound kernel of the step
+    (timestep MLP and modulation GEMV, patch embed, LayerNorm + modulate,
+    output stage, guidance + Euler) at full size, with ~0.5 GB of weights."""
+    import torch
+    import diffusion_transformer_denoising_auraflow_b200 as af
+    wl = WORKLOADS[args.workload]
+    H, W, L, G = wl["H"], wl["W"], wl["L"], wl["G"]
+    Ni = (H // 2) * (W // 2)
+    cfg = af.Config.default(num_mmdit_layers=0, num_single_dit_layers=1, pos_embed_max_size=G * G)
+    w = af.Weights(cfg, 0)
+    make_weights(af, torch, w, args.seed, torch.device("cuda", 0))
+    s = af.Scratch(w, 2, Ni, L)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(args.seed)
+    lat = torch.randn(1, 4, H, W, generator=gen, device="cuda")
+    text = torch.randn(2, L, 2048, generator=gen, device="cuda").to(torch.bfloat16)
+    sig = af.sigma_schedule(N_SCHED, SHIFT)
+    for i in range(args.warmup):
+        af.denoise_step(w, s, lat, text, GUIDANCE, sig[i % N_SCHED], sig[i % N_SCHED + 1])
+    s.sync()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(args.steps):
+        af.denoise_step(w, s, lat, text, GUIDANCE, sig[i % N_SCHED], sig[i % N_SCHED + 1])
+    e1.record()
+    s.sync()
+    print(json.dumps({"case": "small_model", "tokens": 8 + L + Ni, "ms_per_step": e0.elapsed_time(e1) / args.steps,
+                      "finite": bool(torch.isfinite(lat).all().item())}), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     rank = int(os.environ.get("RANK", "0"))
@@ -500,6 +605,8 @@ def main():
         return run_reference(args, rank, world)
     if args.case == "single_block":
         return run_single_block_case(args)
+    if args.case == "small_model":
+        return run_small_model_case(args)
     # CPU baseline first (before any CUDA context), rank 0 at N = 1 only
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
