@@ -78,6 +78,12 @@ _SIGS = {
     "af_single_block": [_P, _P, _I, _P, _P, _I, _I, _I, _P, _P],
     "af_transformer_forward": [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P],
     "af_euler_cfg_step": [_P, _P, _I, _I, _I, _I, _F, _F, _F, _P],
+    "af_euler_cfg_step2": [_P, _P, _P, _I, _I, _I, _I, _F, _F, _F, _P],
+    "af_exchange_create": [_I, ctypes.c_size_t, _P],
+    "af_exchange_handle": [_P, _P],
+    "af_exchange_open_peer": [_P, _P],
+    "af_exchange_ptrs": [_P, _P, _P],
+    "af_exchange_destroy": [_P],
     "af_denoise_step": [_P, _P, _P, _P, _I, _I, _I, _I, _P, _F, _F, _F, _P],
     "af_sigma_schedule": [_I, _F, _I, _P],
     "af_sampler_create": [_P, _P, _P, _P, _I, _I, _I, _I, _P, _I, _P, _F, _I, _P],
@@ -113,6 +119,7 @@ def _load():
     L.af_weights_destroy.restype = None
     L.af_scratch_destroy.restype = None
     L.af_sampler_destroy.restype = None
+    L.af_exchange_destroy.restype = None
     L.af_status_string.restype = ctypes.c_char_p
     L.af_last_error.restype = ctypes.c_char_p
     return L
@@ -638,3 +645,97 @@ def linear_fp8(A8, a_scale, W8, w_scale, C, stream=None):
     cp = c.dev(C, torch.bfloat16, "C")
     c.check()
     _check(lib.af_linear_fp8(ap, asp, wp, wsp, cp, M, N, K, _stream(stream)), where)
+
+
+AF_IPC_HANDLE_BYTES = 64
+
+
+class _DeviceView:
+    """A device buffer seen by torch through the CUDA array interface (no copy)."""
+
+    def __init__(self, ptr: int, shape):
+        self.__cuda_array_interface__ = {"shape": tuple(shape), "typestr": "<f4", "data": (int(ptr), False),
+                                         "version": 3, "strides": None}
+
+
+class Exchange:
+    """Velocity exchange buffer of the two-GPU CFG split (af_exchange): `slots`
+    float32 tensors of `shape` that the peer process maps through CUDA IPC."""
+
+    def __init__(self, shape, slots: int = 2, device: int | None = None):
+        self.shape = tuple(int(x) for x in shape)
+        self.slots = int(slots)
+        self.device = torch.cuda.current_device() if device is None else int(device)
+        self.numel = 1
+        for d in self.shape:
+            self.numel *= d
+        h = ctypes.c_void_p()
+        _check(lib.af_exchange_create(self.device, self.slots * self.numel * 4, ctypes.byref(h)), "af_exchange_create")
+        self.handle_ptr = h
+        self._local = None
+
+    def _ptrs(self):
+        lp, pp = ctypes.c_void_p(), ctypes.c_void_p()
+        _check(lib.af_exchange_ptrs(self.handle_ptr, ctypes.byref(lp), ctypes.byref(pp)), "af_exchange_ptrs")
+        return lp.value, pp.value
+
+    def handle(self) -> bytes:
+        """Opaque IPC handle of this buffer, to send to the peer process."""
+        buf = ctypes.create_string_buffer(AF_IPC_HANDLE_BYTES)
+        _check(lib.af_exchange_handle(self.handle_ptr, buf), "af_exchange_handle")
+        return buf.raw
+
+    def open_peer(self, handle: bytes):
+        _check(lib.af_exchange_open_peer(self.handle_ptr, ctypes.create_string_buffer(bytes(handle),
+                                                                                     AF_IPC_HANDLE_BYTES)),
+               "af_exchange_open_peer")
+
+    def local(self, slot: int) -> torch.Tensor:
+        """Slot `slot` of this process's buffer as a torch tensor (a view)."""
+        if self._local is None:
+            lp, _ = self._ptrs()
+            view = torch.as_tensor(_DeviceView(lp, (self.slots,) + self.shape), device=torch.device("cuda", self.device))
+            self._local = view
+        return self._local[slot]
+
+    def peer(self, slot: int) -> int:
+        """Device address of slot `slot` of the peer's mapped buffer."""
+        _, pp = self._ptrs()
+        if not pp:
+            raise AFError(AF_ERR_INVALID_ARG, "Exchange.peer", "the peer buffer is not open")
+        return pp + slot * self.numel * 4
+
+    def synchronize(self):
+        torch.cuda.current_stream().synchronize()
+
+    def close(self):
+        if self.handle_ptr:
+            self._local = None
+            lib.af_exchange_destroy(self.handle_ptr)
+            self.handle_ptr = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def euler_cfg_step2(latents, v_uncond, v_text, guidance: float, sigma: float, sigma_next: float, stream=None):
+    """Guidance + Euler with the two velocity halves apart; either half may be
+    a torch tensor on this device or the int device address of a peer buffer
+    (Exchange.peer) holding latents.numel() floats."""
+    where = "af_euler_cfg_step2"
+    Bi, C, H, W = latents.shape
+    c = _Call(where)
+    lp = c.dev(latents, torch.float32, "latents")
+    ptrs = []
+    for name, v in (("v_uncond", v_uncond), ("v_text", v_text)):
+        if isinstance(v, int):
+            ptrs.append(ctypes.c_void_p(v))
+        else:
+            _need(v.numel() == latents.numel(), where, f"{name} must hold {latents.numel()} values, got {v.numel()}")
+            ptrs.append(c.dev(v, torch.float32, name))
+    c.check()
+    _check(lib.af_euler_cfg_step2(lp, ptrs[0], ptrs[1], Bi, C, H, W, float(guidance), float(sigma), float(sigma_next),
+                                  _stream(stream)), where)

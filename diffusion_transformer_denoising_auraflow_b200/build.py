@@ -14,7 +14,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libaf.so")
-SOURCES = ["api.cu", "gemm.cu", "attention.cu", "kernels.cu", "init.cu", "fp32.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "gemm.cu", "attention.cu", "kernels.cu", "init.cu", "fp32.cu", "exchange.cu", "noalloc.cu"]
 HEADERS = ["af_internal.h", "ptx.cuh"]
 
 

@@ -55,6 +55,12 @@ bool encode_tmap_3d(CUtensorMap* map, const void* ptr, uint64_t d0, uint64_t d1,
                     uint64_t s2_bytes, uint32_t b0, uint32_t b1, uint32_t b2);
 cudaError_t launch_gemm(const GemmParams& p_in, const void* A, const void* W, int W_rows, cudaStream_t stream,
                         int num_sms);
+// Two problems (same operand type) in one persistent CTA-pair launch, the
+// second's tiles after the first's; falls back to two launches when the
+// problems are too small for CTA pairs.
+cudaError_t launch_gemm_grouped(const GemmParams& p0, const void* A0, const void* W0, int W0_rows,
+                                const GemmParams& p1, const void* A1, const void* W1, int W1_rows,
+                                cudaStream_t stream, int num_sms);
 int device_sm_count();
 
 // Attention (attention.cu)
@@ -104,6 +110,9 @@ cudaError_t small_kernels_set_attributes();
 cudaError_t launch_euler_cfg(float* lat, const float* v, int Bi, int64_t per_sample, float g, float sigma,
                              float sigma_next, cudaStream_t s);
 cudaError_t launch_timestep_features(const float* t, int B, int C, float* feat, cudaStream_t s);
+// x += (sigma' - sigma) (vu + g (vc - vu)) over n elements, the halves given apart
+cudaError_t launch_euler_cfg2(float* lat, const float* v_uncond, const float* v_text, int64_t n, float g, float sigma,
+                              float sigma_next, cudaStream_t s);
 
 // Weight-pack filling (init.cu).  interleave: 0 plain, 1 / 2 = linear_1 /
 // linear_2 rows of an FFN up pair stored in alternating 128-row groups.

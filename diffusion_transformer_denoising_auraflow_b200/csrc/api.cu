@@ -324,10 +324,19 @@ Operand weight_op(const af_weights* w, const std::string& name) {
   return {w->ptr(name), nullptr};
 }
 
+// A tensor-core GEMM call: parameters, operands and the weight rows the
+// tensor map spans.
+struct GemmCall {
+  GemmParams p;
+  const void* A;
+  const void* W;
+  int W_rows;
+  bool ok;  // operand types agree (both bf16 or both e4m3)
+};
+
 // QKV projection of one stream with per-head LayerNorm of Q and K.
-af_status qkv(const af_weights* w, af_scratch* s, Operand y, int B, int rows, Operand wqkv, int row_off,
-              int n_total, cudaStream_t st) {
-  if ((y.scale != nullptr) != (wqkv.scale != nullptr)) return AF_ERR_UNSUPPORTED;
+GemmCall qkv_call(const af_weights* w, af_scratch* s, Operand y, int B, int rows, Operand wqkv, int row_off,
+                  int n_total) {
   const Derived& d = w->d;
   GemmParams p = gemm_base(s, B * rows, 3 * d.D, d.D, EPI_QKV, rows);
   p.q = s->q;
@@ -341,13 +350,12 @@ af_status qkv(const af_weights* w, af_scratch* s, Operand y, int B, int rows, Op
   p.eps = w->cfg.ln_eps;
   p.a_scale = y.scale;
   p.w_scale = wqkv.scale;
-  return run_gemm(s, p, y.ptr, wqkv.ptr, 3 * d.D, st);
+  return {p, y.ptr, wqkv.ptr, 3 * d.D, (y.scale != nullptr) == (wqkv.scale != nullptr)};
 }
 
 // x += gate[b] * (A W^T)
-af_status gated_residual(af_scratch* s, Operand A, int B, int rows, int K, Operand W, int N, uint16_t* x,
-                         const float* gate, int gate_stride, cudaStream_t st) {
-  if ((A.scale != nullptr) != (W.scale != nullptr)) return AF_ERR_UNSUPPORTED;
+GemmCall gres_call(af_scratch* s, Operand A, int B, int rows, int K, Operand W, int N, uint16_t* x,
+                   const float* gate, int gate_stride) {
   GemmParams p = gemm_base(s, B * rows, N, K, EPI_GATE_RES, rows);
   p.out = x;
   p.ldo = N;
@@ -355,7 +363,47 @@ af_status gated_residual(af_scratch* s, Operand A, int B, int rows, int K, Opera
   p.gate_stride = gate_stride;
   p.a_scale = A.scale;
   p.w_scale = W.scale;
-  return run_gemm(s, p, A.ptr, W.ptr, N, st);
+  return {p, A.ptr, W.ptr, N, (A.scale != nullptr) == (W.scale != nullptr)};
+}
+
+// h = silu(y W1^T) * (y W2^T), W1 and W2 interleaved in 128-row groups ([2F, D])
+GemmCall swiglu_call(const af_weights* w, af_scratch* s, Operand y, int M, Operand w12, uint16_t* h) {
+  const Derived& d = w->d;
+  GemmParams p = gemm_base(s, M, d.F, d.D, EPI_SWIGLU, M);
+  p.out = h;
+  p.ldo = d.F;
+  p.a_scale = y.scale;
+  p.w_scale = w12.scale;
+  return {p, y.ptr, w12.ptr, 2 * d.F, (y.scale != nullptr) == (w12.scale != nullptr)};
+}
+
+double gemm_flops(const GemmParams& p) {
+  const double ncols = p.mode == EPI_SWIGLU ? 2.0 * p.N : static_cast<double>(p.N);
+  return 2.0 * p.M * ncols * p.K;
+}
+
+af_status run_call(af_scratch* s, const GemmCall& c, cudaStream_t st) {
+  if (!c.ok) return AF_ERR_UNSUPPORTED;
+  return run_gemm(s, c.p, c.A, c.W, c.W_rows, st);
+}
+
+// Two independent projections (the joint block's image and text streams) in
+// one persistent launch: the text tiles fill the image GEMM's last wave.
+af_status run_calls_grouped(af_scratch* s, const GemmCall& a, const GemmCall& b, cudaStream_t st) {
+  if (!a.ok || !b.ok) return AF_ERR_UNSUPPORTED;
+  LaunchScope ls(s, KC_GEMM, gemm_flops(a.p) + gemm_flops(b.p), st);
+  cudaError_t e = launch_gemm_grouped(a.p, a.A, a.W, a.W_rows, b.p, b.A, b.W, b.W_rows, st, s->sms);
+  return e == cudaSuccess ? AF_OK : cuda_fail(e);
+}
+
+af_status qkv(const af_weights* w, af_scratch* s, Operand y, int B, int rows, Operand wqkv, int row_off,
+              int n_total, cudaStream_t st) {
+  return run_call(s, qkv_call(w, s, y, B, rows, wqkv, row_off, n_total), st);
+}
+
+af_status gated_residual(af_scratch* s, Operand A, int B, int rows, int K, Operand W, int N, uint16_t* x,
+                         const float* gate, int gate_stride, cudaStream_t st) {
+  return run_call(s, gres_call(s, A, B, rows, K, W, N, x, gate, gate_stride), st);
 }
 
 // The 8-bit variant's per-token quantisation of a bf16 activation [rows, K]
@@ -366,16 +414,8 @@ af_status quantize_act(af_scratch* s, const uint16_t* x, int rows, int K, uint8_
   return e == cudaSuccess ? AF_OK : cuda_fail(e);
 }
 
-// h = silu(y W1^T) * (y W2^T), W1 and W2 interleaved in 128-row groups ([2F, D])
 af_status swiglu(const af_weights* w, af_scratch* s, Operand y, int M, Operand w12, uint16_t* h, cudaStream_t st) {
-  if ((y.scale != nullptr) != (w12.scale != nullptr)) return AF_ERR_UNSUPPORTED;
-  const Derived& d = w->d;
-  GemmParams p = gemm_base(s, M, d.F, d.D, EPI_SWIGLU, M);
-  p.out = h;
-  p.ldo = d.F;
-  p.a_scale = y.scale;
-  p.w_scale = w12.scale;
-  return run_gemm(s, p, y.ptr, w12.ptr, 2 * d.F, st);
+  return run_call(s, swiglu_call(w, s, y, M, w12, h), st);
 }
 
 // Padding of the text part: for sample b the keys [base + len[b], end) are
@@ -463,8 +503,9 @@ af_status joint_block_impl(const af_weights* w, af_scratch* s, int layer, uint16
 
   AF_TRY(ln_mod(s, img, mi + 0 * D, mi + 1 * D, mod_stride, y_img, B * Ni, Ni, D, eps, st, q8_img, ys_img));
   AF_TRY(ln_mod(s, txt, mt + 0 * D, mt + 1 * D, mod_stride, y_txt, B * Nt, Nt, D, eps, st, q8_txt, ys_txt));
-  AF_TRY(qkv(w, s, a_txt, B, Nt, weight_op(w, pre + "attn.add_q_proj.weight"), 0, N, st));
-  AF_TRY(qkv(w, s, a_img, B, Ni, weight_op(w, pre + "attn.to_q.weight"), Nt, N, st));
+  // each projection pair (image, text) runs as one grouped launch
+  AF_TRY(run_calls_grouped(s, qkv_call(w, s, a_img, B, Ni, weight_op(w, pre + "attn.to_q.weight"), Nt, N),
+                           qkv_call(w, s, a_txt, B, Nt, weight_op(w, pre + "attn.add_q_proj.weight"), 0, N), st));
   AF_TRY(attention(w, s, B, N, o_txt, o_img, Nt, km, st));
   // 8-bit variant: the attention output and the SwiGLU product are quantised
   // per token (into the same e4m3 buffer, free again once QKV / FFN-up ran)
@@ -475,14 +516,15 @@ af_status joint_block_impl(const af_weights* w, af_scratch* s, int layer, uint16
     oa_img = {q8_img, ys_img};
     oa_txt = {q8_txt, ys_txt};
   }
-  AF_TRY(gated_residual(s, oa_img, B, Ni, D, weight_op(w, pre + "attn.to_out.0.weight"), D, img, mi + 2 * D,
-                        mod_stride, st));
-  AF_TRY(gated_residual(s, oa_txt, B, Nt, D, weight_op(w, pre + "attn.to_add_out.weight"), D, txt, mt + 2 * D,
-                        mod_stride, st));
+  AF_TRY(run_calls_grouped(
+      s, gres_call(s, oa_img, B, Ni, D, weight_op(w, pre + "attn.to_out.0.weight"), D, img, mi + 2 * D, mod_stride),
+      gres_call(s, oa_txt, B, Nt, D, weight_op(w, pre + "attn.to_add_out.weight"), D, txt, mt + 2 * D, mod_stride),
+      st));
   AF_TRY(ln_mod(s, img, mi + 3 * D, mi + 4 * D, mod_stride, y_img, B * Ni, Ni, D, eps, st, q8_img, ys_img));
   AF_TRY(ln_mod(s, txt, mt + 3 * D, mt + 4 * D, mod_stride, y_txt, B * Nt, Nt, D, eps, st, q8_txt, ys_txt));
-  AF_TRY(swiglu(w, s, a_img, B * Ni, weight_op(w, pre + "ff.linear_1.weight"), h_img, st));
-  AF_TRY(swiglu(w, s, a_txt, B * Nt, weight_op(w, pre + "ff_context.linear_1.weight"), h_txt, st));
+  AF_TRY(run_calls_grouped(s, swiglu_call(w, s, a_img, B * Ni, weight_op(w, pre + "ff.linear_1.weight"), h_img),
+                           swiglu_call(w, s, a_txt, B * Nt, weight_op(w, pre + "ff_context.linear_1.weight"), h_txt),
+                           st));
   if (f8) {
     uint8_t* h8_txt = s->y8 + static_cast<size_t>(B) * Ni * d.F;
     AF_TRY(quantize_act(s, h_img, B * Ni, d.F, s->y8, ys_img, st));
@@ -490,10 +532,12 @@ af_status joint_block_impl(const af_weights* w, af_scratch* s, int layer, uint16
     ha_img = {s->y8, ys_img};
     ha_txt = {h8_txt, ys_txt};
   }
-  AF_TRY(gated_residual(s, ha_img, B, Ni, d.F, weight_op(w, pre + "ff.out_projection.weight"), D, img, mi + 5 * D,
-                        mod_stride, st));
-  AF_TRY(gated_residual(s, ha_txt, B, Nt, d.F, weight_op(w, pre + "ff_context.out_projection.weight"), D, txt,
-                        mt + 5 * D, mod_stride, st));
+  AF_TRY(run_calls_grouped(
+      s, gres_call(s, ha_img, B, Ni, d.F, weight_op(w, pre + "ff.out_projection.weight"), D, img, mi + 5 * D,
+                   mod_stride),
+      gres_call(s, ha_txt, B, Nt, d.F, weight_op(w, pre + "ff_context.out_projection.weight"), D, txt, mt + 5 * D,
+                mod_stride),
+      st));
   return AF_OK;
 }
 

@@ -474,10 +474,18 @@ constexpr uint32_t G2_A_BYTES = 128 * GEMM_BK * 2;  // 16 KB
 constexpr uint32_t G2_B_BYTES = 128 * GEMM_BK * 2;  // 16 KB
 constexpr int GEMM2_SMEM = G2_STAGES * (G2_A_BYTES + G2_B_BYTES) + 1024 + 1024;
 
-template <bool FP8>
+//
+// Grouped mode: a second problem (tensor maps tmA1 / tmB1, parameters p1)
+// with its own A, W, epilogue and output rides in the same persistent
+// launch; its tiles follow the first problem's in the tile order (the joint
+// block's text-stream projections after the image-stream ones, filling the
+// image GEMM's last wave instead of a launch of their own).  p1.num_tiles = 0
+// for a single problem, and GROUPED = false compiles the second problem out.
+template <bool FP8, bool GROUPED>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     gemm_tcgen05_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                      const GemmParams p) {
+                      const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
+                      const __grid_constant__ GemmParams p, const __grid_constant__ GemmParams p1) {
   constexpr int KB = FP8 ? 2 * GEMM_BK : GEMM_BK;  // K elements per stage (128 bytes per row)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -525,7 +533,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
   cluster_sync();  // the partner's barriers exist before anything signals them
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int num_k = (p.K + KB - 1) / KB;
+  const int total_tiles = GROUPED ? p.num_tiles + p1.num_tiles : p.num_tiles;
   volatile int never = 0;
 
   if (warp == 0) {
@@ -533,11 +541,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true, issued = false;
-      for (int t = cl; t < p.num_tiles && ok; t += ncl) {
+      for (int t = cl; t < total_tiles && ok; t += ncl) {
+        const bool second = GROUPED && t >= p.num_tiles;
+        const GemmParams& q = second ? p1 : p;
+        const CUtensorMap* ta = second ? &tmA1 : &tmA;
+        const CUtensorMap* tb = second ? &tmB1 : &tmB;
         int mb, nb;
-        tile_coords(t, p.num_m_tiles, p.num_n_tiles, p.group_n, mb, nb);
+        tile_coords(second ? t - p.num_tiles : t, q.num_m_tiles, q.num_n_tiles, q.group_n, mb, nb);
         const int arow = mb * 256 + static_cast<int>(rank) * 128;
         const int wrow = nb * GEMM_BN + static_cast<int>(rank) * 128;
+        const int num_k = (q.K + KB - 1) / KB;
         for (int kb = 0; kb < num_k; ++kb) {
           if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, p.err, abort_flag)) {
             ok = false;
@@ -546,8 +559,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
           const uint32_t fb_local = smem_u32(&full[stage]);
           if (leader) mbar_arrive_expect_tx(fb_local, 2 * (G2_A_BYTES + G2_B_BYTES));
           const uint32_t fb = mapa_shared(fb_local, 0);
-          tma_load_2d_pair(smem_u32(sA + stage * G2_A_BYTES), &tmA, fb, kb * KB, arow);
-          tma_load_2d_pair(smem_u32(sB + stage * G2_B_BYTES), &tmB, fb, kb * KB, wrow);
+          tma_load_2d_pair(smem_u32(sA + stage * G2_A_BYTES), ta, fb, kb * KB, arow);
+          tma_load_2d_pair(smem_u32(sB + stage * G2_B_BYTES), tb, fb, kb * KB, wrow);
           issued = true;
           if (++stage == G2_STAGES) {
             stage = 0;
@@ -567,10 +580,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
       int stage = 0;
       uint32_t phase = 0, acc = 0, acc_phase = 0;
       bool ok = true;
-      for (int t = cl; t < p.num_tiles && ok; t += ncl) {
+      for (int t = cl; t < total_tiles && ok; t += ncl) {
         if (!mbar_wait(smem_u32(&acc_empty[acc]), acc_phase ^ 1u, p.err, abort_flag)) break;
         tc_fence_after();
         const uint32_t d = tmem + acc * GEMM_BN;
+        const int num_k = (((GROUPED && t >= p.num_tiles) ? p1.K : p.K) + KB - 1) / KB;
         for (int kb = 0; kb < num_k; ++kb) {
           if (!mbar_wait(smem_u32(&full[stage]), phase, p.err, abort_flag)) {
             ok = false;
@@ -604,15 +618,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     const int quarter = warp & 3;
     const int row_in_tile = quarter * 32 + lane;
     uint32_t acc = 0, acc_phase = 0;
-    for (int t = cl; t < p.num_tiles; t += ncl) {
+    for (int t = cl; t < total_tiles; t += ncl) {
+      const bool second = GROUPED && t >= p.num_tiles;
+      const GemmParams& q = second ? p1 : p;
       int mb, nb;
-      tile_coords(t, p.num_m_tiles, p.num_n_tiles, p.group_n, mb, nb);
+      tile_coords(second ? t - p.num_tiles : t, q.num_m_tiles, q.num_n_tiles, q.group_n, mb, nb);
       const bool got = mbar_wait(smem_u32(&acc_full[acc]), acc_phase, p.err, abort_flag);
       __syncwarp();
       if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
       const uint32_t tbase = tmem + acc * GEMM_BN + (static_cast<uint32_t>(quarter * 32) << 16);
-      epilogue_tile(p, tbase, mb * 256 + static_cast<int>(rank) * 128, nb, row_in_tile);
+      epilogue_tile(q, tbase, mb * 256 + static_cast<int>(rank) * 128, nb, row_in_tile);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
@@ -649,12 +665,56 @@ cudaError_t gemm_set_attributes() {
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(gemm_tcgen05<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM_SMEM_BYTES);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(gemm_tcgen05_pair<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM2_SMEM);
+    e = cudaFuncSetAttribute(gemm_tcgen05_pair<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM2_SMEM);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(gemm_tcgen05_pair<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM2_SMEM);
+    e = cudaFuncSetAttribute(gemm_tcgen05_pair<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM2_SMEM);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(gemm_tcgen05_pair<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM2_SMEM);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(gemm_tcgen05_pair<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM2_SMEM);
   if (e != cudaSuccess) return e;
   done |= uint64_t(1) << dev;
   return cudaSuccess;
+}
+
+// Tensor maps and tile counts of one problem; pair = 256-row CTA-pair tiles.
+static cudaError_t prepare_gemm(GemmParams& p, const void* A, const void* W, int W_rows, bool pair, CUtensorMap* ta,
+                                CUtensorMap* tb) {
+  const bool fp8 = p.w_scale != nullptr;
+  const int esz = fp8 ? 1 : 2;
+  const int kb = fp8 ? 2 * GEMM_BK : GEMM_BK;  // 128-byte K boxes either way
+  if (p.K <= 0 || (p.K * esz) % 16 != 0) return cudaErrorInvalidValue;
+  if (fp8 && !p.a_scale) return cudaErrorInvalidValue;
+  if (!encode_tmap_2d(ta, A, p.K, p.M, static_cast<uint64_t>(p.K) * esz, kb, GEMM_BM, fp8))
+    return cudaErrorInvalidValue;
+  if (!encode_tmap_2d(tb, W, p.K, W_rows, static_cast<uint64_t>(p.K) * esz, kb, pair ? 128 : GEMM_BN, fp8))
+    return cudaErrorInvalidValue;
+  p.num_n_tiles = p.mode == EPI_SWIGLU ? (p.N + 127) / 128 : (p.N + GEMM_BN - 1) / GEMM_BN;
+  p.group_n = p.num_n_tiles < 16 ? p.num_n_tiles : 16;
+  p.num_m_tiles = pair ? (p.M + 255) / 256 : (p.M + GEMM_BM - 1) / GEMM_BM;
+  p.num_tiles = p.num_m_tiles * p.num_n_tiles;
+  return cudaSuccess;
+}
+
+static cudaError_t launch_pair(const GemmParams& p0, const CUtensorMap& ta0, const CUtensorMap& tb0,
+                               const GemmParams& p1, const CUtensorMap& ta1, const CUtensorMap& tb1,
+                               cudaStream_t stream, int num_sms) {
+  const int total = p0.num_tiles + p1.num_tiles;
+  const int pairs = num_sms / 2;
+  const int grid = 2 * (total < pairs ? total : pairs);
+  const bool grouped = p1.num_tiles > 0;
+  if (p0.w_scale) {
+    if (grouped)
+      gemm_tcgen05_pair<true, true><<<grid, GEMM_THREADS, GEMM2_SMEM, stream>>>(ta0, tb0, ta1, tb1, p0, p1);
+    else
+      gemm_tcgen05_pair<true, false><<<grid, GEMM_THREADS, GEMM2_SMEM, stream>>>(ta0, tb0, ta1, tb1, p0, p1);
+  } else {
+    if (grouped)
+      gemm_tcgen05_pair<false, true><<<grid, GEMM_THREADS, GEMM2_SMEM, stream>>>(ta0, tb0, ta1, tb1, p0, p1);
+    else
+      gemm_tcgen05_pair<false, false><<<grid, GEMM_THREADS, GEMM2_SMEM, stream>>>(ta0, tb0, ta1, tb1, p0, p1);
+  }
+  return cudaGetLastError();
 }
 
 cudaError_t launch_gemm(const GemmParams& p_in, const void* A, const void* W, int W_rows, cudaStream_t stream,
@@ -662,42 +722,42 @@ cudaError_t launch_gemm(const GemmParams& p_in, const void* A, const void* W, in
   GemmParams p = p_in;
   if (p.M <= 0 || p.N <= 0) return cudaSuccess;
   const bool fp8 = p.w_scale != nullptr;
-  const int esz = fp8 ? 1 : 2;
-  const int kb = fp8 ? 2 * GEMM_BK : GEMM_BK;  // 128-byte K boxes either way
-  if (p.K <= 0 || (p.K * esz) % 16 != 0) return cudaErrorInvalidValue;
-  if (fp8 && !p.a_scale) return cudaErrorInvalidValue;
-  CUtensorMap ta, tb;
-  if (!encode_tmap_2d(&ta, A, p.K, p.M, static_cast<uint64_t>(p.K) * esz, kb, GEMM_BM, fp8))
-    return cudaErrorInvalidValue;
   const bool pair = p.M >= 1024 && num_sms >= 2;
-  if (!encode_tmap_2d(&tb, W, p.K, W_rows, static_cast<uint64_t>(p.K) * esz, kb, pair ? 128 : GEMM_BN, fp8))
-    return cudaErrorInvalidValue;
-  {
-    cudaError_t e = gemm_set_attributes();
-    if (e != cudaSuccess) return e;
+  CUtensorMap ta, tb;
+  cudaError_t e = prepare_gemm(p, A, W, W_rows, pair, &ta, &tb);
+  if (e != cudaSuccess) return e;
+  e = gemm_set_attributes();
+  if (e != cudaSuccess) return e;
+  if (pair) {
+    GemmParams none = p;
+    none.num_tiles = 0;
+    return launch_pair(p, ta, tb, none, ta, tb, stream, num_sms);
   }
-  p.num_n_tiles = p.mode == EPI_SWIGLU ? (p.N + 127) / 128 : (p.N + GEMM_BN - 1) / GEMM_BN;
-  p.group_n = p.num_n_tiles < 16 ? p.num_n_tiles : 16;
-  if (p.M >= 1024 && num_sms >= 2) {
-    // CTA pairs on 256-row tiles
-    p.num_m_tiles = (p.M + 255) / 256;
-    p.num_tiles = p.num_m_tiles * p.num_n_tiles;
-    const int pairs = num_sms / 2;
-    const int grid = 2 * (p.num_tiles < pairs ? p.num_tiles : pairs);
-    if (fp8)
-      gemm_tcgen05_pair<true><<<grid, GEMM_THREADS, GEMM2_SMEM, stream>>>(ta, tb, p);
-    else
-      gemm_tcgen05_pair<false><<<grid, GEMM_THREADS, GEMM2_SMEM, stream>>>(ta, tb, p);
-    return cudaGetLastError();
-  }
-  p.num_m_tiles = (p.M + GEMM_BM - 1) / GEMM_BM;
-  p.num_tiles = p.num_m_tiles * p.num_n_tiles;
   const int grid = p.num_tiles < num_sms ? p.num_tiles : num_sms;
   if (fp8)
     gemm_tcgen05<true><<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, stream>>>(ta, tb, p);
   else
     gemm_tcgen05<false><<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, stream>>>(ta, tb, p);
   return cudaGetLastError();
+}
+
+cudaError_t launch_gemm_grouped(const GemmParams& p0_in, const void* A0, const void* W0, int W0_rows,
+                                const GemmParams& p1_in, const void* A1, const void* W1, int W1_rows,
+                                cudaStream_t stream, int num_sms) {
+  GemmParams p0 = p0_in, p1 = p1_in;
+  if ((p0.w_scale != nullptr) != (p1.w_scale != nullptr)) return cudaErrorInvalidValue;
+  const bool empty0 = p0.M <= 0 || p0.N <= 0, empty1 = p1.M <= 0 || p1.N <= 0;
+  if (empty0 || empty1 || p0.M + p1.M < 1024 || num_sms < 2) {  // too small for pairs: one launch each
+    cudaError_t e = empty0 ? cudaSuccess : launch_gemm(p0, A0, W0, W0_rows, stream, num_sms);
+    if (e == cudaSuccess && !empty1) e = launch_gemm(p1, A1, W1, W1_rows, stream, num_sms);
+    return e;
+  }
+  CUtensorMap ta0, tb0, ta1, tb1;
+  cudaError_t e = prepare_gemm(p0, A0, W0, W0_rows, true, &ta0, &tb0);
+  if (e == cudaSuccess) e = prepare_gemm(p1, A1, W1, W1_rows, true, &ta1, &tb1);
+  if (e == cudaSuccess) e = gemm_set_attributes();
+  if (e != cudaSuccess) return e;
+  return launch_pair(p0, ta0, tb0, p1, ta1, tb1, stream, num_sms);
 }
 
 }  // namespace af

@@ -798,25 +798,32 @@ cudaError_t launch_silu_bf16(const float* x, int n, uint16_t* y, cudaStream_t s)
 }
 
 // ------------------------------------------------------------------ Euler + CFG
-__global__ void euler_cfg_kernel(float* __restrict__ x, const float* __restrict__ v, int64_t n_total,
-                                 int64_t per_sample, float g, float dt) {
+// The two halves of the velocity come as separate pointers, so the uncond
+// or the text half may live in another GPU's memory (the two-GPU CFG split
+// reads its peer's half here over NVLink, no separate exchange copy).
+__global__ void euler_cfg_kernel(float* __restrict__ x, const float* __restrict__ vu_p,
+                                 const float* __restrict__ vc_p, int64_t n_total, float g, float dt) {
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n_total;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const float vu = v[i];
-    const float vc = v[i + n_total];
-    (void)per_sample;
+    const float vu = vu_p[i];
+    const float vc = vc_p[i];
     x[i] = x[i] + dt * (vu + g * (vc - vu));
   }
+}
+
+cudaError_t launch_euler_cfg2(float* lat, const float* v_uncond, const float* v_text, int64_t n, float g, float sigma,
+                              float sigma_next, cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  int blocks = static_cast<int>((n + 255) / 256);
+  if (blocks > 4096) blocks = 4096;
+  euler_cfg_kernel<<<blocks, 256, 0, s>>>(lat, v_uncond, v_text, n, g, sigma_next - sigma);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_euler_cfg(float* lat, const float* v, int Bi, int64_t per_sample, float g, float sigma,
                              float sigma_next, cudaStream_t s) {
   const int64_t n = static_cast<int64_t>(Bi) * per_sample;
-  if (n <= 0) return cudaSuccess;
-  int blocks = static_cast<int>((n + 255) / 256);
-  if (blocks > 4096) blocks = 4096;
-  euler_cfg_kernel<<<blocks, 256, 0, s>>>(lat, v, n, per_sample, g, sigma_next - sigma);
-  return cudaGetLastError();
+  return launch_euler_cfg2(lat, v, v + n, n, g, sigma, sigma_next, s);
 }
 
 }  // namespace af

@@ -268,6 +268,40 @@ af_status af_transformer_forward(const af_weights* w, af_scratch* s, const float
 af_status af_euler_cfg_step(float* latents, const float* velocity, int Bi, int C, int H, int W,
                             float guidance, float sigma, float sigma_next, void* stream);
 
+/* ---- CFG split over two GPUs: the exchange fused into the update ---------
+ * The CFG batch [uncond; text] is two independent forwards ([ARCH] §在
+ * AuraFlowPipeline 中的实际调用), so two processes, one per GPU, can each run
+ * one half.  Each writes its half of the velocity into an exchange buffer
+ * that the other maps through CUDA IPC; af_euler_cfg_step2 then reads the
+ * local half and the peer's half straight from the peer GPU's memory (plain
+ * loads over NVLink) while it applies the guidance and the Euler step.
+ *   af_exchange_create: a device buffer of `bytes` on `device` (zeroed).
+ *   af_exchange_handle: its IPC handle (AF_IPC_HANDLE_BYTES opaque bytes), to
+ *     be sent to the peer process by any host channel.
+ *   af_exchange_open_peer: maps the peer's buffer (once per exchange).
+ *   af_exchange_ptrs: device addresses of the local and the mapped peer
+ *     buffer (peer NULL until opened).
+ * Ordering is the caller's: launch the update only after both halves of the
+ * step are complete on both GPUs (stream sync + host barrier), and do not
+ * rewrite a buffer region while the peer may still read it (two slots,
+ * alternating per step, need one barrier per step).  The current device must
+ * be the exchange's device for handle / open. */
+#define AF_IPC_HANDLE_BYTES 64
+typedef struct af_exchange af_exchange;
+af_status af_exchange_create(int device, size_t bytes, af_exchange** out);
+af_status af_exchange_handle(const af_exchange* x, void* handle);
+af_status af_exchange_open_peer(af_exchange* x, const void* peer_handle);
+af_status af_exchange_ptrs(const af_exchange* x, void** local, void** peer);
+void af_exchange_destroy(af_exchange* x);
+
+/* af_euler_cfg_step with the two halves of the velocity given apart, so
+ * either may be a mapped peer buffer ([PIPE] §AuraFlowPipeline 核心参数详解,
+ * [DEEP] §2.3):  x += (sigma_next - sigma) (vu + guidance (vc - vu)).
+ *   latents: device float[Bi, C, H, W] in/out; v_uncond, v_text: device (or
+ *   peer-mapped) float[Bi, C, H, W].  Same arithmetic as af_euler_cfg_step. */
+af_status af_euler_cfg_step2(float* latents, const float* v_uncond, const float* v_text, int Bi, int C, int H, int W,
+                             float guidance, float sigma, float sigma_next, void* stream);
+
 /* One step of the sampling loop ([ARCH] §在 AuraFlowPipeline 中的实际调用):
  * the latents are duplicated into a CFG batch [uncond; text], the forward
  * runs at model time t = sigma on the 2 Bi batch, and af_euler_cfg_step

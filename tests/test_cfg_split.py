@@ -4,7 +4,10 @@ The forward and the Euler update are the oracle's (fp64, CPU tensors) so the
 test runs without a GPU; what is checked is the split itself: which rank
 takes which half, the order of the exchanged velocities, and that both ranks
 end with the single-process result.  A swapped order would flip the sign of
-the guidance term (g = 3.5) and fail.
+the guidance term (g = 3.5) and fail.  Both exchange forms are covered: the
+all-gather, and the peer form, where a file mapped by both processes stands
+in for the IPC-mapped device buffer (handle = its path) and the slots
+alternate per step behind one barrier.
 """
 import os
 import socket
@@ -34,7 +37,32 @@ def _problem():
     return cfg, w, x0, text, O.sigma_schedule(3, 1.73), [2, 8]
 
 
-def _rank(rank, port, out_dir, use_lens):
+class _FileExchange:
+    """The exchange buffer's host stand-in: two float64 slots in a file that
+    the peer process maps (the 'IPC handle' is the file's path)."""
+
+    def __init__(self, shape, out_dir, rank):
+        self.path = os.path.join(out_dir, f"exchange{rank}.npy")
+        self.arr = np.lib.format.open_memmap(self.path, mode="w+", dtype=np.float64, shape=(2,) + tuple(shape))
+        self.peer_arr = None
+
+    def handle(self):
+        return self.path.encode()
+
+    def open_peer(self, handle):
+        self.peer_arr = np.lib.format.open_memmap(handle.decode(), mode="r")
+
+    def local(self, slot):
+        return torch.from_numpy(self.arr[slot])
+
+    def peer(self, slot):
+        return torch.from_numpy(np.array(self.peer_arr[slot]))
+
+    def synchronize(self):
+        self.arr.flush()
+
+
+def _rank(rank, port, out_dir, use_lens, exchange):
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
     dist.init_process_group("gloo", rank=rank, world_size=2)
@@ -52,10 +80,15 @@ def _rank(rank, port, out_dir, use_lens):
         def euler(lat, v, g, a, b):
             lat.copy_(torch.from_numpy(O.euler_cfg_step(lat.numpy(), v.numpy(), g, a, b)))
 
+        def euler2(lat, vu, vc, g, a, b):
+            v = np.concatenate([vu.numpy(), vc.numpy()])
+            lat.copy_(torch.from_numpy(O.euler_cfg_step(lat.numpy(), v, g, a, b)))
+
         lat = torch.from_numpy(x0.copy())
         tl = torch.tensor(lens, dtype=torch.int32) if use_lens else None
-        smp = CFGSplitSampler(None, None, lat, torch.from_numpy(text), sig, 3.5, text_len=tl,
-                              _forward=fwd, _euler=euler)
+        smp = CFGSplitSampler(None, None, lat, torch.from_numpy(text), sig, 3.5, text_len=tl, exchange=exchange,
+                              _forward=fwd, _euler=euler, _euler2=euler2,
+                              _make_exchange=lambda shape: _FileExchange(shape, out_dir, rank))
         for i in range(smp.n_steps):
             smp.step(i)
         np.save(os.path.join(out_dir, f"lat{rank}.npy"), lat.numpy())
@@ -64,9 +97,10 @@ def _rank(rank, port, out_dir, use_lens):
         dist.destroy_process_group()
 
 
+@pytest.mark.parametrize("exchange", ["peer", "nccl"])
 @pytest.mark.parametrize("use_lens", [False, True])
-def test_cfg_split_two_ranks_match_single_process(tmp_path, use_lens):
-    mp.start_processes(_rank, args=(_free_port(), str(tmp_path), use_lens), nprocs=2, start_method="spawn")
+def test_cfg_split_two_ranks_match_single_process(tmp_path, use_lens, exchange):
+    mp.start_processes(_rank, args=(_free_port(), str(tmp_path), use_lens, exchange), nprocs=2, start_method="spawn")
     cfg, w, x0, text, sig, lens = _problem()
     x = x0.copy()
     for i in range(3):
@@ -88,7 +122,8 @@ def _rank_world3(rank, port, out_dir):
     try:
         from diffusion_transformer_denoising_auraflow_b200.cfg_split import CFGSplitSampler
         try:
-            CFGSplitSampler(None, None, torch.zeros(1, 4, 8, 8), torch.zeros(2, 4, 32), [1.0, 0.0], 3.5)
+            CFGSplitSampler(None, None, torch.zeros(1, 4, 8, 8), torch.zeros(2, 4, 32), [1.0, 0.0], 3.5,
+                            exchange="nccl")
             ok = False
         except ValueError:
             ok = True
