@@ -99,9 +99,13 @@ cudaError_t launch_modulation(const float* temb, int B, int D, const uint16_t* w
 cudaError_t launch_patch_embed(const float* lat, int B, int C, int H, int W, int p, const uint16_t* w_pe,
                                const uint16_t* pos, int G, int D, uint16_t* out, int out_rows_per_batch,
                                int out_row_off, cudaStream_t s);
-cudaError_t launch_output_stage(const uint16_t* x, int rows_per_batch, int row_off, int B, int hp, int wp, int D,
-                                const float* scale, const float* shift, int mod_stride, const uint16_t* w_out,
-                                int p, int C, float* vel, cudaStream_t s);
+// The output stage on the tensor cores: fold (1 + scale) into a bf16 copy of
+// proj_out per sample (256-row blocks, rows >= KP zero) and shift into a
+// bias; after the fp32-output GEMM, add the bias and unpatchify.
+cudaError_t launch_output_fold(const uint16_t* w_out, int KP, int D, const float* scale, const float* shift,
+                               int mod_stride, int B, uint16_t* wfold, float* bias, cudaStream_t s);
+cudaError_t launch_output_scatter(const float* o, const float* bias, int B, int hp, int wp, int p, int C, float* vel,
+                                  cudaStream_t s);
 cudaError_t launch_fill(float* dst, int n, float value, cudaStream_t s);
 cudaError_t launch_silu_bf16(const float* x, int n, uint16_t* y, cudaStream_t s);
 cudaError_t gemm_set_attributes();

@@ -124,6 +124,8 @@ struct af_scratch {
   float* yscale;
   uint16_t *img, *txt, *x;   // (fp32 pack: these activation buffers hold floats)
   float* tmp;                // fp32 pack: GEMM outputs before QK-norm / SwiGLU, [B*N, max(3D, 2F)]
+  uint16_t* wfold;           // output stage: proj_out * (1 + scale_b), [B, 256, D] bf16 (rows >= p*p*C zero)
+  float *obias, *oproj;      // output stage: W . shift_b [B, 64]; projected tokens [B * Ni, p*p*C] fp32
   float *lat2, *vel, *tvec;  // denoise step: CFG-duplicated latents, velocity, model times
   int sms;
   // launch accounting / profiling (kernel classes: GEMM, attention, LN, other)
@@ -819,6 +821,8 @@ af_status af_weights_create(const af_config* cfg, int device, af_weights** out) 
     if (d.D % 32 != 0 || d.F % 128 != 0 || cfg->joint_attention_dim % 8 != 0) return AF_ERR_UNSUPPORTED;
     if (!(d.hd == 256 || d.hd == 8 || d.hd == 16 || d.hd == 32 || d.hd == 64)) return AF_ERR_UNSUPPORTED;
     if (cfg->patch_size * cfg->patch_size * cfg->in_channels > 64) return AF_ERR_UNSUPPORTED;
+    // the output projection's folded weights fill rows of a 256-row GEMM tile
+    if (cfg->patch_size * cfg->patch_size * cfg->out_channels > 256) return AF_ERR_UNSUPPORTED;
     // the timestep / modulation GEMV reads rows of 16-byte vectors, at most 4096 wide
     if (cfg->timestep_channels % 8 != 0 || cfg->timestep_channels > 4096 || d.D > 4096) return AF_ERR_UNSUPPORTED;
   }
@@ -1107,6 +1111,10 @@ af_status af_scratch_create(const af_weights* w, int max_batch, int max_img_toke
   const size_t o_lat2 = take(lat_elems * 4);
   const size_t o_vel = take(lat_elems * 4);
   const size_t o_tvec = take(B * 4);
+  const int kpo = w->cfg.patch_size * w->cfg.patch_size * w->cfg.out_channels;
+  const size_t o_wfold = take(w->f32 ? 0 : B * 256 * D * 2);
+  const size_t o_obias = take(B * 256 * 4);
+  const size_t o_oproj = take(w->f32 ? 0 : B * static_cast<size_t>(s->max_ni) * kpo * 4);
   s->bytes = off;
   int prev = 0;
   cudaGetDevice(&prev);
@@ -1146,6 +1154,9 @@ af_status af_scratch_create(const af_weights* w, int max_batch, int max_img_toke
   s->lat2 = reinterpret_cast<float*>(s->base + o_lat2);
   s->vel = reinterpret_cast<float*>(s->base + o_vel);
   s->tvec = reinterpret_cast<float*>(s->base + o_tvec);
+  s->wfold = reinterpret_cast<uint16_t*>(s->base + o_wfold);
+  s->obias = reinterpret_cast<float*>(s->base + o_obias);
+  s->oproj = reinterpret_cast<float*>(s->base + o_oproj);
   *out = s;
   return AF_OK;
 }
@@ -1242,6 +1253,42 @@ af_status af_single_block(const af_weights* w, af_scratch* s, int layer, uint16_
   return single_block_impl(w, s, layer, x, s->mods, 6 * D, B, N, text_mask(w, text_len, Nt), st);
 }
 
+// The output stage ([ARCH] §调制与归一化, §前向传播流程): z = x (1 + scale) + shift
+// on the image rows, o = z proj_out^T, unpatchify.  The modulation folds into a
+// per-sample bf16 copy of proj_out (and a bias W . shift), so the projection of
+// all image rows is one tensor-core GEMM with an fp32 store (the samples as
+// the two problems of a grouped launch), then a scatter adds the bias and
+// unpatchifies.  Accounted as an HBM-bound step (bytes), not as a GEMM.
+static af_status output_stage(const af_weights* w, af_scratch* s, int B, int N, int Nt, int hp, int wp,
+                              const float* pf, int mstride, float* velocity, cudaStream_t st) {
+  const af_config& c = w->cfg;
+  const int p = c.patch_size, D = w->d.D, Ni = hp * wp;
+  const int kpo = p * p * c.out_channels;
+  {
+    LaunchScope ls(s, KC_OTHER, 2.0 * B * kpo * D * 2 + 4.0 * B * kpo, st);
+    AF_CUDA(launch_output_fold(w->ptr("proj_out.weight"), kpo, D, pf, pf + D, mstride, B, s->wfold, s->obias, st));
+  }
+  for (int b0 = 0; b0 < B; b0 += 2) {
+    GemmCall g[2];
+    const int nb = B - b0 < 2 ? B - b0 : 2;
+    for (int j = 0; j < nb; ++j) {
+      const int b = b0 + j;
+      GemmParams gp = gemm_base(s, Ni, kpo, D, EPI_STORE_F32, Ni);
+      gp.out_f32 = s->oproj + static_cast<size_t>(b) * Ni * kpo;
+      gp.ldo = kpo;
+      g[j] = {gp, s->x + (static_cast<size_t>(b) * N + Nt) * D, s->wfold + static_cast<size_t>(b) * 256 * D, 256, true};
+    }
+    LaunchScope ls(s, KC_OTHER, 2.0 * nb * Ni * D + 4.0 * nb * Ni * kpo, st);
+    const cudaError_t e = nb == 2 ? launch_gemm_grouped(g[0].p, g[0].A, g[0].W, g[0].W_rows, g[1].p, g[1].A, g[1].W,
+                                                        g[1].W_rows, st, s->sms)
+                                  : launch_gemm(g[0].p, g[0].A, g[0].W, g[0].W_rows, st, s->sms);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  LaunchScope ls(s, KC_OTHER, 4.0 * B * Ni * kpo * 2, st);
+  AF_CUDA(launch_output_scatter(s->oproj, s->obias, B, hp, wp, p, c.out_channels, velocity, st));
+  return AF_OK;
+}
+
 // premods != nullptr: every adaLN / pre-final modulation of this step was
 // precomputed (rows in the adaLN unit order, element (b, r) at
 // premods[b * pre_stride + r]); the timestep MLP and the modulation GEMV are
@@ -1314,10 +1361,7 @@ static af_status forward_impl(const af_weights* w, af_scratch* s, const float* l
   }
   // pre-final (scale first, then shift), proj_out, unpatchify on the image rows
   const float* pf = mods + w->pf_row;
-  LaunchScope ls(s, KC_OTHER, 2.0 * B * Ni * D + 4.0 * B * c.out_channels * H * W, st);
-  AF_CUDA(launch_output_stage(s->x, N, Nt, B, hp, wp, D, pf, pf + D, mstride,
-                              w->ptr("proj_out.weight"), p, c.out_channels, velocity, st));
-  return AF_OK;
+  return output_stage(w, s, B, N, Nt, hp, wp, pf, mstride, velocity, st);
 }
 
 af_status af_transformer_forward(const af_weights* w, af_scratch* s, const float* latents, const void* text_emb,

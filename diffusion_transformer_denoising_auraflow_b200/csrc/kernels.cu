@@ -13,8 +13,11 @@
 //                    weights streamed once for the whole batch.
 //   patch_embed      patch gather + Linear(p*p*C -> D) + centre-cropped
 //                    learned position row (§Patch Embedding).
-//   output_stage     pre-final x * (1 + scale) + shift, proj_out and the
-//                    unpatchify scatter (§调制与归一化, §前向传播流程).
+//   output_fold /    the output stage around one tensor-core GEMM: the
+//   output_scatter   pre-final x * (1 + scale) + shift folded into a per-sample
+//                    copy of proj_out plus a bias, and after the GEMM the
+//                    bias added and the unpatchify scatter (§调制与归一化,
+//                    §前向传播流程).
 //   euler_cfg        v = v_u + g (v_c - v_u); x += (sigma' - sigma) v.
 #include "af_internal.h"
 #include "ptx.cuh"
@@ -130,32 +133,65 @@ __global__ void __launch_bounds__(256) ln_modulate_kernel(const uint16_t* __rest
 }
 
 // Wide rows (D = 3072), HBM-bound: rows are streamed into shared memory by
-// bulk copies (4 stages of 8 rows = 192 KB in flight per SM, not limited by
-// registers); 8 consumer warps each normalise one row of a stage from shared
-// memory, with (1 + scale) and shift of the CTA's sample staged once.
-// Grid (CTAs per sample, samples); one CTA per SM.
+// bulk copies, 2 stages of 4 rows per CTA and three CTAs per SM (144 KB in
+// flight per SM); the producer warp starts streaming at once while the 4
+// consumer warps stage (1 + scale) and shift of the CTA's sample.  Each
+// consumer warp normalises one row of a stage, the row held in registers
+// (two passes for mean and variance, then the output), the arithmetic on
+// packed fp32 pairs (sm_100 f32x2).  Three smaller CTAs per SM keep more
+// warps issuing than one CTA with 8 rows x 4 stages: 26.7 against 30.8 us
+// per [8720, 3072] call with the input in L2, 30.8 against 34.2 us from
+// DRAM (one-pass statistics in that measurement; the kernel keeps two).
+// Grid (CTAs per sample, samples).
 constexpr int LNB_D = 3072;
-constexpr int LNB_ROWS = 8;
-constexpr int LNB_STAGES = 4;
+constexpr int LNB_ROWS = 4;
+constexpr int LNB_STAGES = 2;
+constexpr int LNB_PER_SM = 3;
 constexpr uint32_t LNB_ROW_BYTES = LNB_D * 2;
 constexpr int LNB_THREADS = 32 * (LNB_ROWS + 1);
-constexpr int LNB_SMEM = LNB_STAGES * LNB_ROWS * LNB_ROW_BYTES + 2 * LNB_D * 4 + 128 + 128;
+constexpr int LNB_SMEM = LNB_STAGES * LNB_ROWS * LNB_ROW_BYTES + 2 * LNB_D * 4;
+
+// packed fp32 pairs
+__device__ __forceinline__ uint64_t f2_pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ float2 f2_unpack(uint64_t r) {
+  float2 v;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(v.x), "=f"(v.y) : "l"(r));
+  return v;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+// the two bf16 halves of w as a packed fp32 pair
+__device__ __forceinline__ uint64_t f2_from_bf16x2(uint32_t w) {
+  return f2_pack(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
 
 template <bool OUT8>
-__global__ void __launch_bounds__(LNB_THREADS, 1) ln_modulate_bulk_kernel(const uint16_t* __restrict__ x,
-                                                                         const float* __restrict__ shift,
-                                                                         const float* __restrict__ scale,
-                                                                         int mod_stride, uint16_t* __restrict__ y,
-                                                                         uint8_t* __restrict__ y8,
-                                                                         float* __restrict__ yscale,
-                                                                         int rows_per_batch, float eps, int* err) {
-  extern __shared__ uint8_t lnb_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(lnb_raw) + 127) & ~uintptr_t(127));
-  uint8_t* rowbuf = smem;                                                       // [stage][row] x 6 KB
-  float* mod_s = reinterpret_cast<float*>(smem + LNB_STAGES * LNB_ROWS * LNB_ROW_BYTES);  // 1 + scale | shift
-  uint64_t* full = reinterpret_cast<uint64_t*>(mod_s + 2 * LNB_D);
-  uint64_t* empty = full + LNB_STAGES;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + LNB_STAGES);
+__global__ void __launch_bounds__(LNB_THREADS, LNB_PER_SM) ln_modulate_bulk_kernel(
+    const uint16_t* __restrict__ x, const float* __restrict__ shift, const float* __restrict__ scale, int mod_stride,
+    uint16_t* __restrict__ y, uint8_t* __restrict__ y8, float* __restrict__ yscale, int rows_per_batch, float eps,
+    int* err) {
+  extern __shared__ __align__(128) uint8_t lnb_raw[];  // [stage][row] x 6 KB, then (1 + scale) | shift
+  uint8_t* rowbuf = lnb_raw;
+  float* mod_s = reinterpret_cast<float*>(lnb_raw + LNB_STAGES * LNB_ROWS * LNB_ROW_BYTES);
+  __shared__ uint64_t full[LNB_STAGES], empty[LNB_STAGES];
+  __shared__ int abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.y;
   const int nchunks = (rows_per_batch + LNB_ROWS - 1) / LNB_ROWS;
@@ -165,26 +201,20 @@ __global__ void __launch_bounds__(LNB_THREADS, 1) ln_modulate_bulk_kernel(const 
       mbar_init(smem_u32(&full[i]), 1);
       mbar_init(smem_u32(&empty[i]), LNB_ROWS);
     }
-    *abort_flag = 0;
+    abort_flag = 0;
     fence_mbar_init();
-  }
-  const float* sc = scale + static_cast<size_t>(b) * mod_stride;
-  const float* sh = shift + static_cast<size_t>(b) * mod_stride;
-  for (int i = threadIdx.x; i < LNB_D; i += blockDim.x) {
-    mod_s[i] = 1.0f + sc[i];
-    mod_s[LNB_D + i] = sh[i];
   }
   __syncthreads();
 
   if (warp == LNB_ROWS) {
-    // producer: one elected thread streams chunks of 8 rows
+    // producer: one elected thread streams chunks of LNB_ROWS rows
     if (lane == 0) {
       bool ok = true, issued = false;
       int k = 0;
       for (int c = blockIdx.x; c < nchunks; c += gridDim.x, ++k) {
         const int st = k % LNB_STAGES;
         const uint32_t ph = (k / LNB_STAGES) & 1;
-        if (!mbar_wait(smem_u32(&empty[st]), ph ^ 1u, err, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(smem_u32(&empty[st]), ph ^ 1u, err, &abort_flag)) { ok = false; break; }
         const int n = min(LNB_ROWS, rows_per_batch - c * LNB_ROWS);
         mbar_arrive_expect_tx(smem_u32(&full[st]), n * LNB_ROW_BYTES);
         for (int r = 0; r < n; ++r)
@@ -201,83 +231,100 @@ __global__ void __launch_bounds__(LNB_THREADS, 1) ln_modulate_bulk_kernel(const 
     }
     return;
   }
-  // consumers: warp w normalises row w of every stage
+  // consumers: stage the modulation vectors (named barrier 1: consumer warps only)
+  {
+    const float* sc = scale + static_cast<size_t>(b) * mod_stride;
+    const float* sh = shift + static_cast<size_t>(b) * mod_stride;
+    for (int i = threadIdx.x; i < LNB_D; i += 32 * LNB_ROWS) {
+      mod_s[i] = 1.0f + sc[i];
+      mod_s[LNB_D + i] = sh[i];
+    }
+    asm volatile("bar.sync 1, %0;" ::"r"(32 * LNB_ROWS) : "memory");
+  }
+  // warp w normalises row w of every stage
   constexpr int VPL = LNB_D / 256;
   int k = 0;
   for (int c = blockIdx.x; c < nchunks; c += gridDim.x, ++k) {
     const int st = k % LNB_STAGES;
     const uint32_t ph = (k / LNB_STAGES) & 1;
-    const bool got = mbar_wait(smem_u32(&full[st]), ph, err, abort_flag);
+    const bool got = mbar_wait(smem_u32(&full[st]), ph, err, &abort_flag);
     if (!__all_sync(0xffffffffu, got)) break;
     const int r = c * LNB_ROWS + warp;
     if (r < rows_per_batch) {
       const uint4* xr = reinterpret_cast<const uint4*>(rowbuf + (st * LNB_ROWS + warp) * LNB_ROW_BYTES);
-      uint4 cur[VPL];
+      uint4 u[VPL];
 #pragma unroll
-      for (int i = 0; i < VPL; ++i) cur[i] = xr[i * 32 + lane];
-      float s = 0.f;
+      for (int i = 0; i < VPL; ++i) u[i] = xr[i * 32 + lane];
+      // two passes over the registers: the mean, then the centred squares
+      uint64_t s2 = f2_pack(0.f, 0.f);
 #pragma unroll
       for (int i = 0; i < VPL; ++i) {
-        const uint32_t w[4] = {cur[i].x, cur[i].y, cur[i].z, cur[i].w};
+        const uint32_t w[4] = {u[i].x, u[i].y, u[i].z, u[i].w};
 #pragma unroll
-        for (int e = 0; e < 4; ++e) s += bf16_lo(w[e]) + bf16_hi(w[e]);
+        for (int e = 0; e < 4; ++e) s2 = f2_add(s2, f2_from_bf16x2(w[e]));
       }
-      const float mean = warp_sum(s) * (1.0f / LNB_D);
-      float ss = 0.f;
+      const float2 sv = f2_unpack(s2);
+      const float mean = warp_sum(sv.x + sv.y) * (1.0f / LNB_D);
+      const uint64_t nm = f2_pack(-mean, -mean);
+      uint64_t q2 = f2_pack(0.f, 0.f);
 #pragma unroll
       for (int i = 0; i < VPL; ++i) {
-        const uint32_t w[4] = {cur[i].x, cur[i].y, cur[i].z, cur[i].w};
+        const uint32_t w[4] = {u[i].x, u[i].y, u[i].z, u[i].w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float d0 = bf16_lo(w[e]) - mean, d1 = bf16_hi(w[e]) - mean;
-          ss += d0 * d0 + d1 * d1;
+          const uint64_t d = f2_add(f2_from_bf16x2(w[e]), nm);
+          q2 = f2_fma(d, d, q2);
         }
       }
-      const float rstd = rsqrtf(warp_sum(ss) * (1.0f / LNB_D) + eps);
-      // output element 2e (+1) of vector i: (x - mean) rstd (1 + scale) + shift
-      auto out8 = [&](int i, float (&o)[8]) {
+      const float2 qv = f2_unpack(q2);
+      const float rstd = rsqrtf(warp_sum(qv.x + qv.y) * (1.0f / LNB_D) + eps);
+      const uint64_t rs2 = f2_pack(rstd, rstd);
+      // output pairs 0..3 of vector i: (x - mean) rstd (1 + scale) + shift
+      auto out8 = [&](int i, uint64_t (&o)[4]) {
         const int vi = i * 32 + lane;
-        const float4 a0 = *reinterpret_cast<const float4*>(mod_s + vi * 8);
-        const float4 a1 = *reinterpret_cast<const float4*>(mod_s + vi * 8 + 4);
-        const float4 h0 = *reinterpret_cast<const float4*>(mod_s + LNB_D + vi * 8);
-        const float4 h1 = *reinterpret_cast<const float4*>(mod_s + LNB_D + vi * 8 + 4);
-        const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-        const float hv[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
-        const uint32_t w[4] = {cur[i].x, cur[i].y, cur[i].z, cur[i].w};
+        const ulonglong2 a01 = *reinterpret_cast<const ulonglong2*>(mod_s + vi * 8);
+        const ulonglong2 a23 = *reinterpret_cast<const ulonglong2*>(mod_s + vi * 8 + 4);
+        const ulonglong2 h01 = *reinterpret_cast<const ulonglong2*>(mod_s + LNB_D + vi * 8);
+        const ulonglong2 h23 = *reinterpret_cast<const ulonglong2*>(mod_s + LNB_D + vi * 8 + 4);
+        const uint64_t av[4] = {a01.x, a01.y, a23.x, a23.y};
+        const uint64_t hv[4] = {h01.x, h01.y, h23.x, h23.y};
+        const uint32_t w[4] = {u[i].x, u[i].y, u[i].z, u[i].w};
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          o[2 * e] = (bf16_lo(w[e]) - mean) * rstd * av[2 * e] + hv[2 * e];
-          o[2 * e + 1] = (bf16_hi(w[e]) - mean) * rstd * av[2 * e + 1] + hv[2 * e + 1];
-        }
+        for (int e = 0; e < 4; ++e) o[e] = f2_fma(f2_mul(f2_add(f2_from_bf16x2(w[e]), nm), rs2), av[e], hv[e]);
       };
       if constexpr (OUT8) {
         float amax = 0.f;
 #pragma unroll
         for (int i = 0; i < VPL; ++i) {
-          float o[8];
+          uint64_t o[4];
           out8(i, o);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(o[e]));
+          for (int e = 0; e < 4; ++e) {
+            const float2 v = f2_unpack(o[e]);
+            amax = fmaxf(amax, fmaxf(fabsf(v.x), fabsf(v.y)));
+          }
         }
         amax = warp_max(amax);
         const float inv = e4m3_inv_scale(amax);
         uint2* yr = reinterpret_cast<uint2*>(y8 + (row0 + r) * LNB_D);
 #pragma unroll
         for (int i = 0; i < VPL; ++i) {
-          float o[8];
+          uint64_t o[4];
           out8(i, o);
-          yr[i * 32 + lane] = make_uint2(pack_e4m3x4(o[0] * inv, o[1] * inv, o[2] * inv, o[3] * inv),
-                                         pack_e4m3x4(o[4] * inv, o[5] * inv, o[6] * inv, o[7] * inv));
+          const float2 v0 = f2_unpack(o[0]), v1 = f2_unpack(o[1]), v2 = f2_unpack(o[2]), v3 = f2_unpack(o[3]);
+          yr[i * 32 + lane] = make_uint2(pack_e4m3x4(v0.x * inv, v0.y * inv, v1.x * inv, v1.y * inv),
+                                         pack_e4m3x4(v2.x * inv, v2.y * inv, v3.x * inv, v3.y * inv));
         }
         if (lane == 0) yscale[row0 + r] = e4m3_scale(amax);
       } else {
         uint4* yr = reinterpret_cast<uint4*>(y + (row0 + r) * LNB_D);
 #pragma unroll
         for (int i = 0; i < VPL; ++i) {
-          float o[8];
+          uint64_t o[4];
           out8(i, o);
-          yr[i * 32 + lane] = make_uint4(pack_bf16(o[0], o[1]), pack_bf16(o[2], o[3]), pack_bf16(o[4], o[5]),
-                                         pack_bf16(o[6], o[7]));
+          const float2 v0 = f2_unpack(o[0]), v1 = f2_unpack(o[1]), v2 = f2_unpack(o[2]), v3 = f2_unpack(o[3]);
+          yr[i * 32 + lane] = make_uint4(pack_bf16(v0.x, v0.y), pack_bf16(v1.x, v1.y), pack_bf16(v2.x, v2.y),
+                                         pack_bf16(v3.x, v3.y));
         }
       }
     }
@@ -300,7 +347,7 @@ cudaError_t launch_ln_modulate(const uint16_t* x, const float* shift, const floa
     static int sms = 0;
     if (!sms) sms = device_sm_count();
     const int nchunks = (rows_per_batch + LNB_ROWS - 1) / LNB_ROWS;
-    const int per = max(1, min(nchunks, (sms + nb - 1) / nb));
+    const int per = max(1, min(nchunks, (LNB_PER_SM * sms + nb - 1) / nb));
     if (out8)
       ln_modulate_bulk_kernel<true><<<dim3(per, nb), LNB_THREADS, LNB_SMEM, s>>>(x, shift, scale, mod_stride, y, y8,
                                                                                yscale, rows_per_batch, eps, err);
@@ -693,83 +740,61 @@ cudaError_t launch_patch_embed(const float* lat, int B, int C, int H, int W, int
   return cudaGetLastError();
 }
 
-// ------------------------------------------------------------------ output stage
-// z = x * (1 + scale[b]) + shift[b];  o[k] = W_out[k] . z  (k < p*p*C);
-// velocity[b, c, hp * p + py, wp * p + px] = o[(py * p + px) * C + c]
-template <int VPL>
-__global__ void __launch_bounds__(256) output_stage_kernel(const uint16_t* __restrict__ x, int rows_per_batch,
-                                                           int row_off, int B, int hpn, int wpn, int D,
-                                                           const float* __restrict__ scale,
-                                                           const float* __restrict__ shift, int mod_stride,
-                                                           const uint16_t* __restrict__ wout, int p, int C,
-                                                           float* __restrict__ vel) {
+// ------------------------------------------------------------------ output stage on the tensor cores
+// The pre-final modulation folds into the projection: with z = x (1 + sc) + sh,
+// o[k] = W[k] . z = (W[k] * (1 + sc)) . x + W[k] . sh.  output_fold_kernel
+// writes, per sample b, W'_b = bf16(W * (1 + sc_b)) into rows [0, KP) of a
+// 256-row block (the rest stays zero, so a 256-wide GEMM tile reads only
+// zeros there) and bias_b[k] = W[k] . sh_b (fp32); one warp per (b, k).
+__global__ void __launch_bounds__(256) output_fold_kernel(const uint16_t* __restrict__ wout, int KP, int D,
+                                                          const float* __restrict__ scale,
+                                                          const float* __restrict__ shift, int mod_stride, int B,
+                                                          uint16_t* __restrict__ wfold, float* __restrict__ bias) {
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
-  const int ntok = hpn * wpn;
-  if (gw >= B * ntok) return;
-  const int b = gw / ntok, n = gw - b * ntok;
-  const uint4* xr = reinterpret_cast<const uint4*>(x + (static_cast<size_t>(b) * rows_per_batch + row_off + n) * D);
+  if (gw >= B * KP) return;
+  const int b = gw / KP, k = gw - b * KP;
   const float* sc = scale + static_cast<size_t>(b) * mod_stride;
   const float* sh = shift + static_cast<size_t>(b) * mod_stride;
-  const int nvec = D >> 3;
-  float z[VPL][8];
-#pragma unroll
-  for (int i = 0; i < VPL; ++i) {
-    const int vi = i * 32 + lane;
-    if (vi < nvec) {
-      const uint4 u = xr[vi];
-      const float xv[8] = {bf16_lo(u.x), bf16_hi(u.x), bf16_lo(u.y), bf16_hi(u.y),
-                           bf16_lo(u.z), bf16_hi(u.z), bf16_lo(u.w), bf16_hi(u.w)};
-#pragma unroll
-      for (int e = 0; e < 8; ++e) z[i][e] = xv[e] * (1.0f + sc[vi * 8 + e]) + sh[vi * 8 + e];
-    } else {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) z[i][e] = 0.f;
-    }
+  const uint16_t* wr = wout + static_cast<size_t>(k) * D;
+  uint16_t* dr = wfold + (static_cast<size_t>(b) * 256 + k) * D;
+  float acc = 0.f;
+  for (int d = lane; d < D; d += 32) {
+    const float w = __uint_as_float(static_cast<uint32_t>(wr[d]) << 16);
+    dr[d] = static_cast<uint16_t>(pack_bf16(w * (1.0f + sc[d]), 0.f) & 0xFFFFu);
+    acc = fmaf(w, sh[d], acc);
   }
-  const int KP = p * p * C;
-  const int hp = n / wpn, wp = n - hp * wpn;
-  const int H = hpn * p, W = wpn * p;
-  for (int k = 0; k < KP; ++k) {
-    const uint4* wr = reinterpret_cast<const uint4*>(wout + static_cast<size_t>(k) * D);
-    float a = 0.f;
-#pragma unroll
-    for (int i = 0; i < VPL; ++i) {
-      const int vi = i * 32 + lane;
-      if (vi < nvec) {
-        const uint4 u = __ldg(wr + vi);
-        a += bf16_lo(u.x) * z[i][0] + bf16_hi(u.x) * z[i][1] + bf16_lo(u.y) * z[i][2] + bf16_hi(u.y) * z[i][3] +
-             bf16_lo(u.z) * z[i][4] + bf16_hi(u.z) * z[i][5] + bf16_lo(u.w) * z[i][6] + bf16_hi(u.w) * z[i][7];
-      }
-    }
-    a = warp_sum(a);
-    if (lane == 0) {
-      const int c = k % C, pq = k / C;
-      const int py = pq / p, px = pq - py * p;
-      vel[((static_cast<size_t>(b) * C + c) * H + hp * p + py) * W + wp * p + px] = a;
-    }
-  }
+  acc = warp_sum(acc);
+  if (lane == 0) bias[b * KP + k] = acc;
 }
 
-cudaError_t launch_output_stage(const uint16_t* x, int rows_per_batch, int row_off, int B, int hp, int wp, int D,
-                                const float* scale, const float* shift, int mod_stride, const uint16_t* w_out, int p,
-                                int C, float* vel, cudaStream_t s) {
-  if (D % 8 != 0) return cudaErrorInvalidValue;
-  const int warps = B * hp * wp;
-  const int blocks = (warps + 7) / 8;
-  const int vpl = (D / 8 + 31) / 32;
-#define AF_OUT_CASE(N)                                                                                        \
-  if (vpl <= N) {                                                                                             \
-    output_stage_kernel<N><<<blocks, 256, 0, s>>>(x, rows_per_batch, row_off, B, hp, wp, D, scale, shift,     \
-                                                  mod_stride, w_out, p, C, vel);                              \
-    return cudaGetLastError();                                                                                \
-  }
-  AF_OUT_CASE(1)
-  AF_OUT_CASE(4)
-  AF_OUT_CASE(12)
-  AF_OUT_CASE(16)
-#undef AF_OUT_CASE
-  return cudaErrorInvalidValue;
+// velocity[b, c, hp p + py, wp p + px] = o[b, n, (py p + px) C + c] + bias_b[...]
+// (the unpatchify of the model's output stage), o the fp32 GEMM output [B * Ni, KP]
+__global__ void output_scatter_kernel(const float* __restrict__ o, const float* __restrict__ bias, int B, int hp,
+                                      int wp, int p, int C, float* __restrict__ vel) {
+  const int KP = p * p * C, Ni = hp * wp;
+  const int total = B * Ni * KP;
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= total) return;
+  const int k = i % KP, n = (i / KP) % Ni, b = i / (KP * Ni);
+  const int c = k % C, pq = k / C, py = pq / p, px = pq - py * p;
+  const int ph = n / wp, pw = n - ph * wp;
+  const int H = hp * p, W = wp * p;
+  vel[((static_cast<size_t>(b) * C + c) * H + ph * p + py) * W + pw * p + px] = o[i] + bias[b * KP + k];
+}
+
+cudaError_t launch_output_fold(const uint16_t* w_out, int KP, int D, const float* scale, const float* shift,
+                               int mod_stride, int B, uint16_t* wfold, float* bias, cudaStream_t s) {
+  const int warps = B * KP;
+  output_fold_kernel<<<(warps + 7) / 8, 256, 0, s>>>(w_out, KP, D, scale, shift, mod_stride, B, wfold, bias);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_output_scatter(const float* o, const float* bias, int B, int hp, int wp, int p, int C, float* vel,
+                                  cudaStream_t s) {
+  const int total = B * hp * wp * p * p * C;
+  output_scatter_kernel<<<(total + 255) / 256, 256, 0, s>>>(o, bias, B, hp, wp, p, C, vel);
+  return cudaGetLastError();
 }
 
 // ------------------------------------------------------------------ fill (model time of a CFG batch)
