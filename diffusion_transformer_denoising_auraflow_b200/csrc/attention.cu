@@ -1015,6 +1015,351 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
   }
 }
 
+// ---------------------------------------------------------------- three K/V stages, four softmax warpgroups
+// attn_hd256_qknorm_pair3: the same computation and cluster layout as
+// attn_hd256_qknorm_pair, arranged for a shorter period per 128-key tile.
+// Two limits each hold the two-stage layout near 2700 cycles per tile
+// against 2048 cycles of MMA work: (a) the K / V stream -- a stage is
+// refilled only when the MMA that read it completes, so with two stages a
+// load has 2T - 1024 cycles to land and a ~4400-cycle load needs
+// T >= 2700 -- and (b) the S -> softmax -> P chain.  Here K and V have three
+// stages each (T >= (1024 + L) / 3), and four softmax warpgroups per CTA
+// (16 warps; warpgroup g owns keys [32 g, 32 g + 32) of every S tile) halve
+// each thread's exponentials per tile.  The shared memory for the third
+// stages comes from using one P buffer: the softmax of tile j + 1 stores its
+// P only after PV_j completes, which the tensor core overlaps with S_{j+2}.
+// The Q tile lands in V stages 0 and 1; the softmax warps move it to TMEM
+// and release those stages (q_moved) before the first V loads.  Shared
+// memory per CTA: P 32 KB, K 3 x 32 KB, V 3 x 32 KB (the row sums reuse the
+// P buffer once the last PV has read it).
+constexpr int AP3_NWG = 4;
+constexpr int AP3_SM_WARPS = 4 * AP3_NWG;
+constexpr int AP3_V_WARP = 2 + AP3_SM_WARPS;
+constexpr int AP3_THREADS = 32 * (AP3_V_WARP + 1);
+constexpr int AP3_KPW = AP_BN / AP3_NWG;   // 32 keys per warpgroup
+constexpr int AP3_STAGES = 3;
+constexpr int AP3_SMEM = AP_P_BYTES + AP3_STAGES * AP_KH_BYTES + AP3_STAGES * AP_VH_BYTES + 256 + 1024;
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AP3_THREADS, 1)
+    attn_hd256_qknorm_pair3(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                            const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sP = smem;                                    // one P buffer (row sums at the end)
+  uint8_t* sK = sP + AP_P_BYTES;                         // AP3_STAGES buffers
+  uint8_t* sV = sK + AP3_STAGES * AP_KH_BYTES;           // AP3_STAGES buffers; the Q tile first (stages 0, 1)
+  float* xsum = reinterpret_cast<float*>(sP);            // [wg 4][row 128], after the last PV
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + AP3_STAGES * AP_VH_BYTES);
+  uint64_t* q_smem = bars + 0;                 // per CTA: this CTA's Q tile has landed
+  uint64_t* k_full = bars + 1;                 // [3] leader: both K halves
+  uint64_t* v_full = bars + 4;                 // [3] leader: both V halves
+  uint64_t* k_empty = bars + 7;                // [3] both CTAs (multicast commit)
+  uint64_t* v_empty = bars + 10;               // [3] both CTAs
+  uint64_t* s_full = bars + 13;                // both CTAs
+  uint64_t* s_empty = bars + 14;               // leader: softmax warps of both CTAs
+  uint64_t* p_full = bars + 15;                // leader: softmax warps of both CTAs
+  uint64_t* pv_done = bars + 16;               // both CTAs
+  uint64_t* q_tmem = bars + 17;                // leader: softmax warps of both CTAs have moved Q to TMEM
+  uint64_t* q_moved = bars + 18;               // per CTA: this CTA's Q copy is done (V stages 0, 1 free)
+  uint64_t* mma_done = bars + 19;              // leader
+  uint64_t* lbar = bars + 20;                  // per CTA: row sums written
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 21);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int bh = b * p.H + h;
+  const int q0 = pair * 256 + static_cast<int>(rank) * 128;
+  const int nkv = (p.N + AP_BN - 1) / AP_BN;
+  const int kv0 = static_cast<int>((static_cast<long long>(pair) * nkv) / npairs);
+  auto kv_tile = [&](int j) { const int t = j + kv0; return t < nkv ? t : t - nkv; };
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(q_smem), 1);
+    for (int i = 0; i < AP3_STAGES; ++i) {
+      mbar_init(smem_u32(&k_full[i]), 1);
+      mbar_init(smem_u32(&v_full[i]), 1);
+      mbar_init(smem_u32(&k_empty[i]), 1);
+      mbar_init(smem_u32(&v_empty[i]), 1);
+    }
+    mbar_init(smem_u32(s_full), 1);
+    mbar_init(smem_u32(s_empty), 2 * AP3_SM_WARPS);
+    mbar_init(smem_u32(p_full), 2 * AP3_SM_WARPS);
+    mbar_init(smem_u32(pv_done), 1);
+    mbar_init(smem_u32(q_tmem), 2 * AP3_SM_WARPS);
+    mbar_init(smem_u32(q_moved), AP3_SM_WARPS);
+    mbar_init(smem_u32(mma_done), 1);
+    mbar_init(smem_u32(lbar), AP3_SM_WARPS);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(tmem_slot), 512);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tO = tmem;
+  const uint32_t tS = tmem + 256;
+  const uint32_t tQ = tmem + 384;
+  volatile int never = 0;
+
+  if (warp == 0 || warp == AP3_V_WARP) {
+    // warp 0: this CTA's Q tile (into V stages 0 and 1), then the K halves
+    // (keys [64 rank, +64) of each tile); last warp: the V halves (head-dim
+    // columns [128 rank, +128)), V stages 0 and 1 only once Q has left them.
+    if (lane == 0) {
+      const bool is_k = warp == 0;
+      uint64_t* full = is_k ? k_full : v_full;
+      uint64_t* empty = is_k ? k_empty : v_empty;
+      const uint32_t half = is_k ? AP_KH_BYTES : AP_VH_BYTES;
+      uint8_t* buf = is_k ? sK : sV;
+      bool ok = true, issued = false;
+      if (is_k) {
+        mbar_arrive_expect_tx(smem_u32(q_smem), 2 * AP_P_BYTES);
+        for (int c = 0; c < 4; ++c)
+          tma_load_3d(smem_u32(sV + c * (128 * 128)), &tmQ, smem_u32(q_smem), c * 64, q0, bh);
+        issued = true;
+      } else {
+        ok = mbar_wait(smem_u32(q_moved), 0, p.err, abort_flag);
+      }
+      for (int j = 0; j < nkv && ok; ++j) {
+        const int s = j % AP3_STAGES;
+        const uint32_t ph = (j / AP3_STAGES) & 1;
+        if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1u, p.err, abort_flag)) { ok = false; break; }
+        if (leader) mbar_arrive_expect_tx(smem_u32(&full[s]), 2 * half);
+        const uint32_t fb = mapa_shared(smem_u32(&full[s]), 0);
+        const int key0 = kv_tile(j) * AP_BN;
+        if (is_k) {
+          for (int c = 0; c < 4; ++c)
+            tma_load_3d_pair(smem_u32(buf + s * half + c * (64 * 128)), &tmK, fb, c * 64,
+                             key0 + static_cast<int>(rank) * 64, bh);
+        } else {
+          for (int c = 0; c < 2; ++c)
+            tma_load_3d_pair(smem_u32(buf + s * half + c * (AP_BN * 128)), &tmV, fb,
+                             static_cast<int>(rank) * 128 + c * 64, key0, bh);
+        }
+        issued = true;
+      }
+      if (!ok && issued) {
+        const uint64_t t0 = globaltimer();
+        while (globaltimer() - t0 < 200000ull) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      const uint32_t idesc_qk = make_idesc_bf16(256, AP_BN, false, false);
+      const uint32_t idesc_pv = make_idesc_bf16(256, AT_HD, false, true);
+      bool ok = mbar_wait(smem_u32(q_tmem), 0, p.err, abort_flag);
+      // S_j into the single S buffer: the K half of tile j has landed and the
+      // softmax warps of both CTAs have read S_{j-1}.
+      auto issue_s = [&](int j) -> bool {
+        const int s = j % AP3_STAGES;
+        if (!mbar_wait(smem_u32(&k_full[s]), (j / AP3_STAGES) & 1, p.err, abort_flag)) return false;
+        if (j > 0 && !mbar_wait(smem_u32(s_empty), (j - 1) & 1, p.err, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t kaddr = smem_u32(sK + s * AP_KH_BYTES);
+        const uint64_t kdesc = make_sdesc(kaddr, 16, 1024, SWZ_128B);
+#pragma unroll
+        for (int kk = 0; kk < AT_HD / 16; ++kk) {
+          const uint32_t c = kk >> 2, off = (kk & 3) * 32;
+          const uint64_t bd = kdesc + static_cast<uint64_t>((c * (64 * 128) + off) >> 4);
+          mma_bf16_ts_pair(tS, tQ + kk * 8, bd, idesc_qk, kk > 0 ? 1u : 0u);
+        }
+        mma_commit_pair(smem_u32(s_full), 0x3);
+        mma_commit_pair(smem_u32(&k_empty[s]), 0x3);
+        return true;
+      };
+      if (ok) ok = issue_s(0);
+      const uint64_t pdesc = make_sdesc(smem_u32(sP), 16, 1024, SWZ_128B);
+      for (int j = 0; j < nkv && ok; ++j) {
+        const int s = j % AP3_STAGES;
+        if (j + 1 < nkv && !issue_s(j + 1)) { ok = false; break; }
+        if (!mbar_wait(smem_u32(p_full), j & 1, p.err, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(smem_u32(&v_full[s]), (j / AP3_STAGES) & 1, p.err, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint64_t vdesc = make_sdesc(smem_u32(sV + s * AP_VH_BYTES), AP_BN * 128, 1024, SWZ_128B);
+#pragma unroll
+        for (int kk = 0; kk < AP_BN / 16; ++kk) {
+          const uint32_t c = kk >> 2, off = (kk & 3) * 32;
+          const uint64_t ad = pdesc + static_cast<uint64_t>((c * (128 * 128) + off) >> 4);
+          const uint64_t bd = vdesc + static_cast<uint64_t>((kk * (16 * 128)) >> 4);
+          mma_bf16_ss_pair(tO, ad, bd, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit_pair(smem_u32(pv_done), 0x3);
+        mma_commit_pair(smem_u32(&v_empty[s]), 0x3);
+      }
+      mma_commit_pair(smem_u32(mma_done), 0x1);
+      mbar_wait(smem_u32(mma_done), 0, nullptr, &never, 100000000ull);
+    }
+  } else {
+    // ---------------------------------------------------------------- softmax: group g owns keys [32 g, 32 g + 32)
+    const int wg = (warp - 2) >> 2;
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const int g64 = wg >> 1;                  // 64-key chunk of a P row this group writes
+    const int u0 = (wg & 1) * 4;              // its first 16-byte unit in that chunk
+    const float c = p.scale_log2;
+    const float off = -QKN_OFFSET_LOG2;
+    int klo, khi;
+    key_mask_range(p, b, klo, khi);
+    const uint32_t s_empty_l = mapa_shared(smem_u32(s_empty), 0);
+    const uint32_t p_full_l = mapa_shared(smem_u32(p_full), 0);
+    float l = 0.f;
+    bool ok = true;
+    {
+      // Q chunk wg (head-dim columns [64 wg, +64)) of this warp's 32 rows,
+      // from V stage wg / 2 into TMEM columns [32 wg, +32); then V stages 0
+      // and 1 are released to the V loads
+      const bool got = mbar_wait(smem_u32(q_smem), 0, p.err, abort_flag);
+      __syncwarp();
+      if (!__all_sync(0xffffffffu, got)) {
+        ok = false;
+      } else {
+        const uint8_t* qrow = sV + wg * (128 * 128) + row * 128;
+        uint32_t qv[32];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const uint4 u = *reinterpret_cast<const uint4*>(qrow + ((q ^ (row & 7)) << 4));
+          qv[4 * q] = u.x;
+          qv[4 * q + 1] = u.y;
+          qv[4 * q + 2] = u.z;
+          qv[4 * q + 3] = u.w;
+        }
+        tmem_st32(tQ + wg * 32 + lane_off, qv);
+        tmem_wait_st();
+        tc_fence_before();
+        fence_proxy_async_smem();   // the generic reads of Q precede the V loads into the same bytes
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive_cluster(mapa_shared(smem_u32(q_tmem), 0));
+          mbar_arrive(smem_u32(q_moved));
+        }
+      }
+    }
+    for (int j = 0; j < nkv && ok; ++j) {
+      const bool got = mbar_wait(smem_u32(s_full), j & 1, p.err, abort_flag);
+      __syncwarp();
+      if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t r[32];
+      tmem_ld32(tS + AP3_KPW * wg + lane_off, r);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(s_empty_l);
+      const int kbase = kv_tile(j) * AP_BN + AP3_KPW * wg;
+      const int kvalid = p.N - kbase, mlo = klo - kbase, mhi = khi - kbase;
+      const bool partial = kvalid < AP3_KPW || (mlo < mhi && mlo < AP3_KPW && mhi > 0);
+      auto dead = [&](int i) { return i >= kvalid || (i >= mlo && i < mhi); };
+      uint32_t pk[16];
+      float rs0 = 0.f, rs1 = 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float e0 = ex2_approx(fmaf(__uint_as_float(r[2 * i]), c, off));
+        float e1 = ex2_approx(fmaf(__uint_as_float(r[2 * i + 1]), c, off));
+        float e2 = ex2_approx(fmaf(__uint_as_float(r[16 + 2 * i]), c, off));
+        float e3 = ex2_approx(fmaf(__uint_as_float(r[16 + 2 * i + 1]), c, off));
+        if (partial) {
+          if (dead(2 * i)) e0 = 0.f;
+          if (dead(2 * i + 1)) e1 = 0.f;
+          if (dead(16 + 2 * i)) e2 = 0.f;
+          if (dead(16 + 2 * i + 1)) e3 = 0.f;
+        }
+        rs0 += e0 + e1;
+        rs1 += e2 + e3;
+        pk[i] = pack_bf16(e0, e1);
+        pk[8 + i] = pack_bf16(e2, e3);
+      }
+      l += rs0 + rs1;
+      // the single P buffer is free once PV_{j-1} has completed
+      if (j >= 1) {
+        const bool g2 = mbar_wait(smem_u32(pv_done), (j - 1) & 1, p.err, abort_flag);
+        __syncwarp();
+        if (!__all_sync(0xffffffffu, g2)) { ok = false; break; }
+      }
+      uint8_t* prow = sP + g64 * (128 * 128) + row * 128;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint4 v = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+        *reinterpret_cast<uint4*>(prow + (((u0 + q) ^ (row & 7)) << 4)) = v;
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(p_full_l);
+    }
+    if (ok) {
+      // the last PV has read P: the buffer takes the row sums
+      const int jl = nkv - 1;
+      const bool g3 = mbar_wait(smem_u32(pv_done), jl & 1, p.err, abort_flag);
+      __syncwarp();
+      if (__all_sync(0xffffffffu, g3)) {
+        xsum[wg * 128 + row] = l;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(lbar));
+        const bool g4 = mbar_wait(smem_u32(lbar), 0, p.err, abort_flag);
+        __syncwarp();
+        if (__all_sync(0xffffffffu, g4)) {
+          tc_fence_after();
+          const float tot = xsum[row] + xsum[128 + row] + xsum[256 + row] + xsum[384 + row];
+          const float inv = 1.0f / tot;
+          const int qrow = q0 + row;
+          const bool row_ok = qrow < p.N;
+          uint16_t* dst = nullptr;
+          if (row_ok) {
+            if (qrow < p.split)
+              dst = p.out_a + (static_cast<size_t>(b) * p.split + qrow) * p.ldo + h * AT_HD;
+            else
+              dst = p.out_b + (static_cast<size_t>(b) * (p.N - p.split) + (qrow - p.split)) * p.ldo + h * AT_HD;
+            dst += 64 * wg;
+          }
+          for (int cc = 0; cc < 2; ++cc) {
+            uint32_t o[32];
+            tmem_ld32(tO + 64 * wg + cc * 32 + lane_off, o);
+            tmem_wait_ld();
+            if (row_ok) {
+              uint4* d = reinterpret_cast<uint4*>(dst + cc * 32);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                uint4 u;
+                u.x = pack_bf16(__uint_as_float(o[8 * i + 0]) * inv, __uint_as_float(o[8 * i + 1]) * inv);
+                u.y = pack_bf16(__uint_as_float(o[8 * i + 2]) * inv, __uint_as_float(o[8 * i + 3]) * inv);
+                u.z = pack_bf16(__uint_as_float(o[8 * i + 4]) * inv, __uint_as_float(o[8 * i + 5]) * inv);
+                u.w = pack_bf16(__uint_as_float(o[8 * i + 6]) * inv, __uint_as_float(o[8 * i + 7]) * inv);
+                d[i] = u;
+              }
+            }
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, 512);
+  }
+}
+
 // ---------------------------------------------------------------- small heads (SIMT)
 template <int HD>
 __global__ void attn_small_simt(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
@@ -1059,6 +1404,8 @@ cudaError_t attention_set_attributes() {
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(attn_hd256_qknorm_pair, cudaFuncAttributeMaxDynamicSharedMemorySize, AP_SMEM);
   if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(attn_hd256_qknorm_pair3, cudaFuncAttributeMaxDynamicSharedMemorySize, AP3_SMEM);
+  if (e != cudaSuccess) return e;
   done |= uint64_t(1) << dev;
   return cudaSuccess;
 }
@@ -1081,7 +1428,7 @@ cudaError_t launch_attention(const AttnParams& p, const uint16_t* q, const uint1
       CUtensorMap tv2;  // V halves: 128 keys x 64 columns per box
       if (!encode_tmap_3d(&tv2, v, AT_HD, p.N, bh, rb, sb, 64, AP_BN, 1)) return cudaErrorInvalidValue;
       dim3 grid2(2 * ((p.N + 255) / 256), p.H, p.B);
-      attn_hd256_qknorm_pair<<<grid2, AT_THREADS, AP_SMEM, stream>>>(tq, tk, tv2, p);
+      attn_hd256_qknorm_pair3<<<grid2, AP3_THREADS, AP3_SMEM, stream>>>(tq, tk, tv2, p);
       return cudaGetLastError();
     }
     dim3 grid((p.N + AT_BM - 1) / AT_BM, p.H, p.B);
