@@ -91,6 +91,22 @@ cudaError_t launch_ln_modulate(const uint16_t* x, const float* shift, const floa
                                uint16_t* y, int rows, int rows_per_batch, int D, float eps, cudaStream_t s,
                                int* err = nullptr, uint8_t* y8 = nullptr, float* yscale = nullptr);
 // y8 != nullptr: write e4m3 codes + per-row scales (y8 [rows, D], yscale [rows]) instead of bf16 y
+// One LayerNorm + modulate problem of nb samples x rows_per_batch rows (D = 3072):
+// scale / shift of sample b at + b * mod_stride; per = CTAs per sample (set by the launcher).
+struct LnSegment {
+  const uint16_t* x;
+  const float* shift;
+  const float* scale;
+  uint16_t* y;
+  uint8_t* y8;
+  float* ys;
+  int rows_per_batch;
+  int nb;
+  int per;
+};
+// Both segments in one launch (the joint block's image and text streams); g1.nb = 0 for one.
+cudaError_t launch_ln_modulate_pair(LnSegment g0, LnSegment g1, int mod_stride, int D, float eps, cudaStream_t s,
+                                    int* err);
 cudaError_t launch_quantize_rows_e4m3(const uint16_t* x, int rows, int K, uint8_t* q, float* scale, cudaStream_t s);
 cudaError_t launch_timestep_mlp(const float* t, int B, const uint16_t* w1, const uint16_t* b1, const uint16_t* w2,
                                 const uint16_t* b2, int C, int D, float* feat, float* h1, float* temb, cudaStream_t s);

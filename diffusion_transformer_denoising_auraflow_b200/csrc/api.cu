@@ -472,6 +472,18 @@ af_status ln_mod(af_scratch* s, const uint16_t* x, const float* shift, const flo
   return e == cudaSuccess ? AF_OK : cuda_fail(e);
 }
 
+// The joint block's image and text LayerNorms in one launch: shift at m, scale
+// at m + D of each stream's modulation rows (same layout rules as ln_mod).
+af_status ln_mod2(af_scratch* s, const uint16_t* xi, const float* mi, uint16_t* yi, uint8_t* yi8, float* ysi,
+                  int Ni, const uint16_t* xt, const float* mt, uint16_t* yt, uint8_t* yt8, float* yst, int Nt,
+                  int B, int mod_stride, int D, float eps, cudaStream_t st) {
+  LaunchScope ls(s, KC_LN, (yi8 ? 3.0 : 4.0) * B * (Ni + Nt) * D, st);
+  const LnSegment g0{xi, mi, mi + D, yi, yi8, ysi, Ni, B, 0};
+  const LnSegment g1{xt, mt, mt + D, yt, yt8, yst, Nt, Nt > 0 ? B : 0, 0};
+  cudaError_t e = launch_ln_modulate_pair(g0, g1, mod_stride, D, eps, st, s->err);
+  return e == cudaSuccess ? AF_OK : cuda_fail(e);
+}
+
 #define AF_TRY(x)                  \
   do {                             \
     af_status st_ = (x);           \
@@ -503,8 +515,9 @@ af_status joint_block_impl(const af_weights* w, af_scratch* s, int layer, uint16
   const Operand a_img = f8 ? Operand{q8_img, ys_img} : Operand{y_img, nullptr};
   const Operand a_txt = f8 ? Operand{q8_txt, ys_txt} : Operand{y_txt, nullptr};
 
-  AF_TRY(ln_mod(s, img, mi + 0 * D, mi + 1 * D, mod_stride, y_img, B * Ni, Ni, D, eps, st, q8_img, ys_img));
-  AF_TRY(ln_mod(s, txt, mt + 0 * D, mt + 1 * D, mod_stride, y_txt, B * Nt, Nt, D, eps, st, q8_txt, ys_txt));
+  // shift = m + 0 D, scale = m + 1 D of each stream, both streams in one launch
+  AF_TRY(ln_mod2(s, img, mi + 0 * D, y_img, q8_img, ys_img, Ni, txt, mt + 0 * D, y_txt, q8_txt, ys_txt, Nt, B,
+                 mod_stride, D, eps, st));
   // each projection pair (image, text) runs as one grouped launch
   AF_TRY(run_calls_grouped(s, qkv_call(w, s, a_img, B, Ni, weight_op(w, pre + "attn.to_q.weight"), Nt, N),
                            qkv_call(w, s, a_txt, B, Nt, weight_op(w, pre + "attn.add_q_proj.weight"), 0, N), st));
@@ -522,8 +535,8 @@ af_status joint_block_impl(const af_weights* w, af_scratch* s, int layer, uint16
       s, gres_call(s, oa_img, B, Ni, D, weight_op(w, pre + "attn.to_out.0.weight"), D, img, mi + 2 * D, mod_stride),
       gres_call(s, oa_txt, B, Nt, D, weight_op(w, pre + "attn.to_add_out.weight"), D, txt, mt + 2 * D, mod_stride),
       st));
-  AF_TRY(ln_mod(s, img, mi + 3 * D, mi + 4 * D, mod_stride, y_img, B * Ni, Ni, D, eps, st, q8_img, ys_img));
-  AF_TRY(ln_mod(s, txt, mt + 3 * D, mt + 4 * D, mod_stride, y_txt, B * Nt, Nt, D, eps, st, q8_txt, ys_txt));
+  AF_TRY(ln_mod2(s, img, mi + 3 * D, y_img, q8_img, ys_img, Ni, txt, mt + 3 * D, y_txt, q8_txt, ys_txt, Nt, B,
+                 mod_stride, D, eps, st));
   AF_TRY(run_calls_grouped(s, swiglu_call(w, s, a_img, B * Ni, weight_op(w, pre + "ff.linear_1.weight"), h_img),
                            swiglu_call(w, s, a_txt, B * Nt, weight_op(w, pre + "ff_context.linear_1.weight"), h_txt),
                            st));

@@ -1035,7 +1035,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
 constexpr int AP3_NWG = 4;
 constexpr int AP3_SM_WARPS = 4 * AP3_NWG;
 constexpr int AP3_V_WARP = 2 + AP3_SM_WARPS;
-constexpr int AP3_THREADS = 32 * (AP3_V_WARP + 1);
+constexpr int AP3_PV_WARP = AP3_V_WARP + 1;
+constexpr int AP3_THREADS = 32 * (AP3_PV_WARP + 1);
 constexpr int AP3_KPW = AP_BN / AP3_NWG;   // 32 keys per warpgroup
 constexpr int AP3_STAGES = 3;
 constexpr int AP3_SMEM = AP_P_BYTES + AP3_STAGES * AP_KH_BYTES + AP3_STAGES * AP_VH_BYTES + 256 + 1024;
@@ -1061,9 +1062,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AP3_THREADS, 1)
   uint64_t* pv_done = bars + 16;               // both CTAs
   uint64_t* q_tmem = bars + 17;                // leader: softmax warps of both CTAs have moved Q to TMEM
   uint64_t* q_moved = bars + 18;               // per CTA: this CTA's Q copy is done (V stages 0, 1 free)
-  uint64_t* mma_done = bars + 19;              // leader
+  uint64_t* mma_done = bars + 19;              // leader: the S issuer's MMAs
   uint64_t* lbar = bars + 20;                  // per CTA: row sums written
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 21);
+  uint64_t* mma_done_pv = bars + 21;           // leader: the PV issuer's MMAs
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 22);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -1093,6 +1095,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AP3_THREADS, 1)
     mbar_init(smem_u32(q_tmem), 2 * AP3_SM_WARPS);
     mbar_init(smem_u32(q_moved), AP3_SM_WARPS);
     mbar_init(smem_u32(mma_done), 1);
+    mbar_init(smem_u32(mma_done_pv), 1);
     mbar_init(smem_u32(lbar), AP3_SM_WARPS);
     *abort_flag = 0;
     fence_mbar_init();
@@ -1160,16 +1163,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AP3_THREADS, 1)
       }
     }
   } else if (warp == 1) {
+    // S issuer: S_j into the single S buffer once the K half of tile j has
+    // landed and the softmax warps of both CTAs have read S_{j-1}
     if (lane == 0 && leader) {
       const uint32_t idesc_qk = make_idesc_bf16(256, AP_BN, false, false);
-      const uint32_t idesc_pv = make_idesc_bf16(256, AT_HD, false, true);
       bool ok = mbar_wait(smem_u32(q_tmem), 0, p.err, abort_flag);
-      // S_j into the single S buffer: the K half of tile j has landed and the
-      // softmax warps of both CTAs have read S_{j-1}.
-      auto issue_s = [&](int j) -> bool {
+      for (int j = 0; j < nkv && ok; ++j) {
         const int s = j % AP3_STAGES;
-        if (!mbar_wait(smem_u32(&k_full[s]), (j / AP3_STAGES) & 1, p.err, abort_flag)) return false;
-        if (j > 0 && !mbar_wait(smem_u32(s_empty), (j - 1) & 1, p.err, abort_flag)) return false;
+        if (!mbar_wait(smem_u32(&k_full[s]), (j / AP3_STAGES) & 1, p.err, abort_flag)) { ok = false; break; }
+        if (j > 0 && !mbar_wait(smem_u32(s_empty), (j - 1) & 1, p.err, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t kaddr = smem_u32(sK + s * AP_KH_BYTES);
         const uint64_t kdesc = make_sdesc(kaddr, 16, 1024, SWZ_128B);
@@ -1181,13 +1183,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AP3_THREADS, 1)
         }
         mma_commit_pair(smem_u32(s_full), 0x3);
         mma_commit_pair(smem_u32(&k_empty[s]), 0x3);
-        return true;
-      };
-      if (ok) ok = issue_s(0);
+      }
+      mma_commit_pair(smem_u32(mma_done), 0x1);
+      mbar_wait(smem_u32(mma_done), 0, nullptr, &never, 100000000ull);
+    }
+  } else if (warp == AP3_PV_WARP) {
+    // PV issuer: O += P_j V_j once P_j is published and the V half of tile j
+    // has landed.  With two issuing threads, one thread's barrier checks
+    // overlap the other's MMAs in the tensor pipe (one thread doing both left
+    // a gap of a few hundred cycles at every S / PV switch for its checks).
+    if (lane == 0 && leader) {
+      const uint32_t idesc_pv = make_idesc_bf16(256, AT_HD, false, true);
       const uint64_t pdesc = make_sdesc(smem_u32(sP), 16, 1024, SWZ_128B);
+      bool ok = true;
       for (int j = 0; j < nkv && ok; ++j) {
         const int s = j % AP3_STAGES;
-        if (j + 1 < nkv && !issue_s(j + 1)) { ok = false; break; }
         if (!mbar_wait(smem_u32(p_full), j & 1, p.err, abort_flag)) { ok = false; break; }
         if (!mbar_wait(smem_u32(&v_full[s]), (j / AP3_STAGES) & 1, p.err, abort_flag)) { ok = false; break; }
         tc_fence_after();
@@ -1202,8 +1212,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AP3_THREADS, 1)
         mma_commit_pair(smem_u32(pv_done), 0x3);
         mma_commit_pair(smem_u32(&v_empty[s]), 0x3);
       }
-      mma_commit_pair(smem_u32(mma_done), 0x1);
-      mbar_wait(smem_u32(mma_done), 0, nullptr, &never, 100000000ull);
+      mma_commit_pair(smem_u32(mma_done_pv), 0x1);
+      mbar_wait(smem_u32(mma_done_pv), 0, nullptr, &never, 100000000ull);
     }
   } else {
     // ---------------------------------------------------------------- softmax: group g owns keys [32 g, 32 g + 32)

@@ -134,21 +134,24 @@ __global__ void __launch_bounds__(256) ln_modulate_kernel(const uint16_t* __rest
 
 // Wide rows (D = 3072), HBM-bound: rows are streamed into shared memory by
 // bulk copies, 2 stages of 4 rows per CTA and three CTAs per SM (144 KB in
-// flight per SM); the producer warp starts streaming at once while the 4
-// consumer warps stage (1 + scale) and shift of the CTA's sample.  Each
-// consumer warp normalises one row of a stage, the row held in registers
-// (two passes for mean and variance, then the output), the arithmetic on
-// packed fp32 pairs (sm_100 f32x2).  Three smaller CTAs per SM keep more
-// warps issuing than one CTA with 8 rows x 4 stages: 26.7 against 30.8 us
-// per [8720, 3072] call with the input in L2, 30.8 against 34.2 us from
-// DRAM (one-pass statistics in that measurement; the kernel keeps two).
-// Grid (CTAs per sample, samples).
+// flight per SM).  The producer warp first copies the CTA's sample's scale
+// and shift (bulk copies as well: staged by a strided load loop they cost
+// ~24 serialised L2 round trips per CTA before the first row), then streams
+// rows.  Each consumer warp normalises one row of a stage, the row held in
+// registers (two passes for mean and variance, then the output), the
+// arithmetic on packed fp32 pairs (sm_100 f32x2).  Three smaller CTAs per SM
+// keep more warps issuing than one CTA with 8 rows x 4 stages: 26.7 against
+// 30.8 us per [8720, 3072] call with the input in L2, 30.8 against 34.2 us
+// from DRAM.  One launch serves up to two problems (the joint block's image
+// and text streams), CTAs split between them in proportion to their rows;
+// 1-D grid: segment 0's samples x CTAs per sample, then segment 1's.
 constexpr int LNB_D = 3072;
-constexpr int LNB_ROWS = 4;
-constexpr int LNB_STAGES = 2;
-constexpr int LNB_PER_SM = 3;
+constexpr int LNB_ROWS = 2;     // rows per stage
+constexpr int LNB_STAGES = 4;
+constexpr int LNB_CW = 4;       // consumer warps
+constexpr int LNB_PER_SM = 2;
 constexpr uint32_t LNB_ROW_BYTES = LNB_D * 2;
-constexpr int LNB_THREADS = 32 * (LNB_ROWS + 1);
+constexpr int LNB_THREADS = 32 * (LNB_CW + 1);
 constexpr int LNB_SMEM = LNB_STAGES * LNB_ROWS * LNB_ROW_BYTES + 2 * LNB_D * 4;
 
 // packed fp32 pairs
@@ -181,37 +184,63 @@ __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
 __device__ __forceinline__ uint64_t f2_from_bf16x2(uint32_t w) {
   return f2_pack(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
 }
+// the same, kept opaque to common-subexpression elimination: a row held as
+// bf16 pairs is expanded again in each pass instead of being cached as fp32
+// (twice the registers)
+__device__ __forceinline__ uint64_t f2_from_bf16x2_each(uint32_t w) {
+  uint64_t r;
+  asm volatile(
+      "{\n\t.reg .b32 lo, hi;\n\t"
+      "shl.b32 lo, %1, 16;\n\t"
+      "and.b32 hi, %1, 0xFFFF0000;\n\t"
+      "mov.b64 %0, {lo, hi};\n\t}"
+      : "=l"(r)
+      : "r"(w));
+  return r;
+}
 
 template <bool OUT8>
-__global__ void __launch_bounds__(LNB_THREADS, LNB_PER_SM) ln_modulate_bulk_kernel(
-    const uint16_t* __restrict__ x, const float* __restrict__ shift, const float* __restrict__ scale, int mod_stride,
-    uint16_t* __restrict__ y, uint8_t* __restrict__ y8, float* __restrict__ yscale, int rows_per_batch, float eps,
-    int* err) {
+__global__ void __launch_bounds__(LNB_THREADS, LNB_PER_SM) ln_modulate_bulk_kernel(LnSegment g0, LnSegment g1,
+                                                                                   int mod_stride, float eps,
+                                                                                   int* err) {
   extern __shared__ __align__(128) uint8_t lnb_raw[];  // [stage][row] x 6 KB, then (1 + scale) | shift
   uint8_t* rowbuf = lnb_raw;
   float* mod_s = reinterpret_cast<float*>(lnb_raw + LNB_STAGES * LNB_ROWS * LNB_ROW_BYTES);
-  __shared__ uint64_t full[LNB_STAGES], empty[LNB_STAGES];
+  __shared__ uint64_t full[LNB_STAGES], empty[LNB_STAGES], mod_full;
   __shared__ int abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int b = blockIdx.y;
+  // the first g0.nb * g0.per CTAs serve segment 0, the rest segment 1
+  const int n0 = g0.nb * g0.per;
+  const bool sec = static_cast<int>(blockIdx.x) >= n0;
+  const int id = sec ? static_cast<int>(blockIdx.x) - n0 : static_cast<int>(blockIdx.x);
+  const int per = sec ? g1.per : g0.per;
+  const int rows_per_batch = sec ? g1.rows_per_batch : g0.rows_per_batch;
+  const int b = id / per, cx = id - b * per;
+  const uint16_t* __restrict__ x = sec ? g1.x : g0.x;
   const int nchunks = (rows_per_batch + LNB_ROWS - 1) / LNB_ROWS;
   const size_t row0 = static_cast<size_t>(b) * rows_per_batch;
   if (threadIdx.x == 0) {
     for (int i = 0; i < LNB_STAGES; ++i) {
       mbar_init(smem_u32(&full[i]), 1);
-      mbar_init(smem_u32(&empty[i]), LNB_ROWS);
+      mbar_init(smem_u32(&empty[i]), LNB_CW);
     }
+    mbar_init(smem_u32(&mod_full), 1);
     abort_flag = 0;
     fence_mbar_init();
   }
   __syncthreads();
 
-  if (warp == LNB_ROWS) {
-    // producer: one elected thread streams chunks of LNB_ROWS rows
+  if (warp == LNB_CW) {
+    // producer: one elected thread copies this sample's scale and shift, then
+    // streams chunks of LNB_ROWS rows
     if (lane == 0) {
-      bool ok = true, issued = false;
+      const size_t mo = static_cast<size_t>(b) * mod_stride;
+      mbar_arrive_expect_tx(smem_u32(&mod_full), 2 * LNB_D * 4);
+      bulk_load(smem_u32(mod_s), (sec ? g1.scale : g0.scale) + mo, LNB_D * 4, smem_u32(&mod_full));
+      bulk_load(smem_u32(mod_s + LNB_D), (sec ? g1.shift : g0.shift) + mo, LNB_D * 4, smem_u32(&mod_full));
+      bool ok = true;
       int k = 0;
-      for (int c = blockIdx.x; c < nchunks; c += gridDim.x, ++k) {
+      for (int c = cx; c < nchunks; c += per, ++k) {
         const int st = k % LNB_STAGES;
         const uint32_t ph = (k / LNB_STAGES) & 1;
         if (!mbar_wait(smem_u32(&empty[st]), ph ^ 1u, err, &abort_flag)) { ok = false; break; }
@@ -221,9 +250,8 @@ __global__ void __launch_bounds__(LNB_THREADS, LNB_PER_SM) ln_modulate_bulk_kern
           bulk_load(smem_u32(rowbuf + (st * LNB_ROWS + r) * LNB_ROW_BYTES),
                     x + (row0 + static_cast<size_t>(c) * LNB_ROWS + r) * LNB_D, LNB_ROW_BYTES,
                     smem_u32(&full[st]));
-        issued = true;
       }
-      if (!ok && issued) {  // let copies already in flight land before the CTA exits
+      if (!ok) {  // let copies already in flight land before the CTA exits
         const uint64_t t0 = globaltimer();
         while (globaltimer() - t0 < 200000ull) {
         }
@@ -231,73 +259,132 @@ __global__ void __launch_bounds__(LNB_THREADS, LNB_PER_SM) ln_modulate_bulk_kern
     }
     return;
   }
-  // consumers: stage the modulation vectors (named barrier 1: consumer warps only)
+  // consumers: warp w owns 16-byte column vectors [32 VPW w, 32 VPW (w + 1))
+  // of both rows of a stage (lane l: vectors 32 VPW w + 32 i + l, i < VPW),
+  // so its (1 + scale) and shift stay in registers; the row statistics are
+  // summed across the LNB_CW warps through shared memory at the consumers'
+  // named barrier 1.  Every barrier is a bar.red.or of "this thread
+  // gave up", so all consumer threads leave the loop together.
+  auto any_failed = [](bool failed) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, 1, %2, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"(static_cast<uint32_t>(failed)), "r"(32 * LNB_CW)
+        : "memory");
+    return r != 0;
+  };
+  __shared__ __align__(16) float red[3][LNB_ROWS][LNB_CW];  // [statistic][row][warp]
+  constexpr int VPW = LNB_D / 8 / LNB_CW / 32;               // 16-byte vectors per lane
+  static_assert(VPW * 32 * LNB_CW * 8 == LNB_D, "columns split evenly over the consumer warps");
+  auto total = [&](const float* t) {
+    float v = 0.f;
+#pragma unroll
+    for (int i = 0; i < LNB_CW; ++i) v += t[i];
+    return v;
+  };
+  auto largest = [&](const float* t) {
+    float v = 0.f;
+#pragma unroll
+    for (int i = 0; i < LNB_CW; ++i) v = fmaxf(v, t[i]);
+    return v;
+  };
+  uint64_t av[VPW][4], hv[VPW][4];                           // (1 + scale), shift as packed pairs
   {
-    const float* sc = scale + static_cast<size_t>(b) * mod_stride;
-    const float* sh = shift + static_cast<size_t>(b) * mod_stride;
-    for (int i = threadIdx.x; i < LNB_D; i += 32 * LNB_ROWS) {
-      mod_s[i] = 1.0f + sc[i];
-      mod_s[LNB_D + i] = sh[i];
+    const bool got = mbar_wait(smem_u32(&mod_full), 0, err, &abort_flag);
+    if (any_failed(!got)) return;
+#pragma unroll
+    for (int i = 0; i < VPW; ++i) {
+      const int c0 = 8 * (warp * 32 * VPW + i * 32 + lane);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        av[i][e] = f2_pack(1.0f + mod_s[c0 + 2 * e], 1.0f + mod_s[c0 + 2 * e + 1]);
+        hv[i][e] = f2_pack(mod_s[LNB_D + c0 + 2 * e], mod_s[LNB_D + c0 + 2 * e + 1]);
+      }
     }
-    asm volatile("bar.sync 1, %0;" ::"r"(32 * LNB_ROWS) : "memory");
   }
-  // warp w normalises row w of every stage
-  constexpr int VPL = LNB_D / 256;
+  // this sample's first output row
+  uint16_t* __restrict__ y = OUT8 ? nullptr : (sec ? g1.y : g0.y) + row0 * LNB_D;
+  uint8_t* __restrict__ y8 = OUT8 ? (sec ? g1.y8 : g0.y8) + row0 * LNB_D : nullptr;
+  float* __restrict__ yscale = OUT8 ? (sec ? g1.ys : g0.ys) + row0 : nullptr;
+  const int v0 = warp * 32 * VPW + lane;  // this lane's first vector; then every 32th
   int k = 0;
-  for (int c = blockIdx.x; c < nchunks; c += gridDim.x, ++k) {
+  for (int c = cx; c < nchunks; c += per, ++k) {
     const int st = k % LNB_STAGES;
     const uint32_t ph = (k / LNB_STAGES) & 1;
     const bool got = mbar_wait(smem_u32(&full[st]), ph, err, &abort_flag);
-    if (!__all_sync(0xffffffffu, got)) break;
-    const int r = c * LNB_ROWS + warp;
-    if (r < rows_per_batch) {
-      const uint4* xr = reinterpret_cast<const uint4*>(rowbuf + (st * LNB_ROWS + warp) * LNB_ROW_BYTES);
-      uint4 u[VPL];
+    uint4 u[LNB_ROWS][VPW];
+    if (got) {
 #pragma unroll
-      for (int i = 0; i < VPL; ++i) u[i] = xr[i * 32 + lane];
-      // two passes over the registers: the mean, then the centred squares
+      for (int rr = 0; rr < LNB_ROWS; ++rr) {
+        const uint4* xr = reinterpret_cast<const uint4*>(rowbuf + (st * LNB_ROWS + rr) * LNB_ROW_BYTES);
+#pragma unroll
+        for (int i = 0; i < VPW; ++i) u[rr][i] = xr[v0 + 32 * i];
+      }
+    }
+    // the rows are in registers: the stage goes back to the producer
+    __syncwarp();
+    if (got && lane == 0) mbar_arrive(smem_u32(&empty[st]));
+    // pass 1: row sums
+#pragma unroll
+    for (int rr = 0; rr < LNB_ROWS; ++rr) {
       uint64_t s2 = f2_pack(0.f, 0.f);
 #pragma unroll
-      for (int i = 0; i < VPL; ++i) {
-        const uint32_t w[4] = {u[i].x, u[i].y, u[i].z, u[i].w};
+      for (int i = 0; i < VPW; ++i) {
+        const uint32_t w[4] = {u[rr][i].x, u[rr][i].y, u[rr][i].z, u[rr][i].w};
 #pragma unroll
-        for (int e = 0; e < 4; ++e) s2 = f2_add(s2, f2_from_bf16x2(w[e]));
+        for (int e = 0; e < 4; ++e) s2 = f2_add(s2, f2_from_bf16x2_each(w[e]));
       }
       const float2 sv = f2_unpack(s2);
-      const float mean = warp_sum(sv.x + sv.y) * (1.0f / LNB_D);
-      const uint64_t nm = f2_pack(-mean, -mean);
+      const float t = warp_sum(sv.x + sv.y);
+      if (lane == 0) red[0][rr][warp] = t;
+    }
+    if (any_failed(!got)) break;
+    uint64_t nm[LNB_ROWS];
+#pragma unroll
+    for (int rr = 0; rr < LNB_ROWS; ++rr) {
+      const float mean = total(red[0][rr]) * (1.0f / LNB_D);
+      nm[rr] = f2_pack(-mean, -mean);
+    }
+    // pass 2: centred squares
+#pragma unroll
+    for (int rr = 0; rr < LNB_ROWS; ++rr) {
       uint64_t q2 = f2_pack(0.f, 0.f);
 #pragma unroll
-      for (int i = 0; i < VPL; ++i) {
-        const uint32_t w[4] = {u[i].x, u[i].y, u[i].z, u[i].w};
+      for (int i = 0; i < VPW; ++i) {
+        const uint32_t w[4] = {u[rr][i].x, u[rr][i].y, u[rr][i].z, u[rr][i].w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const uint64_t d = f2_add(f2_from_bf16x2(w[e]), nm);
+          const uint64_t d = f2_add(f2_from_bf16x2_each(w[e]), nm[rr]);
           q2 = f2_fma(d, d, q2);
         }
       }
       const float2 qv = f2_unpack(q2);
-      const float rstd = rsqrtf(warp_sum(qv.x + qv.y) * (1.0f / LNB_D) + eps);
-      const uint64_t rs2 = f2_pack(rstd, rstd);
-      // output pairs 0..3 of vector i: (x - mean) rstd (1 + scale) + shift
-      auto out8 = [&](int i, uint64_t (&o)[4]) {
-        const int vi = i * 32 + lane;
-        const ulonglong2 a01 = *reinterpret_cast<const ulonglong2*>(mod_s + vi * 8);
-        const ulonglong2 a23 = *reinterpret_cast<const ulonglong2*>(mod_s + vi * 8 + 4);
-        const ulonglong2 h01 = *reinterpret_cast<const ulonglong2*>(mod_s + LNB_D + vi * 8);
-        const ulonglong2 h23 = *reinterpret_cast<const ulonglong2*>(mod_s + LNB_D + vi * 8 + 4);
-        const uint64_t av[4] = {a01.x, a01.y, a23.x, a23.y};
-        const uint64_t hv[4] = {h01.x, h01.y, h23.x, h23.y};
-        const uint32_t w[4] = {u[i].x, u[i].y, u[i].z, u[i].w};
+      const float t = warp_sum(qv.x + qv.y);
+      if (lane == 0) red[1][rr][warp] = t;
+    }
+    asm volatile("bar.sync 1, %0;" ::"r"(32 * LNB_CW) : "memory");
+    const int nrows = min(LNB_ROWS, rows_per_batch - c * LNB_ROWS);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) o[e] = f2_fma(f2_mul(f2_add(f2_from_bf16x2(w[e]), nm), rs2), av[e], hv[e]);
+    for (int rr = 0; rr < LNB_ROWS; ++rr) {
+      const float rstd = rsqrtf(total(red[1][rr]) * (1.0f / LNB_D) + eps);
+      const uint64_t rs2 = f2_pack(rstd, rstd);
+      // (x - mean) rstd (1 + scale) + shift for vector i, pairs 0..3
+      auto outv = [&](int i, uint64_t (&o)[4]) {
+        const uint32_t w[4] = {u[rr][i].x, u[rr][i].y, u[rr][i].z, u[rr][i].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o[e] = f2_fma(f2_mul(f2_add(f2_from_bf16x2_each(w[e]), nm[rr]), rs2), av[i][e], hv[i][e]);
       };
+      const int r = c * LNB_ROWS + rr;
       if constexpr (OUT8) {
         float amax = 0.f;
 #pragma unroll
-        for (int i = 0; i < VPL; ++i) {
+        for (int i = 0; i < VPW; ++i) {
           uint64_t o[4];
-          out8(i, o);
+          outv(i, o);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const float2 v = f2_unpack(o[e]);
@@ -305,32 +392,89 @@ __global__ void __launch_bounds__(LNB_THREADS, LNB_PER_SM) ln_modulate_bulk_kern
           }
         }
         amax = warp_max(amax);
-        const float inv = e4m3_inv_scale(amax);
-        uint2* yr = reinterpret_cast<uint2*>(y8 + (row0 + r) * LNB_D);
+        if (lane == 0) red[2][rr][warp] = amax;
+      } else if (rr < nrows) {
+        uint4* yr = reinterpret_cast<uint4*>(y + static_cast<size_t>(r) * LNB_D);
 #pragma unroll
-        for (int i = 0; i < VPL; ++i) {
+        for (int i = 0; i < VPW; ++i) {
           uint64_t o[4];
-          out8(i, o);
-          const float2 v0 = f2_unpack(o[0]), v1 = f2_unpack(o[1]), v2 = f2_unpack(o[2]), v3 = f2_unpack(o[3]);
-          yr[i * 32 + lane] = make_uint2(pack_e4m3x4(v0.x * inv, v0.y * inv, v1.x * inv, v1.y * inv),
-                                         pack_e4m3x4(v2.x * inv, v2.y * inv, v3.x * inv, v3.y * inv));
-        }
-        if (lane == 0) yscale[row0 + r] = e4m3_scale(amax);
-      } else {
-        uint4* yr = reinterpret_cast<uint4*>(y + (row0 + r) * LNB_D);
-#pragma unroll
-        for (int i = 0; i < VPL; ++i) {
-          uint64_t o[4];
-          out8(i, o);
-          const float2 v0 = f2_unpack(o[0]), v1 = f2_unpack(o[1]), v2 = f2_unpack(o[2]), v3 = f2_unpack(o[3]);
-          yr[i * 32 + lane] = make_uint4(pack_bf16(v0.x, v0.y), pack_bf16(v1.x, v1.y), pack_bf16(v2.x, v2.y),
-                                         pack_bf16(v3.x, v3.y));
+          outv(i, o);
+          const float2 a0 = f2_unpack(o[0]), a1 = f2_unpack(o[1]), a2 = f2_unpack(o[2]), a3 = f2_unpack(o[3]);
+          yr[v0 + 32 * i] = make_uint4(pack_bf16(a0.x, a0.y), pack_bf16(a1.x, a1.y), pack_bf16(a2.x, a2.y),
+                                       pack_bf16(a3.x, a3.y));
         }
       }
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(smem_u32(&empty[st]));
+    if constexpr (OUT8) {
+      // the row's e4m3 scale needs the maximum over all four warps' columns
+      asm volatile("bar.sync 1, %0;" ::"r"(32 * LNB_CW) : "memory");
+#pragma unroll
+      for (int rr = 0; rr < LNB_ROWS; ++rr) {
+        if (rr >= nrows) continue;
+        const float amax = largest(red[2][rr]);
+        const float inv = e4m3_inv_scale(amax);
+        const float mean = total(red[0][rr]) * (1.0f / LNB_D);
+        const float rstd = rsqrtf(total(red[1][rr]) * (1.0f / LNB_D) + eps);
+        const uint64_t nmr = f2_pack(-mean, -mean), rs2 = f2_pack(rstd, rstd);
+        const int r = c * LNB_ROWS + rr;
+        uint2* yr = reinterpret_cast<uint2*>(y8 + static_cast<size_t>(r) * LNB_D);
+#pragma unroll
+        for (int i = 0; i < VPW; ++i) {
+          const uint32_t w[4] = {u[rr][i].x, u[rr][i].y, u[rr][i].z, u[rr][i].w};
+          float2 v[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            v[e] = f2_unpack(f2_fma(f2_mul(f2_add(f2_from_bf16x2_each(w[e]), nmr), rs2), av[i][e], hv[i][e]));
+          yr[v0 + 32 * i] = make_uint2(pack_e4m3x4(v[0].x * inv, v[0].y * inv, v[1].x * inv, v[1].y * inv),
+                                       pack_e4m3x4(v[2].x * inv, v[2].y * inv, v[3].x * inv, v[3].y * inv));
+        }
+        if (threadIdx.x == 0) yscale[r] = e4m3_scale(amax);
+      }
+    }
   }
+}
+
+// Segment sizes: CTAs per sample in proportion to the segment's rows, about
+// LNB_PER_SM CTAs per SM over the whole launch.
+static void ln_plan(LnSegment& g, int total_rows, int sms) {
+  if (g.nb <= 0) { g.nb = 0; g.per = 0; return; }
+  const int nchunks = (g.rows_per_batch + LNB_ROWS - 1) / LNB_ROWS;
+  const double share = static_cast<double>(g.rows_per_batch) * g.nb / total_rows;
+  const int want = static_cast<int>(LNB_PER_SM * sms * share / g.nb + 0.5);
+  g.per = max(1, min(nchunks, want));
+}
+
+static bool ln_bulk_ok(const LnSegment& g, int mod_stride) {
+  auto al = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
+  return al(g.x) && al(g.shift) && al(g.scale) && (mod_stride % 4) == 0;
+}
+
+cudaError_t launch_ln_modulate_pair(LnSegment g0, LnSegment g1, int mod_stride, int D, float eps, cudaStream_t s,
+                                    int* err) {
+  if (g1.nb > 0 && ((g0.y8 == nullptr) != (g1.y8 == nullptr))) return cudaErrorInvalidValue;
+  if (D != LNB_D || !ln_bulk_ok(g0, mod_stride) || (g1.nb > 0 && !ln_bulk_ok(g1, mod_stride))) {
+    // the generic row kernel, one launch per segment
+    cudaError_t e = launch_ln_modulate(g0.x, g0.shift, g0.scale, mod_stride, g0.y, g0.nb * g0.rows_per_batch,
+                                       g0.rows_per_batch, D, eps, s, err, g0.y8, g0.ys);
+    if (e != cudaSuccess || g1.nb <= 0) return e;
+    return launch_ln_modulate(g1.x, g1.shift, g1.scale, mod_stride, g1.y, g1.nb * g1.rows_per_batch,
+                              g1.rows_per_batch, D, eps, s, err, g1.y8, g1.ys);
+  }
+  if (g0.nb <= 0 || g0.rows_per_batch <= 0) return cudaErrorInvalidValue;
+  if (g1.nb > 0 && g1.rows_per_batch <= 0) g1.nb = 0;
+  cudaError_t e = small_kernels_set_attributes();
+  if (e != cudaSuccess) return e;
+  static int sms = 0;
+  if (!sms) sms = device_sm_count();
+  const int total = g0.nb * g0.rows_per_batch + max(g1.nb, 0) * g1.rows_per_batch;
+  ln_plan(g0, total, sms);
+  ln_plan(g1, total, sms);
+  const int grid = g0.nb * g0.per + g1.nb * g1.per;
+  if (g0.y8)
+    ln_modulate_bulk_kernel<true><<<grid, LNB_THREADS, LNB_SMEM, s>>>(g0, g1, mod_stride, eps, err);
+  else
+    ln_modulate_bulk_kernel<false><<<grid, LNB_THREADS, LNB_SMEM, s>>>(g0, g1, mod_stride, eps, err);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_ln_modulate(const uint16_t* x, const float* shift, const float* scale, int mod_stride,
@@ -340,21 +484,10 @@ cudaError_t launch_ln_modulate(const uint16_t* x, const float* shift, const floa
   if (D % 8 != 0) return cudaErrorInvalidValue;
   const bool out8 = y8 != nullptr;
   if (out8 && !yscale) return cudaErrorInvalidValue;
-  if (D == LNB_D && rows % rows_per_batch == 0 && (reinterpret_cast<uintptr_t>(x) & 15) == 0) {
-    cudaError_t e = small_kernels_set_attributes();
-    if (e != cudaSuccess) return e;
-    const int nb = rows / rows_per_batch;
-    static int sms = 0;
-    if (!sms) sms = device_sm_count();
-    const int nchunks = (rows_per_batch + LNB_ROWS - 1) / LNB_ROWS;
-    const int per = max(1, min(nchunks, (LNB_PER_SM * sms + nb - 1) / nb));
-    if (out8)
-      ln_modulate_bulk_kernel<true><<<dim3(per, nb), LNB_THREADS, LNB_SMEM, s>>>(x, shift, scale, mod_stride, y, y8,
-                                                                               yscale, rows_per_batch, eps, err);
-    else
-      ln_modulate_bulk_kernel<false><<<dim3(per, nb), LNB_THREADS, LNB_SMEM, s>>>(x, shift, scale, mod_stride, y, y8,
-                                                                                yscale, rows_per_batch, eps, err);
-    return cudaGetLastError();
+  if (rows_per_batch <= 0) return cudaErrorInvalidValue;
+  if (D == LNB_D && rows % rows_per_batch == 0) {
+    const LnSegment g0{x, shift, scale, y, y8, yscale, rows_per_batch, rows / rows_per_batch, 0};
+    if (ln_bulk_ok(g0, mod_stride)) return launch_ln_modulate_pair(g0, LnSegment{}, mod_stride, D, eps, s, err);
   }
   const int nvec = D / 8;
   const int vpl = (nvec + 31) / 32;
@@ -745,27 +878,31 @@ cudaError_t launch_patch_embed(const float* lat, int B, int C, int H, int W, int
 // o[k] = W[k] . z = (W[k] * (1 + sc)) . x + W[k] . sh.  output_fold_kernel
 // writes, per sample b, W'_b = bf16(W * (1 + sc_b)) into rows [0, KP) of a
 // 256-row block (the rest stays zero, so a 256-wide GEMM tile reads only
-// zeros there) and bias_b[k] = W[k] . sh_b (fp32); one warp per (b, k).
+// zeros there) and bias_b[k] = W[k] . sh_b (fp32); one CTA per (b, k).
 __global__ void __launch_bounds__(256) output_fold_kernel(const uint16_t* __restrict__ wout, int KP, int D,
                                                           const float* __restrict__ scale,
                                                           const float* __restrict__ shift, int mod_stride, int B,
                                                           uint16_t* __restrict__ wfold, float* __restrict__ bias) {
-  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (gw >= B * KP) return;
-  const int b = gw / KP, k = gw - b * KP;
+  __shared__ float part[8];
+  const int b = blockIdx.x / KP, k = blockIdx.x - b * KP;
   const float* sc = scale + static_cast<size_t>(b) * mod_stride;
   const float* sh = shift + static_cast<size_t>(b) * mod_stride;
   const uint16_t* wr = wout + static_cast<size_t>(k) * D;
   uint16_t* dr = wfold + (static_cast<size_t>(b) * 256 + k) * D;
   float acc = 0.f;
-  for (int d = lane; d < D; d += 32) {
+  for (int d = threadIdx.x; d < D; d += blockDim.x) {
     const float w = __uint_as_float(static_cast<uint32_t>(wr[d]) << 16);
     dr[d] = static_cast<uint16_t>(pack_bf16(w * (1.0f + sc[d]), 0.f) & 0xFFFFu);
     acc = fmaf(w, sh[d], acc);
   }
   acc = warp_sum(acc);
-  if (lane == 0) bias[b * KP + k] = acc;
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float t = 0.f;
+    for (int i = 0; i < static_cast<int>(blockDim.x >> 5); ++i) t += part[i];
+    bias[b * KP + k] = t;
+  }
 }
 
 // velocity[b, c, hp p + py, wp p + px] = o[b, n, (py p + px) C + c] + bias_b[...]
@@ -785,8 +922,7 @@ __global__ void output_scatter_kernel(const float* __restrict__ o, const float* 
 
 cudaError_t launch_output_fold(const uint16_t* w_out, int KP, int D, const float* scale, const float* shift,
                                int mod_stride, int B, uint16_t* wfold, float* bias, cudaStream_t s) {
-  const int warps = B * KP;
-  output_fold_kernel<<<(warps + 7) / 8, 256, 0, s>>>(w_out, KP, D, scale, shift, mod_stride, B, wfold, bias);
+  output_fold_kernel<<<B * KP, 256, 0, s>>>(w_out, KP, D, scale, shift, mod_stride, B, wfold, bias);
   return cudaGetLastError();
 }
 
