@@ -39,6 +39,10 @@ struct GemmParams {
   // readable 32 rows past every weight row the GEMM touches (pad to 256)
   const float* a_scale = nullptr;
   const float* w_scale = nullptr;
+  // GATE_RES: nonzero when the residual tiles move by TMA (set by the
+  // launcher when `out` is 16-byte aligned, ldo * 2 a multiple of 16 and the
+  // output rows are the GEMM rows)
+  int res_tma = 0;
 };
 
 constexpr int GEMM_BM = 128;
@@ -46,11 +50,14 @@ constexpr int GEMM_BN = 256;
 constexpr int GEMM_BK = 64;
 constexpr int GEMM_STAGES = 4;
 constexpr int GEMM_THREADS = 192;
-constexpr int GEMM_SMEM_BYTES = GEMM_STAGES * (GEMM_BM + GEMM_BN) * GEMM_BK * 2 + 1024 /*barriers*/ + 1024 /*align*/;
+// per epilogue warp, two 32 x 32 bf16 residual boxes (gated-residual epilogue)
+constexpr int GEMM_RES_BYTES = 4 * 2 * 32 * 32 * 2;
+constexpr int GEMM_SMEM_BYTES =
+    GEMM_STAGES * (GEMM_BM + GEMM_BN) * GEMM_BK * 2 + GEMM_RES_BYTES + 1024 /*barriers*/ + 1024 /*align*/;
 
 // Host helpers (gemm.cu)
 bool encode_tmap_2d(CUtensorMap* map, const void* ptr, uint64_t inner, uint64_t outer, uint64_t row_bytes,
-                    uint32_t box_inner, uint32_t box_outer, bool bytes = false);
+                    uint32_t box_inner, uint32_t box_outer, bool bytes = false, int swizzle_bytes = 128);
 bool encode_tmap_3d(CUtensorMap* map, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1_bytes,
                     uint64_t s2_bytes, uint32_t b0, uint32_t b1, uint32_t b2);
 cudaError_t launch_gemm(const GemmParams& p_in, const void* A, const void* W, int W_rows, cudaStream_t stream,

@@ -46,16 +46,17 @@ static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
 }
 
 bool encode_tmap_2d(CUtensorMap* map, const void* ptr, uint64_t inner, uint64_t outer, uint64_t row_bytes,
-                    uint32_t box_inner, uint32_t box_outer, bool bytes) {
+                    uint32_t box_inner, uint32_t box_outer, bool bytes, int swizzle_bytes) {
   auto enc = get_encode();
   if (!enc) return false;
   cuuint64_t dims[2] = {inner, outer};
   cuuint64_t strides[1] = {row_bytes};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapSwizzle sw = swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
   CUresult r = enc(map, bytes ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
                    const_cast<void*>(ptr), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -227,10 +228,63 @@ __device__ __forceinline__ void epilogue_qkv(const GemmParams& p, uint32_t tbase
   }
 }
 
+// Gated-residual epilogue with TMA-staged residual tiles.  Each epilogue warp
+// owns 32 output rows of a tile and walks them in 32-column chunks; the
+// residual box of a chunk (32 x 32 bf16, 64-byte swizzle) is loaded by TMA
+// into one of the warp's two shared-memory buffers one chunk ahead (the first
+// before the accumulator is ready), updated in place (thread = row, so the
+// reads follow the TMEM lane layout without bank conflicts) and written back
+// by a TMA store: coalesced global traffic instead of every thread walking
+// its own row.
+struct ResStage {
+  uint32_t buf;            // this warp's two 2 KB boxes (1024-byte aligned)
+  uint32_t bar;            // their two mbarriers (8 bytes apart)
+  uint32_t issued, used;   // loads issued / consumed: buffer = n & 1, parity = (n >> 1) & 1
+  volatile int* abort;
+  bool failed;
+};
+constexpr uint32_t RES_BOX_BYTES = 32 * 32 * 2;
+
+// Load the residual box at (col, row) into the next buffer (lane 0 issues).
+__device__ __forceinline__ void res_issue(ResStage& rs, const CUtensorMap* tm, int col, int row, bool lane0) {
+  const uint32_t k = rs.issued & 1u;
+  if (lane0) {
+    bulk_wait_group_read0();  // the store that last read this buffer has read it
+    mbar_arrive_expect_tx(rs.bar + 8 * k, RES_BOX_BYTES);
+    tma_load_2d(rs.buf + k * RES_BOX_BYTES, tm, rs.bar + 8 * k, col, row);
+  }
+  ++rs.issued;
+}
+
+// Wait for the oldest issued box; its shared-memory address (0 on a timeout).
+__device__ __forceinline__ uint32_t res_take(ResStage& rs, int* err) {
+  const uint32_t n = rs.used++;
+  const uint32_t k = n & 1u;
+  const bool got = mbar_wait(rs.bar + 8 * k, (n >> 1) & 1u, err, rs.abort);
+  if (!__all_sync(0xffffffffu, got)) {
+    rs.failed = true;
+    return 0;
+  }
+  return rs.buf + k * RES_BOX_BYTES;
+}
+
+// Before the warp leaves: its stores have completed and no box load is still
+// in flight (an abandoned prefetch lands first; bounded waits).
+__device__ __forceinline__ void res_drain(ResStage& rs, bool lane0) {
+  if (lane0) bulk_wait_group0();
+  volatile int never = 0;
+  while (rs.used < rs.issued) {
+    const uint32_t n = rs.used++;
+    mbar_wait(rs.bar + 8 * (n & 1u), (n >> 1) & 1u, nullptr, &never, 100000000ull);
+  }
+  __syncwarp();
+}
+
 // Epilogue of one accumulator tile for one output row (thread = TMEM lane):
 // tbase addresses this warp's 32-lane quarter of the accumulator, m0 is the
 // first GEMM row of the tile half held in this CTA's TMEM, nb the n-tile.
-__device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tbase, int m0, int nb, int row_in_tile) {
+__device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tbase, int m0, int nb, int row_in_tile,
+                                              ResStage* rs = nullptr, const CUtensorMap* tmo = nullptr) {
   const int r = m0 + row_in_tile;
   const bool row_ok = r < p.M;
   const int b = r / p.rows_per_batch;
@@ -240,6 +294,55 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tbas
 
   if (p.mode == EPI_QKV) {
     epilogue_qkv(p, tbase, nb * GEMM_BN, row_ok, b, n_in, a_s);
+  } else if (p.mode == EPI_GATE_RES && p.res_tma) {
+    // chunk 0's box was issued by the caller before the accumulator was ready
+    const int lane = row_in_tile & 31;
+    const int col0 = nb * GEMM_BN;
+    const int wrow0 = m0 + (row_in_tile & ~31);
+    const int nch = min(GEMM_BN / 32, (p.N - col0 + 31) / 32);
+    const float* gb = row_ok ? p.gate + static_cast<size_t>(b) * p.gate_stride : nullptr;
+    const uint32_t swz = static_cast<uint32_t>((lane >> 1) & 3);
+#pragma unroll 1
+    for (int c = 0; c < nch; ++c) {
+      if (c + 1 < nch) res_issue(*rs, tmo, col0 + 32 * (c + 1), wrow0, lane == 0);
+      float v[32];
+      acc_load32(p, tbase + c * 32, a_s, col0 + c * 32, v);
+      const uint32_t box = res_take(*rs, p.err);
+      if (!box) return;
+      const uint32_t rowa = box + static_cast<uint32_t>(lane) * 64;
+      uint4 xv[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) xv[q] = lds128(rowa + ((static_cast<uint32_t>(q) ^ swz) << 4));
+      if (gb) {
+        const float* g = gb + col0 + c * 32;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float4 g0 = *reinterpret_cast<const float4*>(g + 8 * i);
+          const float4 g1 = *reinterpret_cast<const float4*>(g + 8 * i + 4);
+          v[8 * i + 0] = bf16_lo(xv[i].x) + g0.x * v[8 * i + 0];
+          v[8 * i + 1] = bf16_hi(xv[i].x) + g0.y * v[8 * i + 1];
+          v[8 * i + 2] = bf16_lo(xv[i].y) + g0.z * v[8 * i + 2];
+          v[8 * i + 3] = bf16_hi(xv[i].y) + g0.w * v[8 * i + 3];
+          v[8 * i + 4] = bf16_lo(xv[i].z) + g1.x * v[8 * i + 4];
+          v[8 * i + 5] = bf16_hi(xv[i].z) + g1.y * v[8 * i + 5];
+          v[8 * i + 6] = bf16_lo(xv[i].w) + g1.z * v[8 * i + 6];
+          v[8 * i + 7] = bf16_hi(xv[i].w) + g1.w * v[8 * i + 7];
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint4 u = make_uint4(pack_bf16(v[8 * q + 0], v[8 * q + 1]), pack_bf16(v[8 * q + 2], v[8 * q + 3]),
+                                     pack_bf16(v[8 * q + 4], v[8 * q + 5]), pack_bf16(v[8 * q + 6], v[8 * q + 7]));
+          sts128(rowa + ((static_cast<uint32_t>(q) ^ swz) << 4), u);
+        }
+      }
+      // rows past M (no gate) keep the loaded fill; the store clips them
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_2d(tmo, box, col0 + 32 * c, wrow0);
+        bulk_commit_group();
+      }
+    }
   } else if (p.mode == EPI_SWIGLU) {
     const int col0 = nb * 128;
 #pragma unroll 1
@@ -309,19 +412,21 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tbas
 template <bool FP8>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_tcgen05(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                 const GemmParams p) {
+                 const __grid_constant__ CUtensorMap tmO, const GemmParams p) {
   constexpr int KB = FP8 ? 2 * GEMM_BK : GEMM_BK;  // K elements per stage
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + GEMM_STAGES * A_STAGE_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + GEMM_STAGES * B_STAGE_BYTES);
+  uint8_t* sR = sB + GEMM_STAGES * B_STAGE_BYTES;  // residual boxes, 2 per epilogue warp
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sR + GEMM_RES_BYTES);
   uint64_t* full = bars;
   uint64_t* empty = bars + GEMM_STAGES;
   uint64_t* acc_full = bars + 2 * GEMM_STAGES;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* mma_done = acc_empty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  uint64_t* res_bar = mma_done + 1;  // [epilogue warp][2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(res_bar + 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -337,6 +442,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       mbar_init(smem_u32(&acc_empty[a]), 128);
     }
     mbar_init(smem_u32(mma_done), 1);
+    for (int i = 0; i < 8; ++i) mbar_init(smem_u32(&res_bar[i]), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -434,21 +540,27 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     // ---------------------------------------------------------- epilogue warps
     const int quarter = warp & 3;
     const int row_in_tile = quarter * 32 + lane;
+    const bool res = p.mode == EPI_GATE_RES && p.res_tma;
+    ResStage rs{smem_u32(sR) + static_cast<uint32_t>(warp - 2) * 2 * RES_BOX_BYTES,
+                smem_u32(&res_bar[2 * (warp - 2)]), 0, 0, abort_flag, false};
     uint32_t acc = 0, acc_phase = 0;
     for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
       int mb, nb;
       tile_coords(t, p.num_m_tiles, p.num_n_tiles, p.group_n, mb, nb);
+      if (res) res_issue(rs, &tmO, nb * GEMM_BN, mb * GEMM_BM + quarter * 32, lane == 0);
       const bool got = mbar_wait(smem_u32(&acc_full[acc]), acc_phase, p.err, abort_flag);
       __syncwarp();
       if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
       const uint32_t tbase = tmem + acc * GEMM_BN + (static_cast<uint32_t>(quarter * 32) << 16);
-      epilogue_tile(p, tbase, mb * GEMM_BM, nb, row_in_tile);
+      epilogue_tile(p, tbase, mb * GEMM_BM, nb, row_in_tile, &rs, &tmO);
+      if (rs.failed) break;
       tc_fence_before();
       mbar_arrive(smem_u32(&acc_empty[acc]));
       acc ^= 1u;
       if (acc == 0) acc_phase ^= 1u;
     }
+    res_drain(rs, lane == 0);
   }
 
   tc_fence_before();
@@ -472,7 +584,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 constexpr int G2_STAGES = 6;
 constexpr uint32_t G2_A_BYTES = 128 * GEMM_BK * 2;  // 16 KB
 constexpr uint32_t G2_B_BYTES = 128 * GEMM_BK * 2;  // 16 KB
-constexpr int GEMM2_SMEM = G2_STAGES * (G2_A_BYTES + G2_B_BYTES) + 1024 + 1024;
+constexpr int GEMM2_SMEM = G2_STAGES * (G2_A_BYTES + G2_B_BYTES) + GEMM_RES_BYTES + 1024 + 1024;
 
 //
 // Grouped mode: a second problem (tensor maps tmA1 / tmB1, parameters p1)
@@ -484,20 +596,23 @@ constexpr int GEMM2_SMEM = G2_STAGES * (G2_A_BYTES + G2_B_BYTES) + 1024 + 1024;
 template <bool FP8, bool GROUPED>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     gemm_tcgen05_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                      const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
+                      const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmA1,
+                      const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmO1,
                       const __grid_constant__ GemmParams p, const __grid_constant__ GemmParams p1) {
   constexpr int KB = FP8 ? 2 * GEMM_BK : GEMM_BK;  // K elements per stage (128 bytes per row)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + G2_STAGES * G2_A_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + G2_STAGES * G2_B_BYTES);
+  uint8_t* sR = sB + G2_STAGES * G2_B_BYTES;     // residual boxes, 2 per epilogue warp
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sR + GEMM_RES_BYTES);
   uint64_t* full = bars;                         // [G2_STAGES], used in the leader
   uint64_t* empty = bars + G2_STAGES;            // [G2_STAGES], both CTAs
   uint64_t* acc_full = bars + 2 * G2_STAGES;     // [2], both CTAs
   uint64_t* acc_empty = acc_full + 2;            // [2], used in the leader
   uint64_t* mma_done = acc_empty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  uint64_t* res_bar = mma_done + 1;              // [epilogue warp][2], per CTA
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(res_bar + 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -517,6 +632,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
       mbar_init(smem_u32(&acc_empty[a]), 8);  // 4 epilogue warps in each CTA
     }
     mbar_init(smem_u32(mma_done), 1);
+    for (int i = 0; i < 8; ++i) mbar_init(smem_u32(&res_bar[i]), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -617,18 +733,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
   } else {
     const int quarter = warp & 3;
     const int row_in_tile = quarter * 32 + lane;
+    ResStage rs{smem_u32(sR) + static_cast<uint32_t>(warp - 2) * 2 * RES_BOX_BYTES,
+                smem_u32(&res_bar[2 * (warp - 2)]), 0, 0, abort_flag, false};
     uint32_t acc = 0, acc_phase = 0;
     for (int t = cl; t < total_tiles; t += ncl) {
       const bool second = GROUPED && t >= p.num_tiles;
       const GemmParams& q = second ? p1 : p;
+      const CUtensorMap* to = second ? &tmO1 : &tmO;
       int mb, nb;
       tile_coords(second ? t - p.num_tiles : t, q.num_m_tiles, q.num_n_tiles, q.group_n, mb, nb);
+      const int m0 = mb * 256 + static_cast<int>(rank) * 128;
+      if (q.mode == EPI_GATE_RES && q.res_tma) res_issue(rs, to, nb * GEMM_BN, m0 + quarter * 32, lane == 0);
       const bool got = mbar_wait(smem_u32(&acc_full[acc]), acc_phase, p.err, abort_flag);
       __syncwarp();
       if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
       const uint32_t tbase = tmem + acc * GEMM_BN + (static_cast<uint32_t>(quarter * 32) << 16);
-      epilogue_tile(q, tbase, mb * 256 + static_cast<int>(rank) * 128, nb, row_in_tile);
+      epilogue_tile(q, tbase, m0, nb, row_in_tile, &rs, to);
+      if (rs.failed) break;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
@@ -640,6 +762,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
       acc ^= 1u;
       if (acc == 0) acc_phase ^= 1u;
     }
+    res_drain(rs, lane == 0);
   }
 
   tc_fence_before();
@@ -678,8 +801,11 @@ cudaError_t gemm_set_attributes() {
 }
 
 // Tensor maps and tile counts of one problem; pair = 256-row CTA-pair tiles.
+// `to` maps the gated-residual output in 32 x 32 boxes (64-byte swizzle) when
+// the residual can move by TMA; otherwise it is a copy of `ta` that no
+// epilogue reads.
 static cudaError_t prepare_gemm(GemmParams& p, const void* A, const void* W, int W_rows, bool pair, CUtensorMap* ta,
-                                CUtensorMap* tb) {
+                                CUtensorMap* tb, CUtensorMap* to) {
   const bool fp8 = p.w_scale != nullptr;
   const int esz = fp8 ? 1 : 2;
   const int kb = fp8 ? 2 * GEMM_BK : GEMM_BK;  // 128-byte K boxes either way
@@ -689,6 +815,14 @@ static cudaError_t prepare_gemm(GemmParams& p, const void* A, const void* W, int
     return cudaErrorInvalidValue;
   if (!encode_tmap_2d(tb, W, p.K, W_rows, static_cast<uint64_t>(p.K) * esz, kb, pair ? 128 : GEMM_BN, fp8))
     return cudaErrorInvalidValue;
+  *to = *ta;
+  p.res_tma = 0;
+  if (p.mode == EPI_GATE_RES && p.out && (reinterpret_cast<uintptr_t>(p.out) & 15) == 0 &&
+      (static_cast<uint64_t>(p.ldo) * 2) % 16 == 0 && p.ldo >= p.N && p.rows_per_batch == p.out_rows_per_batch &&
+      p.out_row_off == 0) {
+    if (encode_tmap_2d(to, p.out, p.N, p.M, static_cast<uint64_t>(p.ldo) * 2, 32, 32, false, 64)) p.res_tma = 1;
+    else *to = *ta;
+  }
   p.num_n_tiles = p.mode == EPI_SWIGLU ? (p.N + 127) / 128 : (p.N + GEMM_BN - 1) / GEMM_BN;
   p.group_n = p.num_n_tiles < 16 ? p.num_n_tiles : 16;
   p.num_m_tiles = pair ? (p.M + 255) / 256 : (p.M + GEMM_BM - 1) / GEMM_BM;
@@ -697,22 +831,22 @@ static cudaError_t prepare_gemm(GemmParams& p, const void* A, const void* W, int
 }
 
 static cudaError_t launch_pair(const GemmParams& p0, const CUtensorMap& ta0, const CUtensorMap& tb0,
-                               const GemmParams& p1, const CUtensorMap& ta1, const CUtensorMap& tb1,
-                               cudaStream_t stream, int num_sms) {
+                               const CUtensorMap& to0, const GemmParams& p1, const CUtensorMap& ta1,
+                               const CUtensorMap& tb1, const CUtensorMap& to1, cudaStream_t stream, int num_sms) {
   const int total = p0.num_tiles + p1.num_tiles;
   const int pairs = num_sms / 2;
   const int grid = 2 * (total < pairs ? total : pairs);
   const bool grouped = p1.num_tiles > 0;
   if (p0.w_scale) {
     if (grouped)
-      gemm_tcgen05_pair<true, true><<<grid, GEMM_THREADS, GEMM2_SMEM, stream>>>(ta0, tb0, ta1, tb1, p0, p1);
+      gemm_tcgen05_pair<true, true><<<grid, GEMM_THREADS, GEMM2_SMEM, stream>>>(ta0, tb0, to0, ta1, tb1, to1, p0, p1);
     else
-      gemm_tcgen05_pair<true, false><<<grid, GEMM_THREADS, GEMM2_SMEM, stream>>>(ta0, tb0, ta1, tb1, p0, p1);
+      gemm_tcgen05_pair<true, false><<<grid, GEMM_THREADS, GEMM2_SMEM, stream>>>(ta0, tb0, to0, ta1, tb1, to1, p0, p1);
   } else {
     if (grouped)
-      gemm_tcgen05_pair<false, true><<<grid, GEMM_THREADS, GEMM2_SMEM, stream>>>(ta0, tb0, ta1, tb1, p0, p1);
+      gemm_tcgen05_pair<false, true><<<grid, GEMM_THREADS, GEMM2_SMEM, stream>>>(ta0, tb0, to0, ta1, tb1, to1, p0, p1);
     else
-      gemm_tcgen05_pair<false, false><<<grid, GEMM_THREADS, GEMM2_SMEM, stream>>>(ta0, tb0, ta1, tb1, p0, p1);
+      gemm_tcgen05_pair<false, false><<<grid, GEMM_THREADS, GEMM2_SMEM, stream>>>(ta0, tb0, to0, ta1, tb1, to1, p0, p1);
   }
   return cudaGetLastError();
 }
@@ -723,21 +857,21 @@ cudaError_t launch_gemm(const GemmParams& p_in, const void* A, const void* W, in
   if (p.M <= 0 || p.N <= 0) return cudaSuccess;
   const bool fp8 = p.w_scale != nullptr;
   const bool pair = p.M >= 1024 && num_sms >= 2;
-  CUtensorMap ta, tb;
-  cudaError_t e = prepare_gemm(p, A, W, W_rows, pair, &ta, &tb);
+  CUtensorMap ta, tb, to;
+  cudaError_t e = prepare_gemm(p, A, W, W_rows, pair, &ta, &tb, &to);
   if (e != cudaSuccess) return e;
   e = gemm_set_attributes();
   if (e != cudaSuccess) return e;
   if (pair) {
     GemmParams none = p;
     none.num_tiles = 0;
-    return launch_pair(p, ta, tb, none, ta, tb, stream, num_sms);
+    return launch_pair(p, ta, tb, to, none, ta, tb, to, stream, num_sms);
   }
   const int grid = p.num_tiles < num_sms ? p.num_tiles : num_sms;
   if (fp8)
-    gemm_tcgen05<true><<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, stream>>>(ta, tb, p);
+    gemm_tcgen05<true><<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, stream>>>(ta, tb, to, p);
   else
-    gemm_tcgen05<false><<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, stream>>>(ta, tb, p);
+    gemm_tcgen05<false><<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, stream>>>(ta, tb, to, p);
   return cudaGetLastError();
 }
 
@@ -752,12 +886,12 @@ cudaError_t launch_gemm_grouped(const GemmParams& p0_in, const void* A0, const v
     if (e == cudaSuccess && !empty1) e = launch_gemm(p1, A1, W1, W1_rows, stream, num_sms);
     return e;
   }
-  CUtensorMap ta0, tb0, ta1, tb1;
-  cudaError_t e = prepare_gemm(p0, A0, W0, W0_rows, true, &ta0, &tb0);
-  if (e == cudaSuccess) e = prepare_gemm(p1, A1, W1, W1_rows, true, &ta1, &tb1);
+  CUtensorMap ta0, tb0, to0, ta1, tb1, to1;
+  cudaError_t e = prepare_gemm(p0, A0, W0, W0_rows, true, &ta0, &tb0, &to0);
+  if (e == cudaSuccess) e = prepare_gemm(p1, A1, W1, W1_rows, true, &ta1, &tb1, &to1);
   if (e == cudaSuccess) e = gemm_set_attributes();
   if (e != cudaSuccess) return e;
-  return launch_pair(p0, ta0, tb0, p1, ta1, tb1, stream, num_sms);
+  return launch_pair(p0, ta0, tb0, to0, p1, ta1, tb1, to1, stream, num_sms);
 }
 
 }  // namespace af
