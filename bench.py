@@ -339,7 +339,7 @@ def run_af(args, rank, world, local_rank):
     value = world * args.steps / t_max
     clocks = clk.summary()
 
-    # ---- the per-step path (no plan, no graphs): same kernels, modulations by GEMV each step
+    # ---- the per-step path (no plan, no graphs): same kernels, the step's modulations by one GEMM each step
     direct = None
     if not args.direct:
         for i in range(2):

@@ -1337,8 +1337,21 @@ static af_status forward_impl(const af_weights* w, af_scratch* s, const float* l
                                 s->temb, st));
   }
   if (!premods) {
-    LaunchScope ls(s, KC_OTHER, 2.0 * R_ada * D, st, (B + 7) / 8);
-    AF_CUDA(launch_modulation(s->temb, B, D, ada_base(w), static_cast<int>(R_ada), s->mods, st));
+    // every modulation of the step in one tensor-core GEMM over the adaLN
+    // rows (mods[b, r] = W_ada[r] . silu(temb_b)), silu(temb) rounded to bf16
+    // as in the sampler plan: the 4.6 GB of modulation weights stream once at
+    // HBM rate, where the per-row GEMV ran at about a third of it.  Accounted
+    // by its bytes: the weight stream, not the tensor core, bounds it.
+    uint16_t* silu = reinterpret_cast<uint16_t*>(s->h1);  // h1 is free once temb is formed
+    {
+      LaunchScope ls(s, KC_OTHER, 6.0 * B * D, st);
+      AF_CUDA(launch_silu_bf16(s->temb, B * D, silu, st));
+    }
+    GemmParams gp = gemm_base(s, B, static_cast<int>(R_ada), D, EPI_STORE_F32, B);
+    gp.out_f32 = s->mods;
+    gp.ldo = static_cast<int>(R_ada);
+    LaunchScope ls(s, KC_OTHER, 2.0 * R_ada * D, st);
+    AF_CUDA(launch_gemm(gp, silu, ada_base(w), static_cast<int>(R_ada), st, s->sms));
   }
   {
     LaunchScope ls(s, KC_OTHER, 4.0 * B * Ni * D + 4.0 * B * c.in_channels * H * W, st);

@@ -658,9 +658,9 @@ __global__ void __launch_bounds__(QKN_THREADS, 1)
 }
 
 // ---------------------------------------------------------------- QK-normalised inputs on CTA pairs
-// attn_hd256_qknorm_pair: a cluster of two CTAs takes 256 query rows of one
+// attn_hd256_qknorm_pair3: a cluster of two CTAs takes 256 query rows of one
 // (sample, head), 128 per CTA, and walks the keys in tiles of 128 with
-// tcgen05.mma.cta_group::2 issued by the leader CTA:
+// tcgen05.mma.cta_group::2 issued from the leader CTA:
 //   S = Q K^T   M = 256, N = 128, K = 256: A (Q) is read from each CTA's
 //               TMEM (its 128 rows), B is half of the K tile (64 keys) from
 //               each CTA's shared memory; each CTA's TMEM receives its
@@ -670,25 +670,17 @@ __global__ void __launch_bounds__(QKN_THREADS, 1)
 //               memory; each CTA's TMEM accumulates its 128 x 256 block of O.
 // Per SM that is 64 KB of K/V per 128 keys instead of 128 KB, and every MMA
 // has N >= 128 (full tensor-core rate).  TMEM per CTA: O [0, 256), S
-// [256, 384), Q [384, 512).  Shared memory per CTA: two P buffers (128 x 128
-// bf16, 32 KB each), K and V halves double-buffered (4 x 32 KB).  The Q tile
-// lands in the two P buffers and the softmax warps move it to TMEM before
-// the first P is written; each thread copies exactly the rows of the P slots
-// it later overwrites, so no barrier separates the two uses.
-// With Q in TMEM the S products read only K from shared memory (a third of
-// the operand bytes per cycle), which leaves bandwidth for the softmax
-// warps' P stores; with two P buffers P_{j+1} is written while PV_j still
-// reads P_j, so the softmax of one tile no longer waits for the previous
-// tile's PV.
-// Softmax (fixed shift, as for attn_hd256_qknorm): warpgroup g of each CTA
-// owns keys [64 g, 64 g + 64) of every S tile; their partial row sums are
-// added at the end.  The leader issues S_{j+1} as soon as both CTAs' softmax
-// warps have read S_j out of TMEM, then PV_j once P_j is published, so the
-// tensor core computes the next scores while the softmax warps work.
-// Barriers that gather both CTAs live in the leader (TMA completions, S/P
-// handshakes); commits are multicast to both CTAs.  The follower's softmax
-// warps arrive directly on the leader's S/P barriers (CTA-scope release; a
-// cluster-scope release there costs ~1.2k cycles).
+// [256, 384), Q [384, 512).  With Q in TMEM the S products read only K from
+// shared memory, which leaves bandwidth for the softmax warps' P stores.
+// Softmax (fixed shift, as for attn_hd256_qknorm): each softmax warpgroup
+// owns a slice of the keys of every S tile; the partial row sums are added
+// at the end.  S_{j+1} is issued as soon as both CTAs' softmax warps have
+// read S_j out of TMEM, PV_j once P_j is published, so the tensor core
+// computes the next scores while the softmax warps work.  Barriers that
+// gather both CTAs live in the leader (TMA completions, S/P handshakes);
+// commits are multicast to both CTAs.  The follower's softmax warps arrive
+// directly on the leader's S/P barriers (CTA-scope release; a cluster-scope
+// release there costs ~1.2k cycles).
 // D (+)= A * B over the CTA pair with A in TMEM: each CTA's 128 rows of A are
 // read from its own TMEM at a_tmem (two consecutive K elements per 32-bit
 // column), B split along N between the two CTAs' shared memory.
@@ -705,333 +697,25 @@ __device__ __forceinline__ void mma_bf16_ts_pair(uint32_t d_tmem, uint32_t a_tme
 constexpr int AP_BN = 128;
 constexpr uint32_t AP_KH_BYTES = 64 * AT_HD * 2;      // 32 KB: 64 keys x 256
 constexpr uint32_t AP_VH_BYTES = AP_BN * 128 * 2;     // 32 KB: 128 keys x 128 columns
-constexpr uint32_t AP_P_BYTES = 128 * AP_BN * 2;      // 32 KB (two of them hold the 64 KB Q tile first)
-constexpr int AP_SMEM = 2 * AP_P_BYTES + 2 * AP_KH_BYTES + 2 * AP_VH_BYTES + 2 * 128 * 4 + 256 + 1024;
+constexpr uint32_t AP_P_BYTES = 128 * AP_BN * 2;      // 32 KB: 128 rows x 128 keys
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
-    attn_hd256_qknorm_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                           const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sP = smem;                     // 2 buffers; the Q tile first
-  uint8_t* sK = sP + 2 * AP_P_BYTES;      // 2 buffers
-  uint8_t* sV = sK + 2 * AP_KH_BYTES;     // 2 buffers
-  float* xsum = reinterpret_cast<float*>(sV + 2 * AP_VH_BYTES);  // [wg 2][row 128]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + 2 * AP_VH_BYTES + 2 * 128 * 4);
-  uint64_t* q_smem = bars + 0;     // per CTA: this CTA's Q tile has landed
-  uint64_t* k_full = bars + 1;     // [2] leader: both K halves
-  uint64_t* v_full = bars + 3;     // [2] leader: both V halves
-  uint64_t* k_empty = bars + 5;    // [2] both CTAs (multicast commit)
-  uint64_t* v_empty = bars + 7;    // [2] both CTAs
-  uint64_t* s_full = bars + 9;     // both CTAs
-  uint64_t* s_empty = bars + 10;   // leader: 16 softmax warps of both CTAs
-  uint64_t* p_full = bars + 11;    // [2] leader: 16 softmax warps of both CTAs
-  uint64_t* pv_done = bars + 13;   // [2] both CTAs
-  uint64_t* q_tmem = bars + 15;    // leader: 16 softmax warps have moved Q to TMEM
-  uint64_t* mma_done = bars + 16;  // leader
-  uint64_t* lbar = bars + 17;      // per CTA: 8 softmax warps
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const uint32_t rank = cluster_ctarank();
-  const bool leader = rank == 0;
-  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
-  const int h = blockIdx.y, b = blockIdx.z;
-  const int bh = b * p.H + h;
-  const int q0 = pair * 256 + static_cast<int>(rank) * 128;
-  const int nkv = (p.N + AP_BN - 1) / AP_BN;
-  const int kv0 = static_cast<int>((static_cast<long long>(pair) * nkv) / npairs);
-  auto kv_tile = [&](int j) { const int t = j + kv0; return t < nkv ? t : t - nkv; };
-
-  if (threadIdx.x == 0) {
-    mbar_init(smem_u32(q_smem), 1);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(smem_u32(&k_full[i]), 1);
-      mbar_init(smem_u32(&v_full[i]), 1);
-      mbar_init(smem_u32(&k_empty[i]), 1);
-      mbar_init(smem_u32(&v_empty[i]), 1);
-      mbar_init(smem_u32(&p_full[i]), 2 * AT_SOFTMAX_WARPS);
-      mbar_init(smem_u32(&pv_done[i]), 1);
-    }
-    mbar_init(smem_u32(s_full), 1);
-    mbar_init(smem_u32(s_empty), 2 * AT_SOFTMAX_WARPS);
-    mbar_init(smem_u32(q_tmem), 2 * AT_SOFTMAX_WARPS);
-    mbar_init(smem_u32(mma_done), 1);
-    mbar_init(smem_u32(lbar), AT_SOFTMAX_WARPS);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (warp == 0 && lane == 0) {
-    prefetch_tmap(&tmQ);
-    prefetch_tmap(&tmK);
-    prefetch_tmap(&tmV);
-  }
-  if (warp == 1) {
-    tmem_alloc_pair(smem_u32(tmem_slot), 512);
-    tmem_relinquish_pair();
-  }
-  tc_fence_before();
-  __syncthreads();
-  cluster_sync();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-  const uint32_t tO = tmem;
-  const uint32_t tS = tmem + 256;
-  const uint32_t tQ = tmem + 384;
-  volatile int never = 0;
-
-  if (warp == 0 || warp == AT_V_WARP) {
-    // warp 0: this CTA's Q tile, then the K halves (keys [64 rank, +64) of
-    // each tile); last warp: the V halves (head-dim columns [128 rank, +128)).
-    if (lane == 0) {
-      const bool is_k = warp == 0;
-      uint64_t* full = is_k ? k_full : v_full;
-      uint64_t* empty = is_k ? k_empty : v_empty;
-      const uint32_t half = is_k ? AP_KH_BYTES : AP_VH_BYTES;
-      uint8_t* buf = is_k ? sK : sV;
-      bool ok = true, issued = false;
-      if (is_k) {
-        mbar_arrive_expect_tx(smem_u32(q_smem), 2 * AP_P_BYTES);
-        for (int c = 0; c < 4; ++c)
-          tma_load_3d(smem_u32(sP + c * (128 * 128)), &tmQ, smem_u32(q_smem), c * 64, q0, bh);
-        issued = true;
-      }
-      for (int j = 0; j < nkv; ++j) {
-        const int s = j & 1;
-        const uint32_t ph = (j >> 1) & 1;
-        if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1u, p.err, abort_flag)) { ok = false; break; }
-        if (leader) mbar_arrive_expect_tx(smem_u32(&full[s]), 2 * half);
-        const uint32_t fb = mapa_shared(smem_u32(&full[s]), 0);
-        const int key0 = kv_tile(j) * AP_BN;
-        if (is_k) {
-          for (int c = 0; c < 4; ++c)
-            tma_load_3d_pair(smem_u32(buf + s * half + c * (64 * 128)), &tmK, fb, c * 64,
-                             key0 + static_cast<int>(rank) * 64, bh);
-        } else {
-          for (int c = 0; c < 2; ++c)
-            tma_load_3d_pair(smem_u32(buf + s * half + c * (AP_BN * 128)), &tmV, fb,
-                             static_cast<int>(rank) * 128 + c * 64, key0, bh);
-        }
-        issued = true;
-      }
-      if (!ok && issued) {
-        const uint64_t t0 = globaltimer();
-        while (globaltimer() - t0 < 200000ull) {
-        }
-      }
-    }
-  } else if (warp == 1) {
-    if (lane == 0 && leader) {
-      const uint32_t idesc_qk = make_idesc_bf16(256, AP_BN, false, false);
-      const uint32_t idesc_pv = make_idesc_bf16(256, AT_HD, false, true);
-      bool ok = mbar_wait(smem_u32(q_tmem), 0, p.err, abort_flag);
-      // S_j into the single S buffer: the K half of tile j has landed and the
-      // softmax warps of both CTAs have read S_{j-1}.
-      auto issue_s = [&](int j) -> bool {
-        const int s = j & 1;
-        if (!mbar_wait(smem_u32(&k_full[s]), (j >> 1) & 1, p.err, abort_flag)) return false;
-        if (j > 0 && !mbar_wait(smem_u32(s_empty), (j - 1) & 1, p.err, abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t kaddr = smem_u32(sK + s * AP_KH_BYTES);
-        const uint64_t kdesc = make_sdesc(kaddr, 16, 1024, SWZ_128B);
-#pragma unroll
-        for (int kk = 0; kk < AT_HD / 16; ++kk) {
-          const uint32_t c = kk >> 2, off = (kk & 3) * 32;
-          const uint64_t bd = kdesc + static_cast<uint64_t>((c * (64 * 128) + off) >> 4);
-          mma_bf16_ts_pair(tS, tQ + kk * 8, bd, idesc_qk, kk > 0 ? 1u : 0u);
-        }
-        mma_commit_pair(smem_u32(s_full), 0x3);
-        mma_commit_pair(smem_u32(&k_empty[s]), 0x3);
-        return true;
-      };
-      if (ok) ok = issue_s(0);
-      for (int j = 0; j < nkv && ok; ++j) {
-        const int s = j & 1;
-        if (j + 1 < nkv && !issue_s(j + 1)) { ok = false; break; }
-        if (!mbar_wait(smem_u32(&p_full[s]), (j >> 1) & 1, p.err, abort_flag)) { ok = false; break; }
-        if (!mbar_wait(smem_u32(&v_full[s]), (j >> 1) & 1, p.err, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        const uint64_t pdesc = make_sdesc(smem_u32(sP + s * AP_P_BYTES), 16, 1024, SWZ_128B);
-        const uint64_t vdesc = make_sdesc(smem_u32(sV + s * AP_VH_BYTES), AP_BN * 128, 1024, SWZ_128B);
-#pragma unroll
-        for (int kk = 0; kk < AP_BN / 16; ++kk) {
-          const uint32_t c = kk >> 2, off = (kk & 3) * 32;
-          const uint64_t ad = pdesc + static_cast<uint64_t>((c * (128 * 128) + off) >> 4);
-          const uint64_t bd = vdesc + static_cast<uint64_t>((kk * (16 * 128)) >> 4);
-          mma_bf16_ss_pair(tO, ad, bd, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
-        }
-        mma_commit_pair(smem_u32(&pv_done[s]), 0x3);
-        mma_commit_pair(smem_u32(&v_empty[s]), 0x3);
-      }
-      mma_commit_pair(smem_u32(mma_done), 0x1);
-      mbar_wait(smem_u32(mma_done), 0, nullptr, &never, 100000000ull);
-    }
-  } else {
-    // ---------------------------------------------------------------- softmax: group g owns keys [64 g, 64 g + 64)
-    const int wg = (warp - 2) >> 2;
-    const int quarter = warp & 3;
-    const int row = quarter * 32 + lane;
-    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const float c = p.scale_log2;
-    const float off = -QKN_OFFSET_LOG2;
-    int klo, khi;
-    key_mask_range(p, b, klo, khi);
-    const uint32_t s_empty_l = mapa_shared(smem_u32(s_empty), 0);
-    const uint32_t p_full_l = mapa_shared(smem_u32(p_full), 0);
-    float l = 0.f;
-    bool ok = true;
-    {
-      // This thread's Q row, 64-column chunks wg and wg + 2 (the P slots
-      // (buffer 0, group wg) and (buffer 1, group wg) that it overwrites
-      // later), from shared memory into TMEM columns [32 chunk, +32).
-      const bool got = mbar_wait(smem_u32(q_smem), 0, p.err, abort_flag);
-      __syncwarp();
-      if (!__all_sync(0xffffffffu, got)) {
-        ok = false;
-      } else {
-        for (int cc = wg; cc < 4; cc += 2) {
-          const uint8_t* qrow = sP + cc * (128 * 128) + row * 128;
-          uint32_t qv[32];
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const uint4 u = *reinterpret_cast<const uint4*>(qrow + ((q ^ (row & 7)) << 4));
-            qv[4 * q] = u.x;
-            qv[4 * q + 1] = u.y;
-            qv[4 * q + 2] = u.z;
-            qv[4 * q + 3] = u.w;
-          }
-          tmem_st32(tQ + cc * 32 + lane_off, qv);
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(q_tmem), 0));
-      }
-    }
-    for (int j = 0; j < nkv && ok; ++j) {
-      const int s = j & 1;
-      const bool got = mbar_wait(smem_u32(s_full), j & 1, p.err, abort_flag);
-      __syncwarp();
-      if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
-      tc_fence_after();
-      uint32_t r0[32], r1[32];
-      tmem_ld32(tS + 64 * wg + lane_off, r0);
-      tmem_ld32(tS + 64 * wg + 32 + lane_off, r1);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(s_empty_l);
-      const int kbase = kv_tile(j) * AP_BN + 64 * wg;
-      const int kvalid = p.N - kbase, mlo = klo - kbase, mhi = khi - kbase;
-      const bool partial = kvalid < 64 || (mlo < mhi && mlo < 64 && mhi > 0);
-      auto dead = [&](int i) { return i >= kvalid || (i >= mlo && i < mhi); };
-      uint32_t pk[32];
-      float rs = 0.f;
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        float e0 = ex2_approx(fmaf(__uint_as_float(r0[2 * i]), c, off));
-        float e1 = ex2_approx(fmaf(__uint_as_float(r0[2 * i + 1]), c, off));
-        float e2 = ex2_approx(fmaf(__uint_as_float(r1[2 * i]), c, off));
-        float e3 = ex2_approx(fmaf(__uint_as_float(r1[2 * i + 1]), c, off));
-        if (partial) {
-          if (dead(2 * i)) e0 = 0.f;
-          if (dead(2 * i + 1)) e1 = 0.f;
-          if (dead(32 + 2 * i)) e2 = 0.f;
-          if (dead(32 + 2 * i + 1)) e3 = 0.f;
-        }
-        rs += (e0 + e1) + (e2 + e3);
-        pk[i] = pack_bf16(e0, e1);
-        pk[16 + i] = pack_bf16(e2, e3);
-      }
-      l += rs;
-      // P buffer s is free once PV_{j-2} has completed
-      if (j >= 2) {
-        const bool g2 = mbar_wait(smem_u32(&pv_done[s]), ((j - 2) >> 1) & 1, p.err, abort_flag);
-        __syncwarp();
-        if (!__all_sync(0xffffffffu, g2)) { ok = false; break; }
-      }
-      uint8_t* prow = sP + s * AP_P_BYTES + wg * (128 * 128) + row * 128;
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        uint4 v = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-        *reinterpret_cast<uint4*>(prow + ((q ^ (row & 7)) << 4)) = v;
-      }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(p_full_l + s * 8);
-    }
-    if (ok) {
-      xsum[wg * 128 + row] = l;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(lbar));
-      const int jl = nkv - 1;
-      const bool g3 = mbar_wait(smem_u32(lbar), 0, p.err, abort_flag) &&
-                      mbar_wait(smem_u32(&pv_done[jl & 1]), (jl >> 1) & 1, p.err, abort_flag);
-      __syncwarp();
-      if (__all_sync(0xffffffffu, g3)) {
-        tc_fence_after();
-        const float inv = 1.0f / (l + xsum[(wg ^ 1) * 128 + row]);
-        const int qrow = q0 + row;
-        const bool row_ok = qrow < p.N;
-        uint16_t* dst = nullptr;
-        if (row_ok) {
-          if (qrow < p.split)
-            dst = p.out_a + (static_cast<size_t>(b) * p.split + qrow) * p.ldo + h * AT_HD;
-          else
-            dst = p.out_b + (static_cast<size_t>(b) * (p.N - p.split) + (qrow - p.split)) * p.ldo + h * AT_HD;
-          dst += 128 * wg;
-        }
-        for (int cc = 0; cc < 4; ++cc) {
-          uint32_t o[32];
-          tmem_ld32(tO + 128 * wg + cc * 32 + lane_off, o);
-          tmem_wait_ld();
-          if (row_ok) {
-            uint4* d = reinterpret_cast<uint4*>(dst + cc * 32);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              uint4 u;
-              u.x = pack_bf16(__uint_as_float(o[8 * i + 0]) * inv, __uint_as_float(o[8 * i + 1]) * inv);
-              u.y = pack_bf16(__uint_as_float(o[8 * i + 2]) * inv, __uint_as_float(o[8 * i + 3]) * inv);
-              u.z = pack_bf16(__uint_as_float(o[8 * i + 4]) * inv, __uint_as_float(o[8 * i + 5]) * inv);
-              u.w = pack_bf16(__uint_as_float(o[8 * i + 6]) * inv, __uint_as_float(o[8 * i + 7]) * inv);
-              d[i] = u;
-            }
-          }
-        }
-      }
-    }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  cluster_sync();
-  if (warp == 1) {
-    __syncwarp();
-    tc_fence_after();
-    tmem_dealloc_pair(tmem, 512);
-  }
-}
-
-// ---------------------------------------------------------------- three K/V stages, four softmax warpgroups
-// attn_hd256_qknorm_pair3: the same computation and cluster layout as
-// attn_hd256_qknorm_pair, arranged for a shorter period per 128-key tile.
-// Two limits each hold the two-stage layout near 2700 cycles per tile
-// against 2048 cycles of MMA work: (a) the K / V stream -- a stage is
-// refilled only when the MMA that read it completes, so with two stages a
-// load has 2T - 1024 cycles to land and a ~4400-cycle load needs
-// T >= 2700 -- and (b) the S -> softmax -> P chain.  Here K and V have three
-// stages each (T >= (1024 + L) / 3), and four softmax warpgroups per CTA
-// (16 warps; warpgroup g owns keys [32 g, 32 g + 32) of every S tile) halve
-// each thread's exponentials per tile.  The shared memory for the third
-// stages comes from using one P buffer: the softmax of tile j + 1 stores its
-// P only after PV_j completes, which the tensor core overlaps with S_{j+2}.
-// The Q tile lands in V stages 0 and 1; the softmax warps move it to TMEM
-// and release those stages (q_moved) before the first V loads.  Shared
-// memory per CTA: P 32 KB, K 3 x 32 KB, V 3 x 32 KB (the row sums reuse the
-// P buffer once the last PV has read it).
+// The layout of attn_hd256_qknorm_pair3 is arranged for a short period per
+// 128-key tile.  Two limits each held an earlier two-stage layout (two P
+// buffers, two softmax warpgroups) near 2700 cycles per tile against 2048
+// cycles of MMA work: (a) the K / V stream -- a stage is refilled only when
+// the MMA that read it completes, so with two stages a load has 2T - 1024
+// cycles to land and a ~4400-cycle load needs T >= 2700 -- and (b) the
+// S -> softmax -> P chain.  Here K and V have three stages each
+// (T >= (1024 + L) / 3), and four softmax warpgroups per CTA (16 warps;
+// warpgroup g owns keys [32 g, 32 g + 32) of every S tile) halve each
+// thread's exponentials per tile.  The shared memory for the third stages
+// comes from using one P buffer: the softmax of tile j + 1 stores its P only
+// after PV_j completes, which the tensor core overlaps with S_{j+2}.  The Q
+// tile lands in V stages 0 and 1; the softmax warps move it to TMEM and
+// release those stages (q_moved) before the first V loads.  Shared memory
+// per CTA: P 32 KB, K 3 x 32 KB, V 3 x 32 KB (the row sums reuse the P
+// buffer once the last PV has read it).  The S and PV products are issued
+// by two threads (below).
 constexpr int AP3_NWG = 4;
 constexpr int AP3_SM_WARPS = 4 * AP3_NWG;
 constexpr int AP3_V_WARP = 2 + AP3_SM_WARPS;
@@ -1411,8 +1095,6 @@ cudaError_t attention_set_attributes() {
   cudaError_t e = cudaFuncSetAttribute(attn_hd256_online, cudaFuncAttributeMaxDynamicSharedMemorySize, AT_SMEM);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(attn_hd256_qknorm, cudaFuncAttributeMaxDynamicSharedMemorySize, QKN_SMEM);
-  if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(attn_hd256_qknorm_pair, cudaFuncAttributeMaxDynamicSharedMemorySize, AP_SMEM);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(attn_hd256_qknorm_pair3, cudaFuncAttributeMaxDynamicSharedMemorySize, AP3_SMEM);
   if (e != cudaSuccess) return e;

@@ -101,9 +101,10 @@ def test_sampler_graph_replay_is_bit_identical(af):
 
 
 def test_sampler_close_to_direct_steps(af):
-    """Precomputed modulations round silu(temb) to bf16 for the tensor-core
-    GEMM; the per-step path keeps it in fp32.  The two loops agree to well
-    inside the stack tolerance."""
+    """The plan precomputes every step's modulations; the per-step path
+    computes the step's own with the same tensor-core GEMM (silu(temb)
+    rounded to bf16 on both).  The two loops agree to well inside the stack
+    tolerance."""
     cfg = tiny_config()
     n = 3
     w, s, drawn, x0, text = _setup(af, cfg, 77, 1, 16, 16, 8)
