@@ -658,29 +658,27 @@ __global__ void __launch_bounds__(QKN_THREADS, 1)
 }
 
 // ---------------------------------------------------------------- QK-normalised inputs on CTA pairs
-// attn_hd256_qknorm_pair3: a cluster of two CTAs takes 256 query rows of one
+// attn_hd256_qknorm_pair: a cluster of two CTAs takes 256 query rows of one
 // (sample, head), 128 per CTA, and walks the keys in tiles of 128 with
 // tcgen05.mma.cta_group::2 issued from the leader CTA:
-//   S = Q K^T   M = 256, N = 128, K = 256: A (Q) is read from each CTA's
-//               TMEM (its 128 rows), B is half of the K tile (64 keys) from
-//               each CTA's shared memory; each CTA's TMEM receives its
-//               128 x 128 block of S.
-//   O += P V    M = 256, N = 256, K = 128: each CTA supplies its 128 rows of
-//               P and half of the V tile (128 head-dim columns) from shared
-//               memory; each CTA's TMEM accumulates its 128 x 256 block of O.
+//   S = Q K^T   M = 256, N = 128, K = 256: A is each CTA's 128 Q rows, B half
+//               of the K tile (64 keys), both from that CTA's shared memory;
+//               each CTA's TMEM receives its 128 x 128 block of S.
+//   O += P V    M = 256, N = 256, K = 128: A is each CTA's 128 rows of P, read
+//               from its own TMEM; B is half of the V tile (128 head-dim
+//               columns) from shared memory; each CTA's TMEM accumulates its
+//               128 x 256 block of O.
 // Per SM that is 64 KB of K/V per 128 keys instead of 128 KB, and every MMA
-// has N >= 128 (full tensor-core rate).  TMEM per CTA: O [0, 256), S
-// [256, 384), Q [384, 512).  With Q in TMEM the S products read only K from
-// shared memory, which leaves bandwidth for the softmax warps' P stores.
-// Softmax (fixed shift, as for attn_hd256_qknorm): each softmax warpgroup
-// owns a slice of the keys of every S tile; the partial row sums are added
-// at the end.  S_{j+1} is issued as soon as both CTAs' softmax warps have
-// read S_j out of TMEM, PV_j once P_j is published, so the tensor core
-// computes the next scores while the softmax warps work.  Barriers that
-// gather both CTAs live in the leader (TMA completions, S/P handshakes);
-// commits are multicast to both CTAs.  The follower's softmax warps arrive
-// directly on the leader's S/P barriers (CTA-scope release; a cluster-scope
-// release there costs ~1.2k cycles).
+// has N >= 128 (full tensor-core rate).  Softmax (fixed shift, as for
+// attn_hd256_qknorm): each softmax warpgroup owns a slice of the keys of
+// every S tile; the partial row sums are added at the end.  S_{j+1} is
+// issued as soon as both CTAs' softmax warps have read S_j out of TMEM,
+// PV_j once P_j is published, so the tensor core computes the next scores
+// while the softmax warps work.  Barriers that gather both CTAs live in the
+// leader (TMA completions, S/P handshakes); commits are multicast to both
+// CTAs.  The follower's softmax warps arrive directly on the leader's S/P
+// barriers (CTA-scope release; a cluster-scope release there costs ~1.2k
+// cycles).
 // D (+)= A * B over the CTA pair with A in TMEM: each CTA's 128 rows of A are
 // read from its own TMEM at a_tmem (two consecutive K elements per 32-bit
 // column), B split along N between the two CTAs' shared memory.
@@ -697,55 +695,77 @@ __device__ __forceinline__ void mma_bf16_ts_pair(uint32_t d_tmem, uint32_t a_tme
 constexpr int AP_BN = 128;
 constexpr uint32_t AP_KH_BYTES = 64 * AT_HD * 2;      // 32 KB: 64 keys x 256
 constexpr uint32_t AP_VH_BYTES = AP_BN * 128 * 2;     // 32 KB: 128 keys x 128 columns
-constexpr uint32_t AP_P_BYTES = 128 * AP_BN * 2;      // 32 KB: 128 rows x 128 keys
+constexpr uint32_t AP_Q_BYTES = 128 * AT_HD * 2;      // 64 KB: 128 rows x 256
 
-// The layout of attn_hd256_qknorm_pair3 is arranged for a short period per
-// 128-key tile.  Two limits each held an earlier two-stage layout (two P
-// buffers, two softmax warpgroups) near 2700 cycles per tile against 2048
-// cycles of MMA work: (a) the K / V stream -- a stage is refilled only when
-// the MMA that read it completes, so with two stages a load has 2T - 1024
-// cycles to land and a ~4400-cycle load needs T >= 2700 -- and (b) the
-// S -> softmax -> P chain.  Here K and V have three stages each
-// (T >= (1024 + L) / 3), and four softmax warpgroups per CTA (16 warps;
-// warpgroup g owns keys [32 g, 32 g + 32) of every S tile) halve each
-// thread's exponentials per tile.  The shared memory for the third stages
-// comes from using one P buffer: the softmax of tile j + 1 stores its P only
-// after PV_j completes, which the tensor core overlaps with S_{j+2}.  The Q
-// tile lands in V stages 0 and 1; the softmax warps move it to TMEM and
-// release those stages (q_moved) before the first V loads.  Shared memory
-// per CTA: P 32 KB, K 3 x 32 KB, V 3 x 32 KB (the row sums reuse the P
-// buffer once the last PV has read it).  The S and PV products are issued
-// by two threads (below).
-constexpr int AP3_NWG = 4;
-constexpr int AP3_SM_WARPS = 4 * AP3_NWG;
-constexpr int AP3_V_WARP = 2 + AP3_SM_WARPS;
-constexpr int AP3_PV_WARP = AP3_V_WARP + 1;
-constexpr int AP3_THREADS = 32 * (AP3_PV_WARP + 1);
-constexpr int AP3_KPW = AP_BN / AP3_NWG;   // 32 keys per warpgroup
-constexpr int AP3_STAGES = 3;
-constexpr int AP3_SMEM = AP_P_BYTES + AP3_STAGES * AP_KH_BYTES + AP3_STAGES * AP_VH_BYTES + 256 + 1024;
+// Layout.  Q stays in shared memory for the S products, which leaves TMEM
+// room for two P buffers: the softmax warps write P_j into TMEM with
+// tcgen05.st (no shared-memory store, no proxy fence) and the PV product
+// reads it from there.  TMEM per CTA: O [0, 256), S [256, 384), P_0
+// [384, 448), P_1 [448, 512).  Shared memory per CTA: Q 64 KB, K 3 x 32 KB,
+// V 2 x 32 KB (the row sums reuse a V stage after the last PV).  K has three
+// stages (a K half takes ~900-4400 cycles from load to landing, and a stage
+// is refilled only when the S product that read it completes), V two (a V
+// stage is refilled when its PV completes and is next needed two tiles
+// later).  Four softmax warpgroups of 32 keys each (TMEM lane quarters
+// shared by warps w, w + 4, w + 8, w + 12); P buffer j & 1 is rewritten only
+// after PV_{j-2} completes, so the softmax never waits for the PV product
+// just before it.  Each softmax warp reads S_{j+1} out of TMEM before
+// publishing P_j when S_{j+1} has already completed.  The S and PV products
+// are issued by two threads: the barrier checks of one overlap the other's
+// MMAs in the tensor pipe (one thread doing both left a gap of a few hundred
+// cycles at every switch).  Earlier layouts, measured: Q in TMEM with P in
+// shared memory (one or two P buffers, K and V stages 2 + 2, 3 + 3, 3 + 2 or
+// a shared ring of 5) ran at ~2580-2870 cycles per tile, bound by the
+// softmax warps' P store, proxy fence and arrival; this one is 6-8% faster.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+constexpr int PAIR_NWG = 4;
+constexpr int PAIR_SM_WARPS = 4 * PAIR_NWG;
+constexpr int PAIR_V_WARP = 2 + PAIR_SM_WARPS;
+constexpr int PAIR_PV_WARP = PAIR_V_WARP + 1;
+constexpr int PAIR_THREADS = 32 * (PAIR_PV_WARP + 1);
+constexpr int PAIR_KPW = AP_BN / PAIR_NWG;   // 32 keys per warpgroup
+constexpr int PAIR_KST = 3;
+constexpr int PAIR_VST = 2;
+constexpr int PAIR_SMEM = AP_Q_BYTES + PAIR_KST * AP_KH_BYTES + PAIR_VST * AP_VH_BYTES + 256 + 1024;
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AP3_THREADS, 1)
-    attn_hd256_qknorm_pair3(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+// Non-suspending test of an mbarrier phase.
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred P1;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 P1, [%1], %2;\n\t"
+      "selp.b32 %0, 1, 0, P1;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
+    attn_hd256_qknorm_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                             const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sP = smem;                                    // one P buffer (row sums at the end)
-  uint8_t* sK = sP + AP_P_BYTES;                         // AP3_STAGES buffers
-  uint8_t* sV = sK + AP3_STAGES * AP_KH_BYTES;           // AP3_STAGES buffers; the Q tile first (stages 0, 1)
-  float* xsum = reinterpret_cast<float*>(sP);            // [wg 4][row 128], after the last PV
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + AP3_STAGES * AP_VH_BYTES);
-  uint64_t* q_smem = bars + 0;                 // per CTA: this CTA's Q tile has landed
+  uint8_t* sQ = smem;                                    // this CTA's 128 Q rows (64 KB)
+  uint8_t* sK = sQ + AP_Q_BYTES;                     // PAIR_KST stages
+  uint8_t* sV = sK + PAIR_KST * AP_KH_BYTES;              // PAIR_VST stages (row sums at the end)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + PAIR_VST * AP_VH_BYTES);
+  uint64_t* q_full = bars + 0;                 // leader: both CTAs' Q tiles
   uint64_t* k_full = bars + 1;                 // [3] leader: both K halves
-  uint64_t* v_full = bars + 4;                 // [3] leader: both V halves
-  uint64_t* k_empty = bars + 7;                // [3] both CTAs (multicast commit)
-  uint64_t* v_empty = bars + 10;               // [3] both CTAs
-  uint64_t* s_full = bars + 13;                // both CTAs
-  uint64_t* s_empty = bars + 14;               // leader: softmax warps of both CTAs
-  uint64_t* p_full = bars + 15;                // leader: softmax warps of both CTAs
-  uint64_t* pv_done = bars + 16;               // both CTAs
-  uint64_t* q_tmem = bars + 17;                // leader: softmax warps of both CTAs have moved Q to TMEM
-  uint64_t* q_moved = bars + 18;               // per CTA: this CTA's Q copy is done (V stages 0, 1 free)
+  uint64_t* k_empty = bars + 4;                // [3] both CTAs (multicast commit)
+  uint64_t* v_full = bars + 7;                 // [2] leader: both V halves
+  uint64_t* v_empty = bars + 9;                // [2] both CTAs
+  uint64_t* s_full = bars + 11;                // both CTAs
+  uint64_t* s_empty = bars + 12;               // leader: softmax warps of both CTAs
+  uint64_t* p_full = bars + 13;                // [2] leader: softmax warps of both CTAs
+  uint64_t* pv_done = bars + 15;               // [2] both CTAs
   uint64_t* mma_done = bars + 19;              // leader: the S issuer's MMAs
   uint64_t* lbar = bars + 20;                  // per CTA: row sums written
   uint64_t* mma_done_pv = bars + 21;           // leader: the PV issuer's MMAs
@@ -765,22 +785,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AP3_THREADS, 1)
   auto kv_tile = [&](int j) { const int t = j + kv0; return t < nkv ? t : t - nkv; };
 
   if (threadIdx.x == 0) {
-    mbar_init(smem_u32(q_smem), 1);
-    for (int i = 0; i < AP3_STAGES; ++i) {
+    mbar_init(smem_u32(q_full), 1);
+    for (int i = 0; i < PAIR_KST; ++i) {
       mbar_init(smem_u32(&k_full[i]), 1);
-      mbar_init(smem_u32(&v_full[i]), 1);
       mbar_init(smem_u32(&k_empty[i]), 1);
+    }
+    for (int i = 0; i < PAIR_VST; ++i) {
+      mbar_init(smem_u32(&v_full[i]), 1);
       mbar_init(smem_u32(&v_empty[i]), 1);
     }
     mbar_init(smem_u32(s_full), 1);
-    mbar_init(smem_u32(s_empty), 2 * AP3_SM_WARPS);
-    mbar_init(smem_u32(p_full), 2 * AP3_SM_WARPS);
-    mbar_init(smem_u32(pv_done), 1);
-    mbar_init(smem_u32(q_tmem), 2 * AP3_SM_WARPS);
-    mbar_init(smem_u32(q_moved), AP3_SM_WARPS);
+    mbar_init(smem_u32(s_empty), 2 * PAIR_SM_WARPS);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&p_full[i]), 2 * PAIR_SM_WARPS);
+      mbar_init(smem_u32(&pv_done[i]), 1);
+    }
     mbar_init(smem_u32(mma_done), 1);
     mbar_init(smem_u32(mma_done_pv), 1);
-    mbar_init(smem_u32(lbar), AP3_SM_WARPS);
+    mbar_init(smem_u32(lbar), PAIR_SM_WARPS);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -800,31 +822,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AP3_THREADS, 1)
   const uint32_t tmem = *tmem_slot;
   const uint32_t tO = tmem;
   const uint32_t tS = tmem + 256;
-  const uint32_t tQ = tmem + 384;
+  const uint32_t tP = tmem + 384;  // P buffer b at tP + 64 b
   volatile int never = 0;
 
-  if (warp == 0 || warp == AP3_V_WARP) {
-    // warp 0: this CTA's Q tile (into V stages 0 and 1), then the K halves
-    // (keys [64 rank, +64) of each tile); last warp: the V halves (head-dim
-    // columns [128 rank, +128)), V stages 0 and 1 only once Q has left them.
+  if (warp == 0 || warp == PAIR_V_WARP) {
+    // warp 0: this CTA's Q tile (into the V stages), then the K halves (keys
+    // [64 rank, +64) of each tile); the V warp: the V halves (head-dim
+    // columns [128 rank, +128))
     if (lane == 0) {
       const bool is_k = warp == 0;
+      const int nst = is_k ? PAIR_KST : PAIR_VST;
       uint64_t* full = is_k ? k_full : v_full;
       uint64_t* empty = is_k ? k_empty : v_empty;
       const uint32_t half = is_k ? AP_KH_BYTES : AP_VH_BYTES;
       uint8_t* buf = is_k ? sK : sV;
-      bool ok = true, issued = false;
+      bool ok = true;
       if (is_k) {
-        mbar_arrive_expect_tx(smem_u32(q_smem), 2 * AP_P_BYTES);
-        for (int c = 0; c < 4; ++c)
-          tma_load_3d(smem_u32(sV + c * (128 * 128)), &tmQ, smem_u32(q_smem), c * 64, q0, bh);
-        issued = true;
-      } else {
-        ok = mbar_wait(smem_u32(q_moved), 0, p.err, abort_flag);
+        // both CTAs' Q tiles complete on the leader's barrier
+        if (leader) mbar_arrive_expect_tx(smem_u32(q_full), 2 * AP_Q_BYTES);
+        const uint32_t qb = mapa_shared(smem_u32(q_full), 0);
+        for (int c = 0; c < 4; ++c) tma_load_3d_pair(smem_u32(sQ + c * (128 * 128)), &tmQ, qb, c * 64, q0, bh);
       }
       for (int j = 0; j < nkv && ok; ++j) {
-        const int s = j % AP3_STAGES;
-        const uint32_t ph = (j / AP3_STAGES) & 1;
+        const int s = j % nst;
+        const uint32_t ph = (j / nst) & 1;
         if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1u, p.err, abort_flag)) { ok = false; break; }
         if (leader) mbar_arrive_expect_tx(smem_u32(&full[s]), 2 * half);
         const uint32_t fb = mapa_shared(smem_u32(&full[s]), 0);
@@ -838,32 +859,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AP3_THREADS, 1)
             tma_load_3d_pair(smem_u32(buf + s * half + c * (AP_BN * 128)), &tmV, fb,
                              static_cast<int>(rank) * 128 + c * 64, key0, bh);
         }
-        issued = true;
       }
-      if (!ok && issued) {
+      if (!ok) {  // let copies already in flight land before the CTA exits
         const uint64_t t0 = globaltimer();
         while (globaltimer() - t0 < 200000ull) {
         }
       }
     }
   } else if (warp == 1) {
-    // S issuer: S_j into the single S buffer once the K half of tile j has
-    // landed and the softmax warps of both CTAs have read S_{j-1}
+    // S issuer: S_j into the single S buffer once K_j has landed and the
+    // softmax warps of both CTAs have read S_{j-1}
     if (lane == 0 && leader) {
       const uint32_t idesc_qk = make_idesc_bf16(256, AP_BN, false, false);
-      bool ok = mbar_wait(smem_u32(q_tmem), 0, p.err, abort_flag);
+      bool ok = mbar_wait(smem_u32(q_full), 0, p.err, abort_flag);
+      const uint64_t qdesc = make_sdesc(smem_u32(sQ), 16, 1024, SWZ_128B);
       for (int j = 0; j < nkv && ok; ++j) {
-        const int s = j % AP3_STAGES;
-        if (!mbar_wait(smem_u32(&k_full[s]), (j / AP3_STAGES) & 1, p.err, abort_flag)) { ok = false; break; }
+        const int s = j % PAIR_KST;
+        if (!mbar_wait(smem_u32(&k_full[s]), (j / PAIR_KST) & 1, p.err, abort_flag)) { ok = false; break; }
         if (j > 0 && !mbar_wait(smem_u32(s_empty), (j - 1) & 1, p.err, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t kaddr = smem_u32(sK + s * AP_KH_BYTES);
-        const uint64_t kdesc = make_sdesc(kaddr, 16, 1024, SWZ_128B);
+        const uint64_t kdesc = make_sdesc(smem_u32(sK + s * AP_KH_BYTES), 16, 1024, SWZ_128B);
 #pragma unroll
         for (int kk = 0; kk < AT_HD / 16; ++kk) {
           const uint32_t c = kk >> 2, off = (kk & 3) * 32;
+          const uint64_t ad = qdesc + static_cast<uint64_t>((c * (128 * 128) + off) >> 4);
           const uint64_t bd = kdesc + static_cast<uint64_t>((c * (64 * 128) + off) >> 4);
-          mma_bf16_ts_pair(tS, tQ + kk * 8, bd, idesc_qk, kk > 0 ? 1u : 0u);
+          mma_bf16_ss_pair(tS, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
         }
         mma_commit_pair(smem_u32(s_full), 0x3);
         mma_commit_pair(smem_u32(&k_empty[s]), 0x3);
@@ -871,29 +892,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AP3_THREADS, 1)
       mma_commit_pair(smem_u32(mma_done), 0x1);
       mbar_wait(smem_u32(mma_done), 0, nullptr, &never, 100000000ull);
     }
-  } else if (warp == AP3_PV_WARP) {
-    // PV issuer: O += P_j V_j once P_j is published and the V half of tile j
-    // has landed.  With two issuing threads, one thread's barrier checks
-    // overlap the other's MMAs in the tensor pipe (one thread doing both left
-    // a gap of a few hundred cycles at every S / PV switch for its checks).
+  } else if (warp == PAIR_PV_WARP) {
+    // PV issuer: O += P_j V_j once P_j is published (TMEM buffer j & 1, the A
+    // operand) and V_j has landed
     if (lane == 0 && leader) {
       const uint32_t idesc_pv = make_idesc_bf16(256, AT_HD, false, true);
-      const uint64_t pdesc = make_sdesc(smem_u32(sP), 16, 1024, SWZ_128B);
       bool ok = true;
       for (int j = 0; j < nkv && ok; ++j) {
-        const int s = j % AP3_STAGES;
-        if (!mbar_wait(smem_u32(p_full), j & 1, p.err, abort_flag)) { ok = false; break; }
-        if (!mbar_wait(smem_u32(&v_full[s]), (j / AP3_STAGES) & 1, p.err, abort_flag)) { ok = false; break; }
+        const int s = j % PAIR_VST;
+        if (!mbar_wait(smem_u32(&p_full[j & 1]), (j >> 1) & 1, p.err, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(smem_u32(&v_full[s]), (j / PAIR_VST) & 1, p.err, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint64_t vdesc = make_sdesc(smem_u32(sV + s * AP_VH_BYTES), AP_BN * 128, 1024, SWZ_128B);
 #pragma unroll
         for (int kk = 0; kk < AP_BN / 16; ++kk) {
-          const uint32_t c = kk >> 2, off = (kk & 3) * 32;
-          const uint64_t ad = pdesc + static_cast<uint64_t>((c * (128 * 128) + off) >> 4);
           const uint64_t bd = vdesc + static_cast<uint64_t>((kk * (16 * 128)) >> 4);
-          mma_bf16_ss_pair(tO, ad, bd, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+          mma_bf16_ts_pair(tO, tP + 64 * (j & 1) + kk * 8, bd, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
         }
-        mma_commit_pair(smem_u32(pv_done), 0x3);
+        mma_commit_pair(smem_u32(&pv_done[j & 1]), 0x3);
         mma_commit_pair(smem_u32(&v_empty[s]), 0x3);
       }
       mma_commit_pair(smem_u32(mma_done_pv), 0x1);
@@ -905,60 +921,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AP3_THREADS, 1)
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const int g64 = wg >> 1;                  // 64-key chunk of a P row this group writes
-    const int u0 = (wg & 1) * 4;              // its first 16-byte unit in that chunk
     const float c = p.scale_log2;
     const float off = -QKN_OFFSET_LOG2;
     int klo, khi;
     key_mask_range(p, b, klo, khi);
     const uint32_t s_empty_l = mapa_shared(smem_u32(s_empty), 0);
-    const uint32_t p_full_l = mapa_shared(smem_u32(p_full), 0);
     float l = 0.f;
     bool ok = true;
-    {
-      // Q chunk wg (head-dim columns [64 wg, +64)) of this warp's 32 rows,
-      // from V stage wg / 2 into TMEM columns [32 wg, +32); then V stages 0
-      // and 1 are released to the V loads
-      const bool got = mbar_wait(smem_u32(q_smem), 0, p.err, abort_flag);
-      __syncwarp();
-      if (!__all_sync(0xffffffffu, got)) {
-        ok = false;
-      } else {
-        const uint8_t* qrow = sV + wg * (128 * 128) + row * 128;
-        uint32_t qv[32];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const uint4 u = *reinterpret_cast<const uint4*>(qrow + ((q ^ (row & 7)) << 4));
-          qv[4 * q] = u.x;
-          qv[4 * q + 1] = u.y;
-          qv[4 * q + 2] = u.z;
-          qv[4 * q + 3] = u.w;
-        }
-        tmem_st32(tQ + wg * 32 + lane_off, qv);
-        tmem_wait_st();
-        tc_fence_before();
-        fence_proxy_async_smem();   // the generic reads of Q precede the V loads into the same bytes
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive_cluster(mapa_shared(smem_u32(q_tmem), 0));
-          mbar_arrive(smem_u32(q_moved));
-        }
-      }
-    }
-    for (int j = 0; j < nkv && ok; ++j) {
+    // S_j out of TMEM into r (this group's 32 columns), then S is released
+    uint32_t r[32];
+    auto read_s = [&](int j) -> bool {
       const bool got = mbar_wait(smem_u32(s_full), j & 1, p.err, abort_flag);
       __syncwarp();
-      if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+      if (!__all_sync(0xffffffffu, got)) return false;
       tc_fence_after();
-      uint32_t r[32];
-      tmem_ld32(tS + AP3_KPW * wg + lane_off, r);
+      tmem_ld32(tS + PAIR_KPW * wg + lane_off, r);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(s_empty_l);
-      const int kbase = kv_tile(j) * AP_BN + AP3_KPW * wg;
+      return true;
+    };
+    if (ok && nkv > 0) ok = read_s(0);
+    bool have_next = true;  // r holds S_j at the top of iteration j
+    for (int j = 0; j < nkv && ok; ++j) {
+      if (!have_next && !read_s(j)) { ok = false; break; }
+      const int kbase = kv_tile(j) * AP_BN + PAIR_KPW * wg;
       const int kvalid = p.N - kbase, mlo = klo - kbase, mhi = khi - kbase;
-      const bool partial = kvalid < AP3_KPW || (mlo < mhi && mlo < AP3_KPW && mhi > 0);
+      const bool partial = kvalid < PAIR_KPW || (mlo < mhi && mlo < PAIR_KPW && mhi > 0);
       auto dead = [&](int i) { return i >= kvalid || (i >= mlo && i < mhi); };
       uint32_t pk[16];
       float rs0 = 0.f, rs1 = 0.f;
@@ -980,29 +970,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AP3_THREADS, 1)
         pk[8 + i] = pack_bf16(e2, e3);
       }
       l += rs0 + rs1;
-      // the single P buffer is free once PV_{j-1} has completed
-      if (j >= 1) {
-        const bool g2 = mbar_wait(smem_u32(pv_done), (j - 1) & 1, p.err, abort_flag);
+      // S_{j+1} now if it has completed (the S product after it can start
+      // while P_j is stored), otherwise after P_j
+      have_next = false;
+      if (j + 1 < nkv && __all_sync(0xffffffffu, mbar_test(smem_u32(s_full), (j + 1) & 1))) {
+        if (!read_s(j + 1)) { ok = false; break; }
+        have_next = true;
+      }
+      // P buffer j & 1 is free once PV_{j-2} has completed
+      if (j >= 2) {
+        const bool g2 = mbar_wait(smem_u32(&pv_done[j & 1]), ((j - 2) >> 1) & 1, p.err, abort_flag);
         __syncwarp();
         if (!__all_sync(0xffffffffu, g2)) { ok = false; break; }
       }
-      uint8_t* prow = sP + g64 * (128 * 128) + row * 128;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint4 v = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-        *reinterpret_cast<uint4*>(prow + (((u0 + q) ^ (row & 7)) << 4)) = v;
-      }
-      fence_proxy_async_smem();
+      // this group's 32 keys of P_j (two per 32-bit column, in key order) into
+      // columns [16 wg, 16 wg + 16) of TMEM buffer j & 1
+      tmem_st16(tP + 64 * (j & 1) + 16 * wg + lane_off, pk);
+      tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(p_full_l);
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&p_full[j & 1]), 0));
     }
     if (ok) {
-      // the last PV has read P: the buffer takes the row sums
+      // after the last PV no V stage is read any more: V stage 0 takes the row sums
       const int jl = nkv - 1;
-      const bool g3 = mbar_wait(smem_u32(pv_done), jl & 1, p.err, abort_flag);
+      const bool g3 = mbar_wait(smem_u32(&pv_done[jl & 1]), (jl >> 1) & 1, p.err, abort_flag);
       __syncwarp();
       if (__all_sync(0xffffffffu, g3)) {
+        float* xsum = reinterpret_cast<float*>(sV);  // [wg 4][row 128]
         xsum[wg * 128 + row] = l;
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(lbar));
@@ -1096,7 +1091,7 @@ cudaError_t attention_set_attributes() {
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(attn_hd256_qknorm, cudaFuncAttributeMaxDynamicSharedMemorySize, QKN_SMEM);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(attn_hd256_qknorm_pair3, cudaFuncAttributeMaxDynamicSharedMemorySize, AP3_SMEM);
+  e = cudaFuncSetAttribute(attn_hd256_qknorm_pair, cudaFuncAttributeMaxDynamicSharedMemorySize, PAIR_SMEM);
   if (e != cudaSuccess) return e;
   done |= uint64_t(1) << dev;
   return cudaSuccess;
@@ -1120,7 +1115,7 @@ cudaError_t launch_attention(const AttnParams& p, const uint16_t* q, const uint1
       CUtensorMap tv2;  // V halves: 128 keys x 64 columns per box
       if (!encode_tmap_3d(&tv2, v, AT_HD, p.N, bh, rb, sb, 64, AP_BN, 1)) return cudaErrorInvalidValue;
       dim3 grid2(2 * ((p.N + 255) / 256), p.H, p.B);
-      attn_hd256_qknorm_pair3<<<grid2, AP3_THREADS, AP3_SMEM, stream>>>(tq, tk, tv2, p);
+      attn_hd256_qknorm_pair<<<grid2, PAIR_THREADS, PAIR_SMEM, stream>>>(tq, tk, tv2, p);
       return cudaGetLastError();
     }
     dim3 grid((p.N + AT_BM - 1) / AT_BM, p.H, p.B);
