@@ -900,8 +900,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
       bool ok = true;
       for (int j = 0; j < nkv && ok; ++j) {
         const int s = j % PAIR_VST;
-        if (!mbar_wait(smem_u32(&p_full[j & 1]), (j >> 1) & 1, p.err, abort_flag)) { ok = false; break; }
+        // V first: it has normally landed long before P_j, so its check is
+        // off the path from P_j's publication to the first PV instruction
         if (!mbar_wait(smem_u32(&v_full[s]), (j / PAIR_VST) & 1, p.err, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(smem_u32(&p_full[j & 1]), (j >> 1) & 1, p.err, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint64_t vdesc = make_sdesc(smem_u32(sV + s * AP_VH_BYTES), AP_BN * 128, 1024, SWZ_128B);
 #pragma unroll
