@@ -1009,31 +1009,39 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
           tc_fence_after();
           const float tot = xsum[row] + xsum[128 + row] + xsum[256 + row] + xsum[384 + row];
           const float inv = 1.0f / tot;
-          const int qrow = q0 + row;
-          const bool row_ok = qrow < p.N;
-          uint16_t* dst = nullptr;
-          if (row_ok) {
-            if (qrow < p.split)
-              dst = p.out_a + (static_cast<size_t>(b) * p.split + qrow) * p.ldo + h * AT_HD;
-            else
-              dst = p.out_b + (static_cast<size_t>(b) * (p.N - p.split) + (qrow - p.split)) * p.ldo + h * AT_HD;
-            dst += 64 * wg;
-          }
+          // this warp's 32 rows x 64 columns of O, normalised, through shared
+          // memory (the Q tile's bytes: every S product has completed) so that
+          // the global stores are row-contiguous: thread = row when reading
+          // TMEM, 8 lanes per 128-byte row segment when writing out
+          uint8_t* stage = sQ + wg * (128 * 128);  // [128 rows][128 bytes], 16-byte units XOR-swizzled
           for (int cc = 0; cc < 2; ++cc) {
             uint32_t o[32];
             tmem_ld32(tO + 64 * wg + cc * 32 + lane_off, o);
             tmem_wait_ld();
-            if (row_ok) {
-              uint4* d = reinterpret_cast<uint4*>(dst + cc * 32);
 #pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                uint4 u;
-                u.x = pack_bf16(__uint_as_float(o[8 * i + 0]) * inv, __uint_as_float(o[8 * i + 1]) * inv);
-                u.y = pack_bf16(__uint_as_float(o[8 * i + 2]) * inv, __uint_as_float(o[8 * i + 3]) * inv);
-                u.z = pack_bf16(__uint_as_float(o[8 * i + 4]) * inv, __uint_as_float(o[8 * i + 5]) * inv);
-                u.w = pack_bf16(__uint_as_float(o[8 * i + 6]) * inv, __uint_as_float(o[8 * i + 7]) * inv);
-                d[i] = u;
-              }
+            for (int i = 0; i < 4; ++i) {
+              uint4 u;
+              u.x = pack_bf16(__uint_as_float(o[8 * i + 0]) * inv, __uint_as_float(o[8 * i + 1]) * inv);
+              u.y = pack_bf16(__uint_as_float(o[8 * i + 2]) * inv, __uint_as_float(o[8 * i + 3]) * inv);
+              u.z = pack_bf16(__uint_as_float(o[8 * i + 4]) * inv, __uint_as_float(o[8 * i + 5]) * inv);
+              u.w = pack_bf16(__uint_as_float(o[8 * i + 6]) * inv, __uint_as_float(o[8 * i + 7]) * inv);
+              const int unit = cc * 4 + i;
+              *reinterpret_cast<uint4*>(stage + row * 128 + ((unit ^ (row & 7)) << 4)) = u;
+            }
+          }
+          __syncwarp();
+          const int unit = lane & 7;
+#pragma unroll
+          for (int it = 0; it < 8; ++it) {
+            const int rr = quarter * 32 + it * 4 + (lane >> 3);  // a row of this warp
+            const int qrow = q0 + rr;
+            if (qrow < p.N) {
+              uint16_t* dst =
+                  qrow < p.split
+                      ? p.out_a + (static_cast<size_t>(b) * p.split + qrow) * p.ldo
+                      : p.out_b + (static_cast<size_t>(b) * (p.N - p.split) + (qrow - p.split)) * p.ldo;
+              const uint4 u = *reinterpret_cast<const uint4*>(stage + rr * 128 + ((unit ^ (rr & 7)) << 4));
+              *reinterpret_cast<uint4*>(dst + h * AT_HD + 64 * wg + unit * 8) = u;
             }
           }
         }
