@@ -829,9 +829,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
   volatile int never = 0;
 
   if (warp == 0 || warp == PAIR_V_WARP) {
-    // warp 0: this CTA's Q tile (into the V stages), then the K halves (keys
-    // [64 rank, +64) of each tile); the V warp: the V halves (head-dim
-    // columns [128 rank, +128))
+    // warp 0: this CTA's Q tile, then the K halves (keys [64 rank, +64) of
+    // each tile); the V warp: the V halves (head-dim columns [128 rank, +128))
     if (lane == 0) {
       const bool is_k = warp == 0;
       const int nst = is_k ? PAIR_KST : PAIR_VST;
