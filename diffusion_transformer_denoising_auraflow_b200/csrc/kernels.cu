@@ -180,13 +180,9 @@ __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
   asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
-// the two bf16 halves of w as a packed fp32 pair
-__device__ __forceinline__ uint64_t f2_from_bf16x2(uint32_t w) {
-  return f2_pack(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
-}
-// the same, kept opaque to common-subexpression elimination: a row held as
-// bf16 pairs is expanded again in each pass instead of being cached as fp32
-// (twice the registers)
+// the two bf16 halves of w as a packed fp32 pair, kept opaque to
+// common-subexpression elimination: a row held as bf16 pairs is expanded
+// again in each pass instead of being cached as fp32 (twice the registers)
 __device__ __forceinline__ uint64_t f2_from_bf16x2_each(uint32_t w) {
   uint64_t r;
   asm volatile(
