@@ -29,16 +29,19 @@ __device__ __forceinline__ float warp_sum(float v) {
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
 }
-__device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
-}
 
 // Per-row e4m3 scaling (the 8-bit GEMM inputs): a = max |row|, codes
 // e4m3(x * (448 / a)), scale a / 448 (1 and zeros for an all-zero row).
 __device__ __forceinline__ float e4m3_inv_scale(float amax) { return amax > 0.f ? 448.0f / amax : 1.0f; }
 __device__ __forceinline__ float e4m3_scale(float amax) { return amax > 0.f ? amax / 448.0f : 1.0f; }
+
+// max |v| over the full warp in one instruction (sm_100a f32 redux; NaN
+// inputs are ignored, as fmaxf does)
+__device__ __forceinline__ float redux_max_abs(float v) {
+  float r;
+  asm volatile("redux.sync.max.abs.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+  return r;
+}
 
 // ------------------------------------------------------------------ LN + modulate
 template <int VPL, bool OUT8>  // 8-element vectors per lane; OUT8: e4m3 codes + row scale
@@ -104,7 +107,7 @@ __global__ void __launch_bounds__(256) ln_modulate_kernel(const uint16_t* __rest
     }
   }
   if constexpr (OUT8) {
-    amax = warp_max(amax);
+    amax = redux_max_abs(amax);
     const float inv = e4m3_inv_scale(amax);
     uint2* yr = reinterpret_cast<uint2*>(y8 + static_cast<size_t>(warp) * D);
 #pragma unroll
@@ -132,19 +135,19 @@ __global__ void __launch_bounds__(256) ln_modulate_kernel(const uint16_t* __rest
   }
 }
 
-// Wide rows (D = 3072), HBM-bound: rows are streamed into shared memory by
-// bulk copies, 2 stages of 4 rows per CTA and three CTAs per SM (144 KB in
-// flight per SM).  The producer warp first copies the CTA's sample's scale
-// and shift (bulk copies as well: staged by a strided load loop they cost
-// ~24 serialised L2 round trips per CTA before the first row), then streams
-// rows.  Each consumer warp normalises one row of a stage, the row held in
-// registers (two passes for mean and variance, then the output), the
-// arithmetic on packed fp32 pairs (sm_100 f32x2).  Three smaller CTAs per SM
-// keep more warps issuing than one CTA with 8 rows x 4 stages: 26.7 against
-// 30.8 us per [8720, 3072] call with the input in L2, 30.8 against 34.2 us
-// from DRAM.  One launch serves up to two problems (the joint block's image
-// and text streams), CTAs split between them in proportion to their rows;
-// 1-D grid: segment 0's samples x CTAs per sample, then segment 1's.
+// Wide rows (D = 3072), HBM-bound: rows stream into shared memory by bulk
+// copies, stages of LNB_ROWS rows (LNB_STAGES stages) per CTA, LNB_PER_SM
+// CTAs per SM.  The producer warp first bulk-copies the CTA's sample's scale
+// and shift, then streams rows.  The LNB_CW consumer warps split the columns,
+// not the rows: each owns a fixed set of 16-byte column vectors of every row,
+// so its (1 + scale) and shift stay in registers for the CTA's lifetime; a
+// warp loads its part of the stage's rows into registers and hands the stage
+// back at once, and the row statistics (two-pass mean and variance, then the
+// e4m3 row maximum for 8-bit output) are combined across the consumer warps
+// through shared memory at named barrier 1.  Arithmetic on packed fp32 pairs
+// (sm_100 f32x2).  One launch serves up to two problems (the joint block's
+// image and text streams), CTAs split between them in proportion to their
+// rows; 1-D grid: segment 0's samples x CTAs per sample, then segment 1's.
 constexpr int LNB_D = 3072;
 constexpr int LNB_ROWS = 2;     // rows per stage
 constexpr int LNB_STAGES = 4;
@@ -364,6 +367,7 @@ __global__ void __launch_bounds__(LNB_THREADS, LNB_PER_SM) ln_modulate_bulk_kern
     }
     asm volatile("bar.sync 1, %0;" ::"r"(32 * LNB_CW) : "memory");
     const int nrows = min(LNB_ROWS, rows_per_batch - c * LNB_ROWS);
+    uint64_t q[LNB_ROWS][VPW][4];  // 8-bit output: the rows' outputs, kept until the row maxima are known
 #pragma unroll
     for (int rr = 0; rr < LNB_ROWS; ++rr) {
       const float rstd = rsqrtf(total(red[1][rr]) * (1.0f / LNB_D) + eps);
@@ -379,15 +383,14 @@ __global__ void __launch_bounds__(LNB_THREADS, LNB_PER_SM) ln_modulate_bulk_kern
         float amax = 0.f;
 #pragma unroll
         for (int i = 0; i < VPW; ++i) {
-          uint64_t o[4];
-          outv(i, o);
+          outv(i, q[rr][i]);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float2 v = f2_unpack(o[e]);
+            const float2 v = f2_unpack(q[rr][i][e]);
             amax = fmaxf(amax, fmaxf(fabsf(v.x), fabsf(v.y)));
           }
         }
-        amax = warp_max(amax);
+        amax = redux_max_abs(amax);
         if (lane == 0) red[2][rr][warp] = amax;
       } else if (rr < nrows) {
         uint4* yr = reinterpret_cast<uint4*>(y + static_cast<size_t>(r) * LNB_D);
@@ -409,18 +412,13 @@ __global__ void __launch_bounds__(LNB_THREADS, LNB_PER_SM) ln_modulate_bulk_kern
         if (rr >= nrows) continue;
         const float amax = largest(red[2][rr]);
         const float inv = e4m3_inv_scale(amax);
-        const float mean = total(red[0][rr]) * (1.0f / LNB_D);
-        const float rstd = rsqrtf(total(red[1][rr]) * (1.0f / LNB_D) + eps);
-        const uint64_t nmr = f2_pack(-mean, -mean), rs2 = f2_pack(rstd, rstd);
         const int r = c * LNB_ROWS + rr;
         uint2* yr = reinterpret_cast<uint2*>(y8 + static_cast<size_t>(r) * LNB_D);
 #pragma unroll
         for (int i = 0; i < VPW; ++i) {
-          const uint32_t w[4] = {u[rr][i].x, u[rr][i].y, u[rr][i].z, u[rr][i].w};
           float2 v[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            v[e] = f2_unpack(f2_fma(f2_mul(f2_add(f2_from_bf16x2_each(w[e]), nmr), rs2), av[i][e], hv[i][e]));
+          for (int e = 0; e < 4; ++e) v[e] = f2_unpack(q[rr][i][e]);
           yr[v0 + 32 * i] = make_uint2(pack_e4m3x4(v[0].x * inv, v[0].y * inv, v[1].x * inv, v[1].y * inv),
                                        pack_e4m3x4(v[2].x * inv, v[2].y * inv, v[3].x * inv, v[3].y * inv));
         }
@@ -525,7 +523,7 @@ __global__ void __launch_bounds__(256) quantize_rows_e4m3_kernel(const uint16_t*
 #pragma unroll
     for (int e = 0; e < 4; ++e) amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(w[e])), fabsf(bf16_hi(w[e]))));
   }
-  amax = warp_max(amax);
+  amax = redux_max_abs(amax);
   const float inv = e4m3_inv_scale(amax);
   uint2* qr = reinterpret_cast<uint2*>(q + static_cast<size_t>(row) * K);
   for (int vi = lane; vi < nvec; vi += 32) {
@@ -557,7 +555,7 @@ __global__ void __launch_bounds__(256) quantize_wide_rows_e4m3_kernel(const uint
 #pragma unroll
     for (int e = 0; e < 4; ++e) amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(w[e])), fabsf(bf16_hi(w[e]))));
   }
-  amax = warp_max(amax);
+  amax = redux_max_abs(amax);
   if (lane == 0) wmax[warp] = amax;
   __syncthreads();
   amax = wmax[0];
