@@ -71,6 +71,7 @@ _SIGS = {
     "af_scratch_create": [_P, _I, _I, _I, _P],
     "af_scratch_destroy": [_P],
     "af_sync": [_P, _P],
+    "af_check_wait_timeout": [_P, ctypes.c_int64, _P],
     "af_timestep_embed": [_P, _P, _P, _I, _P, _P],
     "af_timestep_embed_noalloc": [_P, _P, _I, _P, _P],
     "af_patch_embed": [_P, _P, _P, _I, _I, _I, _P, _P],
@@ -369,6 +370,11 @@ class Scratch:
 
     def sync(self, stream=None):
         _check(lib.af_sync(self.handle, _stream(stream)), "af_sync")
+
+    def check_wait_timeout(self, limit_ns=20_000_000, stream=None):
+        """Run the device timeout path on purpose (af_check_wait_timeout): the
+        next sync() raises AFError with AF_ERR_TIMEOUT."""
+        _check(lib.af_check_wait_timeout(self.handle, int(limit_ns), _stream(stream)), "af_check_wait_timeout")
 
     def launch_counts(self):
         """Launches of this library's kernels through this scratch: [gemm, attention, ln, other]."""

@@ -115,6 +115,9 @@ struct LnSegment {
 cudaError_t launch_ln_modulate_pair(LnSegment g0, LnSegment g1, int mod_stride, int D, float eps, cudaStream_t s,
                                     int* err);
 cudaError_t launch_quantize_rows_e4m3(const uint16_t* x, int rows, int K, uint8_t* q, float* scale, cudaStream_t s);
+// The bounded-wait check: one CTA waits on an mbarrier phase nothing completes
+// for limit_ns, records the timeout in *err and returns (kernels.cu).
+cudaError_t launch_wait_timeout_check(int* err, uint64_t limit_ns, cudaStream_t s);
 cudaError_t launch_timestep_mlp(const float* t, int B, const uint16_t* w1, const uint16_t* b1, const uint16_t* w2,
                                 const uint16_t* b2, int C, int D, float* feat, float* h1, float* temb, cudaStream_t s);
 cudaError_t launch_modulation(const float* temb, int B, int D, const uint16_t* w, int rows, float* out,

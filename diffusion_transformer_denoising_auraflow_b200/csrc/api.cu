@@ -1194,6 +1194,15 @@ af_status af_sync(af_scratch* s, void* stream) {
   return AF_OK;
 }
 
+af_status af_check_wait_timeout(af_scratch* s, int64_t limit_ns, void* stream) {
+  if (!s) return AF_ERR_INVALID_ARG;
+  const int64_t lim = limit_ns < 1000000 ? 1000000 : (limit_ns > 1000000000 ? 1000000000 : limit_ns);
+  LaunchScope ls(s, KC_OTHER, 0.0, static_cast<cudaStream_t>(stream));
+  cudaError_t e = launch_wait_timeout_check(s->err, static_cast<uint64_t>(lim), static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  return AF_OK;
+}
+
 af_status af_timestep_embed(const af_weights* w, af_scratch* s, const float* t, int B, float* temb, void* stream) {
   AF_TRY(check_scratch(w, s));
   if (!t || !temb || B <= 0) return AF_ERR_INVALID_ARG;

@@ -648,6 +648,41 @@ static cudaError_t gemv_attr() {
                               GEMV_MAX_B * VPL * 256 * static_cast<int>(sizeof(float)));
 }
 
+// ------------------------------------------------------------------ bounded-wait check
+// The timeout path of every pipeline wait, run on purpose and without any
+// fault: the warp takes 32 TMEM columns as the tensor-core kernels do, waits
+// on an mbarrier phase that no thread completes, gives up after limit_ns
+// (recording the timeout in *err, as mbar_wait does for any expired wait),
+// and frees the columns before it exits.
+__global__ void __launch_bounds__(32) wait_timeout_check_kernel(int* err, uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ uint32_t slot;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncwarp();
+  tmem_alloc(smem_u32(&slot), 32);
+  tmem_relinquish();
+  tc_fence_before();
+  __syncwarp();
+  tc_fence_after();
+  const uint32_t tmem = slot;
+  mbar_wait(smem_u32(&bar), 0, err, &abort_flag, limit_ns);  // nothing arrives: runs out
+  tc_fence_before();
+  __syncwarp();
+  tc_fence_after();
+  tmem_dealloc(tmem, 32);
+}
+
+cudaError_t launch_wait_timeout_check(int* err, uint64_t limit_ns, cudaStream_t s) {
+  if (!err) return cudaErrorInvalidValue;
+  wait_timeout_check_kernel<<<1, 32, 0, s>>>(err, limit_ns);
+  return cudaGetLastError();
+}
+
 // Shared-memory opt-ins of this file's kernels, once per device.
 cudaError_t small_kernels_set_attributes() {
   static uint64_t done = 0;

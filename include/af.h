@@ -385,6 +385,20 @@ af_status af_linear_fp8(const uint8_t* A, const float* a_scale, const uint8_t* W
  * out: host float[n_steps + 1].  No device work. */
 af_status af_sigma_schedule(int n_steps, float shift, int num_train_timesteps, float* out);
 
+/* ---- failure detection --------------------------------------------------
+ * Every wait of the device code (mbarrier phases of the TMA / MMA / softmax
+ * pipelines) is bounded: a wait that runs out records AF_ERR_TIMEOUT in the
+ * scratch's error word, the kernel lets its in-flight copies and MMAs land
+ * (bounded as well), frees its TMEM and returns, and the next af_sync
+ * reports the timeout.  af_check_wait_timeout exercises that path without
+ * any fault: one CTA takes 32 TMEM columns, waits on an mbarrier phase that
+ * nothing completes, gives up after limit_ns nanoseconds (clamped to
+ * [1 ms, 1 s]; the pipelines' own limit is 4 s), records the timeout in
+ * s's error word, frees its TMEM and exits.  The next af_sync(s) then
+ * returns AF_ERR_TIMEOUT and clears the word; the context stays usable.
+ * Asynchronous on `stream`; AF_ERR_INVALID_ARG for a null scratch. */
+af_status af_check_wait_timeout(af_scratch* s, int64_t limit_ns, void* stream);
+
 /* ---- launch accounting and per-kernel-class timing ----------------------
  * Kernel classes: 0 tensor-core GEMM, 1 attention, 2 LayerNorm+modulate,
  * 3 other kernels (timestep/modulation GEMV, patch embed, output stage,

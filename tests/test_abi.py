@@ -58,6 +58,7 @@ def test_argument_errors_are_host_side():
     assert L.af_euler_cfg_step(None, None, 1, 4, 8, 8, 3.5, 1.0, 0.9, None) == 1
     assert L.af_ln_modulate(None, None, None, 0, None, 1, 1, 32, 1e-6, None) == 1
     assert L.af_sync(None, None) == 1
+    assert L.af_check_wait_timeout(None, 20_000_000, None) == 1
     assert L.af_transformer_forward(None, None, None, None, None, 1, 8, 8, 4, None, None, None) == 1
     assert L.af_status_string(6) == b"device wait timed out"
     out = ctypes.c_void_p()
