@@ -96,6 +96,7 @@ _SIGS = {
     "af_profile_end": [_P, _P, _P, _P, _P],
     "af_ln_modulate": [_P, _P, _P, _I, _P, _I, _I, _I, _F, _P],
     "af_linear": [_P, _P, _P, _I, _I, _I, _P],
+    "af_linear_grouped": [_P, _P, _P, _I, _I, _I, _P, _P, _P, _I, _I, _I, _P],
     "af_attention": [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _I, _I, _P],
     "af_weights_quantize_fp8": [_P, _I, _P],
     "af_quantize_rows_e4m3": [_P, _I, _I, _P, _P, _P],
@@ -591,6 +592,24 @@ def linear(A, W, C, stream=None):
     ap, wp, cp = c.dev(A, torch.bfloat16, "A"), c.dev(W, torch.bfloat16, "W"), c.dev(C, torch.bfloat16, "C")
     c.check()
     _check(lib.af_linear(ap, wp, cp, M, N, K, _stream(stream)), where)
+
+
+def linear_grouped(A0, W0, C0, A1, W1, C1, stream=None):
+    """C0 = A0 W0^T and C1 = A1 W1^T in one launch (af_linear_grouped)."""
+    where = "af_linear_grouped"
+    M0, K0 = A0.shape
+    N0 = W0.shape[0]
+    M1, K1 = A1.shape
+    N1 = W1.shape[0]
+    _need_shape(W0, (N0, K0), "W0", where)
+    _need_shape(C0, (M0, N0), "C0", where)
+    _need_shape(W1, (N1, K1), "W1", where)
+    _need_shape(C1, (M1, N1), "C1", where)
+    c = _Call(where)
+    a0, w0, c0 = c.dev(A0, torch.bfloat16, "A0"), c.dev(W0, torch.bfloat16, "W0"), c.dev(C0, torch.bfloat16, "C0")
+    a1, w1, c1 = c.dev(A1, torch.bfloat16, "A1"), c.dev(W1, torch.bfloat16, "W1"), c.dev(C1, torch.bfloat16, "C1")
+    c.check()
+    _check(lib.af_linear_grouped(a0, w0, c0, M0, N0, K0, a1, w1, c1, M1, N1, K1, _stream(stream)), where)
 
 
 def attention(q, k, v, o, qk_normalized: bool = False, key_len=None, key_base: int = 0, key_end: int = 0,

@@ -1703,9 +1703,8 @@ af_status af_linear_fp8(const uint8_t* A, const float* a_scale, const uint8_t* W
   return AF_OK;
 }
 
-af_status af_linear(const uint16_t* A, const uint16_t* W, uint16_t* C, int M, int N, int K, void* stream) {
-  if (!A || !W || !C || M <= 0 || N <= 0 || K <= 0) return AF_ERR_INVALID_ARG;
-  if (K % 8 != 0 || N % 8 != 0) return AF_ERR_UNSUPPORTED;
+// A plain bf16 product C[M, N] = A W^T as GEMM parameters.
+static GemmParams plain_gemm(uint16_t* C, int M, int N, int K) {
   GemmParams p;
   memset(&p, 0, sizeof(p));
   p.M = M;
@@ -1717,9 +1716,28 @@ af_status af_linear(const uint16_t* A, const uint16_t* W, uint16_t* C, int M, in
   p.out = C;
   p.ldo = N;
   p.err = nullptr;
+  return p;
+}
+
+af_status af_linear(const uint16_t* A, const uint16_t* W, uint16_t* C, int M, int N, int K, void* stream) {
+  if (!A || !W || !C || M <= 0 || N <= 0 || K <= 0) return AF_ERR_INVALID_ARG;
+  if (K % 8 != 0 || N % 8 != 0) return AF_ERR_UNSUPPORTED;
   static int sms = 0;
   if (!sms) sms = device_sm_count();
-  AF_CUDA(launch_gemm(p, A, W, N, static_cast<cudaStream_t>(stream), sms));
+  AF_CUDA(launch_gemm(plain_gemm(C, M, N, K), A, W, N, static_cast<cudaStream_t>(stream), sms));
+  return AF_OK;
+}
+
+af_status af_linear_grouped(const uint16_t* A0, const uint16_t* W0, uint16_t* C0, int M0, int N0, int K0,
+                            const uint16_t* A1, const uint16_t* W1, uint16_t* C1, int M1, int N1, int K1,
+                            void* stream) {
+  if (!A0 || !W0 || !C0 || M0 <= 0 || N0 <= 0 || K0 <= 0) return AF_ERR_INVALID_ARG;
+  if (!A1 || !W1 || !C1 || M1 <= 0 || N1 <= 0 || K1 <= 0) return AF_ERR_INVALID_ARG;
+  if (K0 % 8 != 0 || N0 % 8 != 0 || K1 % 8 != 0 || N1 % 8 != 0) return AF_ERR_UNSUPPORTED;
+  static int sms = 0;
+  if (!sms) sms = device_sm_count();
+  AF_CUDA(launch_gemm_grouped(plain_gemm(C0, M0, N0, K0), A0, W0, N0, plain_gemm(C1, M1, N1, K1), A1, W1, N1,
+                              static_cast<cudaStream_t>(stream), sms));
   return AF_OK;
 }
 

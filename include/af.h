@@ -428,6 +428,16 @@ af_status af_ln_modulate(const uint16_t* x, const float* shift, const float* sca
  *   K must be a multiple of 8 (16-byte rows for the TMA engine). */
 af_status af_linear(const uint16_t* A, const uint16_t* W, uint16_t* C, int M, int N, int K, void* stream);
 
+/* Two independent products C0 = A0 W0^T and C1 = A1 W1^T in one persistent
+ * CTA-pair launch, the second problem's tiles after the first's: the form
+ * the joint block gives its image- and text-stream projections ([ARCH]
+ * §联合注意力块, one set of projections per stream).  Shapes, layout and
+ * constraints as af_linear for each problem; when M0 + M1 < 1024 the two
+ * products run as two af_linear launches. */
+af_status af_linear_grouped(const uint16_t* A0, const uint16_t* W0, uint16_t* C0, int M0, int N0, int K0,
+                            const uint16_t* A1, const uint16_t* W1, uint16_t* C1, int M1, int N1, int K1,
+                            void* stream);
+
 /* Non-causal softmax(q k^T / sqrt(hd)) v per (batch, head) ([ARCH]
  * §注意力处理器与 QKV 融合).
  *   q, k, v: device bf16[B, H, N, hd];  o: device bf16[B, N, H*hd].

@@ -54,6 +54,7 @@ def test_argument_errors_are_host_side():
     import diffusion_transformer_denoising_auraflow_b200 as af
     L = af.lib
     assert L.af_linear(None, None, None, 4, 4, 4, None) == 1
+    assert L.af_linear_grouped(None, None, None, 4, 4, 4, None, None, None, 4, 4, 4, None) == 1
     assert L.af_attention(None, None, None, None, 1, 1, 1, 256, 0, None, 0, 0, None) == 1
     assert L.af_euler_cfg_step(None, None, 1, 4, 8, 8, 3.5, 1.0, 0.9, None) == 1
     assert L.af_ln_modulate(None, None, None, 0, None, 1, 1, 32, 1e-6, None) == 1

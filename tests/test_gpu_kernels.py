@@ -44,6 +44,36 @@ def test_linear_matches_fp64(af, M, N, K):
     assert np.all(np.abs(got - ref) <= 2 ** -8 * np.abs(ref) + 1e-4 * np.sqrt(K) * 0.02 * 4)
 
 
+# The joint block's grouped form (image- and text-stream projections in one
+# persistent launch) against the two products launched alone ("fused ==
+# unfused"): every output element is one full-K chain of tensor-core MMAs
+# in the same K order whichever tile, launch or CTA-group width computes it
+# (a problem below 1024 rows runs on the 1-CTA kernel alone and on CTA pairs
+# when grouped), so the two agree bit for bit; both are also held to fp64.
+@pytest.mark.parametrize("M0,N0,K0,M1,N1,K1", [(8192, 3072, 3072, 528, 3072, 3072),
+                                               (4096, 9216, 3072, 1030, 9216, 3072),
+                                               (1100, 776, 520, 300, 520, 200),
+                                               (300, 520, 200, 64, 96, 32)])
+def test_linear_grouped_equals_separate(af, M0, N0, K0, M1, N1, K1):
+    A0 = synth.normal(21, f"gA0_{M0}_{N0}_{K0}", (M0, K0), 1.0)
+    W0 = synth.normal(22, f"gW0_{M0}_{N0}_{K0}", (N0, K0), 0.02)
+    A1 = synth.normal(23, f"gA1_{M1}_{N1}_{K1}", (M1, K1), 1.0)
+    W1 = synth.normal(24, f"gW1_{M1}_{N1}_{K1}", (N1, K1), 0.02)
+    a0, w0, a1, w1 = to_bf16(A0), to_bf16(W0), to_bf16(A1), to_bf16(W1)
+    G0 = torch.empty(M0, N0, dtype=torch.bfloat16, device="cuda")
+    G1 = torch.empty(M1, N1, dtype=torch.bfloat16, device="cuda")
+    S0 = torch.empty_like(G0)
+    S1 = torch.empty_like(G1)
+    af.linear_grouped(a0, w0, G0, a1, w1, G1)
+    af.linear(a0, w0, S0)
+    af.linear(a1, w1, S1)
+    torch.cuda.synchronize()
+    for G, S, A, W in ((G0, S0, A0, W0), (G1, S1, A1, W1)):
+        assert torch.equal(G, S)
+        ref = A.astype(np.float64) @ W.astype(np.float64).T
+        assert O.rel_l2(to_np(G), ref) < 3e-3
+
+
 def test_linear_rejects_unaligned_k(af):
     A = torch.zeros(4, 12, dtype=torch.bfloat16, device="cuda")
     W = torch.zeros(8, 12, dtype=torch.bfloat16, device="cuda")
