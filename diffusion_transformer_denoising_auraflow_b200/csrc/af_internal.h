@@ -39,9 +39,11 @@ struct GemmParams {
   // readable 32 rows past every weight row the GEMM touches (pad to 256)
   const float* a_scale = nullptr;
   const float* w_scale = nullptr;
-  // GATE_RES: nonzero when the residual tiles move by TMA (set by the
-  // launcher when `out` is 16-byte aligned, ldo * 2 a multiple of 16 and the
-  // output rows are the GEMM rows)
+  // nonzero when the epilogue's output tiles move by TMA through shared
+  // memory (set by the launcher): GATE_RES (residual in and out) and SWIGLU
+  // when `out` is 16-byte aligned, ldo * 2 a multiple of 16 and the output
+  // rows are the GEMM rows; QKV when q, k and v are equally spaced buffers
+  // (one 3-D tensor map over the three)
   int res_tma = 0;
 };
 
@@ -59,7 +61,7 @@ constexpr int GEMM_SMEM_BYTES =
 bool encode_tmap_2d(CUtensorMap* map, const void* ptr, uint64_t inner, uint64_t outer, uint64_t row_bytes,
                     uint32_t box_inner, uint32_t box_outer, bool bytes = false, int swizzle_bytes = 128);
 bool encode_tmap_3d(CUtensorMap* map, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1_bytes,
-                    uint64_t s2_bytes, uint32_t b0, uint32_t b1, uint32_t b2);
+                    uint64_t s2_bytes, uint32_t b0, uint32_t b1, uint32_t b2, int swizzle_bytes = 128);
 cudaError_t launch_gemm(const GemmParams& p_in, const void* A, const void* W, int W_rows, cudaStream_t stream,
                         int num_sms);
 // Two problems (same operand type) in one persistent CTA-pair launch, the

@@ -62,15 +62,16 @@ bool encode_tmap_2d(CUtensorMap* map, const void* ptr, uint64_t inner, uint64_t 
 }
 
 bool encode_tmap_3d(CUtensorMap* map, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1_bytes,
-                    uint64_t s2_bytes, uint32_t b0, uint32_t b1, uint32_t b2) {
+                    uint64_t s2_bytes, uint32_t b0, uint32_t b1, uint32_t b2, int swizzle_bytes) {
   auto enc = get_encode();
   if (!enc) return false;
   cuuint64_t dims[3] = {d0, d1, d2};
   cuuint64_t strides[2] = {s1_bytes, s2_bytes};
   cuuint32_t box[3] = {b0, b1, b2};
   cuuint32_t estr[3] = {1, 1, 1};
+  const CUtensorMapSwizzle sw = swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -150,84 +151,6 @@ __device__ __forceinline__ void acc_load32(const GemmParams& p, uint32_t taddr, 
   }
 }
 
-// QK-norm epilogue for one output row: columns [c0, c0 + width) of the tile
-// hold (256 / hd) heads of Q, K or V.  Q and K are LayerNorm-ed over each
-// head's hd values (two passes over TMEM: mean, then variance), V is stored as is.
-__device__ __forceinline__ void epilogue_qkv(const GemmParams& p, uint32_t tbase, int n0, bool row_ok, int b,
-                                             int n_in, float a_s) {
-  const int hd = p.hd;
-  const int tok = p.qkv_row_off + n_in;
-  if (hd >= 32) {
-    const int chunks = hd >> 5;
-    for (int h0 = 0; h0 < GEMM_BN; h0 += hd) {
-      const int col = n0 + h0;
-      if (col >= p.N) break;                       // uniform across the warp
-      const int which = col / p.D;
-      const int head = (col - which * p.D) / hd;
-      uint16_t* base = which == 0 ? p.q : (which == 1 ? p.k : p.v);
-      uint16_t* dst = base + ((static_cast<size_t>(b) * p.heads + head) * p.n_total + tok) * hd;
-      float mean = 0.f, rstd = 1.f;
-      float v[32];
-      if (which < 2) {
-        // one pass over TMEM: sums of (x - k) and (x - k)^2 with the shift k =
-        // the head's first value, so E[x^2] - mean^2 does not cancel when the
-        // mean is large against the spread
-        float k = 0.f, s1 = 0.f, s2 = 0.f;
-        for (int c = 0; c < chunks; ++c) {
-          acc_load32(p, tbase + h0 + c * 32, a_s, col + c * 32, v);
-          if (c == 0) k = v[0];
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const float d = v[j] - k;
-            s1 += d;
-            s2 += d * d;
-          }
-        }
-        const float m1 = s1 / hd;
-        mean = k + m1;
-        rstd = rsqrtf(fmaxf(s2 / hd - m1 * m1, 0.f) + p.eps);
-      }
-      for (int c = 0; c < chunks; ++c) {
-        acc_load32(p, tbase + h0 + c * 32, a_s, col + c * 32, v);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = (v[j] - mean) * rstd;
-        if (row_ok) store_bf16x32(dst + c * 32, v);
-      }
-    }
-  } else {
-    // small heads (hd in {8, 16}): each 32-column chunk holds 32 / hd heads
-    for (int c = 0; c < GEMM_BN / 32; ++c) {
-      if (n0 + c * 32 >= p.N) break;
-      float r[32];
-      acc_load32(p, tbase + c * 32, a_s, n0 + c * 32, r);
-      for (int s0 = 0; s0 < 32; s0 += hd) {
-        const int col = n0 + c * 32 + s0;
-        if (col >= p.N) break;
-        const int which = col / p.D;
-        const int head = (col - which * p.D) / hd;
-        uint16_t* base = which == 0 ? p.q : (which == 1 ? p.k : p.v);
-        uint16_t* dst = base + ((static_cast<size_t>(b) * p.heads + head) * p.n_total + tok) * hd;
-        float v[32];
-        float mean = 0.f, rstd = 1.f;
-        if (which < 2) {
-          float s = 0.f;
-          for (int j = 0; j < hd; ++j) s += r[s0 + j];
-          mean = s / hd;
-          float ss = 0.f;
-          for (int j = 0; j < hd; ++j) {
-            const float d = r[s0 + j] - mean;
-            ss += d * d;
-          }
-          rstd = rsqrtf(ss / hd + p.eps);
-        }
-        for (int j = 0; j < hd; ++j) v[j] = (r[s0 + j] - mean) * rstd;
-        if (row_ok)
-          for (int j = 0; j < hd; ++j) dst[j] = static_cast<uint16_t>(pack_bf16(v[j], 0.f) & 0xFFFFu);
-      }
-    }
-  }
-}
-
 // Gated-residual epilogue with TMA-staged residual tiles.  Each epilogue warp
 // owns 32 output rows of a tile and walks them in 32-column chunks; the
 // residual box of a chunk (32 x 32 bf16, 64-byte swizzle) is loaded by TMA
@@ -280,6 +203,121 @@ __device__ __forceinline__ void res_drain(ResStage& rs, bool lane0) {
   __syncwarp();
 }
 
+// Outputs through shared memory: a warp writes one 32 x 32 bf16 chunk of its
+// rows (thread = row, as read from TMEM) into the next of its two boxes and
+// lane 0 stores the box with one TMA store, so the global writes are whole
+// 64-byte row segments instead of every thread writing its own row; the
+// store that last read the box (two chunks earlier) has read it first.
+__device__ __forceinline__ uint32_t box_put(ResStage& rs, int lane, const float (&v)[32]) {
+  const uint32_t box = rs.buf + (rs.issued & 1u) * RES_BOX_BYTES;
+  if (lane == 0) bulk_wait_group_read1();
+  __syncwarp();
+  const uint32_t rowa = box + static_cast<uint32_t>(lane) * 64;
+  const uint32_t swz = static_cast<uint32_t>((lane >> 1) & 3);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint4 u = make_uint4(pack_bf16(v[8 * q + 0], v[8 * q + 1]), pack_bf16(v[8 * q + 2], v[8 * q + 3]),
+                               pack_bf16(v[8 * q + 4], v[8 * q + 5]), pack_bf16(v[8 * q + 6], v[8 * q + 7]));
+    sts128(rowa + ((static_cast<uint32_t>(q) ^ swz) << 4), u);
+  }
+  fence_proxy_async_smem();
+  __syncwarp();
+  ++rs.issued;  // no load uses the box: issued and used advance together
+  ++rs.used;
+  return box;
+}
+
+// QK-norm epilogue for one output row: the tile's columns hold (256 / hd)
+// heads of Q, K or V.  Q and K are LayerNorm-ed over each head's hd values,
+// V is stored as is.  With rs set (hd >= 32 and the warp's 32 rows valid
+// rows of sample b0, from token tok0 on) the normalised heads leave through
+// shared memory by TMA (tensor map tmo over q, k, v: [3][B H n_total][hd]).
+__device__ __forceinline__ void epilogue_qkv(const GemmParams& p, uint32_t tbase, int n0, bool row_ok, int b,
+                                             int n_in, float a_s, ResStage* rs = nullptr,
+                                             const CUtensorMap* tmo = nullptr, int lane = 0, int b0 = 0,
+                                             int tok0 = 0) {
+  const int hd = p.hd;
+  const int tok = p.qkv_row_off + n_in;
+  if (hd >= 32) {
+    const int chunks = hd >> 5;
+    for (int h0 = 0; h0 < GEMM_BN; h0 += hd) {
+      const int col = n0 + h0;
+      if (col >= p.N) break;                       // uniform across the warp
+      const int which = col / p.D;
+      const int head = (col - which * p.D) / hd;
+      uint16_t* base = which == 0 ? p.q : (which == 1 ? p.k : p.v);
+      uint16_t* dst = base + ((static_cast<size_t>(b) * p.heads + head) * p.n_total + tok) * hd;
+      float mean = 0.f, rstd = 1.f;
+      float v[32];
+      if (which < 2) {
+        // one pass over TMEM: sums of (x - k) and (x - k)^2 with the shift k =
+        // the head's first value, so E[x^2] - mean^2 does not cancel when the
+        // mean is large against the spread
+        float k = 0.f, s1 = 0.f, s2 = 0.f;
+        for (int c = 0; c < chunks; ++c) {
+          acc_load32(p, tbase + h0 + c * 32, a_s, col + c * 32, v);
+          if (c == 0) k = v[0];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float d = v[j] - k;
+            s1 += d;
+            s2 += d * d;
+          }
+        }
+        const float m1 = s1 / hd;
+        mean = k + m1;
+        rstd = rsqrtf(fmaxf(s2 / hd - m1 * m1, 0.f) + p.eps);
+      }
+      const int drow0 = (b0 * p.heads + head) * p.n_total + tok0;  // the warp's first destination row
+      for (int c = 0; c < chunks; ++c) {
+        acc_load32(p, tbase + h0 + c * 32, a_s, col + c * 32, v);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = (v[j] - mean) * rstd;
+        if (rs) {
+          const uint32_t box = box_put(*rs, lane, v);
+          if (lane == 0) {
+            tma_store_3d(tmo, box, c * 32, drow0, which);
+            bulk_commit_group();
+          }
+        } else if (row_ok) {
+          store_bf16x32(dst + c * 32, v);
+        }
+      }
+    }
+  } else {
+    // small heads (hd in {8, 16}): each 32-column chunk holds 32 / hd heads
+    for (int c = 0; c < GEMM_BN / 32; ++c) {
+      if (n0 + c * 32 >= p.N) break;
+      float r[32];
+      acc_load32(p, tbase + c * 32, a_s, n0 + c * 32, r);
+      for (int s0 = 0; s0 < 32; s0 += hd) {
+        const int col = n0 + c * 32 + s0;
+        if (col >= p.N) break;
+        const int which = col / p.D;
+        const int head = (col - which * p.D) / hd;
+        uint16_t* base = which == 0 ? p.q : (which == 1 ? p.k : p.v);
+        uint16_t* dst = base + ((static_cast<size_t>(b) * p.heads + head) * p.n_total + tok) * hd;
+        float v[32];
+        float mean = 0.f, rstd = 1.f;
+        if (which < 2) {
+          float s = 0.f;
+          for (int j = 0; j < hd; ++j) s += r[s0 + j];
+          mean = s / hd;
+          float ss = 0.f;
+          for (int j = 0; j < hd; ++j) {
+            const float d = r[s0 + j] - mean;
+            ss += d * d;
+          }
+          rstd = rsqrtf(ss / hd + p.eps);
+        }
+        for (int j = 0; j < hd; ++j) v[j] = (r[s0 + j] - mean) * rstd;
+        if (row_ok)
+          for (int j = 0; j < hd; ++j) dst[j] = static_cast<uint16_t>(pack_bf16(v[j], 0.f) & 0xFFFFu);
+      }
+    }
+  }
+}
+
 // Epilogue of one accumulator tile for one output row (thread = TMEM lane):
 // tbase addresses this warp's 32-lane quarter of the accumulator, m0 is the
 // first GEMM row of the tile half held in this CTA's TMEM, nb the n-tile.
@@ -292,13 +330,18 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tbas
   const size_t orow = static_cast<size_t>(b) * p.out_rows_per_batch + p.out_row_off + n_in;
   const float a_s = (p.a_scale && row_ok) ? p.a_scale[r] : 1.0f;
 
+  const int lane = row_in_tile & 31;
+  const int r0 = m0 + (row_in_tile & ~31);  // the warp's first row
   if (p.mode == EPI_QKV) {
-    epilogue_qkv(p, tbase, nb * GEMM_BN, row_ok, b, n_in, a_s);
+    // by TMA when the warp's 32 rows are valid rows of one sample
+    const int b0 = r0 / p.rows_per_batch;
+    const bool tma = p.res_tma && p.hd >= 32 && r0 + 31 < p.M && (r0 + 31) / p.rows_per_batch == b0;
+    epilogue_qkv(p, tbase, nb * GEMM_BN, row_ok, b, n_in, a_s, tma ? rs : nullptr, tmo, lane, b0,
+                 p.qkv_row_off + (r0 - b0 * p.rows_per_batch));
   } else if (p.mode == EPI_GATE_RES && p.res_tma) {
     // chunk 0's box was issued by the caller before the accumulator was ready
-    const int lane = row_in_tile & 31;
     const int col0 = nb * GEMM_BN;
-    const int wrow0 = m0 + (row_in_tile & ~31);
+    const int wrow0 = r0;
     const int nch = min(GEMM_BN / 32, (p.N - col0 + 31) / 32);
     const float* gb = row_ok ? p.gate + static_cast<size_t>(b) * p.gate_stride : nullptr;
     const uint32_t swz = static_cast<uint32_t>((lane >> 1) & 3);
@@ -354,7 +397,17 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tbas
 #pragma unroll
       for (int j = 0; j < 32; ++j) v[j] = silu_f(va[j]) * v[j];
       const int col = col0 + c * 32;
-      if (row_ok && col < p.N) store_bf16_n(p.out + orow * p.ldo + col, v, p.N - col);
+      if (p.res_tma) {  // rows past M and columns past N are clipped by the tensor map
+        if (col < p.N) {
+          const uint32_t box = box_put(*rs, lane, v);
+          if (lane == 0) {
+            tma_store_2d(tmo, box, col, r0);
+            bulk_commit_group();
+          }
+        }
+      } else if (row_ok && col < p.N) {
+        store_bf16_n(p.out + orow * p.ldo + col, v, p.N - col);
+      }
     }
   } else {
     const int col0 = nb * GEMM_BN;
@@ -822,6 +875,25 @@ static cudaError_t prepare_gemm(GemmParams& p, const void* A, const void* W, int
       p.out_row_off == 0) {
     if (encode_tmap_2d(to, p.out, p.N, p.M, static_cast<uint64_t>(p.ldo) * 2, 32, 32, false, 64)) p.res_tma = 1;
     else *to = *ta;
+  }
+  auto al16 = [](const void* a) { return (reinterpret_cast<uintptr_t>(a) & 15) == 0; };
+  if (p.mode == EPI_SWIGLU && p.out && al16(p.out) && (static_cast<uint64_t>(p.ldo) * 2) % 16 == 0 &&
+      p.ldo >= p.N && p.rows_per_batch == p.out_rows_per_batch && p.out_row_off == 0) {
+    if (encode_tmap_2d(to, p.out, p.N, p.M, static_cast<uint64_t>(p.ldo) * 2, 32, 32, false, 64)) p.res_tma = 1;
+    else *to = *ta;
+  }
+  if (p.mode == EPI_QKV && p.q && p.k && p.v && p.hd >= 32 && p.hd % 32 == 0 && p.rows_per_batch > 0 &&
+      p.M % p.rows_per_batch == 0 && p.n_total >= p.qkv_row_off + p.rows_per_batch) {
+    const char* q = reinterpret_cast<const char*>(p.q);
+    const ptrdiff_t dk = reinterpret_cast<const char*>(p.k) - q, dv = reinterpret_cast<const char*>(p.v) - q;
+    const uint64_t rows = static_cast<uint64_t>(p.M / p.rows_per_batch) * p.heads * p.n_total;
+    if (al16(q) && dk > 0 && dv == 2 * dk && dk % 16 == 0 &&
+        static_cast<uint64_t>(dk) >= rows * p.hd * 2 &&
+        encode_tmap_3d(to, p.q, p.hd, rows, 3, static_cast<uint64_t>(p.hd) * 2, static_cast<uint64_t>(dk), 32, 32, 1,
+                       64))
+      p.res_tma = 1;
+    else
+      *to = *ta;
   }
   p.num_n_tiles = p.mode == EPI_SWIGLU ? (p.N + 127) / 128 : (p.N + GEMM_BN - 1) / GEMM_BN;
   p.group_n = p.num_n_tiles < 16 ? p.num_n_tiles : 16;
