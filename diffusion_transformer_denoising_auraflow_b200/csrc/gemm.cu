@@ -16,8 +16,12 @@
 //               tcgen05.mma (M=128, N=256, K=16) into one of two 256-column
 //               fp32 accumulators, committing each stage back to the producer.
 //   warps 2..5  epilogue: tcgen05.ld of their 32-lane quarter (one thread =
-//               one output row), fused epilogue, global stores; the other
-//               accumulator is being filled meanwhile.
+//               one output row), fused epilogue; the outputs (and the gated
+//               residual) move through the warp's shared-memory boxes by TMA
+//               in 32 x 32 chunks where the layout allows, else by per-thread
+//               stores; the other accumulator is being filled meanwhile.
+// The large projections (M >= 1024) run the CTA-pair form below
+// (gemm_tcgen05_pair: 256 x 256 tiles, cta_group::2) with the same epilogues.
 // Every wait is bounded (ptx.cuh); a timeout sets the error word and the CTA
 // drains its outstanding copies and MMAs before releasing TMEM.
 #include <cstdio>
